@@ -1,0 +1,195 @@
+"""fp64 CPU oracle of the Mixtral sparse-MoE feed-forward layer.
+
+TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the
+benchmark's CPU-baseline leg may import or run this module. The CUDA path never
+does, and this module imports nothing from it: it shares no code, table or helper
+with the kernels. Inputs arrive as arrays of bf16 values (torch CPU tensors or numpy
+arrays); everything below is numpy in float64.
+
+What it computes, in the pages' own order (nnterp encyclopedia, "Mixtral"):
+
+1. router logits   l = x W_r^T, one per expert, no bias ("Values, by host":
+                   router_logits is the output of the router's F.linear, before the
+                   scoring; "Attention has no window": no projection has a bias);
+2. scoring         softmax over all E experts, keep the k largest, divide them by
+                   their sum; slot 0 holds the larger weight ("The router
+                   renormalizes its top 2, in float32");
+3. experts         per routed slot, down(act(gate x) * up x) with act = silu
+                   ("Values, by host": mlp_neurons is act(gate)*up, what the down
+                   projection receives; Hugging Face "Mixtral" doc, MixtralConfig:
+                   hidden_act silu);
+4. combine         expert_outputs[t, j] = w[t, j] * y[t, j]; routed_output is their
+                   sum over the slot axis ("expert_outputs needs the default experts
+                   implementation"); mlp_output == routed_output (no shared expert);
+                   the block adds it to the residual ("The block, in order").
+
+Two modes. ``exact`` rounds nothing. ``bf16_storage`` rounds, to the nearest bf16
+with ties to even, at the two places where a bf16 load stores bf16 values on this
+path: the expert's hidden activation h (mlp_neurons) and the block's output
+("The router renormalizes its top 2, in float32": in a bf16 load routed_output is
+bf16 while expert_weights stay float32).
+
+Readings where the pages are silent:
+* The top-k decision is taken on the router logits rounded to float32 (the scoring
+  precision the pages fix; softmax is strictly increasing, so ranking logits ranks
+  probabilities); equal float32 logits go to the lower expert index. The weights
+  themselves are computed in fp64 from the unrounded logits.
+* The expert-contiguous order of routed rows is a stable counting sort on
+  (expert, token, slot); every expert group is padded to a multiple of ``pad`` rows,
+  pad rows carry token -1.
+* With k = 1 the single weight is renormalised to exactly 1.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "to_f64", "round_bf16", "silu", "router_logits", "route_topk", "stable_permute",
+    "swiglu_expert", "moe_layer",
+]
+
+
+def to_f64(a) -> np.ndarray:
+    """float64 numpy copy of ``a`` (a torch tensor of any float dtype, or an array)."""
+    if hasattr(a, "detach"):
+        return a.detach().cpu().double().numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+def round_bf16(a) -> np.ndarray:
+    """Nearest bf16 value of each fp64 element, ties to even, returned as fp64.
+
+    bf16 keeps 8 significant bits and float32's exponent range (smallest normal
+    2**-126, subnormal spacing 2**-133). For |a| = m * 2**e with 0.5 <= m < 1 the
+    spacing of bf16 values near a is 2**(e - 8), floored at 2**-133; dividing by a
+    power of two is exact, and np.rint rounds half-way cases to even.
+    """
+    a = np.asarray(a, dtype=np.float64)
+    _, e = np.frexp(a)
+    quantum = np.ldexp(1.0, np.maximum(e, -125) - 8)
+    return np.rint(a / quantum) * quantum
+
+
+def silu(g: np.ndarray) -> np.ndarray:
+    """silu(g) = g * sigmoid(g) = g / (1 + exp(-g))."""
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g))
+
+
+def router_logits(x, w_router, logit_bias=None) -> np.ndarray:
+    """[T, E] fp64 logits l[t, e] = sum_h x[t, h] * W_r[e, h] (+ logit_bias[e] if given).
+
+    ``logit_bias`` is not part of Mixtral; the benchmark's imbalanced workload uses it
+    to skew routing.
+    """
+    logits = to_f64(x) @ to_f64(w_router).T
+    if logit_bias is not None:
+        logits = logits + to_f64(logit_bias)[None, :]
+    return logits
+
+
+def route_topk(logits: np.ndarray, k: int):
+    """Softmax over all experts, the k largest, renormalised to sum to one.
+
+    Returns (idx [T, k] int32, weights [T, k] fp64, probs [T, E] fp64); slot 0 holds
+    the largest weight.
+    """
+    logits = np.asarray(logits, dtype=np.float64)
+    t_count, e_count = logits.shape
+    shifted = logits - logits.max(axis=1, keepdims=True)
+    p = np.exp(shifted)
+    p = p / p.sum(axis=1, keepdims=True)
+    key32 = logits.astype(np.float32)
+    idx = np.empty((t_count, k), dtype=np.int32)
+    for t in range(t_count):
+        # stable sort of -key keeps lower expert indices first among equal keys
+        order = np.argsort(-key32[t].astype(np.float64), kind="stable")
+        idx[t] = order[:k]
+    top = np.take_along_axis(p, idx.astype(np.int64), axis=1)
+    weights = top / top.sum(axis=1, keepdims=True)
+    return idx, weights, p
+
+
+def stable_permute(idx: np.ndarray, num_experts: int, pad: int = 128):
+    """Expert-contiguous order of the routed (token, slot) pairs.
+
+    Counting sort: count[e] = #{(t, j): idx[t, j] == e}; group e starts at
+    offset[e] = sum_{e' < e} pad_up(count[e']); within a group rows follow token,
+    then slot, order. Returns (count [E], offset [E+1], row_of [T, k],
+    token_of_row [offset[E]] with -1 on pad rows).
+    """
+    idx = np.asarray(idx)
+    t_count, k = idx.shape
+    count = np.zeros(num_experts, dtype=np.int64)
+    for e in idx.reshape(-1):
+        count[e] += 1
+    padded = (count + pad - 1) // pad * pad
+    offset = np.zeros(num_experts + 1, dtype=np.int64)
+    offset[1:] = np.cumsum(padded)
+    cursor = offset[:-1].copy()
+    row_of = np.empty((t_count, k), dtype=np.int64)
+    token_of_row = np.full(int(offset[-1]), -1, dtype=np.int64)
+    for t in range(t_count):
+        for j in range(k):
+            e = idx[t, j]
+            row_of[t, j] = cursor[e]
+            token_of_row[cursor[e]] = t
+            cursor[e] += 1
+    return count, offset, row_of, token_of_row
+
+
+def swiglu_expert(x_rows: np.ndarray, w1_e, w3_e, w2_e, h_bf16: bool = False) -> np.ndarray:
+    """y = down(silu(gate x) * up x) for each row of ``x_rows`` ([n, H] fp64).
+
+    gate = w1 [I, H], up = w3 [I, H], down = w2 [H, I], all in nn.Linear
+    [out, in] form. With ``h_bf16`` the hidden activation is rounded to bf16 before
+    the down projection, as a bf16 load stores it.
+    """
+    g = x_rows @ to_f64(w1_e).T
+    u = x_rows @ to_f64(w3_e).T
+    h = silu(g) * u
+    if h_bf16:
+        h = round_bf16(h)
+    return h @ to_f64(w2_e).T
+
+
+def moe_layer(x, w_router, w1, w3, w2, k: int, residual=None, logit_bias=None,
+              mode: str = "exact", tokens=None) -> dict:
+    """The layer on tokens ``tokens`` (all tokens when None).
+
+    Returns a dict of fp64 arrays over the chosen tokens: ``logits`` [n, E], ``idx``
+    [n, k], ``weights`` [n, k], ``y`` [n, k, H] (unweighted expert outputs),
+    ``expert_outputs`` [n, k, H] (weighted), ``routed`` [n, H] and ``out`` [n, H]
+    (residual + routed; rounded to bf16 in ``bf16_storage`` mode).
+    """
+    if mode not in ("exact", "bf16_storage"):
+        raise ValueError(mode)
+    storage = mode == "bf16_storage"
+    xs = to_f64(x)
+    if tokens is not None:
+        tokens = np.asarray(tokens, dtype=np.int64)
+        xs = xs[tokens]
+    n, hidden = xs.shape
+    logits = router_logits(xs, w_router, logit_bias)
+    idx, weights, _ = route_topk(logits, k)
+    num_experts = logits.shape[1]
+    y = np.zeros((n, k, hidden), dtype=np.float64)
+    for e in range(num_experts):
+        tok, slot = np.nonzero(idx == e)
+        if tok.size == 0:
+            continue
+        y[tok, slot] = swiglu_expert(xs[tok], w1[e], w3[e], w2[e], h_bf16=storage)
+    expert_outputs = weights[:, :, None] * y
+    routed = np.zeros((n, hidden), dtype=np.float64)
+    for j in range(k):
+        routed = routed + expert_outputs[:, j]
+    out = routed.copy()
+    if residual is not None:
+        res = to_f64(residual)
+        if tokens is not None:
+            res = res[tokens]
+        out = res + routed
+    if storage:
+        out = round_bf16(out)
+    return {"logits": logits, "idx": idx, "weights": weights, "y": y,
+            "expert_outputs": expert_outputs, "routed": routed, "out": out}

@@ -1,0 +1,289 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Each check is independent of the oracle's own code path: closed forms, library
+routines (torch's bf16 conversion, F.silu, F.linear), brute force over tiny inputs,
+and the invariants the nnterp "Mixtral" page states for the layer.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle import moe_oracle as O
+from oracle.screen import min_gap, screen_margin
+from sparse_mixture_experts_09_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- bf16 rounding
+
+def test_round_bf16_matches_torch_on_float32_values():
+    g = torch.Generator().manual_seed(0)
+    a = torch.randn(200000, generator=g, dtype=torch.float32) * torch.exp(
+        torch.randn(200000, generator=g) * 10)
+    want = a.to(torch.bfloat16).double().numpy()
+    got = O.round_bf16(a.double().numpy())
+    assert np.array_equal(got, want)
+
+
+def test_round_bf16_ties_to_even_closed_form():
+    # 1 + 2^-8 is half-way between 1 and 1 + 2^-7 (bf16 spacing at 1 is 2^-7)
+    assert O.round_bf16(1 + 2.0 ** -8) == 1.0
+    assert O.round_bf16(1 + 3 * 2.0 ** -8) == 1 + 2.0 ** -6
+    assert O.round_bf16(-(1 + 3 * 2.0 ** -8)) == -(1 + 2.0 ** -6)
+    # just above half-way rounds up
+    assert O.round_bf16(1 + 2.0 ** -8 + 2.0 ** -30) == 1 + 2.0 ** -7
+    # smallest bf16 subnormal is 2^-133
+    assert O.round_bf16(2.0 ** -133 * 0.75) == 2.0 ** -133
+    assert O.round_bf16(0.0) == 0.0
+
+
+# ---------------------------------------------------------------- silu
+
+def test_silu_closed_forms():
+    l3 = math.log(3.0)
+    # sigmoid(ln 3) = 3/4, sigmoid(-ln 3) = 1/4
+    assert O.silu(np.array([l3]))[0] == pytest.approx(0.75 * l3, rel=1e-15)
+    assert O.silu(np.array([-l3]))[0] == pytest.approx(-0.25 * l3, rel=1e-15)
+    assert O.silu(np.array([0.0]))[0] == 0.0
+    assert O.silu(np.array([800.0]))[0] == 800.0
+    assert O.silu(np.array([-800.0]))[0] == 0.0
+
+
+def test_silu_matches_torch():
+    g = np.linspace(-30, 30, 10001)
+    want = F.silu(torch.from_numpy(g)).numpy()
+    assert np.allclose(O.silu(g), want, rtol=1e-14, atol=1e-300)
+
+
+# ---------------------------------------------------------------- router
+
+def test_router_logits_pick_columns():
+    # x = unit vector e_h selects column h of W_r: logits[t, e] = W_r[e, h]
+    rng = np.random.default_rng(0)
+    wr = rng.standard_normal((5, 7))
+    x = np.eye(7)[[3, 0, 6]]
+    assert np.array_equal(O.router_logits(x, wr), wr[:, [3, 0, 6]].T)
+    bias = np.arange(5.0)
+    assert np.array_equal(O.router_logits(x, wr, bias), wr[:, [3, 0, 6]].T + bias)
+
+
+def test_route_closed_form_example():
+    # logits ln[1, 4, 2, 1]: softmax = [1, 4, 2, 1] / 8; top-2 = experts 1, 2;
+    # renormalised weights 4/6 and 2/6.
+    logits = np.log(np.array([[1.0, 4.0, 2.0, 1.0]]))
+    idx, w, p = O.route_topk(logits, 2)
+    assert idx.tolist() == [[1, 2]]
+    assert np.allclose(p, [[1 / 8, 4 / 8, 2 / 8, 1 / 8]], rtol=1e-15)
+    assert np.allclose(w, [[2 / 3, 1 / 3]], rtol=1e-15)
+
+
+def test_route_weights_sum_to_one_and_match_two_logit_softmax():
+    rng = np.random.default_rng(1)
+    logits = rng.standard_normal((500, 8)) * 3
+    idx, w, _ = O.route_topk(logits, 2)
+    # "a token's weights are p and 1 - p"
+    assert np.all(np.abs(w.sum(1) - 1) <= 1e-15)
+    # softmax -> top-2 -> renormalise == softmax over the two selected logits
+    l0 = np.take_along_axis(logits, idx.astype(np.int64)[:, :1], 1)[:, 0]
+    l1 = np.take_along_axis(logits, idx.astype(np.int64)[:, 1:], 1)[:, 0]
+    assert np.allclose(w[:, 0], 1 / (1 + np.exp(l1 - l0)), rtol=1e-14)
+    assert np.all(w[:, 0] >= w[:, 1])
+
+
+def test_route_brute_force_pair_search():
+    # The top-2 set is the pair of experts with the largest total probability.
+    rng = np.random.default_rng(2)
+    logits = rng.standard_normal((200, 6)) * 2
+    idx, _, p = O.route_topk(logits, 2)
+    for t in range(200):
+        best = max(itertools.combinations(range(6), 2), key=lambda ab: p[t, ab[0]] + p[t, ab[1]])
+        assert set(idx[t].tolist()) == set(best)
+        assert p[t, idx[t, 0]] >= p[t, idx[t, 1]]
+
+
+def test_route_ties_to_lower_index_and_k1():
+    idx, w, _ = O.route_topk(np.array([[0.5, 2.0, 2.0, 2.0]]), 2)
+    assert idx.tolist() == [[1, 2]]
+    assert np.allclose(w, [[0.5, 0.5]])
+    idx1, w1, _ = O.route_topk(np.array([[0.1, 0.9, 0.3]]), 1)
+    assert idx1.tolist() == [[1]] and w1.tolist() == [[1.0]]
+
+
+# ---------------------------------------------------------------- permutation
+
+@pytest.mark.parametrize("t_count,e_count,k", [(37, 8, 2), (300, 5, 3), (1, 8, 2), (64, 1, 1)])
+def test_stable_permute_against_library_sort(t_count, e_count, k):
+    rng = np.random.default_rng(t_count)
+    idx = np.stack([rng.permutation(e_count)[:k] for _ in range(t_count)]).astype(np.int32)
+    count, offset, row_of, tok = O.stable_permute(idx, e_count)
+    assert count.sum() == t_count * k
+    assert np.all(offset[1:] % 128 == 0) and offset[0] == 0
+    # order of (expert, token, slot) keys by a library stable sort
+    flat = idx.reshape(-1).astype(np.int64)
+    order = np.argsort(flat, kind="stable")       # flat index = t*k + j, already in (t, j) order
+    for e in range(e_count):
+        members = order[flat[order] == e]
+        rows = offset[e] + np.arange(members.size)
+        assert np.array_equal(row_of.reshape(-1)[members], rows)
+        assert np.array_equal(tok[rows], members // k)
+        assert np.all(tok[offset[e] + members.size: offset[e + 1]] == -1)
+    assert np.unique(row_of).size == t_count * k
+
+
+# ---------------------------------------------------------------- experts and layer
+
+def _tiny_layer(seed, t_count=24, h=16, i=32, e_count=4, k=2):
+    rng = np.random.default_rng(seed)
+    x = O.round_bf16(rng.standard_normal((t_count, h)))
+    wr = O.round_bf16(rng.standard_normal((e_count, h)) / math.sqrt(h))
+    w1 = O.round_bf16(rng.standard_normal((e_count, i, h)) / math.sqrt(h))
+    w3 = O.round_bf16(rng.standard_normal((e_count, i, h)) / math.sqrt(h))
+    w2 = O.round_bf16(rng.standard_normal((e_count, h, i)) / math.sqrt(i))
+    res = O.round_bf16(rng.standard_normal((t_count, h)))
+    return x, wr, w1, w3, w2, res
+
+
+def test_single_expert_top1_is_plain_swiglu_mlp():
+    # E = 1, k = 1: the layer is the SwiGLU MLP down(silu(gate x) * up x), written
+    # here with torch's own F.linear and F.silu in float64.
+    x, wr, w1, w3, w2, res = _tiny_layer(3, e_count=1, k=1)
+    got = O.moe_layer(x, wr[:1], w1, w3, w2, k=1)["out"]
+    xt = torch.from_numpy(x)
+    want = F.linear(F.silu(F.linear(xt, torch.from_numpy(w1[0]))) * F.linear(xt, torch.from_numpy(w3[0])),
+                    torch.from_numpy(w2[0])).numpy()
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-14)
+
+
+def test_diagonal_experts_closed_form():
+    # H = I with diagonal weights: y_i = c_i * silu(a_i x_i) * b_i x_i.
+    h = 8
+    a, b, c = np.linspace(0.5, 2, h), np.linspace(-1, 1, h), np.linspace(1, 3, h)
+    x = np.linspace(-2, 2, h)[None, :]
+    y = O.swiglu_expert(x, np.diag(a), np.diag(b), np.diag(c))
+    want = c * (a * x / (1 + np.exp(-a * x))) * (b * x)
+    assert np.allclose(y, want, rtol=1e-14, atol=1e-15)
+
+
+@pytest.mark.parametrize("seed,k", [(4, 2), (5, 2), (6, 3)])
+def test_sparse_layer_equals_dense_masked_evaluation(seed, k):
+    # Evaluate all E experts on every token and mix them with a dense gate that is
+    # zero off the top-k and the renormalised softmax on it (brute force).
+    x, wr, w1, w3, w2, res = _tiny_layer(seed, k=k)
+    got = O.moe_layer(x, wr, w1, w3, w2, k=k, residual=res)
+    logits = x @ wr.T
+    e_count = wr.shape[0]
+    p = np.exp(logits - logits.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    dense = np.zeros_like(x)
+    for t in range(x.shape[0]):
+        top = sorted(range(e_count), key=lambda e: -p[t, e])[:k]
+        gate = np.zeros(e_count)
+        gate[top] = p[t, top] / p[t, top].sum()
+        for e in range(e_count):
+            xt = torch.from_numpy(x[t:t + 1])
+            ye = F.linear(F.silu(F.linear(xt, torch.from_numpy(w1[e]))) * F.linear(xt, torch.from_numpy(w3[e])),
+                          torch.from_numpy(w2[e])).numpy()[0]
+            dense[t] += gate[e] * ye
+    assert np.allclose(got["routed"], dense, rtol=1e-12, atol=1e-13)
+    assert np.allclose(got["out"], res + dense, rtol=1e-12, atol=1e-13)
+
+
+def test_slot_sum_and_ablation_invariants():
+    x, wr, w1, w3, w2, res = _tiny_layer(7)
+    r = O.moe_layer(x, wr, w1, w3, w2, k=2)
+    # expert_outputs sums over its slot axis to routed_output
+    assert np.array_equal(r["expert_outputs"].sum(1), r["routed"])
+    # zeroing expert e's weight changes the output on exactly the tokens that chose e
+    for e in range(wr.shape[0]):
+        w_abl = np.where(r["idx"] == e, 0.0, r["weights"])
+        ablated = (w_abl[:, :, None] * r["y"]).sum(1)
+        changed = (ablated != r["routed"]).any(-1)
+        assert np.array_equal(changed, (r["idx"] == e).any(-1))
+
+
+def test_token_subset_matches_full_layer():
+    x, wr, w1, w3, w2, res = _tiny_layer(8)
+    full = O.moe_layer(x, wr, w1, w3, w2, k=2, residual=res, mode="bf16_storage")
+    sub = [0, 5, 17, 23]
+    part = O.moe_layer(x, wr, w1, w3, w2, k=2, residual=res, mode="bf16_storage", tokens=sub)
+    for key in ("idx", "weights", "routed", "out"):
+        assert np.array_equal(part[key], full[key][sub])
+
+
+def test_storage_mode_differs_only_by_bf16_rounding():
+    x, wr, w1, w3, w2, _ = _tiny_layer(9)
+    ex = O.moe_layer(x, wr, w1, w3, w2, k=2, mode="exact")
+    st = O.moe_layer(x, wr, w1, w3, w2, k=2, mode="bf16_storage")
+    assert np.array_equal(ex["idx"], st["idx"])
+    # bound: h rounded with relative error <= 2^-9 feeds |w2| |h|; then one more 2^-9
+    bound = np.zeros_like(ex["routed"])
+    for e in range(wr.shape[0]):
+        tok, slot = np.nonzero(ex["idx"] == e)
+        g = x[tok] @ w1[e].T
+        u = x[tok] @ w3[e].T
+        hmag = np.abs(O.silu(g) * u)
+        contrib = (hmag @ np.abs(w2[e]).T) * 2.0 ** -9 * ex["weights"][tok, slot][:, None]
+        np.add.at(bound, tok, contrib)
+    bound = bound * (1 + 1e-9) + np.abs(ex["routed"] + bound) * 2.0 ** -9 + 1e-300
+    assert np.all(np.abs(st["out"] - ex["routed"]) <= bound)
+    assert np.any(st["out"] != ex["routed"])
+
+
+# ---------------------------------------------------------------- margin screen
+
+def test_margin_screen_enforces_gaps():
+    w = W.WORKLOADS["tiny"]
+    inp = W.draw(w)
+    x, att, near = screen_margin(inp.x, inp.w_router, None, 2,
+                                 lambda rows, a: W.redraw_x_rows(w, rows, a))
+    gaps = min_gap(O.router_logits(x, inp.w_router), 2)
+    ok = np.ones(x.shape[0], dtype=bool)
+    ok[near.numpy()] = False
+    assert np.all(gaps[ok] >= 1e-2)
+    assert int(att.max()) >= 0 and near.numel() == 0
+    # rows that were never redrawn are untouched
+    same = att == 0
+    assert torch.equal(x[same], inp.x[same])
+
+
+# ---------------------------------------------------------------- the pages' printed values
+
+def _golden_config():
+    vals = {}
+    with open(os.path.join(GOLDEN, "mixtral_8x7b_config.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                k, v = line.split()
+                vals[k] = float(v)
+    return vals
+
+
+def test_workload_shapes_match_printed_config():
+    g = _golden_config()
+    for name in ("decode", "prefill", "imbalanced_a", "imbalanced_b"):
+        w = W.WORKLOADS[name]
+        assert w.hidden_size == g["hidden_size"] and w.intermediate_size == g["intermediate_size"]
+        assert w.num_experts == g["num_local_experts"] and w.num_experts_per_tok == g["num_experts_per_tok"]
+    assert W.WORKLOADS["larger"].intermediate_size == g["intermediate_size_8x22b"]
+
+
+def test_parameter_count_reconciles_45b_and_47b():
+    # Experts: layers * E * 3 * H * I. Attention: q, k, v, o projections. Plus
+    # untied embedding and head. The pages print 45B (doc) and 47B (model card):
+    # the first is the expert total, the second the model total.
+    g = _golden_config()
+    h, i, layers = g["hidden_size"], g["intermediate_size"], g["num_hidden_layers"]
+    experts = layers * g["num_local_experts"] * 3 * h * i
+    attn = layers * h * (g["q_proj_out"] + g["k_proj_out"] + g["v_proj_out"] + g["o_proj_out"])
+    router = layers * g["num_local_experts"] * h
+    embed = 2 * g["vocab_size"] * h
+    total = experts + attn + router + embed
+    assert round(experts / 1e9) == g["params_total_billion_doc"]
+    assert round(total / 1e9) == g["params_total_billion_card"]
