@@ -1,0 +1,177 @@
+/*
+ * moe.h - C ABI of libmoe.so, the Mixtral sparse-MoE feed-forward layer on one
+ * B200 (sm_100a).
+ *
+ * The layer (nnterp encyclopedia, "Mixtral": "The block, in order"; "The router
+ * renormalizes its top 2, in float32"; "Values, by host"; "expert_outputs needs the
+ * default experts implementation"):
+ *
+ *   logits[t,e] = sum_h x[t,h] * w_router[e,h]                 (no bias)
+ *   p[t,:]      = softmax(logits[t,:]) in float32
+ *   idx[t,0..k) = the k largest, slot 0 the largest; w[t,j] = p[idx[t,j]] / sum_j p
+ *   y[t,j]      = w2[e] (silu(w1[e] x[t]) * (w3[e] x[t])),  e = idx[t,j]
+ *   out[t]      = residual[t] + sum_j w[t,j] * y[t,j]
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ * - Pointers are DEVICE pointers unless the name ends in _host. The caller owns
+ *   every buffer; the library allocates and frees nothing. Every entry point
+ *   validates its arguments on the host, then enqueues kernels on `stream` and
+ *   returns without synchronising (moe_forward_host excepted).
+ * - bf16 tensors are raw IEEE bfloat16 bit patterns (moe_bf16_t), row-major,
+ *   contiguous. Weights use nn.Linear [out, in] form stacked over experts:
+ *   w_router [E, H]; w1 (gate) and w3 (up) [E, I, H]; w2 (down) [E, H, I].
+ * - Requirements (else MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED): num_tokens >= 1,
+ *   1 <= num_experts_per_tok <= num_experts <= 64, num_experts_per_tok <= 8,
+ *   hidden_size and intermediate_size positive multiples of 128, every pointer
+ *   non-NULL (except those documented as nullable) and 16-byte aligned.
+ * - Routed rows are stored expert-contiguous: a stable order on (expert, token,
+ *   slot), each expert group padded to a multiple of MOE_ROW_PAD rows. Pad rows
+ *   have token -1 and zero activations. moe_max_padded_rows() bounds the total.
+ * - `ws` is a device workspace of at least moe_workspace_size() bytes, 256-byte
+ *   aligned; each entry point that takes it uses its own region of it. Kernels
+ *   whose waits run out (a bounded spin that never completes) record
+ *   MOE_ERR_TIMEOUT in the workspace; moe_device_status() reads and clears it.
+ * - On failure the returned code is non-zero and moe_last_error() (thread-local)
+ *   describes it. Launch failures return MOE_ERR_CUDA.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16_t;              /* bfloat16 bit pattern */
+typedef struct CUstream_st* moe_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+#define MOE_ROW_PAD 128
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,
+  MOE_ERR_UNSUPPORTED = 2,
+  MOE_ERR_WORKSPACE = 3,
+  MOE_ERR_CUDA = 4,
+  MOE_ERR_TIMEOUT = 5
+} moe_status_t;
+
+/* The layer's sizes, named as in MixtralConfig (Hugging Face "Mixtral" doc):
+ * hidden_size, intermediate_size, num_local_experts (here num_experts) and
+ * num_experts_per_tok. num_tokens = batch * sequence length. */
+typedef struct {
+  int64_t num_tokens;
+  int32_t hidden_size;
+  int32_t intermediate_size;
+  int32_t num_experts;
+  int32_t num_experts_per_tok;
+} moe_shape_t;
+
+/* Bytes of device workspace every workspace-taking entry point needs for `shape`;
+ * 0 if the shape is invalid. */
+size_t moe_workspace_size(const moe_shape_t* shape);
+
+/* Bytes of workspace moe_forward_host needs: moe_workspace_size plus device
+ * staging for x, residual and out. 0 if the shape is invalid. */
+size_t moe_workspace_size_host(const moe_shape_t* shape);
+
+/* Upper bound on the padded routed-row count R_pad = sum_e pad128(count[e]):
+ * round_up(T * k, 128) + 128 * E. Size x_perm, token_of_row and y_perm with it.
+ * Returns -1 if the shape is invalid. */
+int64_t moe_max_padded_rows(const moe_shape_t* shape);
+
+/* Router and scoring (nnterp "Mixtral", "The router renormalizes its top 2, in
+ * float32"): one warp per token computes the E logits x . w_router[e] with fp32
+ * accumulation, the float32 softmax over all E, the k largest (ranked on the
+ * float32 logit, equal logits to the lower expert index, slot 0 the largest) and
+ * their renormalised weights.
+ *   x [T, H] bf16; w_router [E, H] bf16;
+ *   logit_bias [E] fp32, nullable: added to the logits (not part of Mixtral; lets a
+ *     benchmark skew the routing);
+ *   topk_idx [T, k] int32 out; topk_w [T, k] fp32 out (each row sums to 1);
+ *   router_logits [T, E] fp32 out, nullable (the pre-softmax logits). */
+moe_status_t moe_router_topk(const moe_shape_t* shape, const moe_bf16_t* x,
+                             const moe_bf16_t* w_router, const float* logit_bias,
+                             int32_t* topk_idx, float* topk_w, float* router_logits,
+                             moe_stream_t stream);
+
+/* Expert-contiguous permutation (the pages hand expert indices and weights to the
+ * experts module, nnterp "Mixtral", "Values, by host"; the order is this library's
+ * own): a deterministic per-expert histogram, padded prefix offsets, a stable
+ * rank of each (token, slot) and the gather of x rows.
+ *   topk_idx [T, k] int32 in, every value in [0, E);
+ *   x [T, H] bf16 in;
+ *   expert_counts [E] int32 out; expert_offsets [E+1] int32 out (multiples of 128,
+ *     offsets[E] = R_pad);
+ *   row_of [T, k] int32 out (row of each routed slot);
+ *   token_of_row [moe_max_padded_rows] int32 out (token of each row, -1 on pads;
+ *     entries past R_pad untouched);
+ *   x_perm [moe_max_padded_rows, H] bf16 out (pad rows zero; rows past R_pad
+ *     untouched). */
+moe_status_t moe_permute(const moe_shape_t* shape, const int32_t* topk_idx,
+                         const moe_bf16_t* x, int32_t* expert_counts,
+                         int32_t* expert_offsets, int32_t* row_of,
+                         int32_t* token_of_row, moe_bf16_t* x_perm, void* ws,
+                         size_t ws_bytes, moe_stream_t stream);
+
+/* The experts (nnterp "Mixtral", "Values, by host": mlp_neurons = act(gate)*up is
+ * what the down projection receives; act = silu per MixtralConfig hidden_act):
+ * two persistent tcgen05 grouped GEMMs over the ragged expert groups.
+ *   GEMM1: h = bf16(silu(x_perm w1[e]^T) * (x_perm w3[e]^T)), fp32 accumulation in
+ *          tensor memory, h kept in the workspace;
+ *   GEMM2: y_perm = h w2[e]^T, fp32.
+ *   x_perm [R_pad, H] bf16 and expert_offsets [E+1] int32 as written by moe_permute;
+ *   w1, w3 [E, I, H] bf16; w2 [E, H, I] bf16;
+ *   y_perm [moe_max_padded_rows, H] fp32 out (rows past R_pad untouched). */
+moe_status_t moe_grouped_swiglu(const moe_shape_t* shape, const moe_bf16_t* x_perm,
+                                const int32_t* expert_offsets, const moe_bf16_t* w1,
+                                const moe_bf16_t* w3, const moe_bf16_t* w2,
+                                float* y_perm, void* ws, size_t ws_bytes,
+                                moe_stream_t stream);
+
+/* Weighted combine into the residual (nnterp "Mixtral": expert_outputs summed over
+ * the slot axis is routed_output; the block adds mlp_output to the residual):
+ *   out[t] = bf16( residual[t] + sum_j topk_w[t,j] * y_perm[row_of[t,j]] ),
+ * fp32 arithmetic, slots in order, a single round-to-nearest-even at the end.
+ *   residual [T, H] bf16, nullable (treated as zero); out [T, H] bf16. */
+moe_status_t moe_combine(const moe_shape_t* shape, const float* y_perm,
+                         const int32_t* row_of, const float* topk_w,
+                         const moe_bf16_t* residual, moe_bf16_t* out,
+                         moe_stream_t stream);
+
+/* The whole layer: router, permutation, experts and combine, every intermediate in
+ * `ws`. residual and logit_bias are nullable. */
+moe_status_t moe_forward(const moe_shape_t* shape, const moe_bf16_t* x,
+                         const moe_bf16_t* w_router, const float* logit_bias,
+                         const moe_bf16_t* w1, const moe_bf16_t* w3,
+                         const moe_bf16_t* w2, const moe_bf16_t* residual,
+                         moe_bf16_t* out, void* ws, size_t ws_bytes,
+                         moe_stream_t stream);
+
+/* moe_forward with HOST activations: copies x_host (and residual_host, nullable)
+ * into the workspace, runs the layer, copies out back into out_host, and waits for
+ * the stream. Host buffers should be pinned for asynchronous copies. Weights and
+ * ws stay on the device; ws_bytes >= moe_workspace_size_host(shape). */
+moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_bf16_t* x_host,
+                              const moe_bf16_t* w_router, const float* logit_bias,
+                              const moe_bf16_t* w1, const moe_bf16_t* w3,
+                              const moe_bf16_t* w2, const moe_bf16_t* residual_host,
+                              moe_bf16_t* out_host, void* ws, size_t ws_bytes,
+                              moe_stream_t stream);
+
+/* Waits for `stream`, then reads and clears the device status word in `ws`:
+ * MOE_OK, or MOE_ERR_TIMEOUT if a kernel gave up a bounded wait since the last
+ * call. */
+moe_status_t moe_device_status(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Thread-local description of the last failure on this thread ("" if none). */
+const char* moe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

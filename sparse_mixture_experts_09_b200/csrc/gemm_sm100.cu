@@ -1,0 +1,509 @@
+// Persistent grouped GEMMs of the experts on sm_100a: TMA loads into 128-byte
+// swizzled shared-memory stages, tcgen05.mma (kind::f16, bf16 in, fp32 accumulate)
+// into tensor memory, a four-warp epilogue reading tensor memory with tcgen05.ld.
+//
+// The experts (nnterp encyclopedia, "Mixtral", "Values, by host"): mlp_neurons =
+// act(gate x) * up x is what the down projection receives; act = silu (Hugging Face
+// "Mixtral" doc, MixtralConfig hidden_act). The pages name a grouped matmul over
+// the stacked experts as the default implementation ("expert_outputs needs the
+// default experts implementation"); this is our own design of it for B200.
+//
+//   GEMM1 (kSwiGLU): for a 128-row tile of one expert's routed rows and 128
+//     intermediate columns, B is the 128 w1 rows stacked on the 128 w3 rows, so one
+//     M=128 x N=256 MMA chain yields gate (columns 0..127) and up (128..255) side by
+//     side; the epilogue writes h = bf16(silu(gate) * up).
+//   GEMM2 (kPlain): y = h w2^T for a 128-row tile and BN output columns, fp32 out.
+//
+// Roles per CTA (192 threads): warp 0 issues TMA, warp 1 owns tensor memory and
+// issues MMAs, warps 2..5 drain accumulators. Two accumulators in tensor memory let
+// the epilogue of one tile overlap the MMAs of the next. Tiles are visited in a
+// static round-robin over a tile order that keeps an expert's rows together and
+// walks its row tiles fastest, so concurrently running CTAs share weight tiles in L2.
+//
+// Every wait is bounded: after `timeout_ns` a role records kStatusTimeout in the
+// device status word, raises a CTA-wide abort flag, and all roles unwind; the
+// producer waits (bounded) for its copies in flight and the MMA warp for its MMAs
+// before tensor memory is freed.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;        // bf16 elements per 128-byte swizzled row
+constexpr int kThreads = 192;
+constexpr int kStages = 4;
+constexpr int kSwiGLU = 0;
+constexpr int kPlain = 1;
+
+template <int BN>
+struct Tile {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + BAR_BYTES + 4 * 72;
+  // instruction descriptor: D f32 (bit 4), A bf16 (bits 7-9 = 1), B bf16 (bits 10-12 = 1),
+  // both K-major, N >> 3 at bit 17, M >> 4 at bit 24
+  static constexpr uint32_t IDESC =
+      (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+};
+
+struct KParams {
+  const int32_t* offsets;
+  int32_t* status;
+  void* out;
+  int64_t out_ld;
+  int E;
+  int k_blocks;
+  int n_tiles;
+  int b_rows;  // rows of the B tensor per expert
+  unsigned long long timeout_ns;
+};
+
+// ---------------------------------------------------------------- PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// shared-memory matrix descriptor, K-major, 128-byte swizzle: start address >> 4,
+// leading byte offset 16 B (unused for swizzled K-major), stride byte offset 1024 B
+// (one 8-row x 128-byte swizzle atom), version 1 (bit 46), layout SWIZZLE_128B = 2.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Bounded wait on an mbarrier phase. Returns false if the CTA aborted or the wait
+// ran past timeout_ns (then it records the timeout and raises the abort flag).
+__device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                        int32_t* status, unsigned long long timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > timeout_ns) {
+        *abort_flag = 1;
+        atomicOr(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait used while unwinding: ignores the abort flag.
+__device__ __noinline__ void drain_phase(uint32_t bar, uint32_t parity,
+                                         unsigned long long timeout_ns) {
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > timeout_ns) return;
+  }
+}
+
+// Tile L -> (expert e, row tile m, column tile n). row_tiles[e] = offsets[e] / 128.
+// Tiles of expert e occupy [row_tiles[e] * n_tiles, row_tiles[e+1] * n_tiles) and
+// walk the expert's row tiles fastest.
+__device__ __forceinline__ void tile_coords(int L, const int* row_tiles, int E, int n_tiles, int& e,
+                                            int& m, int& n) {
+  const int mrow = L / n_tiles;
+  e = 0;
+  while (e + 1 < E && row_tiles[e + 1] <= mrow) ++e;
+  const int cnt = row_tiles[e + 1] - row_tiles[e];
+  const int local = L - row_tiles[e] * n_tiles;
+  n = local / cnt;
+  m = row_tiles[e] + local % cnt;
+}
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
+                   const __grid_constant__ CUtensorMap mapB1, const KParams p) {
+  using C = Tile<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * C::STAGE_BYTES);
+  // bars: full[kStages], empty[kStages], tfull[2], tempty[2], final
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* row_tiles = reinterpret_cast<int*>(tmem_holder + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * kStages + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * kStages + 2 + a); };
+  const uint32_t final_bar = bar0 + 8u * (2 * kStages + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 4);
+    }
+    mbar_init(final_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (threadIdx.x == 32) {
+    prefetch_map(&mapA);
+    prefetch_map(&mapB0);
+    prefetch_map(&mapB1);
+  }
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) row_tiles[i] = p.offsets[i] / BM;
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int total = row_tiles[p.E] * p.n_tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      int it = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        int e, m, n;
+        tile_coords(L, row_tiles, p.E, p.n_tiles, e, m, n);
+        const int a_row = m * BM;
+        int b_row0, b_row1;
+        if (MODE == kSwiGLU) {
+          b_row0 = e * p.b_rows + n * 128;
+          b_row1 = b_row0;
+        } else {
+          b_row0 = e * p.b_rows + n * BN;
+          b_row1 = b_row0 + 128;
+        }
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          if (!wait_phase(empty_bar(s), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+          mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
+          tma_load_2d(sa, &mapA, kb * BK, a_row, full_bar(s));
+          tma_load_2d(sa + C::A_BYTES, &mapB0, kb * BK, b_row0, full_bar(s));
+          if (BN == 256) tma_load_2d(sa + C::A_BYTES + 128 * BK * 2, &mapB1, kb * BK, b_row1, full_bar(s));
+        }
+      }
+      if (!ok) {
+        // let the copies already issued land before the CTA can exit
+        const int first = it > kStages ? it - kStages : 0;
+        for (int i = first; i < it; ++i)
+          drain_phase(full_bar(i % kStages), (uint32_t)(i / kStages) & 1u, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      int it = 0, tc = 0;
+      bool ok = true, issued = false;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tc) {
+        const int a = tc & 1;
+        const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
+        if (!wait_phase(tempty_bar(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
+        fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(a * BN);
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          if (!wait_phase(full_bar(s), ph, abort_flag, p.status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            mma_bf16(d, sdesc(sa + kk * 32), sdesc(sb + kk * 32), C::IDESC, (kb | kk) ? 1u : 0u);
+          }
+          mma_commit(empty_bar(s));
+          issued = true;
+        }
+        if (ok) mma_commit(tfull_bar(a));
+      }
+      // every MMA issued so far completes before tensor memory is released
+      if (issued) {
+        mma_commit(final_bar);
+        drain_phase(final_bar, 0, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: warps 2..5, warp w reads TMEM lanes 32*(w%4) ..
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    int tc = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x, ++tc) {
+      int e, m, n;
+      tile_coords(L, row_tiles, p.E, p.n_tiles, e, m, n);
+      const int a = tc & 1;
+      const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
+      int ok = 0;
+      if (lane == 0) ok = wait_phase(tfull_bar(a), aph, abort_flag, p.status, p.timeout_ns) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * BN);
+      const int64_t row = (int64_t)m * BM + row_in_tile;
+      if (MODE == kSwiGLU) {
+        uint16_t* h = reinterpret_cast<uint16_t*>(p.out) + row * p.out_ld + (int64_t)n * 128;
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 16) {
+          uint32_t g[16], u[16];
+          tmem_ld16(taddr + c, g);
+          tmem_ld16(taddr + 128 + c, u);
+          tmem_wait_ld();
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+            const float h0 = g0 / (1.f + __expf(-g0)) * u0;
+            const float h1 = g1 / (1.f + __expf(-g1)) * u1;
+            pk[i] = pack_bf16x2_rn(h0, h1);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(h + c);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+      } else {
+        float* y = reinterpret_cast<float*>(p.out) + row * p.out_ld + (int64_t)n * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(taddr + c, v);
+          tmem_wait_ld();
+          float4* dst = reinterpret_cast<float4*>(y + c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(a));
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [rows, inner] row-major; box = 64 x box_rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE, int BN>
+cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                       const KParams& p, int64_t max_tiles, cudaStream_t st) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int smem = Tile<BN>::SMEM_BYTES;
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm<MODE, BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  int64_t grid = num_sms();
+  if (grid > max_tiles) grid = max_tiles;
+  k_grouped_gemm<MODE, BN><<<(unsigned)grid, kThreads, smem, st>>>(a, b0, b1, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_swiglu(const Shape& s, const GemmArgs& g, cudaStream_t st,
+                                  const char** why) {
+  CUtensorMap mx, mw1, mw3, mh, mw2;
+  const uint64_t EI = (uint64_t)s.E * s.I, EH = (uint64_t)s.E * s.H;
+  if (!make_map(&mx, g.a, s.H, g.rmax, 128) || !make_map(&mw1, g.w1, s.H, EI, 128) ||
+      !make_map(&mw3, g.w3, s.H, EI, 128) || !make_map(&mh, g.h, s.I, g.rmax, 128) ||
+      !make_map(&mw2, g.w2, s.I, EH, 128)) {
+    *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad tensor)";
+    return cudaErrorInvalidValue;
+  }
+  const int64_t mt_max = g.rmax / BM;
+
+  KParams p1;
+  p1.offsets = g.offsets;
+  p1.status = g.status;
+  p1.out = g.h;
+  p1.out_ld = s.I;
+  p1.E = s.E;
+  p1.k_blocks = s.H / BK;
+  p1.n_tiles = s.I / 128;
+  p1.b_rows = s.I;
+  p1.timeout_ns = g.timeout_ns;
+  cudaError_t e = launch_one<kSwiGLU, 256>(mx, mw1, mw3, p1, mt_max * p1.n_tiles, st);
+  if (e != cudaSuccess) {
+    *why = "GEMM1 launch failed";
+    return e;
+  }
+
+  KParams p2 = p1;
+  p2.out = g.y;
+  p2.out_ld = s.H;
+  p2.k_blocks = s.I / BK;
+  p2.b_rows = s.H;
+  if (s.H % 256 == 0) {
+    p2.n_tiles = s.H / 256;
+    e = launch_one<kPlain, 256>(mh, mw2, mw2, p2, mt_max * p2.n_tiles, st);
+  } else {
+    p2.n_tiles = s.H / 128;
+    e = launch_one<kPlain, 128>(mh, mw2, mw2, p2, mt_max * p2.n_tiles, st);
+  }
+  if (e != cudaSuccess) *why = "GEMM2 launch failed";
+  return e;
+}
+
+}  // namespace moe

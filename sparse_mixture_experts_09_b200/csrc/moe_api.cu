@@ -1,0 +1,355 @@
+// C ABI of libmoe.so: argument validation, workspace layout and kernel launches.
+// Declarations and the contract of each entry point are in include/moe.h.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/moe.h"
+#include "moe_internal.h"
+
+namespace moe {
+
+int num_sms() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 64 && cache[dev]) return cache[dev];
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (n <= 0) n = 148;
+  if (dev < 64) cache[dev] = n;
+  return n;
+}
+
+namespace {
+
+thread_local char g_err[512];
+
+moe_status_t fail(moe_status_t code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+moe_status_t cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_err, sizeof g_err, "%s: %s", where, cudaGetErrorString(e));
+  return MOE_ERR_CUDA;
+}
+
+constexpr size_t kAlign = 1024;
+inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+// Workspace regions, in order; each starts on a 1024-byte boundary.
+struct Layout {
+  size_t status, topk_idx, topk_w, block_base, counts, offsets, row_of, token_of_row, x_perm, h, y,
+      end;
+  size_t x_in, res_in, out_st, end_host;  // staging of moe_forward_host
+};
+
+Layout layout(const Shape& s) {
+  Layout L;
+  const size_t tk = (size_t)s.T * s.k;
+  const size_t rmax = (size_t)max_padded_rows(s);
+  size_t o = 0;
+  L.status = o; o += up(256);
+  L.topk_idx = o; o += up(tk * 4);
+  L.topk_w = o; o += up(tk * 4);
+  L.block_base = o; o += up((size_t)num_token_blocks(s) * s.E * 4);
+  L.counts = o; o += up((size_t)s.E * 4);
+  L.offsets = o; o += up((size_t)(s.E + 1) * 4);
+  L.row_of = o; o += up(tk * 4);
+  L.token_of_row = o; o += up(rmax * 4);
+  L.x_perm = o; o += up(rmax * s.H * 2);
+  L.h = o; o += up(rmax * s.I * 2);
+  L.y = o; o += up(rmax * s.H * 4);
+  L.end = o;
+  L.x_in = o; o += up((size_t)s.T * s.H * 2);
+  L.res_in = o; o += up((size_t)s.T * s.H * 2);
+  L.out_st = o; o += up((size_t)s.T * s.H * 2);
+  L.end_host = o;
+  return L;
+}
+
+moe_status_t check_shape(const moe_shape_t* sh, Shape* out) {
+  if (!sh) return fail(MOE_ERR_INVALID_ARG, "shape is NULL");
+  if (sh->num_tokens < 1) return fail(MOE_ERR_INVALID_ARG, "num_tokens must be >= 1 (got %lld)", (long long)sh->num_tokens);
+  if (sh->num_experts < 1 || sh->num_experts > 64)
+    return fail(MOE_ERR_UNSUPPORTED, "num_experts must be in [1, 64] (got %d)", sh->num_experts);
+  if (sh->num_experts_per_tok < 1 || sh->num_experts_per_tok > sh->num_experts ||
+      sh->num_experts_per_tok > 8)
+    return fail(MOE_ERR_UNSUPPORTED, "num_experts_per_tok must be in [1, min(8, num_experts)] (got %d)",
+                sh->num_experts_per_tok);
+  if (sh->hidden_size <= 0 || sh->hidden_size % 128)
+    return fail(MOE_ERR_UNSUPPORTED, "hidden_size must be a positive multiple of 128 (got %d)",
+                sh->hidden_size);
+  if (sh->intermediate_size <= 0 || sh->intermediate_size % 128)
+    return fail(MOE_ERR_UNSUPPORTED, "intermediate_size must be a positive multiple of 128 (got %d)",
+                sh->intermediate_size);
+  if (sh->num_tokens * sh->num_experts_per_tok > (int64_t)1 << 30)
+    return fail(MOE_ERR_UNSUPPORTED, "num_tokens * num_experts_per_tok must be <= 2^30 (got %lld)",
+                (long long)(sh->num_tokens * sh->num_experts_per_tok));
+  out->T = sh->num_tokens;
+  out->H = sh->hidden_size;
+  out->I = sh->intermediate_size;
+  out->E = sh->num_experts;
+  out->k = sh->num_experts_per_tok;
+  const int64_t rmax = max_padded_rows(*out);
+  if ((rmax / 128) * (int64_t)(out->I / 128) > INT32_MAX || (int64_t)out->E * out->I > INT32_MAX)
+    return fail(MOE_ERR_UNSUPPORTED, "shape too large for 32-bit tile indices");
+  return MOE_OK;
+}
+
+moe_status_t check_ptr(const void* p, const char* name, bool nullable = false) {
+  if (!p) {
+    if (nullable) return MOE_OK;
+    return fail(MOE_ERR_INVALID_ARG, "%s is NULL", name);
+  }
+  if (reinterpret_cast<uintptr_t>(p) % 16)
+    return fail(MOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return MOE_OK;
+}
+
+moe_status_t check_ws(const void* ws, size_t ws_bytes, size_t need) {
+  if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % 256) return fail(MOE_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  if (ws_bytes < need) return fail(MOE_ERR_WORKSPACE, "workspace too small: need %zu bytes, got %zu", need, ws_bytes);
+  return MOE_OK;
+}
+
+#define MOE_TRY(x)                  \
+  do {                              \
+    moe_status_t _s = (x);          \
+    if (_s != MOE_OK) return _s;    \
+  } while (0)
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per wait
+
+moe_status_t run_forward(const Shape& s, const uint16_t* x, const uint16_t* wr, const float* bias,
+                         const uint16_t* w1, const uint16_t* w3, const uint16_t* w2,
+                         const uint16_t* res, uint16_t* out, void* ws, cudaStream_t st) {
+  const Layout L = layout(s);
+  cudaError_t e = launch_router(s, x, wr, bias, at<int32_t>(ws, L.topk_idx), at<float>(ws, L.topk_w),
+                                nullptr, st);
+  if (e != cudaSuccess) return cuda_fail(e, "router launch");
+  e = launch_permute(s, at<int32_t>(ws, L.topk_idx), x, at<int32_t>(ws, L.counts),
+                     at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.row_of),
+                     at<int32_t>(ws, L.token_of_row), at<uint16_t>(ws, L.x_perm),
+                     at<int32_t>(ws, L.block_base), st);
+  if (e != cudaSuccess) return cuda_fail(e, "permute launch");
+  GemmArgs g;
+  g.a = at<uint16_t>(ws, L.x_perm);
+  g.offsets = at<int32_t>(ws, L.offsets);
+  g.w1 = w1;
+  g.w3 = w3;
+  g.w2 = w2;
+  g.h = at<uint16_t>(ws, L.h);
+  g.y = at<float>(ws, L.y);
+  g.status = at<int32_t>(ws, L.status);
+  g.rmax = max_padded_rows(s);
+  g.timeout_ns = kTimeoutNs;
+  const char* why = "";
+  e = launch_grouped_swiglu(s, g, st, &why);
+  if (e != cudaSuccess) return cuda_fail(e, why);
+  e = launch_combine(s, at<float>(ws, L.y), at<int32_t>(ws, L.row_of), at<float>(ws, L.topk_w), res,
+                     out, st);
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_shape_t* shape) {
+  Shape s;
+  if (check_shape(shape, &s) != MOE_OK) return 0;
+  return layout(s).end;
+}
+
+size_t moe_workspace_size_host(const moe_shape_t* shape) {
+  Shape s;
+  if (check_shape(shape, &s) != MOE_OK) return 0;
+  return layout(s).end_host;
+}
+
+int64_t moe_max_padded_rows(const moe_shape_t* shape) {
+  Shape s;
+  if (check_shape(shape, &s) != MOE_OK) return -1;
+  return max_padded_rows(s);
+}
+
+const char* moe_last_error(void) { return g_err; }
+
+moe_status_t moe_router_topk(const moe_shape_t* shape, const moe_bf16_t* x,
+                             const moe_bf16_t* w_router, const float* logit_bias,
+                             int32_t* topk_idx, float* topk_w, float* router_logits,
+                             moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(x, "x"));
+  MOE_TRY(check_ptr(w_router, "w_router"));
+  MOE_TRY(check_ptr(logit_bias, "logit_bias", true));
+  MOE_TRY(check_ptr(topk_idx, "topk_idx"));
+  MOE_TRY(check_ptr(topk_w, "topk_w"));
+  MOE_TRY(check_ptr(router_logits, "router_logits", true));
+  cudaError_t e = launch_router(s, x, w_router, logit_bias, topk_idx, topk_w, router_logits,
+                                (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "router launch");
+}
+
+moe_status_t moe_permute(const moe_shape_t* shape, const int32_t* topk_idx, const moe_bf16_t* x,
+                         int32_t* expert_counts, int32_t* expert_offsets, int32_t* row_of,
+                         int32_t* token_of_row, moe_bf16_t* x_perm, void* ws, size_t ws_bytes,
+                         moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(topk_idx, "topk_idx"));
+  MOE_TRY(check_ptr(x, "x"));
+  MOE_TRY(check_ptr(expert_counts, "expert_counts"));
+  MOE_TRY(check_ptr(expert_offsets, "expert_offsets"));
+  MOE_TRY(check_ptr(row_of, "row_of"));
+  MOE_TRY(check_ptr(token_of_row, "token_of_row"));
+  MOE_TRY(check_ptr(x_perm, "x_perm"));
+  const Layout L = layout(s);
+  MOE_TRY(check_ws(ws, ws_bytes, L.end));
+  cudaError_t e = launch_permute(s, topk_idx, x, expert_counts, expert_offsets, row_of,
+                                 token_of_row, x_perm, at<int32_t>(ws, L.block_base),
+                                 (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "permute launch");
+}
+
+moe_status_t moe_grouped_swiglu(const moe_shape_t* shape, const moe_bf16_t* x_perm,
+                                const int32_t* expert_offsets, const moe_bf16_t* w1,
+                                const moe_bf16_t* w3, const moe_bf16_t* w2, float* y_perm,
+                                void* ws, size_t ws_bytes, moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(x_perm, "x_perm"));
+  MOE_TRY(check_ptr(expert_offsets, "expert_offsets"));
+  MOE_TRY(check_ptr(w1, "w1"));
+  MOE_TRY(check_ptr(w3, "w3"));
+  MOE_TRY(check_ptr(w2, "w2"));
+  MOE_TRY(check_ptr(y_perm, "y_perm"));
+  const Layout L = layout(s);
+  MOE_TRY(check_ws(ws, ws_bytes, L.end));
+  GemmArgs g;
+  g.a = x_perm;
+  g.offsets = expert_offsets;
+  g.w1 = w1;
+  g.w3 = w3;
+  g.w2 = w2;
+  g.h = at<uint16_t>(ws, L.h);
+  g.y = y_perm;
+  g.status = at<int32_t>(ws, L.status);
+  g.rmax = max_padded_rows(s);
+  g.timeout_ns = kTimeoutNs;
+  const char* why = "";
+  cudaError_t e = launch_grouped_swiglu(s, g, (cudaStream_t)stream, &why);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, why);
+}
+
+moe_status_t moe_combine(const moe_shape_t* shape, const float* y_perm, const int32_t* row_of,
+                         const float* topk_w, const moe_bf16_t* residual, moe_bf16_t* out,
+                         moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(y_perm, "y_perm"));
+  MOE_TRY(check_ptr(row_of, "row_of"));
+  MOE_TRY(check_ptr(topk_w, "topk_w"));
+  MOE_TRY(check_ptr(residual, "residual", true));
+  MOE_TRY(check_ptr(out, "out"));
+  cudaError_t e = launch_combine(s, y_perm, row_of, topk_w, residual, out, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "combine launch");
+}
+
+moe_status_t moe_forward(const moe_shape_t* shape, const moe_bf16_t* x, const moe_bf16_t* w_router,
+                         const float* logit_bias, const moe_bf16_t* w1, const moe_bf16_t* w3,
+                         const moe_bf16_t* w2, const moe_bf16_t* residual, moe_bf16_t* out,
+                         void* ws, size_t ws_bytes, moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(x, "x"));
+  MOE_TRY(check_ptr(w_router, "w_router"));
+  MOE_TRY(check_ptr(logit_bias, "logit_bias", true));
+  MOE_TRY(check_ptr(w1, "w1"));
+  MOE_TRY(check_ptr(w3, "w3"));
+  MOE_TRY(check_ptr(w2, "w2"));
+  MOE_TRY(check_ptr(residual, "residual", true));
+  MOE_TRY(check_ptr(out, "out"));
+  MOE_TRY(check_ws(ws, ws_bytes, layout(s).end));
+  return run_forward(s, x, w_router, logit_bias, w1, w3, w2, residual, out, ws,
+                     (cudaStream_t)stream);
+}
+
+moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_bf16_t* x_host,
+                              const moe_bf16_t* w_router, const float* logit_bias,
+                              const moe_bf16_t* w1, const moe_bf16_t* w3, const moe_bf16_t* w2,
+                              const moe_bf16_t* residual_host, moe_bf16_t* out_host, void* ws,
+                              size_t ws_bytes, moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  if (!x_host) return fail(MOE_ERR_INVALID_ARG, "x_host is NULL");
+  if (!out_host) return fail(MOE_ERR_INVALID_ARG, "out_host is NULL");
+  MOE_TRY(check_ptr(w_router, "w_router"));
+  MOE_TRY(check_ptr(logit_bias, "logit_bias", true));
+  MOE_TRY(check_ptr(w1, "w1"));
+  MOE_TRY(check_ptr(w3, "w3"));
+  MOE_TRY(check_ptr(w2, "w2"));
+  const Layout L = layout(s);
+  MOE_TRY(check_ws(ws, ws_bytes, L.end_host));
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t bytes = (size_t)s.T * s.H * 2;
+  uint16_t* xd = at<uint16_t>(ws, L.x_in);
+  uint16_t* rd = residual_host ? at<uint16_t>(ws, L.res_in) : nullptr;
+  uint16_t* od = at<uint16_t>(ws, L.out_st);
+  cudaError_t e = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e, "copy of x to the device");
+  if (rd) {
+    e = cudaMemcpyAsync(rd, residual_host, bytes, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "copy of residual to the device");
+  }
+  MOE_TRY(run_forward(s, xd, w_router, logit_bias, w1, w3, w2, rd, od, ws, st));
+  e = cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e, "copy of out to the host");
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  return MOE_OK;
+}
+
+moe_status_t moe_device_status(void* ws, size_t ws_bytes, moe_stream_t stream) {
+  g_err[0] = 0;
+  if (!ws || ws_bytes < 256) return fail(MOE_ERR_WORKSPACE, "workspace is NULL or too small");
+  cudaStream_t st = (cudaStream_t)stream;
+  int32_t word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof word, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (word == 0) return MOE_OK;
+  e = cudaMemsetAsync(ws, 0, sizeof word, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  if (word & kStatusTimeout)
+    return fail(MOE_ERR_TIMEOUT, "a kernel gave up a bounded wait (device status 0x%x)",
+                (unsigned)word);
+  return fail(MOE_ERR_CUDA, "unknown device status 0x%x", (unsigned)word);
+}
+
+}  // extern "C"

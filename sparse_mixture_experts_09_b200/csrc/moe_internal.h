@@ -1,0 +1,65 @@
+// Internal declarations shared by the libmoe.so translation units (not installed).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Routed (token, slot) pairs handled by one CTA of the histogram / scatter kernels:
+// one warp's worth of tokens, so a CTA ranks its pairs with warp ballots.
+constexpr int kTokensPerBlock = 32;
+constexpr int kRowPad = 128;
+
+// Device status word, first int32 of the workspace.
+constexpr int32_t kStatusTimeout = 1;
+
+struct Shape {
+  int64_t T;
+  int H, I, E, k;
+};
+
+inline int64_t max_padded_rows(const Shape& s) {
+  int64_t r = s.T * s.k;
+  return (r + kRowPad - 1) / kRowPad * kRowPad + (int64_t)kRowPad * s.E;
+}
+
+inline int64_t num_token_blocks(const Shape& s) {
+  return (s.T + kTokensPerBlock - 1) / kTokensPerBlock;
+}
+
+// ---- launchers (each returns the launch's cudaError_t) ----
+
+cudaError_t launch_router(const Shape& s, const uint16_t* x, const uint16_t* w_router,
+                          const float* logit_bias, int32_t* topk_idx, float* topk_w,
+                          float* logits, cudaStream_t st);
+
+cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16_t* x,
+                           int32_t* counts, int32_t* offsets, int32_t* row_of,
+                           int32_t* token_of_row, uint16_t* x_perm, int32_t* block_base,
+                           cudaStream_t st);
+
+struct GemmArgs {
+  const uint16_t* a;        // x_perm [Rmax, K1] (GEMM1) or h [Rmax, I] (GEMM2)
+  const int32_t* offsets;   // [E+1], multiples of 128
+  const uint16_t* w1;
+  const uint16_t* w3;
+  const uint16_t* w2;
+  uint16_t* h;              // [Rmax, I]
+  float* y;                 // [Rmax, H]
+  int32_t* status;          // device status word
+  int64_t rmax;
+  unsigned long long timeout_ns;
+};
+
+// GEMM1 (gate/up + SwiGLU -> h) then GEMM2 (h w2^T -> y), both persistent tcgen05.
+cudaError_t launch_grouped_swiglu(const Shape& s, const GemmArgs& g, cudaStream_t st,
+                                  const char** why);
+
+cudaError_t launch_combine(const Shape& s, const float* y, const int32_t* row_of,
+                           const float* topk_w, const uint16_t* residual, uint16_t* out,
+                           cudaStream_t st);
+
+int num_sms();
+
+}  // namespace moe

@@ -1,0 +1,299 @@
+// Router + scoring, expert histogram, padded offsets, stable ranks and the gather of
+// routed rows: the integer and HBM-bound steps of the sparse-MoE layer on sm_100a.
+//
+// Sources (nnterp encyclopedia, "Mixtral"): the router gives one logit per expert
+// with no bias ("Values, by host", router_logits; "Attention has no window": no
+// projection has a bias); softmax over all E in float32, keep the k largest, divide
+// them by their sum, slot 0 the larger ("The router renormalizes its top 2, in
+// float32"). The expert-contiguous row order is this library's own: stable on
+// (expert, token, slot), groups padded to 128 rows.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.cs.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+// One warp per token. Each lane accumulates, in fp32 and in a fixed order, the dot
+// products of its 8-element slices of x[t] with every router row; a butterfly sum
+// gives every lane the E logits. Lane 0 then scores them.
+template <int EMAX>
+__global__ void __launch_bounds__(256) k_router(const uint16_t* __restrict__ x,
+                                                const uint16_t* __restrict__ wr,
+                                                const float* __restrict__ bias, int64_t T,
+                                                int H, int E, int k,
+                                                int32_t* __restrict__ idx_out,
+                                                float* __restrict__ w_out,
+                                                float* __restrict__ logits_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int chunks = H >> 3;
+  for (int64_t t = warp0; t < T; t += nwarps) {
+    float acc[EMAX];
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) acc[e] = 0.f;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + t * H);
+    for (int c = lane; c < chunks; c += 32) {
+      const uint4 xv = ld_stream(xr + c);
+      const float x0 = bf16_lo(xv.x), x1 = bf16_hi(xv.x), x2 = bf16_lo(xv.y), x3 = bf16_hi(xv.y);
+      const float x4 = bf16_lo(xv.z), x5 = bf16_hi(xv.z), x6 = bf16_lo(xv.w), x7 = bf16_hi(xv.w);
+#pragma unroll
+      for (int e = 0; e < EMAX; ++e) {
+        if (e < E) {
+          const uint4 wv = __ldg(reinterpret_cast<const uint4*>(wr + (size_t)e * H) + c);
+          float a = acc[e];
+          a = fmaf(x0, bf16_lo(wv.x), a);
+          a = fmaf(x1, bf16_hi(wv.x), a);
+          a = fmaf(x2, bf16_lo(wv.y), a);
+          a = fmaf(x3, bf16_hi(wv.y), a);
+          a = fmaf(x4, bf16_lo(wv.z), a);
+          a = fmaf(x5, bf16_hi(wv.z), a);
+          a = fmaf(x6, bf16_lo(wv.w), a);
+          a = fmaf(x7, bf16_hi(wv.w), a);
+          acc[e] = a;
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+    }
+    if (lane == 0) {
+      float l[EMAX], p[EMAX];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < EMAX; ++e) {
+        if (e < E) {
+          l[e] = acc[e] + (bias ? bias[e] : 0.f);
+          mx = fmaxf(mx, l[e]);
+          if (logits_out) logits_out[t * E + e] = l[e];
+        }
+      }
+      // float32 softmax over all E experts
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < EMAX; ++e)
+        if (e < E) { p[e] = expf(l[e] - mx); s += p[e]; }
+#pragma unroll
+      for (int e = 0; e < EMAX; ++e)
+        if (e < E) p[e] = p[e] / s;
+      // the k largest, ranked on the float32 logit; equal logits -> lower index
+      uint64_t taken = 0;
+      int sel[8];
+      float psum = 0.f;
+      for (int j = 0; j < k; ++j) {
+        int best = -1;
+        float bl = 0.f;
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) {
+          if (e < E && !((taken >> e) & 1ull) && (best < 0 || l[e] > bl)) { best = e; bl = l[e]; }
+        }
+        taken |= 1ull << best;
+        sel[j] = best;
+        float pb = 0.f;
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e)
+          if (e == best) pb = p[e];
+        psum += pb;
+      }
+      for (int j = 0; j < k; ++j) {
+        float pb = 0.f;
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e)
+          if (e == sel[j]) pb = p[e];
+        idx_out[t * k + j] = sel[j];
+        w_out[t * k + j] = pb / psum;
+      }
+    }
+  }
+}
+
+// Lanes of this warp (one token each) whose routed slots include expert e.
+__device__ __forceinline__ unsigned expert_lanes(const int* my, int k, bool valid, int e) {
+  unsigned bits = 0;
+  for (int j = 0; j < k; ++j) bits |= __ballot_sync(0xffffffffu, valid && my[j] == e);
+  return bits;
+}
+
+// Per token block (32 tokens, one warp): count of routed slots per expert.
+__global__ void __launch_bounds__(256) k_block_hist(const int32_t* __restrict__ idx, int64_t T,
+                                                    int E, int k, int64_t nb,
+                                                    int32_t* __restrict__ block_counts) {
+  const int lane = threadIdx.x & 31;
+  const int64_t b = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (b >= nb) return;
+  const int64_t t = b * kTokensPerBlock + lane;
+  const bool valid = t < T;
+  int my[8];
+  for (int j = 0; j < k; ++j) my[j] = valid ? idx[t * k + j] : -1;
+  for (int e = 0; e < E; ++e) {
+    const unsigned bits = expert_lanes(my, k, valid, e);
+    if (lane == 0) block_counts[b * E + e] = __popc(bits);
+  }
+}
+
+// One CTA: per-expert exclusive prefix over token blocks (in place), total counts,
+// and the padded group offsets; then every block base is shifted by its group's
+// offset.
+__global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ block_base, int64_t nb,
+                                               int E, int32_t* __restrict__ counts,
+                                               int32_t* __restrict__ offsets) {
+  __shared__ int32_t s_count[64];
+  __shared__ int32_t s_off[65];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int e = warp; e < E; e += nwarps) {
+    int32_t run = 0;
+    for (int64_t b0 = 0; b0 < nb; b0 += 32) {
+      const int64_t b = b0 + lane;
+      const int32_t v = b < nb ? block_base[b * E + e] : 0;
+      int32_t incl = v;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int32_t n = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += n;
+      }
+      if (b < nb) block_base[b * E + e] = run + incl - v;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_count[e] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t acc = 0;
+    for (int e = 0; e < E; ++e) {
+      s_off[e] = acc;
+      acc += (s_count[e] + kRowPad - 1) / kRowPad * kRowPad;
+    }
+    s_off[E] = acc;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    offsets[e] = s_off[e];
+    if (e < E) counts[e] = s_count[e];
+  }
+  for (int64_t i = threadIdx.x; i < nb * E; i += blockDim.x) block_base[i] += s_off[i % E];
+}
+
+// Per token block: the stable rank of each routed slot among its expert's slots,
+// hence its row; writes row_of and token_of_row for real rows.
+__global__ void __launch_bounds__(256) k_rank(const int32_t* __restrict__ idx, int64_t T, int E,
+                                              int k, int64_t nb,
+                                              const int32_t* __restrict__ block_base,
+                                              int32_t* __restrict__ row_of,
+                                              int32_t* __restrict__ token_of_row) {
+  const int lane = threadIdx.x & 31;
+  const int64_t b = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (b >= nb) return;
+  const int64_t t = b * kTokensPerBlock + lane;
+  const bool valid = t < T;
+  int my[8];
+  for (int j = 0; j < k; ++j) my[j] = valid ? idx[t * k + j] : -1;
+  const unsigned below = (1u << lane) - 1u;
+  for (int e = 0; e < E; ++e) {
+    const unsigned bits = expert_lanes(my, k, valid, e);
+    if (!bits) continue;
+    const int32_t base = block_base[b * E + e];
+    // a token's k slots name k distinct experts, so at most one slot matches e
+    for (int j = 0; j < k; ++j) {
+      if (valid && my[j] == e) {
+        const int32_t row = base + __popc(bits & below);
+        row_of[t * k + j] = row;
+        token_of_row[row] = (int32_t)t;
+      }
+    }
+  }
+}
+
+// One warp per row of x_perm below R_pad: copies x[token] or, on pad rows, writes
+// zeros and token -1.
+__global__ void __launch_bounds__(256) k_gather(const uint16_t* __restrict__ x, int H, int E,
+                                                const int32_t* __restrict__ counts,
+                                                const int32_t* __restrict__ offsets,
+                                                int32_t* __restrict__ token_of_row,
+                                                uint16_t* __restrict__ x_perm) {
+  __shared__ int32_t s_off[65], s_cnt[64];
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    s_off[e] = offsets[e];
+    if (e < E) s_cnt[e] = counts[e];
+  }
+  __syncthreads();
+  const int64_t rows = s_off[E];
+  const int lane = threadIdx.x & 31;
+  const int64_t w0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int chunks = H >> 3;
+  for (int64_t r = w0; r < rows; r += nw) {
+    int e = 0;
+    while (e + 1 < E && s_off[e + 1] <= r) ++e;
+    const bool pad = r >= s_off[e] + s_cnt[e];
+    uint4* dst = reinterpret_cast<uint4*>(x_perm + r * H);
+    if (pad) {
+      if (lane == 0) token_of_row[r] = -1;
+      for (int c = lane; c < chunks; c += 32) dst[c] = make_uint4(0, 0, 0, 0);
+    } else {
+      const int64_t t = token_of_row[r];
+      const uint4* src = reinterpret_cast<const uint4*>(x + t * H);
+      int c = lane;
+      for (; c + 96 < chunks; c += 128) {
+        const uint4 a = __ldg(src + c), b2 = __ldg(src + c + 32), c2 = __ldg(src + c + 64),
+                    d = __ldg(src + c + 96);
+        dst[c] = a;
+        dst[c + 32] = b2;
+        dst[c + 64] = c2;
+        dst[c + 96] = d;
+      }
+      for (; c < chunks; c += 32) dst[c] = __ldg(src + c);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_router(const Shape& s, const uint16_t* x, const uint16_t* w_router,
+                          const float* logit_bias, int32_t* topk_idx, float* topk_w,
+                          float* logits, cudaStream_t st) {
+  const int threads = 256;
+  int64_t blocks = (s.T + 7) / 8;
+  const int64_t cap = (int64_t)num_sms() * 16;
+  if (blocks > cap) blocks = cap;
+#define MOE_ROUTER(EM)                                                                  \
+  k_router<EM><<<(unsigned)blocks, threads, 0, st>>>(x, w_router, logit_bias, s.T, s.H, \
+                                                     s.E, s.k, topk_idx, topk_w, logits)
+  if (s.E <= 8) MOE_ROUTER(8);
+  else if (s.E <= 16) MOE_ROUTER(16);
+  else if (s.E <= 32) MOE_ROUTER(32);
+  else MOE_ROUTER(64);
+#undef MOE_ROUTER
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16_t* x,
+                           int32_t* counts, int32_t* offsets, int32_t* row_of,
+                           int32_t* token_of_row, uint16_t* x_perm, int32_t* block_base,
+                           cudaStream_t st) {
+  const int64_t nb = num_token_blocks(s);
+  const unsigned wblocks = (unsigned)((nb + 7) / 8);
+  k_block_hist<<<wblocks, 256, 0, st>>>(topk_idx, s.T, s.E, s.k, nb, block_base);
+  k_scan<<<1, 1024, 0, st>>>(block_base, nb, s.E, counts, offsets);
+  k_rank<<<wblocks, 256, 0, st>>>(topk_idx, s.T, s.E, s.k, nb, block_base, row_of, token_of_row);
+  int64_t gblocks = (max_padded_rows(s) + 7) / 8;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  if (gblocks > cap) gblocks = cap;
+  k_gather<<<(unsigned)gblocks, 256, 0, st>>>(x, s.H, s.E, counts, offsets, token_of_row, x_perm);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,241 @@
+"""ctypes binding of libmoe.so (include/moe.h): argument marshalling only.
+
+Every step of the layer runs in the library's CUDA kernels. PyTorch supplies device
+memory and the current stream; nothing here computes any part of the layer, and
+there is no fallback: if the library is missing or a tensor is not on a CUDA device,
+the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+ROW_PAD = 128
+
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+          4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
+
+EXPORTS = ("moe_workspace_size", "moe_workspace_size_host", "moe_max_padded_rows",
+           "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_forward",
+           "moe_forward_host", "moe_device_status", "moe_last_error")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("num_tokens", ctypes.c_int64), ("hidden_size", ctypes.c_int32),
+                ("intermediate_size", ctypes.c_int32), ("num_experts", ctypes.c_int32),
+                ("num_experts_per_tok", ctypes.c_int32)]
+
+
+_lib = None
+_P = ctypes.c_void_p
+_SZ = ctypes.c_size_t
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmoe.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m sparse_mixture_experts_09_b200.build_lib`")
+        L = ctypes.CDLL(LIB_PATH)
+        sp = ctypes.POINTER(Shape)
+        st = ctypes.c_int
+        L.moe_workspace_size.argtypes = [sp]
+        L.moe_workspace_size.restype = _SZ
+        L.moe_workspace_size_host.argtypes = [sp]
+        L.moe_workspace_size_host.restype = _SZ
+        L.moe_max_padded_rows.argtypes = [sp]
+        L.moe_max_padded_rows.restype = ctypes.c_int64
+        L.moe_router_topk.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P]
+        L.moe_router_topk.restype = st
+        L.moe_permute.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.moe_permute.restype = st
+        L.moe_grouped_swiglu.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.moe_grouped_swiglu.restype = st
+        L.moe_combine.argtypes = [sp, _P, _P, _P, _P, _P, _P]
+        L.moe_combine.restype = st
+        L.moe_forward.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.moe_forward.restype = st
+        L.moe_forward_host.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.moe_forward_host.restype = st
+        L.moe_device_status.argtypes = [_P, _SZ, _P]
+        L.moe_device_status.restype = st
+        L.moe_last_error.argtypes = []
+        L.moe_last_error.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise MoeError(status, lib().moe_last_error().decode(errors="replace"))
+
+
+def make_shape(num_tokens: int, hidden_size: int, intermediate_size: int, num_experts: int,
+               num_experts_per_tok: int) -> Shape:
+    return Shape(int(num_tokens), int(hidden_size), int(intermediate_size), int(num_experts),
+                 int(num_experts_per_tok))
+
+
+def _dev(t: Optional[torch.Tensor], name: str, dtype=None, nullable=False) -> Optional[int]:
+    if t is None:
+        if nullable:
+            return None
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def workspace_size(shape: Shape) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(shape)))
+
+
+def workspace_size_host(shape: Shape) -> int:
+    return int(lib().moe_workspace_size_host(ctypes.byref(shape)))
+
+
+def max_padded_rows(shape: Shape) -> int:
+    return int(lib().moe_max_padded_rows(ctypes.byref(shape)))
+
+
+def make_workspace(shape: Shape, device="cuda", host: bool = False) -> torch.Tensor:
+    """A zeroed device workspace (zero status word) big enough for ``shape``."""
+    n = workspace_size_host(shape) if host else workspace_size(shape)
+    if n == 0:
+        raise MoeError(2, lib().moe_last_error().decode(errors="replace"))
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def router_topk(x, w_router, k: int, logit_bias=None, return_logits=False, stream=None):
+    """(topk_idx [T,k] int32, topk_w [T,k] fp32[, logits [T,E] fp32])."""
+    t, h = x.shape
+    e = w_router.shape[0]
+    shape = make_shape(t, h, ROW_PAD, e, k)
+    idx = torch.empty((t, k), dtype=torch.int32, device=x.device)
+    w = torch.empty((t, k), dtype=torch.float32, device=x.device)
+    logits = torch.empty((t, e), dtype=torch.float32, device=x.device) if return_logits else None
+    _check(lib().moe_router_topk(ctypes.byref(shape), _dev(x, "x", torch.bfloat16),
+                                 _dev(w_router, "w_router", torch.bfloat16),
+                                 _dev(logit_bias, "logit_bias", torch.float32, True),
+                                 _dev(idx, "idx"), _dev(w, "w"), _dev(logits, "logits", None, True),
+                                 _stream(stream)))
+    return (idx, w, logits) if return_logits else (idx, w)
+
+
+def permute(topk_idx, x, num_experts: int, intermediate_size: int, ws, stream=None) -> dict:
+    """Expert-contiguous permutation of the routed rows (see moe_permute)."""
+    t, k = topk_idx.shape
+    h = x.shape[1]
+    shape = make_shape(t, h, intermediate_size, num_experts, k)
+    rmax = max_padded_rows(shape)
+    dev = x.device
+    out = {
+        "counts": torch.empty(num_experts, dtype=torch.int32, device=dev),
+        "offsets": torch.empty(num_experts + 1, dtype=torch.int32, device=dev),
+        "row_of": torch.empty((t, k), dtype=torch.int32, device=dev),
+        "token_of_row": torch.full((rmax,), -2, dtype=torch.int32, device=dev),
+        "x_perm": torch.zeros((rmax, h), dtype=torch.bfloat16, device=dev),
+    }
+    _check(lib().moe_permute(ctypes.byref(shape), _dev(topk_idx, "topk_idx", torch.int32),
+                             _dev(x, "x", torch.bfloat16), _dev(out["counts"], "counts"),
+                             _dev(out["offsets"], "offsets"), _dev(out["row_of"], "row_of"),
+                             _dev(out["token_of_row"], "token_of_row"), _dev(out["x_perm"], "x_perm"),
+                             _dev(ws, "ws"), ws.numel(), _stream(stream)))
+    return out
+
+
+def grouped_swiglu(x_perm, offsets, w1, w3, w2, num_tokens: int, k: int, ws, stream=None):
+    """y_perm [R_max, H] fp32 = w2[e] (silu(w1[e] x) * w3[e] x) per routed row."""
+    e, i, h = w1.shape
+    shape = make_shape(num_tokens, h, i, e, k)
+    y = torch.zeros((max_padded_rows(shape), h), dtype=torch.float32, device=x_perm.device)
+    _check(lib().moe_grouped_swiglu(ctypes.byref(shape), _dev(x_perm, "x_perm", torch.bfloat16),
+                                    _dev(offsets, "offsets", torch.int32),
+                                    _dev(w1, "w1", torch.bfloat16), _dev(w3, "w3", torch.bfloat16),
+                                    _dev(w2, "w2", torch.bfloat16), _dev(y, "y_perm"),
+                                    _dev(ws, "ws"), ws.numel(), _stream(stream)))
+    return y
+
+
+def combine(y_perm, row_of, topk_w, residual=None, num_experts: int = 8, intermediate_size: int = ROW_PAD,
+            stream=None):
+    """out [T,H] bf16 = residual + sum_j topk_w[:,j] * y_perm[row_of[:,j]]."""
+    t, k = row_of.shape
+    h = y_perm.shape[1]
+    shape = make_shape(t, h, intermediate_size, max(num_experts, k), k)
+    out = torch.empty((t, h), dtype=torch.bfloat16, device=y_perm.device)
+    _check(lib().moe_combine(ctypes.byref(shape), _dev(y_perm, "y_perm", torch.float32),
+                             _dev(row_of, "row_of", torch.int32), _dev(topk_w, "topk_w", torch.float32),
+                             _dev(residual, "residual", torch.bfloat16, True), _dev(out, "out"),
+                             _stream(stream)))
+    return out
+
+
+def forward(x, w_router, w1, w3, w2, k: int, residual=None, logit_bias=None, ws=None, out=None,
+            stream=None):
+    """The whole layer on device tensors; returns out [T,H] bf16."""
+    t, h = x.shape
+    e, i, _ = w1.shape
+    shape = make_shape(t, h, i, e, k)
+    if ws is None:
+        ws = make_workspace(shape, x.device)
+    if out is None:
+        out = torch.empty((t, h), dtype=torch.bfloat16, device=x.device)
+    _check(lib().moe_forward(ctypes.byref(shape), _dev(x, "x", torch.bfloat16),
+                             _dev(w_router, "w_router", torch.bfloat16),
+                             _dev(logit_bias, "logit_bias", torch.float32, True),
+                             _dev(w1, "w1", torch.bfloat16), _dev(w3, "w3", torch.bfloat16),
+                             _dev(w2, "w2", torch.bfloat16),
+                             _dev(residual, "residual", torch.bfloat16, True), _dev(out, "out"),
+                             _dev(ws, "ws"), ws.numel(), _stream(stream)))
+    return out
+
+
+def forward_host(x_host, w_router, w1, w3, w2, k: int, residual_host=None, logit_bias=None,
+                 ws=None, out_host=None, stream=None):
+    """The layer with host (ideally pinned) activations; returns out_host (synchronous)."""
+    t, h = x_host.shape
+    e, i, _ = w1.shape
+    shape = make_shape(t, h, i, e, k)
+    for name, a in (("x_host", x_host), ("residual_host", residual_host)):
+        if a is not None and (a.is_cuda or a.dtype != torch.bfloat16 or not a.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous bf16 host tensor")
+    if ws is None:
+        ws = make_workspace(shape, w1.device, host=True)
+    if out_host is None:
+        out_host = torch.empty((t, h), dtype=torch.bfloat16, pin_memory=True)
+    _check(lib().moe_forward_host(ctypes.byref(shape), x_host.data_ptr(),
+                                  _dev(w_router, "w_router", torch.bfloat16),
+                                  _dev(logit_bias, "logit_bias", torch.float32, True),
+                                  _dev(w1, "w1", torch.bfloat16), _dev(w3, "w3", torch.bfloat16),
+                                  _dev(w2, "w2", torch.bfloat16),
+                                  None if residual_host is None else residual_host.data_ptr(),
+                                  out_host.data_ptr(), _dev(ws, "ws"), ws.numel(), _stream(stream)))
+    return out_host
+
+
+def device_status(ws, stream=None) -> None:
+    """Raise MoeError(MOE_ERR_TIMEOUT) if a kernel gave up a bounded wait since last checked."""
+    _check(lib().moe_device_status(_dev(ws, "ws"), ws.numel(), _stream(stream)))

@@ -1,0 +1,91 @@
+"""The C-ABI library: it builds, loads, exports every declared symbol, and rejects bad
+arguments on the host before any CUDA call (so these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_mixture_experts_09_b200 import build_lib
+from sparse_mixture_experts_09_b200 import moe as M
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build_lib.build()
+    return M.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
+                     "moe_forward", "moe_workspace_size", "moe_last_error"):
+        assert required in names
+    assert set(names) == set(M.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def shape(t=64, h=128, i=256, e=8, k=2):
+    return M.make_shape(t, h, i, e, k)
+
+
+def test_workspace_and_padded_rows(L):
+    s = shape()
+    assert M.max_padded_rows(s) == 128 + 128 * 8
+    assert M.workspace_size(s) > 0
+    assert M.workspace_size_host(s) > M.workspace_size(s)
+    big = shape(t=4096, h=4096, i=14336)
+    rmax = M.max_padded_rows(big)
+    # x_perm + h + y dominate
+    assert M.workspace_size(big) >= rmax * (4096 * 2 + 14336 * 2 + 4096 * 4)
+
+
+@pytest.mark.parametrize("bad", [dict(t=0), dict(h=100), dict(i=200), dict(e=0), dict(e=65),
+                                 dict(k=0), dict(k=9, e=16), dict(k=3, e=2)])
+def test_invalid_shapes_are_rejected(L, bad):
+    s = shape(**bad)
+    assert M.workspace_size(s) == 0
+    assert M.max_padded_rows(s) == -1
+    st = L.moe_forward(ctypes.byref(s), 16, 16, None, 16, 16, 16, None, 16, 256, 1 << 30, None)
+    assert st in (1, 2)
+    assert L.moe_last_error()
+
+
+def test_null_and_misaligned_pointers_are_rejected(L):
+    s = shape()
+    st = L.moe_forward(ctypes.byref(s), None, 16, None, 16, 16, 16, None, 16, 256, 1 << 30, None)
+    assert st == 1 and b"x is NULL" in L.moe_last_error()
+    st = L.moe_forward(ctypes.byref(s), 24, 16, None, 16, 16, 16, None, 16, 256, 1 << 30, None)
+    assert st == 1 and b"aligned" in L.moe_last_error()
+    st = L.moe_router_topk(ctypes.byref(s), 16, 16, None, 16, None, None, None)
+    assert st == 1 and b"topk_w" in L.moe_last_error()
+
+
+def test_small_workspace_is_rejected(L):
+    s = shape()
+    need = M.workspace_size(s)
+    st = L.moe_forward(ctypes.byref(s), 16, 16, None, 16, 16, 16, None, 16, 256, need - 1, None)
+    assert st == 3 and b"workspace too small" in L.moe_last_error()
+    st = L.moe_forward(ctypes.byref(s), 16, 16, None, 16, 16, 16, None, 16, 128, need, None)
+    assert st == 3
+    st = L.moe_grouped_swiglu(ctypes.byref(s), 16, 16, 16, 16, 16, 16, 256, 10, None)
+    assert st == 3
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    x = torch.zeros(4, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        M.router_topk(x, torch.zeros(8, 128, dtype=torch.bfloat16), 2)

@@ -1,0 +1,121 @@
+"""Whole-layer GPU parity through the C ABI (moe_forward), in the benchmark's launch
+configuration, against the fp64 oracle; plus the invariants the nnterp "Mixtral"
+page states for the layer, checked on the GPU."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from sparse_mixture_experts_09_b200 import moe as M
+from sparse_mixture_experts_09_b200 import workloads as W
+
+from ._cases import assert_layer_close, layer_errors, sample_tokens, screened, to_cpu
+from .test_gpu_kernels import SMALL
+
+pytestmark = pytest.mark.gpu
+
+SINGLE_EXPERT = W.Workload("single_expert", 200, 128, 256, 1, 1, seed=16)
+
+
+def _forward_and_check(w, inp, tokens=None, residual=True):
+    res = inp.residual if residual else None
+    shape = M.make_shape(*w.shape)
+    ws = M.make_workspace(shape)
+    out = M.forward(inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, w.num_experts_per_tok,
+                    residual=res, logit_bias=inp.logit_bias, ws=ws)
+    M.device_status(ws)
+    c = to_cpu(inp)
+    ref = O.moe_layer(c.x, c.w_router, c.w1, c.w3, c.w2, w.num_experts_per_tok,
+                      residual=None if res is None else c.residual, logit_bias=c.logit_bias,
+                      mode="bf16_storage", tokens=tokens)
+    got = O.to_f64(out.cpu())
+    if tokens is not None:
+        got = got[tokens]
+    return got, ref, out
+
+
+@pytest.mark.parametrize("name", list(SMALL) + ["single_expert"])
+def test_forward_small(name):
+    w = SINGLE_EXPERT if name == "single_expert" else SMALL[name]
+    inp, near = screened(w)
+    assert near.numel() == 0
+    # the gate is on the routed output (no residual), which a unit-RMS residual would mask
+    got, ref, _ = _forward_and_check(w, inp, residual=False)
+    assert_layer_close(got, ref["out"], name)
+    got, ref, _ = _forward_and_check(w, inp, residual=True)
+    assert_layer_close(got, ref["out"], name + "+residual")
+
+
+def test_single_expert_is_plain_swiglu():
+    # E = 1, k = 1: the layer is w2 (silu(w1 x) * w3 x), checked here against torch's
+    # own fp64 F.linear / F.silu on the same bf16 values
+    import torch.nn.functional as F
+    w = SINGLE_EXPERT
+    inp, _ = screened(w)
+    got, _, _ = _forward_and_check(w, inp, residual=False)
+    c = to_cpu(inp)
+    x = c.x.double()
+    want = F.linear(F.silu(F.linear(x, c.w1[0].double())) * F.linear(x, c.w3[0].double()),
+                    c.w2[0].double()).numpy()
+    max_rel, mae = layer_errors(got, want)
+    assert max_rel <= 2e-2 and mae <= 5e-3       # h rounded to bf16 on the GPU, not in `want`
+
+
+def test_forward_is_deterministic_and_host_entry_matches():
+    w = SMALL["ragged"]
+    inp, _ = screened(w)
+    a = M.forward(inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, 2, residual=inp.residual)
+    b = M.forward(inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, 2, residual=inp.residual)
+    assert torch.equal(a, b)
+    xh = inp.x.cpu().pin_memory()
+    rh = inp.residual.cpu().pin_memory()
+    h = M.forward_host(xh, inp.w_router, inp.w1, inp.w3, inp.w2, 2, residual_host=rh)
+    assert torch.equal(h, a.cpu())
+
+
+def test_ablating_an_expert_changes_exactly_its_tokens():
+    # nnterp "Mixtral", "Ablating an expert": zero expert e's weight where it was chosen;
+    # the output changes on exactly the tokens that chose e.
+    w = SMALL["ragged"]
+    inp, _ = screened(w)
+    shape = M.make_shape(*w.shape)
+    ws = M.make_workspace(shape)
+    idx, wt = M.router_topk(inp.x, inp.w_router, 2)
+    p = M.permute(idx, inp.x, w.num_experts, w.intermediate_size, ws)
+    y = M.grouped_swiglu(p["x_perm"], p["offsets"], inp.w1, inp.w3, inp.w2, w.num_tokens, 2, ws)
+    clean = M.combine(y, p["row_of"], wt, inp.residual, w.num_experts, w.intermediate_size)
+    for e in (0, 3, 7):
+        abl_w = wt.masked_fill(idx == e, 0.0)
+        ablated = M.combine(y, p["row_of"], abl_w, inp.residual, w.num_experts, w.intermediate_size)
+        changed = (ablated != clean).any(-1)
+        assert torch.equal(changed, (idx == e).any(-1))
+
+
+@pytest.mark.parametrize("name", ["decode", "prefill", "imbalanced_a", "imbalanced_b", "larger"])
+def test_forward_full_size(name):
+    w = W.WORKLOADS[name]
+    inp, near = screened(w)
+    assert near.numel() <= max(1, w.num_tokens // 1000)
+    c = to_cpu(inp)
+    # routing of every token, bit-exact
+    idx, wt = M.router_topk(inp.x, inp.w_router, 2, inp.logit_bias)
+    ref_idx, ref_w, _ = O.route_topk(O.router_logits(c.x, c.w_router, c.logit_bias), 2)
+    ok = np.ones(w.num_tokens, dtype=bool)
+    ok[near.numpy()] = False
+    assert np.array_equal(idx.cpu().numpy()[ok], ref_idx[ok])
+    count, offset, row_of, tok = O.stable_permute(ref_idx, w.num_experts)
+    if w.logit_bias is not None:
+        assert count[0] > 0.4 * count.sum()          # about half the slots go to expert 0
+    # outputs on sampled tokens (all tokens when T <= 256)
+    tokens = sample_tokens(w.num_tokens)
+    got, ref, _ = _forward_and_check(w, inp, tokens=tokens, residual=False)
+    assert_layer_close(got, ref["out"], name)
+
+
+@pytest.mark.parametrize("t", W.DECODE_SWEEP_TOKENS)
+def test_forward_decode_sweep(t):
+    w = W.WORKLOADS["larger"].with_tokens(t)
+    inp, near = screened(w)
+    assert near.numel() == 0
+    got, ref, _ = _forward_and_check(w, inp, residual=False)
+    assert_layer_close(got, ref["out"], w.name)
