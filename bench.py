@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Throughput of the Mixtral sparse-MoE feed-forward layer on B200, one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|...]
+    python bench.py --impl reference ...     # the fp64 CPU oracle on the host cores
+
+A step is one pass of the whole layer (router, scoring, permutation, both expert
+GEMMs, combine) over the workload's synthetic batch. ``value`` is tokens/s with every
+input resident in HBM, timed with CUDA events around K back-to-back moe_forward calls.
+A second loop of K steps runs the same kernels through the split entry points with
+events between stages, which gives each kernel's average duration for the roofline
+line. ``e2e`` times K calls of moe_forward_host: host-to-device copy of x and the
+residual from pinned memory, the layer, device-to-host copy of the output.
+
+Under torchrun every rank runs its own replica of the workload (the layer shards
+over independent batches; there is no data-path collective): ``value`` is all ranks'
+tokens over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s and % of roofline (BF16 tensor peak / HBM BW) at 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+GEMM_SOURCE = os.path.join(ROOT, "sparse_mixture_experts_09_b200", "csrc", "gemm_sm100.cu")
+# kernels one moe_forward launches: router, 4 permutation kernels (histogram, scan,
+# rank, gather), the two expert GEMMs and the combine
+KERNELS_PER_FORWARD = 8
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(w):
+    return {"workload": w.name, "num_tokens": w.num_tokens, "hidden_size": w.hidden_size,
+            "intermediate_size": w.intermediate_size, "num_experts": w.num_experts,
+            "num_experts_per_tok": w.num_experts_per_tok,
+            "logit_bias": list(w.logit_bias) if w.logit_bias else None}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock, power and throttle reasons while running."""
+    QUERY = ("index,pci.bus_id,utilization.gpu,clocks.sm,clocks.max.sm,power.draw,"
+             "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id=None):
+        self.bus_id = bus_id
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                   "-lms", "100"]
+            if self.bus_id:
+                cmd += ["-i", self.bus_id]
+            self.proc = subprocess.Popen(cmd, stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [r.split(", ") for r in f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        rows = [r for r in rows if len(r) >= 11]
+        if not rows:
+            return None
+        loaded = [r for r in rows if r[2].strip().isdigit() and int(r[2]) >= 30] or rows
+        sm = [float(r[3]) for r in loaded if _isnum(r[3])]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i in range(4) if r[7 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(loaded[0][4]) if _isnum(loaded[0][4]) else None,
+                "reasons": reasons, "samples_under_load": len(loaded),
+                "power_w_max": max(float(r[5]) for r in loaded if _isnum(r[5])) if loaded else None}
+
+
+def _isnum(s):
+    try:
+        float(s)
+        return True
+    except ValueError:
+        return False
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else None
+    except Exception:
+        return None
+
+
+def oracle_timing(inp_cpu, w, budget_s, max_runs=None, tokens=None):
+    """Run the oracle (as it stands) on the workload until ``budget_s`` of CPU time
+    has passed; returns (seconds per run, runs, tokens per run)."""
+    import torch
+    from oracle import moe_oracle as O
+    runs, t0 = 0, time.perf_counter()
+    while True:
+        O.moe_layer(inp_cpu.x, inp_cpu.w_router, inp_cpu.w1, inp_cpu.w3, inp_cpu.w2,
+                    w.num_experts_per_tok, residual=inp_cpu.residual, logit_bias=inp_cpu.logit_bias,
+                    mode="exact", tokens=tokens)
+        runs += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or (max_runs and runs >= max_runs):
+            break
+    n_tok = w.num_tokens if tokens is None else len(tokens)
+    return el / runs, runs, n_tok, torch.get_num_threads()
+
+
+def cpu_sample_tokens(w):
+    """Token subset for the CPU baseline: whole batch up to 64 tokens, else 64 tokens."""
+    if w.num_tokens <= 64:
+        return None
+    step = w.num_tokens // 64
+    return list(range(0, w.num_tokens, step))[:64]
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    from sparse_mixture_experts_09_b200 import workloads as W
+    w = W.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = W.draw(w, dev)
+    inp = W.LayerInputs(*(None if t is None else t.cpu() for t in
+                          (inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, inp.residual, inp.logit_bias)))
+    tokens = cpu_sample_tokens(w)
+    # probe one step, then size the run to a few minutes
+    per_step, _, n_tok, threads = oracle_timing(inp, w, 0.0, max_runs=1, tokens=tokens)
+    budget = 150.0
+    steps = max(1, min(args.steps, int((budget - per_step) / per_step) - args.warmup))
+    warm = min(args.warmup, max(0, int(budget / per_step) - steps - 1))
+    if warm:
+        oracle_timing(inp, w, 0.0, max_runs=warm, tokens=tokens)
+    t0 = time.perf_counter()
+    oracle_timing(inp, w, 0.0, max_runs=steps, tokens=tokens)
+    el = time.perf_counter() - t0
+    value = n_tok * steps / el
+    sample = (f"{'all ' if tokens is None else ''}{n_tok} tokens of the {w.name} batch per step, "
+              f"fp64 exact mode, {steps} timed steps after {warm} warm-up")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 0,
+            "steps": steps, "warmup": warm, "ms_per_step": 1e3 * el / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads() or threads,
+                             "kind": "oracle", "sample": sample, "host_cpus": os.cpu_count()},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+
+def kernel_roofline(w, stage_ms, counts, peaks, peak_kind, long_run):
+    """Roofline object of the dominant kernel (largest average duration)."""
+    H, I, k, T = w.hidden_size, w.intermediate_size, w.num_experts_per_tok, w.num_tokens
+    R = T * k
+    n_active = int(sum(1 for c in counts if c > 0))
+    wbytes = 2  # bf16
+    work = {
+        # name: (bytes per launch, flops per launch)
+        "router": (T * H * wbytes + w.num_experts * H * wbytes + T * k * 8, 2 * T * H * w.num_experts),
+        "permute": (2 * R * H * wbytes + T * k * 12, 0),
+        "gate_up": (n_active * 2 * I * H * wbytes + R * H * wbytes + R * I * wbytes, 4 * R * H * I),
+        "down": (n_active * H * I * wbytes + R * I * wbytes + R * H * 4, 2 * R * H * I),
+        "combine": (R * H * 4 + 2 * T * H * wbytes + T * k * 8, 2 * R * H),
+    }
+    name = max(stage_ms, key=stage_ms.get)
+    bytes_, flops = work[name]
+    sec = stage_ms[name] * 1e-3
+    hbm_peak = peaks["hbm_gbs"]
+    tensor_peak = peaks["bf16_tflops_sustained" if long_run else "bf16_tflops"]
+    hbm_time = bytes_ / (hbm_peak * 1e9)
+    tensor_time = flops / (tensor_peak * 1e12) if flops else 0.0
+    if name in ("gate_up", "down") and tensor_time > hbm_time:
+        r = {"bound": "tensor", "achieved": flops / sec / 1e12, "peak": tensor_peak,
+             "unit": "TFLOP/s"}
+    else:
+        r = {"bound": "hbm", "achieved": bytes_ / sec / 1e9, "peak": hbm_peak, "unit": "GB/s"}
+    r["frac"] = r["achieved"] / r["peak"]
+    r["kernel"] = name
+    r["peak_source"] = peak_kind + (" sustained" if (r["bound"] == "tensor" and long_run) else " burst")
+    r["algorithmic_bytes"] = bytes_
+    r["algorithmic_flops"] = flops
+    r["active_experts"] = n_active
+    r["traffic"] = ncu_traffic(w.name, name)
+    return r
+
+
+def ncu_traffic(workload, kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current GEMM source; else None."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            d = json.load(f)
+        with open(GEMM_SOURCE, "rb") as f:
+            src = hashlib.sha256(f.read()).hexdigest()[:16]
+        e = d.get(workload, {}).get(kernel)
+        if e and e.get("source_sha256_16") == src:
+            return e["dram_bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from sparse_mixture_experts_09_b200 import moe
+    from sparse_mixture_experts_09_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    moe.lib()  # fail loudly if the library is missing
+    w = W.WORKLOADS[args.workload]
+    inp = W.draw(w, dev)
+    k = w.num_experts_per_tok
+    shape = moe.make_shape(*w.shape)
+    ws = moe.make_workspace(shape, dev)
+    out = torch.empty((w.num_tokens, w.hidden_size), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        moe.forward(inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, k, residual=inp.residual,
+                    logit_bias=inp.logit_bias, ws=ws, out=out)
+
+    # split-path buffers for the per-kernel breakdown
+    rmax = moe.max_padded_rows(shape)
+    idx = torch.empty((w.num_tokens, k), dtype=torch.int32, device=dev)
+    wt = torch.empty((w.num_tokens, k), dtype=torch.float32, device=dev)
+    perm = {"counts": torch.empty(w.num_experts, dtype=torch.int32, device=dev),
+            "offsets": torch.empty(w.num_experts + 1, dtype=torch.int32, device=dev),
+            "row_of": torch.empty((w.num_tokens, k), dtype=torch.int32, device=dev),
+            "token_of_row": torch.empty(rmax, dtype=torch.int32, device=dev),
+            "x_perm": torch.empty((rmax, w.hidden_size), dtype=torch.bfloat16, device=dev)}
+    hbuf = torch.empty((rmax, w.intermediate_size), dtype=torch.bfloat16, device=dev)
+    ybuf = torch.empty((rmax, w.hidden_size), dtype=torch.float32, device=dev)
+    L = moe.lib()
+    import ctypes
+    sp = ctypes.byref(shape)
+    st = stream.cuda_stream
+    p = lambda t: t.data_ptr()  # noqa: E731
+    bias = None if inp.logit_bias is None else p(inp.logit_bias)
+
+    def split_step(ev):
+        ev[0].record(stream)
+        moe._check(L.moe_router_topk(sp, p(inp.x), p(inp.w_router), bias, p(idx), p(wt), None, st))
+        ev[1].record(stream)
+        moe._check(L.moe_permute(sp, p(idx), p(inp.x), p(perm["counts"]), p(perm["offsets"]),
+                                 p(perm["row_of"]), p(perm["token_of_row"]), p(perm["x_perm"]),
+                                 p(ws), ws.numel(), st))
+        ev[2].record(stream)
+        moe._check(L.moe_expert_gate_up(sp, p(perm["x_perm"]), p(perm["offsets"]), p(inp.w1),
+                                        p(inp.w3), p(hbuf), p(ws), ws.numel(), st))
+        ev[3].record(stream)
+        moe._check(L.moe_expert_down(sp, p(hbuf), p(perm["offsets"]), p(inp.w2), p(ybuf), p(ws),
+                                     ws.numel(), st))
+        ev[4].record(stream)
+        moe._check(L.moe_combine(sp, p(ybuf), p(perm["row_of"]), p(wt), p(inp.residual), p(out), st))
+        ev[5].record(stream)
+
+    xh = inp.x.cpu().pin_memory()
+    rh = inp.residual.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    wsh = moe.make_workspace(shape, dev, host=True)
+
+    def host_step():
+        moe.forward_host(xh, inp.w_router, inp.w1, inp.w3, inp.w2, k, residual_host=rh,
+                         logit_bias=inp.logit_bias, ws=wsh, out_host=oh)
+
+    K, Wm = args.steps, max(3, args.warmup)
+    for _ in range(Wm):
+        step()
+    scratch = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    for _ in range(3):
+        split_step(scratch)
+        host_step()
+    torch.cuda.synchronize(dev)
+    moe.device_status(ws)
+    barrier()
+
+    bus = None
+    try:
+        props = torch.cuda.get_device_properties(dev)
+        bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+    except Exception:
+        pass
+    clocks = ClockSampler(bus)
+    clocks.start()
+    time.sleep(0.3)
+
+    # (1) value: K back-to-back moe_forward calls, inputs resident in HBM
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = e0.elapsed_time(e1) / K
+
+    # (2) per-kernel breakdown through the split entry points
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        split_step(evs[i])
+    torch.cuda.synchronize(dev)
+    names = ["router", "permute", "gate_up", "down", "combine"]
+    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
+                for j, n in enumerate(names)}
+
+    # (3) end to end from pinned host memory
+    barrier()
+    torch.cuda.synchronize(dev)
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record(stream)
+    for _ in range(K):
+        host_step()
+    h1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = h0.elapsed_time(h1) / K
+    clk = clocks.stop()
+    moe.device_status(ws)
+    moe.device_status(wsh)
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+
+    counts = perm["counts"].cpu().tolist()
+    peaks, peak_kind = load_peaks()
+    long_run = ms * K > 1000.0
+    roof = kernel_roofline(w, stage_ms, counts, peaks, peak_kind, long_run)
+
+    line = None
+    if rank == 0:
+        tokens_all = w.num_tokens * world
+        bytes_io = w.num_tokens * w.hidden_size * 2
+        line = {
+            "metric": METRIC, "value": tokens_all / (ms * 1e-3), "unit": "tokens/s",
+            "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded SplitMix64/Box-Muller draws, weights ~N(0,1/fan_in), x rows RMS 1",
+            "config": dict(workload_config(w), parallelism=f"replicas x{world}",
+                           l2=("no flush: each step streams %.2f GB of expert weights, more than "
+                               "the 126 MB L2" % (roof["active_experts"] * w.expert_bytes() / 1e9))),
+            "roofline": roof,
+            "kernels_ms": stage_ms,
+            "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": 2 * bytes_io, "d2h_bytes_per_step": bytes_io,
+                    "api": "moe_forward_host"},
+            "gpu_launches": KERNELS_PER_FORWARD * K,
+            "clocks": clk,
+            "expert_counts": counts,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = W.LayerInputs(*(None if t is None else t.cpu() for t in
+                                  (inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, inp.residual,
+                                   inp.logit_bias)))
+            tokens = cpu_sample_tokens(w)
+            per, runs, n_tok, threads = oracle_timing(cpu, w, args.cpu_seconds, tokens=tokens)
+            line["cpu_baseline"] = {
+                "value": n_tok / per, "unit": "tokens/s", "cores": blas_threads() or threads,
+                "kind": "oracle", "host_cpus": os.cpu_count(),
+                "sample": (f"{'all ' if tokens is None else ''}{n_tok} tokens of the {w.name} batch "
+                           f"through the fp64 oracle (exact mode), {runs} runs, {per:.2f} s each")}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

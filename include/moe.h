@@ -29,7 +29,8 @@
  *   slot), each expert group padded to a multiple of MOE_ROW_PAD rows. Pad rows
  *   have token -1 and zero activations. moe_max_padded_rows() bounds the total.
  * - `ws` is a device workspace of at least moe_workspace_size() bytes, 256-byte
- *   aligned; each entry point that takes it uses its own region of it. Kernels
+ *   aligned, whose first 256 bytes (the status word) are zero before first use;
+ *   each entry point that takes it uses its own region of it. Kernels
  *   whose waits run out (a bounded spin that never completes) record
  *   MOE_ERR_TIMEOUT in the workspace; moe_device_status() reads and clears it.
  * - On failure the returned code is non-zero and moe_last_error() (thread-local)
@@ -131,6 +132,19 @@ moe_status_t moe_grouped_swiglu(const moe_shape_t* shape, const moe_bf16_t* x_pe
                                 const moe_bf16_t* w3, const moe_bf16_t* w2,
                                 float* y_perm, void* ws, size_t ws_bytes,
                                 moe_stream_t stream);
+
+/* The two halves of moe_grouped_swiglu, for callers that keep h themselves or time
+ * the GEMMs apart. `ws` as for moe_grouped_swiglu (ws_bytes >= moe_workspace_size).
+ *   moe_expert_gate_up: h [moe_max_padded_rows, I] bf16 out = bf16(silu(x_perm
+ *     w1[e]^T) * (x_perm w3[e]^T)) for the rows below R_pad;
+ *   moe_expert_down: y_perm [moe_max_padded_rows, H] fp32 out = h w2[e]^T. */
+moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* x_perm,
+                                const int32_t* expert_offsets, const moe_bf16_t* w1,
+                                const moe_bf16_t* w3, moe_bf16_t* h, void* ws,
+                                size_t ws_bytes, moe_stream_t stream);
+moe_status_t moe_expert_down(const moe_shape_t* shape, const moe_bf16_t* h,
+                             const int32_t* expert_offsets, const moe_bf16_t* w2,
+                             float* y_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Weighted combine into the residual (nnterp "Mixtral": expert_outputs summed over
  * the slot axis is routed_output; the block adds mlp_output to the residual):

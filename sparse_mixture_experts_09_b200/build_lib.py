@@ -36,25 +36,27 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose_ptxas: bool = False, extra_flags=(), out: str = LIB) -> str:
+    """Compile into ``out`` (default: the in-tree libmoe.so) unless it is up to date."""
+    if not force and out == LIB and not _stale():
         return LIB
-    objdir = os.path.join(ROOT, "_build")
+    objdir = os.path.join(ROOT, "_build", os.path.basename(os.path.dirname(os.path.abspath(out))))
     os.makedirs(objdir, exist_ok=True)
     objs = []
     flags = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
                     "-I", os.path.join(ROOT, "include")]
     if verbose_ptxas:
         flags += ["-Xptxas", "-v"]
+    flags += list(extra_flags)
     for src in SOURCES:
         obj = os.path.join(objdir, src.replace(".cu", ".o"))
         cmd = [nvcc()] + flags + ["-c", os.path.join(CSRC, src), "-o", obj]
         subprocess.run(cmd, check=True)
         objs.append(obj)
-    tmp = LIB + ".tmp"
+    tmp = out + ".tmp"
     subprocess.run([nvcc()] + ARCH + ["-shared", "-o", tmp] + objs, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

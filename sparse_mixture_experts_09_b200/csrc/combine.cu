@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ y,
                                                  const uint16_t* __restrict__ res,
                                                  uint16_t* __restrict__ out, int64_t T, int H,
                                                  int k) {
+  pdl_trigger();
+  pdl_wait();
   const int per_tok = H >> 3;
   const int64_t n = T * per_tok;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -77,8 +79,8 @@ cudaError_t launch_combine(const Shape& s, const float* y, const int32_t* row_of
   int64_t blocks = (n + 255) / 256;
   const int64_t cap = (int64_t)num_sms() * 8;
   if (blocks > cap) blocks = cap;
-  k_combine<<<(unsigned)blocks, 256, 0, st>>>(y, row_of, topk_w, residual, out, s.T, s.H, s.k);
-  return cudaGetLastError();
+  return launch_pdl(k_combine, dim3((unsigned)blocks), dim3(256), 0, st, y, row_of, topk_w, residual,
+                    out, s.T, s.H, s.k);
 }
 
 }  // namespace moe

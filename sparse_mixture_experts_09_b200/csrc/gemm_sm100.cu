@@ -250,7 +250,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_map(&mapB0);
     prefetch_map(&mapB1);
   }
-  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) row_tiles[i] = p.offsets[i] / BM;
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_holder)),
@@ -258,6 +257,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  // everything above is on-chip set-up; global inputs are read only after the
+  // previous kernel on the stream has completed
+  pdl_trigger();
+  pdl_wait();
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) row_tiles[i] = p.offsets[i] / BM;
   fence_before();
   __syncthreads();
   fence_after();
@@ -456,54 +460,68 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
   }
   int64_t grid = num_sms();
   if (grid > max_tiles) grid = max_tiles;
-  k_grouped_gemm<MODE, BN><<<(unsigned)grid, kThreads, smem, st>>>(a, b0, b1, p);
-  return cudaGetLastError();
+  return launch_pdl(k_grouped_gemm<MODE, BN>, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, st,
+                    a, b0, b1, p);
 }
 
 }  // namespace
 
-cudaError_t launch_grouped_swiglu(const Shape& s, const GemmArgs& g, cudaStream_t st,
-                                  const char** why) {
-  CUtensorMap mx, mw1, mw3, mh, mw2;
-  const uint64_t EI = (uint64_t)s.E * s.I, EH = (uint64_t)s.E * s.H;
+cudaError_t launch_gate_up(const Shape& s, const GemmArgs& g, cudaStream_t st, const char** why) {
+  CUtensorMap mx, mw1, mw3;
+  const uint64_t EI = (uint64_t)s.E * s.I;
   if (!make_map(&mx, g.a, s.H, g.rmax, 128) || !make_map(&mw1, g.w1, s.H, EI, 128) ||
-      !make_map(&mw3, g.w3, s.H, EI, 128) || !make_map(&mh, g.h, s.I, g.rmax, 128) ||
-      !make_map(&mw2, g.w2, s.I, EH, 128)) {
+      !make_map(&mw3, g.w3, s.H, EI, 128)) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad tensor)";
     return cudaErrorInvalidValue;
   }
-  const int64_t mt_max = g.rmax / BM;
-
-  KParams p1;
-  p1.offsets = g.offsets;
-  p1.status = g.status;
-  p1.out = g.h;
-  p1.out_ld = s.I;
-  p1.E = s.E;
-  p1.k_blocks = s.H / BK;
-  p1.n_tiles = s.I / 128;
-  p1.b_rows = s.I;
-  p1.timeout_ns = g.timeout_ns;
-  cudaError_t e = launch_one<kSwiGLU, 256>(mx, mw1, mw3, p1, mt_max * p1.n_tiles, st);
-  if (e != cudaSuccess) {
-    *why = "GEMM1 launch failed";
-    return e;
-  }
-
-  KParams p2 = p1;
-  p2.out = g.y;
-  p2.out_ld = s.H;
-  p2.k_blocks = s.I / BK;
-  p2.b_rows = s.H;
-  if (s.H % 256 == 0) {
-    p2.n_tiles = s.H / 256;
-    e = launch_one<kPlain, 256>(mh, mw2, mw2, p2, mt_max * p2.n_tiles, st);
-  } else {
-    p2.n_tiles = s.H / 128;
-    e = launch_one<kPlain, 128>(mh, mw2, mw2, p2, mt_max * p2.n_tiles, st);
-  }
-  if (e != cudaSuccess) *why = "GEMM2 launch failed";
+  KParams p;
+  p.offsets = g.offsets;
+  p.status = g.status;
+  p.out = g.h;
+  p.out_ld = s.I;
+  p.E = s.E;
+  p.k_blocks = s.H / BK;
+  p.n_tiles = s.I / 128;
+  p.b_rows = s.I;
+  p.timeout_ns = g.timeout_ns;
+  cudaError_t e = launch_one<kSwiGLU, 256>(mx, mw1, mw3, p, (g.rmax / BM) * p.n_tiles, st);
+  if (e != cudaSuccess) *why = "gate/up GEMM launch failed";
   return e;
+}
+
+cudaError_t launch_down(const Shape& s, const GemmArgs& g, cudaStream_t st, const char** why) {
+  CUtensorMap mh, mw2;
+  const uint64_t EH = (uint64_t)s.E * s.H;
+  if (!make_map(&mh, g.h, s.I, g.rmax, 128) || !make_map(&mw2, g.w2, s.I, EH, 128)) {
+    *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad tensor)";
+    return cudaErrorInvalidValue;
+  }
+  KParams p;
+  p.offsets = g.offsets;
+  p.status = g.status;
+  p.out = g.y;
+  p.out_ld = s.H;
+  p.E = s.E;
+  p.k_blocks = s.I / BK;
+  p.b_rows = s.H;
+  p.timeout_ns = g.timeout_ns;
+  cudaError_t e;
+  if (s.H % 256 == 0) {
+    p.n_tiles = s.H / 256;
+    e = launch_one<kPlain, 256>(mh, mw2, mw2, p, (g.rmax / BM) * p.n_tiles, st);
+  } else {
+    p.n_tiles = s.H / 128;
+    e = launch_one<kPlain, 128>(mh, mw2, mw2, p, (g.rmax / BM) * p.n_tiles, st);
+  }
+  if (e != cudaSuccess) *why = "down GEMM launch failed";
+  return e;
+}
+
+cudaError_t launch_grouped_swiglu(const Shape& s, const GemmArgs& g, cudaStream_t st,
+                                  const char** why) {
+  cudaError_t e = launch_gate_up(s, g, st, why);
+  if (e != cudaSuccess) return e;
+  return launch_down(s, g, st, why);
 }
 
 }  // namespace moe

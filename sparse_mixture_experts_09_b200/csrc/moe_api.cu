@@ -45,8 +45,8 @@ inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 // Workspace regions, in order; each starts on a 1024-byte boundary.
 struct Layout {
-  size_t status, topk_idx, topk_w, block_base, counts, offsets, row_of, token_of_row, x_perm, h, y,
-      end;
+  size_t status, topk_idx, topk_w, block_base, counts, offsets, row_of, token_of_row, x_perm, h,
+      y, end;
   size_t x_in, res_in, out_st, end_host;  // staging of moe_forward_host
 };
 
@@ -260,6 +260,59 @@ moe_status_t moe_grouped_swiglu(const moe_shape_t* shape, const moe_bf16_t* x_pe
   g.timeout_ns = kTimeoutNs;
   const char* why = "";
   cudaError_t e = launch_grouped_swiglu(s, g, (cudaStream_t)stream, &why);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, why);
+}
+
+moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* x_perm,
+                                const int32_t* expert_offsets, const moe_bf16_t* w1,
+                                const moe_bf16_t* w3, moe_bf16_t* h, void* ws, size_t ws_bytes,
+                                moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(x_perm, "x_perm"));
+  MOE_TRY(check_ptr(expert_offsets, "expert_offsets"));
+  MOE_TRY(check_ptr(w1, "w1"));
+  MOE_TRY(check_ptr(w3, "w3"));
+  MOE_TRY(check_ptr(h, "h"));
+  const Layout L = layout(s);
+  MOE_TRY(check_ws(ws, ws_bytes, L.end));
+  GemmArgs g = {};
+  g.a = x_perm;
+  g.offsets = expert_offsets;
+  g.w1 = w1;
+  g.w3 = w3;
+  g.h = h;
+  g.status = at<int32_t>(ws, 0);
+  g.rmax = max_padded_rows(s);
+  g.timeout_ns = kTimeoutNs;
+  const char* why = "";
+  cudaError_t e = launch_gate_up(s, g, (cudaStream_t)stream, &why);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, why);
+}
+
+moe_status_t moe_expert_down(const moe_shape_t* shape, const moe_bf16_t* h,
+                             const int32_t* expert_offsets, const moe_bf16_t* w2, float* y_perm,
+                             void* ws, size_t ws_bytes, moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(h, "h"));
+  MOE_TRY(check_ptr(expert_offsets, "expert_offsets"));
+  MOE_TRY(check_ptr(w2, "w2"));
+  MOE_TRY(check_ptr(y_perm, "y_perm"));
+  const Layout L = layout(s);
+  MOE_TRY(check_ws(ws, ws_bytes, L.end));
+  GemmArgs g = {};
+  g.offsets = expert_offsets;
+  g.w2 = w2;
+  g.h = const_cast<uint16_t*>(h);
+  g.y = y_perm;
+  g.status = at<int32_t>(ws, 0);
+  g.rmax = max_padded_rows(s);
+  g.timeout_ns = kTimeoutNs;
+  const char* why = "";
+  cudaError_t e = launch_down(s, g, (cudaStream_t)stream, &why);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, why);
 }
 

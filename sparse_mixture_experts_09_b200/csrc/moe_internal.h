@@ -11,6 +11,7 @@ namespace moe {
 constexpr int kTokensPerBlock = 32;
 constexpr int kRowPad = 128;
 
+
 // Device status word, first int32 of the workspace.
 constexpr int32_t kStatusTimeout = 1;
 
@@ -53,6 +54,8 @@ struct GemmArgs {
 };
 
 // GEMM1 (gate/up + SwiGLU -> h) then GEMM2 (h w2^T -> y), both persistent tcgen05.
+cudaError_t launch_gate_up(const Shape& s, const GemmArgs& g, cudaStream_t st, const char** why);
+cudaError_t launch_down(const Shape& s, const GemmArgs& g, cudaStream_t st, const char** why);
 cudaError_t launch_grouped_swiglu(const Shape& s, const GemmArgs& g, cudaStream_t st,
                                   const char** why);
 
@@ -61,5 +64,32 @@ cudaError_t launch_combine(const Shape& s, const float* y, const int32_t* row_of
                            cudaStream_t st);
 
 int num_sms();
+
+// ---- programmatic dependent launch ----
+// Every kernel of the layer is launched with programmatic stream serialization: it
+// may be scheduled while the previous kernel on the stream is still draining. Each
+// kernel lets its own dependents launch at entry (pdl_trigger) and, before it
+// touches global memory, waits until the previous grid has completed and its writes
+// are visible (pdl_wait). Only launch latency and on-chip prologue work overlap.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 }  // namespace moe

@@ -25,10 +25,14 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   return r;
 }
 
-// One warp per token. Each lane accumulates, in fp32 and in a fixed order, the dot
-// products of its 8-element slices of x[t] with every router row; a butterfly sum
-// gives every lane the E logits. Lane 0 then scores them.
-template <int EMAX>
+// Router and scoring. S warps cooperate on one token (S = 1, 2, 4 or 8; S > 1 when
+// there are too few tokens to keep the GPU busy): warp w of a token takes the w-th
+// of S equal slices of x[t] and of every router row. Each lane accumulates its
+// 8-element chunks in fp32 in a fixed order, a butterfly sum gives the warp's
+// partial logits, and one thread adds the S partials in warp order, adds the bias,
+// and scores: float32 softmax over all E, the k largest logits (ties to the lower
+// expert index, slot 0 the largest), weights renormalised to sum to one.
+template <int EMAX, int S>
 __global__ void __launch_bounds__(256) k_router(const uint16_t* __restrict__ x,
                                                 const uint16_t* __restrict__ wr,
                                                 const float* __restrict__ bias, int64_t T,
@@ -36,33 +40,52 @@ __global__ void __launch_bounds__(256) k_router(const uint16_t* __restrict__ x,
                                                 int32_t* __restrict__ idx_out,
                                                 float* __restrict__ w_out,
                                                 float* __restrict__ logits_out) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int chunks = H >> 3;
-  for (int64_t t = warp0; t < T; t += nwarps) {
+  pdl_trigger();
+  pdl_wait();
+  constexpr int TOK_PER_CTA = 8 / S;
+  __shared__ float part[8][EMAX];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int slot = warp / S, sub = warp % S;
+  const int per = (H >> 3) / S;  // 8-element chunks per warp; H % 128 == 0 keeps it whole
+  for (int64_t t0 = (int64_t)blockIdx.x * TOK_PER_CTA; t0 < T;
+       t0 += (int64_t)gridDim.x * TOK_PER_CTA) {
+    const int64_t t = t0 + slot;
     float acc[EMAX];
 #pragma unroll
     for (int e = 0; e < EMAX; ++e) acc[e] = 0.f;
-    const uint4* xr = reinterpret_cast<const uint4*>(x + t * H);
-    for (int c = lane; c < chunks; c += 32) {
-      const uint4 xv = ld_stream(xr + c);
-      const float x0 = bf16_lo(xv.x), x1 = bf16_hi(xv.x), x2 = bf16_lo(xv.y), x3 = bf16_hi(xv.y);
-      const float x4 = bf16_lo(xv.z), x5 = bf16_hi(xv.z), x6 = bf16_lo(xv.w), x7 = bf16_hi(xv.w);
+    if (t < T) {
+      const uint4* xr = reinterpret_cast<const uint4*>(x + t * H) + sub * per;
+      const uint4* wrow = reinterpret_cast<const uint4*>(wr) + sub * per;
+      const int rstride = H >> 3;
+      for (int c = lane; c < per; c += 32) {
+        const uint4 xv = ld_stream(xr + c);
+        const float x0 = bf16_lo(xv.x), x1 = bf16_hi(xv.x), x2 = bf16_lo(xv.y), x3 = bf16_hi(xv.y);
+        const float x4 = bf16_lo(xv.z), x5 = bf16_hi(xv.z), x6 = bf16_lo(xv.w), x7 = bf16_hi(xv.w);
+        // router rows in groups of 8: all loads of a group are issued before any use
+        // (rows past E read row E-1 and are discarded), so they overlap in flight
 #pragma unroll
-      for (int e = 0; e < EMAX; ++e) {
-        if (e < E) {
-          const uint4 wv = __ldg(reinterpret_cast<const uint4*>(wr + (size_t)e * H) + c);
-          float a = acc[e];
-          a = fmaf(x0, bf16_lo(wv.x), a);
-          a = fmaf(x1, bf16_hi(wv.x), a);
-          a = fmaf(x2, bf16_lo(wv.y), a);
-          a = fmaf(x3, bf16_hi(wv.y), a);
-          a = fmaf(x4, bf16_lo(wv.z), a);
-          a = fmaf(x5, bf16_hi(wv.z), a);
-          a = fmaf(x6, bf16_lo(wv.w), a);
-          a = fmaf(x7, bf16_hi(wv.w), a);
-          acc[e] = a;
+        for (int e0 = 0; e0 < EMAX; e0 += 8) {
+          if (e0 < E) {
+            uint4 wv[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int row = e0 + q < E ? e0 + q : E - 1;
+              wv[q] = __ldg(wrow + (size_t)row * rstride + c);
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              float a = acc[e0 + q];
+              a = fmaf(x0, bf16_lo(wv[q].x), a);
+              a = fmaf(x1, bf16_hi(wv[q].x), a);
+              a = fmaf(x2, bf16_lo(wv[q].y), a);
+              a = fmaf(x3, bf16_hi(wv[q].y), a);
+              a = fmaf(x4, bf16_lo(wv[q].z), a);
+              a = fmaf(x5, bf16_hi(wv[q].z), a);
+              a = fmaf(x6, bf16_lo(wv[q].w), a);
+              a = fmaf(x7, bf16_hi(wv[q].w), a);
+              acc[e0 + q] = a;
+            }
+          }
         }
       }
     }
@@ -71,53 +94,65 @@ __global__ void __launch_bounds__(256) k_router(const uint16_t* __restrict__ x,
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
     }
-    if (lane == 0) {
+    if (S > 1) {
+      if (lane == 0) {
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) part[warp][e] = acc[e];
+      }
+      __syncthreads();
+    }
+    if (sub == 0 && lane == 0 && t < T) {
       float l[EMAX], p[EMAX];
       float mx = -INFINITY;
 #pragma unroll
       for (int e = 0; e < EMAX; ++e) {
         if (e < E) {
-          l[e] = acc[e] + (bias ? bias[e] : 0.f);
+          float v = acc[e];
+          if (S > 1) {
+            v = part[slot * S][e];
+#pragma unroll
+            for (int w = 1; w < S; ++w) v += part[slot * S + w][e];
+          }
+          l[e] = v + (bias ? bias[e] : 0.f);
           mx = fmaxf(mx, l[e]);
           if (logits_out) logits_out[t * E + e] = l[e];
         }
       }
       // float32 softmax over all E experts
-      float s = 0.f;
+      float sum = 0.f;
 #pragma unroll
       for (int e = 0; e < EMAX; ++e)
-        if (e < E) { p[e] = expf(l[e] - mx); s += p[e]; }
+        if (e < E) { p[e] = expf(l[e] - mx); sum += p[e]; }
 #pragma unroll
       for (int e = 0; e < EMAX; ++e)
-        if (e < E) p[e] = p[e] / s;
+        if (e < E) p[e] = p[e] / sum;
       // the k largest, ranked on the float32 logit; equal logits -> lower index
       uint64_t taken = 0;
       int sel[8];
+      float psel[8];
       float psum = 0.f;
       for (int j = 0; j < k; ++j) {
         int best = -1;
-        float bl = 0.f;
+        float bl = 0.f, bp = 0.f;
 #pragma unroll
         for (int e = 0; e < EMAX; ++e) {
-          if (e < E && !((taken >> e) & 1ull) && (best < 0 || l[e] > bl)) { best = e; bl = l[e]; }
+          if (e < E && !((taken >> e) & 1ull) && (best < 0 || l[e] > bl)) {
+            best = e;
+            bl = l[e];
+            bp = p[e];
+          }
         }
         taken |= 1ull << best;
         sel[j] = best;
-        float pb = 0.f;
-#pragma unroll
-        for (int e = 0; e < EMAX; ++e)
-          if (e == best) pb = p[e];
-        psum += pb;
+        psel[j] = bp;
+        psum += bp;
       }
       for (int j = 0; j < k; ++j) {
-        float pb = 0.f;
-#pragma unroll
-        for (int e = 0; e < EMAX; ++e)
-          if (e == sel[j]) pb = p[e];
         idx_out[t * k + j] = sel[j];
-        w_out[t * k + j] = pb / psum;
+        w_out[t * k + j] = psel[j] / psum;
       }
     }
+    if (S > 1) __syncthreads();
   }
 }
 
@@ -132,6 +167,8 @@ __device__ __forceinline__ unsigned expert_lanes(const int* my, int k, bool vali
 __global__ void __launch_bounds__(256) k_block_hist(const int32_t* __restrict__ idx, int64_t T,
                                                     int E, int k, int64_t nb,
                                                     int32_t* __restrict__ block_counts) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t b = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (b >= nb) return;
@@ -151,6 +188,8 @@ __global__ void __launch_bounds__(256) k_block_hist(const int32_t* __restrict__ 
 __global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ block_base, int64_t nb,
                                                int E, int32_t* __restrict__ counts,
                                                int32_t* __restrict__ offsets) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int32_t s_count[64];
   __shared__ int32_t s_off[65];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
@@ -194,6 +233,8 @@ __global__ void __launch_bounds__(256) k_rank(const int32_t* __restrict__ idx, i
                                               const int32_t* __restrict__ block_base,
                                               int32_t* __restrict__ row_of,
                                               int32_t* __restrict__ token_of_row) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t b = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (b >= nb) return;
@@ -217,6 +258,75 @@ __global__ void __launch_bounds__(256) k_rank(const int32_t* __restrict__ idx, i
   }
 }
 
+// Histogram, scan and ranks in one CTA when there are at most 32 token blocks
+// (T <= 1024): warp b counts its block's slots per expert with ballots, one thread per
+// expert prefixes the block counts in order, thread 0 lays out the padded groups,
+// then every warp ranks its slots. Same results as k_block_hist + k_scan + k_rank.
+__global__ void __launch_bounds__(1024) k_plan_small(const int32_t* __restrict__ idx, int64_t T,
+                                                     int E, int k, int nb,
+                                                     int32_t* __restrict__ counts,
+                                                     int32_t* __restrict__ offsets,
+                                                     int32_t* __restrict__ row_of,
+                                                     int32_t* __restrict__ token_of_row) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int32_t s_base[32][64];
+  __shared__ int32_t s_tot[64];
+  __shared__ int32_t s_off[65];
+  const int b = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)b * kTokensPerBlock + lane;
+  const bool active = b < nb;
+  const bool valid = active && t < T;
+  int my[8];
+  for (int j = 0; j < k; ++j) my[j] = valid ? idx[t * k + j] : -1;
+  if (active) {
+    for (int e = 0; e < E; ++e) {
+      const unsigned bits = expert_lanes(my, k, valid, e);
+      if (lane == 0) s_base[b][e] = __popc(bits);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < E) {
+    const int e = threadIdx.x;
+    int32_t run = 0;
+    for (int bb = 0; bb < nb; ++bb) {
+      const int32_t v = s_base[bb][e];
+      s_base[bb][e] = run;
+      run += v;
+    }
+    s_tot[e] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t acc = 0;
+    for (int e = 0; e < E; ++e) {
+      s_off[e] = acc;
+      acc += (s_tot[e] + kRowPad - 1) / kRowPad * kRowPad;
+    }
+    s_off[E] = acc;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    offsets[e] = s_off[e];
+    if (e < E) counts[e] = s_tot[e];
+  }
+  if (active) {
+    const unsigned below = (1u << lane) - 1u;
+    for (int e = 0; e < E; ++e) {
+      const unsigned bits = expert_lanes(my, k, valid, e);
+      if (!bits) continue;
+      const int32_t base = s_off[e] + s_base[b][e];
+      for (int j = 0; j < k; ++j) {
+        if (valid && my[j] == e) {
+          const int32_t row = base + __popc(bits & below);
+          row_of[t * k + j] = row;
+          token_of_row[row] = (int32_t)t;
+        }
+      }
+    }
+  }
+}
+
 // One warp per row of x_perm below R_pad: copies x[token] or, on pad rows, writes
 // zeros and token -1.
 __global__ void __launch_bounds__(256) k_gather(const uint16_t* __restrict__ x, int H, int E,
@@ -224,6 +334,8 @@ __global__ void __launch_bounds__(256) k_gather(const uint16_t* __restrict__ x, 
                                                 const int32_t* __restrict__ offsets,
                                                 int32_t* __restrict__ token_of_row,
                                                 uint16_t* __restrict__ x_perm) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int32_t s_off[65], s_cnt[64];
   for (int e = threadIdx.x; e <= E; e += blockDim.x) {
     s_off[e] = offsets[e];
@@ -265,19 +377,32 @@ __global__ void __launch_bounds__(256) k_gather(const uint16_t* __restrict__ x, 
 cudaError_t launch_router(const Shape& s, const uint16_t* x, const uint16_t* w_router,
                           const float* logit_bias, int32_t* topk_idx, float* topk_w,
                           float* logits, cudaStream_t st) {
-  const int threads = 256;
-  int64_t blocks = (s.T + 7) / 8;
-  const int64_t cap = (int64_t)num_sms() * 16;
+  // enough warps to cover the GPU: split each token over S warps when T is small
+  const int64_t want_warps = (int64_t)num_sms() * 32;
+  int S = 1;
+  while (S < 8 && s.T * S < want_warps) S *= 2;
+  const int64_t tok_per_cta = 8 / S;
+  int64_t blocks = (s.T + tok_per_cta - 1) / tok_per_cta;
+  const int64_t cap = (int64_t)num_sms() * 8;
   if (blocks > cap) blocks = cap;
-#define MOE_ROUTER(EM)                                                                  \
-  k_router<EM><<<(unsigned)blocks, threads, 0, st>>>(x, w_router, logit_bias, s.T, s.H, \
-                                                     s.E, s.k, topk_idx, topk_w, logits)
-  if (s.E <= 8) MOE_ROUTER(8);
-  else if (s.E <= 16) MOE_ROUTER(16);
-  else if (s.E <= 32) MOE_ROUTER(32);
-  else MOE_ROUTER(64);
+  cudaError_t err = cudaSuccess;
+#define MOE_ROUTER(EM, SS)                                                                  \
+  err = launch_pdl(k_router<EM, SS>, dim3((unsigned)blocks), dim3(256), 0, st, x, w_router,   \
+                   logit_bias, s.T, s.H, s.E, s.k, topk_idx, topk_w, logits)
+#define MOE_ROUTER_E(EM)           \
+  switch (S) {                     \
+    case 1: MOE_ROUTER(EM, 1); break; \
+    case 2: MOE_ROUTER(EM, 2); break; \
+    case 4: MOE_ROUTER(EM, 4); break; \
+    default: MOE_ROUTER(EM, 8); break; \
+  }
+  if (s.E <= 8) { MOE_ROUTER_E(8) }
+  else if (s.E <= 16) { MOE_ROUTER_E(16) }
+  else if (s.E <= 32) { MOE_ROUTER_E(32) }
+  else { MOE_ROUTER_E(64) }
+#undef MOE_ROUTER_E
 #undef MOE_ROUTER
-  return cudaGetLastError();
+  return err;
 }
 
 cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16_t* x,
@@ -285,15 +410,28 @@ cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16
                            int32_t* token_of_row, uint16_t* x_perm, int32_t* block_base,
                            cudaStream_t st) {
   const int64_t nb = num_token_blocks(s);
-  const unsigned wblocks = (unsigned)((nb + 7) / 8);
-  k_block_hist<<<wblocks, 256, 0, st>>>(topk_idx, s.T, s.E, s.k, nb, block_base);
-  k_scan<<<1, 1024, 0, st>>>(block_base, nb, s.E, counts, offsets);
-  k_rank<<<wblocks, 256, 0, st>>>(topk_idx, s.T, s.E, s.k, nb, block_base, row_of, token_of_row);
+  cudaError_t e;
+  if (nb <= 32) {
+    const int threads = (int)(nb < 2 ? 2 : nb) * 32;
+    e = launch_pdl(k_plan_small, dim3(1), dim3(threads), 0, st, topk_idx, s.T, s.E, s.k, (int)nb,
+                   counts, offsets, row_of, token_of_row);
+    if (e != cudaSuccess) return e;
+  } else {
+    const unsigned wblocks = (unsigned)((nb + 7) / 8);
+    e = launch_pdl(k_block_hist, dim3(wblocks), dim3(256), 0, st, topk_idx, s.T, s.E, s.k, nb,
+                   block_base);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(k_scan, dim3(1), dim3(1024), 0, st, block_base, nb, s.E, counts, offsets);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(k_rank, dim3(wblocks), dim3(256), 0, st, topk_idx, s.T, s.E, s.k, nb, block_base,
+                   row_of, token_of_row);
+    if (e != cudaSuccess) return e;
+  }
   int64_t gblocks = (max_padded_rows(s) + 7) / 8;
   const int64_t cap = (int64_t)num_sms() * 8;
   if (gblocks > cap) gblocks = cap;
-  k_gather<<<(unsigned)gblocks, 256, 0, st>>>(x, s.H, s.E, counts, offsets, token_of_row, x_perm);
-  return cudaGetLastError();
+  return launch_pdl(k_gather, dim3((unsigned)gblocks), dim3(256), 0, st, x, s.H, s.E, counts,
+                    offsets, token_of_row, x_perm);
 }
 
 }  // namespace moe

@@ -14,14 +14,16 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoe.so")
+# MOE_LIB_PATH selects another build of the same library (it must exist)
+LIB_PATH = os.environ.get("MOE_LIB_PATH") or os.path.join(_HERE, "libmoe.so")
 ROW_PAD = 128
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
 
 EXPORTS = ("moe_workspace_size", "moe_workspace_size_host", "moe_max_padded_rows",
-           "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_forward",
+           "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_expert_gate_up",
+           "moe_expert_down", "moe_combine", "moe_forward",
            "moe_forward_host", "moe_device_status", "moe_last_error")
 
 
@@ -64,6 +66,10 @@ def lib() -> ctypes.CDLL:
         L.moe_permute.restype = st
         L.moe_grouped_swiglu.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
         L.moe_grouped_swiglu.restype = st
+        L.moe_expert_gate_up.argtypes = [sp, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.moe_expert_gate_up.restype = st
+        L.moe_expert_down.argtypes = [sp, _P, _P, _P, _P, _P, _SZ, _P]
+        L.moe_expert_down.restype = st
         L.moe_combine.argtypes = [sp, _P, _P, _P, _P, _P, _P]
         L.moe_combine.restype = st
         L.moe_forward.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
@@ -176,6 +182,33 @@ def grouped_swiglu(x_perm, offsets, w1, w3, w2, num_tokens: int, k: int, ws, str
                                     _dev(w1, "w1", torch.bfloat16), _dev(w3, "w3", torch.bfloat16),
                                     _dev(w2, "w2", torch.bfloat16), _dev(y, "y_perm"),
                                     _dev(ws, "ws"), ws.numel(), _stream(stream)))
+    return y
+
+
+def expert_gate_up(x_perm, offsets, w1, w3, num_tokens: int, k: int, ws, h=None, stream=None):
+    """h [R_max, I] bf16 = bf16(silu(x_perm w1[e]^T) * (x_perm w3[e]^T)) (GEMM1 alone)."""
+    e, i, hd = w1.shape
+    shape = make_shape(num_tokens, hd, i, e, k)
+    if h is None:
+        h = torch.zeros((max_padded_rows(shape), i), dtype=torch.bfloat16, device=x_perm.device)
+    _check(lib().moe_expert_gate_up(ctypes.byref(shape), _dev(x_perm, "x_perm", torch.bfloat16),
+                                    _dev(offsets, "offsets", torch.int32),
+                                    _dev(w1, "w1", torch.bfloat16), _dev(w3, "w3", torch.bfloat16),
+                                    _dev(h, "h", torch.bfloat16), _dev(ws, "ws"), ws.numel(),
+                                    _stream(stream)))
+    return h
+
+
+def expert_down(h, offsets, w2, num_tokens: int, k: int, ws, y=None, stream=None):
+    """y_perm [R_max, H] fp32 = h w2[e]^T (GEMM2 alone)."""
+    e, hd, i = w2.shape
+    shape = make_shape(num_tokens, hd, i, e, k)
+    if y is None:
+        y = torch.zeros((max_padded_rows(shape), hd), dtype=torch.float32, device=h.device)
+    _check(lib().moe_expert_down(ctypes.byref(shape), _dev(h, "h", torch.bfloat16),
+                                 _dev(offsets, "offsets", torch.int32), _dev(w2, "w2", torch.bfloat16),
+                                 _dev(y, "y_perm", torch.float32), _dev(ws, "ws"), ws.numel(),
+                                 _stream(stream)))
     return y
 
 
