@@ -118,6 +118,27 @@ moe_status_t moe_permute(const moe_shape_t* shape, const int32_t* topk_idx,
                          int32_t* token_of_row, moe_bf16_t* x_perm, void* ws,
                          size_t ws_bytes, moe_stream_t stream);
 
+/* Allocation-free moe_permute. The paper has no counterpart: this entry point exists
+ * for callers that cannot call cudaMalloc, and so cannot supply the workspace that
+ * moe_permute takes -- for example a plug-in whose host application owns every
+ * device allocation through its own pool, or a serving path that must not allocate
+ * once it is running. Arguments, results and checks are those of moe_permute
+ * without ws and ws_bytes.
+ * Its one piece of scratch, the per-block expert base table (ceil(num_tokens / 32)
+ * x num_experts int32, used only when num_tokens > 1024), lives in a 256 KiB static
+ * device array inside the library, which every GPU that loads the library holds
+ * until the process exits. Shapes needing more than 65536 entries return
+ * MOE_ERR_UNSUPPORTED. The first call on each device, made with that device
+ * current, looks up the array's device address (cudaGetSymbolAddress); make that
+ * first call before any stream capture. Every call shares the array: calls whose
+ * kernels overlap on the GPU race on it, so the caller must serialise them. A call
+ * writes every table entry it reads, so nothing needs clearing between calls. */
+moe_status_t moe_permute_static(const moe_shape_t* shape, const int32_t* topk_idx,
+                                const moe_bf16_t* x, int32_t* expert_counts,
+                                int32_t* expert_offsets, int32_t* row_of,
+                                int32_t* token_of_row, moe_bf16_t* x_perm,
+                                moe_stream_t stream);
+
 /* The experts (nnterp "Mixtral", "Values, by host": mlp_neurons = act(gate)*up is
  * what the down projection receives; act = silu per MixtralConfig hidden_act):
  * two persistent tcgen05 grouped GEMMs over the ragged expert groups.

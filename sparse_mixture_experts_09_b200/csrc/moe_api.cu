@@ -166,6 +166,11 @@ moe_status_t run_forward(const Shape& s, const uint16_t* x, const uint16_t* wr, 
 }
 
 }  // namespace
+
+int validate_shape(const moe_shape_t* shape, Shape* out) { return (int)check_shape(shape, out); }
+
+void set_error_message(const char* msg) { snprintf(g_err, sizeof g_err, "%s", msg); }
+
 }  // namespace moe
 
 using namespace moe;

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/moe.h"
+
 namespace moe {
 
 // Routed (token, slot) pairs handled by one CTA of the histogram / scatter kernels:
@@ -64,6 +66,11 @@ cudaError_t launch_combine(const Shape& s, const float* y, const int32_t* row_of
                            cudaStream_t st);
 
 int num_sms();
+
+// Host helpers of the C ABI (moe_api.cu): shape validation returning a moe_status_t
+// (message in moe_last_error), and setting the thread's moe_last_error message.
+int validate_shape(const moe_shape_t* shape, Shape* out);
+void set_error_message(const char* msg);
 
 // ---- programmatic dependent launch ----
 // Every kernel of the layer is launched with programmatic stream serialization: it

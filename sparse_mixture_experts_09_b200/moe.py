@@ -24,7 +24,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
 EXPORTS = ("moe_workspace_size", "moe_workspace_size_host", "moe_max_padded_rows",
            "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_expert_gate_up",
            "moe_expert_down", "moe_combine", "moe_forward",
-           "moe_forward_host", "moe_device_status", "moe_last_error")
+           "moe_forward_host", "moe_device_status", "moe_last_error", "moe_permute_static")
 
 
 class MoeError(RuntimeError):
@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_host.restype = st
         L.moe_device_status.argtypes = [_P, _SZ, _P]
         L.moe_device_status.restype = st
+        L.moe_permute_static.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P]
+        L.moe_permute_static.restype = st
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         _lib = L
@@ -169,6 +171,30 @@ def permute(topk_idx, x, num_experts: int, intermediate_size: int, ws, stream=No
                              _dev(out["offsets"], "offsets"), _dev(out["row_of"], "row_of"),
                              _dev(out["token_of_row"], "token_of_row"), _dev(out["x_perm"], "x_perm"),
                              _dev(ws, "ws"), ws.numel(), _stream(stream)))
+    return out
+
+
+def permute_static(topk_idx, x, num_experts: int, intermediate_size: int, stream=None) -> dict:
+    """moe_permute_static: the permutation without a workspace, for callers that cannot
+    allocate device memory (its scratch is a static array in the library; calls that
+    overlap on the GPU race on it). Same results as ``permute``."""
+    t, k = topk_idx.shape
+    h = x.shape[1]
+    shape = make_shape(t, h, intermediate_size, num_experts, k)
+    rmax = max_padded_rows(shape)
+    dev = x.device
+    out = {
+        "counts": torch.empty(num_experts, dtype=torch.int32, device=dev),
+        "offsets": torch.empty(num_experts + 1, dtype=torch.int32, device=dev),
+        "row_of": torch.empty((t, k), dtype=torch.int32, device=dev),
+        "token_of_row": torch.full((rmax,), -2, dtype=torch.int32, device=dev),
+        "x_perm": torch.zeros((rmax, h), dtype=torch.bfloat16, device=dev),
+    }
+    _check(lib().moe_permute_static(ctypes.byref(shape), _dev(topk_idx, "topk_idx", torch.int32),
+                                    _dev(x, "x", torch.bfloat16), _dev(out["counts"], "counts"),
+                                    _dev(out["offsets"], "offsets"), _dev(out["row_of"], "row_of"),
+                                    _dev(out["token_of_row"], "token_of_row"),
+                                    _dev(out["x_perm"], "x_perm"), _stream(stream)))
     return out
 
 
