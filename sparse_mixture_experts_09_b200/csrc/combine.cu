@@ -21,6 +21,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
 
 // One thread per 8 consecutive outputs of a token: reads k rows of y (32 B each)
 // and 16 B of residual, writes 16 B.
+template <int KMAX>
 __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ y,
                                                  const int32_t* __restrict__ row_of,
                                                  const float* __restrict__ w,
@@ -38,22 +39,42 @@ __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ y,
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int64_t r = row_of[t * k + j];
-      const float wj = w[t * k + j];
-      const float4* yp = reinterpret_cast<const float4*>(y + r * H + c);
-      const float4 a = __ldg(yp), b = __ldg(yp + 1);
-      acc[0] = fmaf(wj, a.x, acc[0]);
-      acc[1] = fmaf(wj, a.y, acc[1]);
-      acc[2] = fmaf(wj, a.z, acc[2]);
-      acc[3] = fmaf(wj, a.w, acc[3]);
-      acc[4] = fmaf(wj, b.x, acc[4]);
-      acc[5] = fmaf(wj, b.y, acc[5]);
-      acc[6] = fmaf(wj, b.z, acc[6]);
-      acc[7] = fmaf(wj, b.w, acc[7]);
+    // all rows' loads are issued before the first multiply-add; slots are then
+    // accumulated in order
+    int64_t r[KMAX];
+    float wj[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j < k) {
+        r[j] = row_of[t * k + j];
+        wj[j] = w[t * k + j];
+      }
+    }
+    float4 ya[KMAX], yb[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j < k) {
+        const float4* yp = reinterpret_cast<const float4*>(y + r[j] * H + c);
+        ya[j] = __ldg(yp);
+        yb[j] = __ldg(yp + 1);
+      }
+    }
+    uint4 rv = make_uint4(0, 0, 0, 0);
+    if (res) rv = __ldg(reinterpret_cast<const uint4*>(res + t * H + c));
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j < k) {
+        acc[0] = fmaf(wj[j], ya[j].x, acc[0]);
+        acc[1] = fmaf(wj[j], ya[j].y, acc[1]);
+        acc[2] = fmaf(wj[j], ya[j].z, acc[2]);
+        acc[3] = fmaf(wj[j], ya[j].w, acc[3]);
+        acc[4] = fmaf(wj[j], yb[j].x, acc[4]);
+        acc[5] = fmaf(wj[j], yb[j].y, acc[5]);
+        acc[6] = fmaf(wj[j], yb[j].z, acc[6]);
+        acc[7] = fmaf(wj[j], yb[j].w, acc[7]);
+      }
     }
     if (res) {
-      const uint4 rv = __ldg(reinterpret_cast<const uint4*>(res + t * H + c));
       const uint32_t rr[4] = {rv.x, rv.y, rv.z, rv.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -77,10 +98,16 @@ cudaError_t launch_combine(const Shape& s, const float* y, const int32_t* row_of
                            cudaStream_t st) {
   const int64_t n = s.T * (s.H / 8);
   int64_t blocks = (n + 255) / 256;
-  const int64_t cap = (int64_t)num_sms() * 8;
+  const int64_t cap = (int64_t)num_sms() * 32;
   if (blocks > cap) blocks = cap;
-  return launch_pdl(k_combine, dim3((unsigned)blocks), dim3(256), 0, st, y, row_of, topk_w, residual,
-                    out, s.T, s.H, s.k);
+  if (s.k <= 2)
+    return launch_pdl(k_combine<2>, dim3((unsigned)blocks), dim3(256), 0, st, y, row_of, topk_w,
+                      residual, out, s.T, s.H, s.k);
+  if (s.k <= 4)
+    return launch_pdl(k_combine<4>, dim3((unsigned)blocks), dim3(256), 0, st, y, row_of, topk_w,
+                      residual, out, s.T, s.H, s.k);
+  return launch_pdl(k_combine<8>, dim3((unsigned)blocks), dim3(256), 0, st, y, row_of, topk_w,
+                    residual, out, s.T, s.H, s.k);
 }
 
 }  // namespace moe

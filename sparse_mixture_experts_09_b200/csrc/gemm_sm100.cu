@@ -209,11 +209,47 @@ __device__ __forceinline__ void tile_coords(int L, const int* row_tiles, int E, 
   m = row_tiles[e] + local % cnt;
 }
 
+// Work items. Whole waves of tiles run at full width (item = tile, round-robin over
+// the CTAs). When the tiles left over for the last wave would fill at most half of the
+// CTAs, each of them is cut into `split` (2 or 4) pieces along N, so the last wave is
+// shorter by that factor and more CTAs share it.
+struct Work {
+  int full_items, split, items;
+  __device__ void init(int total_tiles, int grid) {
+    full_items = (total_tiles / grid) * grid;
+    const int rest = total_tiles - full_items;
+    split = 1;
+    if (rest > 0) {
+      if (4 * rest <= grid) split = 4;
+      else if (2 * rest <= grid) split = 2;
+    }
+    items = full_items + split * rest;
+  }
+  // item -> (tile, piece, pieces)
+  __device__ void get(int item, int& tile, int& piece, int& pieces) const {
+    if (item < full_items) {
+      tile = item;
+      piece = 0;
+      pieces = 1;
+    } else {
+      const int j = item - full_items;
+      tile = full_items + j / split;
+      piece = j % split;
+      pieces = split;
+    }
+  }
+};
+
 template <int MODE, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
-                   const __grid_constant__ CUtensorMap mapB1, const KParams p) {
+                   const __grid_constant__ CUtensorMap mapB1,
+                   const __grid_constant__ CUtensorMap mapB0s,
+                   const __grid_constant__ CUtensorMap mapB1s, const KParams p) {
   using C = Tile<BN>;
+  // B rows of one weight matrix in a full tile: 128 w1 and 128 w3 rows (gate/up),
+  // or BN w2 rows (down)
+  constexpr int ROWS = (MODE == kSwiGLU) ? 128 : BN;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -249,6 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_map(&mapA);
     prefetch_map(&mapB0);
     prefetch_map(&mapB1);
+    prefetch_map(&mapB0s);
+    prefetch_map(&mapB1s);
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -266,25 +304,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int total = row_tiles[p.E] * p.n_tiles;
+  Work work;
+  work.init(row_tiles[p.E] * p.n_tiles, gridDim.x);
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer
       int it = 0;
       bool ok = true;
-      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-        int e, m, n;
-        tile_coords(L, row_tiles, p.E, p.n_tiles, e, m, n);
+      for (int w = blockIdx.x; w < work.items && ok; w += gridDim.x) {
+        int tile, piece, pieces, e, m, n;
+        work.get(w, tile, piece, pieces);
+        tile_coords(tile, row_tiles, p.E, p.n_tiles, e, m, n);
         const int a_row = m * BM;
-        int b_row0, b_row1;
-        if (MODE == kSwiGLU) {
-          b_row0 = e * p.b_rows + n * 128;
-          b_row1 = b_row0;
-        } else {
-          b_row0 = e * p.b_rows + n * BN;
-          b_row1 = b_row0 + 128;
-        }
+        const int rp = ROWS / pieces;  // B rows per weight matrix in this item
+        const int b_row = e * p.b_rows + n * ROWS + piece * rp;
+        const uint32_t bytes = C::A_BYTES + (MODE == kSwiGLU ? 2 : 1) * rp * BK * 2;
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
@@ -293,10 +328,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
-          mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+          mbar_expect_tx(full_bar(s), bytes);
           tma_load_2d(sa, &mapA, kb * BK, a_row, full_bar(s));
-          tma_load_2d(sa + C::A_BYTES, &mapB0, kb * BK, b_row0, full_bar(s));
-          if (BN == 256) tma_load_2d(sa + C::A_BYTES + 128 * BK * 2, &mapB1, kb * BK, b_row1, full_bar(s));
+          if (pieces == 1) {
+            if (MODE == kSwiGLU) {
+              tma_load_2d(sb, &mapB0, kb * BK, b_row, full_bar(s));
+              tma_load_2d(sb + 128 * BK * 2, &mapB1, kb * BK, b_row, full_bar(s));
+            } else {
+              tma_load_2d(sb, &mapB0, kb * BK, b_row, full_bar(s));
+              if (BN == 256) tma_load_2d(sb + 128 * BK * 2, &mapB0, kb * BK, b_row + 128, full_bar(s));
+            }
+          } else {
+            // 32-row boxes; gate (or down) rows first, then the up rows
+            for (int j = 0; j < rp; j += 32)
+              tma_load_2d(sb + j * BK * 2, &mapB0s, kb * BK, b_row + j, full_bar(s));
+            if (MODE == kSwiGLU)
+              for (int j = 0; j < rp; j += 32)
+                tma_load_2d(sb + (rp + j) * BK * 2, &mapB1s, kb * BK, b_row + j, full_bar(s));
+          }
         }
       }
       if (!ok) {
@@ -312,7 +362,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------- MMA issuer
       int it = 0, tc = 0;
       bool ok = true, issued = false;
-      for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tc) {
+      for (int w = blockIdx.x; w < work.items && ok; w += gridDim.x, ++tc) {
+        int tile, piece, pieces;
+        work.get(w, tile, piece, pieces);
+        const uint32_t nmma = (uint32_t)((MODE == kSwiGLU ? 2 : 1) * (ROWS / pieces));
+        const uint32_t idesc = (C::IDESC & ~(0x3Fu << 17)) | ((nmma >> 3) << 17);
         const int a = tc & 1;
         const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
         if (!wait_phase(tempty_bar(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
@@ -330,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sb = sa + C::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            mma_bf16(d, sdesc(sa + kk * 32), sdesc(sb + kk * 32), C::IDESC, (kb | kk) ? 1u : 0u);
+            mma_bf16(d, sdesc(sa + kk * 32), sdesc(sb + kk * 32), idesc, (kb | kk) ? 1u : 0u);
           }
           mma_commit(empty_bar(s));
           issued = true;
@@ -349,9 +403,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int row_in_tile = q * 32 + lane;
     int tc = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x, ++tc) {
-      int e, m, n;
-      tile_coords(L, row_tiles, p.E, p.n_tiles, e, m, n);
+    for (int w = blockIdx.x; w < work.items; w += gridDim.x, ++tc) {
+      int tile, piece, pieces, e, m, n;
+      work.get(w, tile, piece, pieces);
+      tile_coords(tile, row_tiles, p.E, p.n_tiles, e, m, n);
+      const int rp = ROWS / pieces;  // output columns of this item
       const int a = tc & 1;
       const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
       int ok = 0;
@@ -361,13 +417,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * BN);
       const int64_t row = (int64_t)m * BM + row_in_tile;
+      const int64_t col0 = (int64_t)n * ROWS + (int64_t)piece * rp;
       if (MODE == kSwiGLU) {
-        uint16_t* h = reinterpret_cast<uint16_t*>(p.out) + row * p.out_ld + (int64_t)n * 128;
+        uint16_t* h = reinterpret_cast<uint16_t*>(p.out) + row * p.out_ld + col0;
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 16) {
+        for (int c = 0; c < rp; c += 16) {
           uint32_t g[16], u[16];
           tmem_ld16(taddr + c, g);
-          tmem_ld16(taddr + 128 + c, u);
+          tmem_ld16(taddr + rp + c, u);
           tmem_wait_ld();
           uint32_t pk[8];
 #pragma unroll
@@ -383,9 +440,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       } else {
-        float* y = reinterpret_cast<float*>(p.out) + row * p.out_ld + (int64_t)n * BN;
+        float* y = reinterpret_cast<float*>(p.out) + row * p.out_ld + col0;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
+        for (int c = 0; c < rp; c += 16) {
           uint32_t v[16];
           tmem_ld16(taddr + c, v);
           tmem_wait_ld();
@@ -447,7 +504,8 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
 
 template <int MODE, int BN>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                       const KParams& p, int64_t max_tiles, cudaStream_t st) {
+                       const CUtensorMap& b0s, const CUtensorMap& b1s, const KParams& p,
+                       int64_t max_tiles, cudaStream_t st) {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -461,16 +519,17 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
   int64_t grid = num_sms();
   if (grid > max_tiles) grid = max_tiles;
   return launch_pdl(k_grouped_gemm<MODE, BN>, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, st,
-                    a, b0, b1, p);
+                    a, b0, b1, b0s, b1s, p);
 }
 
 }  // namespace
 
 cudaError_t launch_gate_up(const Shape& s, const GemmArgs& g, cudaStream_t st, const char** why) {
-  CUtensorMap mx, mw1, mw3;
+  CUtensorMap mx, mw1, mw3, mw1s, mw3s;
   const uint64_t EI = (uint64_t)s.E * s.I;
   if (!make_map(&mx, g.a, s.H, g.rmax, 128) || !make_map(&mw1, g.w1, s.H, EI, 128) ||
-      !make_map(&mw3, g.w3, s.H, EI, 128)) {
+      !make_map(&mw3, g.w3, s.H, EI, 128) || !make_map(&mw1s, g.w1, s.H, EI, 32) ||
+      !make_map(&mw3s, g.w3, s.H, EI, 32)) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad tensor)";
     return cudaErrorInvalidValue;
   }
@@ -484,15 +543,17 @@ cudaError_t launch_gate_up(const Shape& s, const GemmArgs& g, cudaStream_t st, c
   p.n_tiles = s.I / 128;
   p.b_rows = s.I;
   p.timeout_ns = g.timeout_ns;
-  cudaError_t e = launch_one<kSwiGLU, 256>(mx, mw1, mw3, p, (g.rmax / BM) * p.n_tiles, st);
+  cudaError_t e =
+      launch_one<kSwiGLU, 256>(mx, mw1, mw3, mw1s, mw3s, p, (g.rmax / BM) * p.n_tiles, st);
   if (e != cudaSuccess) *why = "gate/up GEMM launch failed";
   return e;
 }
 
 cudaError_t launch_down(const Shape& s, const GemmArgs& g, cudaStream_t st, const char** why) {
-  CUtensorMap mh, mw2;
+  CUtensorMap mh, mw2, mw2s;
   const uint64_t EH = (uint64_t)s.E * s.H;
-  if (!make_map(&mh, g.h, s.I, g.rmax, 128) || !make_map(&mw2, g.w2, s.I, EH, 128)) {
+  if (!make_map(&mh, g.h, s.I, g.rmax, 128) || !make_map(&mw2, g.w2, s.I, EH, 128) ||
+      !make_map(&mw2s, g.w2, s.I, EH, 32)) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad tensor)";
     return cudaErrorInvalidValue;
   }
@@ -508,10 +569,10 @@ cudaError_t launch_down(const Shape& s, const GemmArgs& g, cudaStream_t st, cons
   cudaError_t e;
   if (s.H % 256 == 0) {
     p.n_tiles = s.H / 256;
-    e = launch_one<kPlain, 256>(mh, mw2, mw2, p, (g.rmax / BM) * p.n_tiles, st);
+    e = launch_one<kPlain, 256>(mh, mw2, mw2, mw2s, mw2s, p, (g.rmax / BM) * p.n_tiles, st);
   } else {
     p.n_tiles = s.H / 128;
-    e = launch_one<kPlain, 128>(mh, mw2, mw2, p, (g.rmax / BM) * p.n_tiles, st);
+    e = launch_one<kPlain, 128>(mh, mw2, mw2, mw2s, mw2s, p, (g.rmax / BM) * p.n_tiles, st);
   }
   if (e != cudaSuccess) *why = "down GEMM launch failed";
   return e;

@@ -57,12 +57,12 @@ __global__ void __launch_bounds__(256) k_router(const uint16_t* __restrict__ x,
       const uint4* xr = reinterpret_cast<const uint4*>(x + t * H) + sub * per;
       const uint4* wrow = reinterpret_cast<const uint4*>(wr) + sub * per;
       const int rstride = H >> 3;
+      // router rows in groups of 8: all loads of a group are issued before any use
+      // (rows past E read row E-1 and are discarded), so they overlap in flight
       for (int c = lane; c < per; c += 32) {
         const uint4 xv = ld_stream(xr + c);
         const float x0 = bf16_lo(xv.x), x1 = bf16_hi(xv.x), x2 = bf16_lo(xv.y), x3 = bf16_hi(xv.y);
         const float x4 = bf16_lo(xv.z), x5 = bf16_hi(xv.z), x6 = bf16_lo(xv.w), x7 = bf16_hi(xv.w);
-        // router rows in groups of 8: all loads of a group are issued before any use
-        // (rows past E read row E-1 and are discarded), so they overlap in flight
 #pragma unroll
         for (int e0 = 0; e0 < EMAX; e0 += 8) {
           if (e0 < E) {

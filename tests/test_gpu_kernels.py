@@ -26,6 +26,9 @@ SMALL = {
     # tiles per expert with more than five waves of tiles (k32_waves)
     "k16": W.Workload("k16", 300, 1024, 1024, 8, 2, seed=17),
     "k32_waves": W.Workload("k32_waves", 3000, 1024, 2048, 8, 2, seed=18),
+    # hidden 640: the down GEMM uses 128-column tiles, and its last wave is cut
+    # into 32-column pieces
+    "bn128_split": W.Workload("bn128_split", 4000, 640, 512, 8, 2, seed=19),
 }
 
 
