@@ -36,7 +36,10 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;        // bf16 elements per 128-byte swizzled row
 constexpr int kThreads = 192;
-constexpr int kStages = 4;
+#ifndef MOE_GEMM_STAGES
+#define MOE_GEMM_STAGES 4
+#endif
+constexpr int kStages = MOE_GEMM_STAGES;
 constexpr int kSwiGLU = 0;
 constexpr int kPlain = 1;
 
