@@ -257,6 +257,22 @@ def ncu_traffic(workload, kernel):
     return None
 
 
+def slowest_rank(ms, e2e_ms, world, device):
+    """Per-step times of the slowest rank (max over ranks; identity for one rank)."""
+    if world == 1:
+        return ms, e2e_ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t[0]), float(t[1])
+
+
+def job_throughput(tokens_per_rank, world, ms):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's step time."""
+    return tokens_per_rank * world / (ms * 1e-3)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -393,10 +409,7 @@ def run_ours(args):
     moe.device_status(ws)
     moe.device_status(wsh)
 
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
+    ms, e2e_ms = slowest_rank(ms, e2e_ms, world, dev)
 
     counts = perm["counts"].cpu().tolist()
     peaks, peak_kind = load_peaks()
@@ -405,10 +418,9 @@ def run_ours(args):
 
     line = None
     if rank == 0:
-        tokens_all = w.num_tokens * world
         bytes_io = w.num_tokens * w.hidden_size * 2
         line = {
-            "metric": METRIC, "value": tokens_all / (ms * 1e-3), "unit": "tokens/s",
+            "metric": METRIC, "value": job_throughput(w.num_tokens, world, ms), "unit": "tokens/s",
             "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic: seeded SplitMix64/Box-Muller draws, weights ~N(0,1/fan_in), x rows RMS 1",
@@ -417,7 +429,7 @@ def run_ours(args):
                                "the 126 MB L2" % (roof["active_experts"] * w.expert_bytes() / 1e9))),
             "roofline": roof,
             "kernels_ms": stage_ms,
-            "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": job_throughput(w.num_tokens, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": 2 * bytes_io, "d2h_bytes_per_step": bytes_io,
                     "api": "moe_forward_host"},
             "gpu_launches": KERNELS_PER_FORWARD * K,

@@ -202,6 +202,14 @@ moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_bf16_t* x_host
  * call. */
 moe_status_t moe_device_status(void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Diagnostic of the failure path: launches one thread that waits, with the same
+ * bounded wait the GEMM kernels use, on a barrier phase that nothing completes. After
+ * timeout_ns (0 < timeout_ns <= 10 s) the wait gives up and records MOE_ERR_TIMEOUT
+ * in the status word of `ws` (ws_bytes >= 256), which moe_device_status() then
+ * reports; the context stays usable. Returns after the launch. */
+moe_status_t moe_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t timeout_ns,
+                                       moe_stream_t stream);
+
 /* Thread-local description of the last failure on this thread ("" if none). */
 const char* moe_last_error(void);
 

@@ -392,6 +392,16 @@ moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_bf16_t* x_host
   return MOE_OK;
 }
 
+moe_status_t moe_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t timeout_ns,
+                                       moe_stream_t stream) {
+  g_err[0] = 0;
+  MOE_TRY(check_ws(ws, ws_bytes, 256));
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull)
+    return fail(MOE_ERR_INVALID_ARG, "timeout_ns must be in (0, 10 s]");
+  cudaError_t e = launch_wait_selftest(at<int32_t>(ws, 0), timeout_ns, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "self-test launch");
+}
+
 moe_status_t moe_device_status(void* ws, size_t ws_bytes, moe_stream_t stream) {
   g_err[0] = 0;
   if (!ws || ws_bytes < 256) return fail(MOE_ERR_WORKSPACE, "workspace is NULL or too small");

@@ -61,6 +61,9 @@ cudaError_t launch_down(const Shape& s, const GemmArgs& g, cudaStream_t st, cons
 cudaError_t launch_grouped_swiglu(const Shape& s, const GemmArgs& g, cudaStream_t st,
                                   const char** why);
 
+// One thread's bounded wait on a barrier nothing arrives on (checks timeout reporting).
+cudaError_t launch_wait_selftest(int32_t* status, unsigned long long timeout_ns, cudaStream_t st);
+
 cudaError_t launch_combine(const Shape& s, const float* y, const int32_t* row_of,
                            const float* topk_w, const uint16_t* residual, uint16_t* out,
                            cudaStream_t st);

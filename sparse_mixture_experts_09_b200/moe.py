@@ -24,7 +24,8 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
 EXPORTS = ("moe_workspace_size", "moe_workspace_size_host", "moe_max_padded_rows",
            "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_expert_gate_up",
            "moe_expert_down", "moe_combine", "moe_forward",
-           "moe_forward_host", "moe_device_status", "moe_last_error", "moe_permute_static")
+           "moe_forward_host", "moe_device_status", "moe_last_error", "moe_permute_static",
+           "moe_selftest_wait_timeout")
 
 
 class MoeError(RuntimeError):
@@ -80,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.moe_device_status.restype = st
         L.moe_permute_static.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P]
         L.moe_permute_static.restype = st
+        L.moe_selftest_wait_timeout.argtypes = [_P, _SZ, ctypes.c_uint64, _P]
+        L.moe_selftest_wait_timeout.restype = st
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         _lib = L
@@ -293,6 +296,12 @@ def forward_host(x_host, w_router, w1, w3, w2, k: int, residual_host=None, logit
                                   None if residual_host is None else residual_host.data_ptr(),
                                   out_host.data_ptr(), _dev(ws, "ws"), ws.numel(), _stream(stream)))
     return out_host
+
+
+def selftest_wait_timeout(ws, timeout_ns: int, stream=None) -> None:
+    """Launch the bounded-wait check: a wait that nothing completes gives up after
+    ``timeout_ns`` and records MOE_ERR_TIMEOUT in ``ws``'s status word."""
+    _check(lib().moe_selftest_wait_timeout(_dev(ws, "ws"), ws.numel(), int(timeout_ns), _stream(stream)))
 
 
 def device_status(ws, stream=None) -> None:

@@ -29,6 +29,9 @@ SMALL = {
     # hidden 640: the down GEMM uses 128-column tiles, and its last wave is cut
     # into 32-column pieces
     "bn128_split": W.Workload("bn128_split", 4000, 640, 512, 8, 2, seed=19),
+    # at least 1024 routed rows per expert: the down GEMM runs on CTA pairs
+    # (tcgen05 cta_group::2), experts with odd and even row-tile counts
+    "pair_down": W.Workload("pair_down", 4500, 512, 512, 8, 2, seed=20),
 }
 
 
