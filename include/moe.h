@@ -186,6 +186,21 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_bf16_t* x,
                          moe_bf16_t* out, void* ws, size_t ws_bytes,
                          moe_stream_t stream);
 
+/* The mixture half of the decoder block (nnterp "Mixtral", "The block, in order":
+ * out = h + mlp(post_attention_layernorm(h)); the norm is MixtralRMSNorm with
+ * rms_norm_eps, 1e-5 on every checkpoint):
+ *   xn[t]  = bf16( (h[t] * r[t]) * norm_weight ),  r[t] = 1 / sqrt(mean(h[t]^2) + eps),
+ *   out[t] = bf16( h[t] + sum_j w[t,j] * y[t,j](xn) ).
+ * The norm is fused into the router (which computes r, fp32) and the gather (which
+ * writes the normed rows); h is also the residual. norm_weight [H] bf16;
+ * 0 <= eps <= 1. */
+moe_status_t moe_forward_rmsnorm(const moe_shape_t* shape, const moe_bf16_t* h,
+                                 const moe_bf16_t* norm_weight, float eps,
+                                 const moe_bf16_t* w_router, const float* logit_bias,
+                                 const moe_bf16_t* w1, const moe_bf16_t* w3,
+                                 const moe_bf16_t* w2, moe_bf16_t* out, void* ws,
+                                 size_t ws_bytes, moe_stream_t stream);
+
 /* moe_forward with HOST activations: copies x_host (and residual_host, nullable)
  * into the workspace, runs the layer, copies out back into out_host, and waits for
  * the stream. Host buffers should be pinned for asynchronous copies. Weights and

@@ -45,7 +45,7 @@ import numpy as np
 
 __all__ = [
     "to_f64", "round_bf16", "silu", "router_logits", "route_topk", "stable_permute",
-    "swiglu_expert", "moe_layer",
+    "swiglu_expert", "moe_layer", "rms_norm", "moe_block",
 ]
 
 
@@ -193,3 +193,35 @@ def moe_layer(x, w_router, w1, w3, w2, k: int, residual=None, logit_bias=None,
         out = round_bf16(out)
     return {"logits": logits, "idx": idx, "weights": weights, "y": y,
             "expert_outputs": expert_outputs, "routed": routed, "out": out}
+
+
+def rms_norm(h, weight, eps: float) -> np.ndarray:
+    """RMSNorm of each row: h / sqrt(mean(h^2) + eps) * weight, in fp64.
+
+    The block norms the residual stream before the mixture (nnterp "Mixtral", "The
+    block, in order": out = h + mlp(post_attention_layernorm(h)); Printout:
+    MixtralRMSNorm((4096,), eps=1e-05); Config: rms_norm_eps 1e-05). The pages name the
+    norm and its epsilon but do not write it out; this is the standard root-mean-square
+    layer norm with a learned per-channel gain and no bias, eps inside the root.
+    """
+    h = to_f64(h)
+    ms = (h * h).mean(axis=1, keepdims=True)
+    return h / np.sqrt(ms + eps) * to_f64(weight)[None, :]
+
+
+def moe_block(h, norm_weight, eps: float, w_router, w1, w3, w2, k: int, logit_bias=None,
+              mode: str = "exact", tokens=None) -> dict:
+    """The mixture half of the decoder block: out = h + moe(rms_norm(h)).
+
+    In ``bf16_storage`` mode the normed activations are rounded to bf16 (they are the
+    mixture's bf16 input in a bf16 load) and the output is rounded once.
+    """
+    hs = to_f64(h)
+    if tokens is not None:
+        hs = hs[np.asarray(tokens, dtype=np.int64)]
+    x = rms_norm(hs, norm_weight, eps)
+    if mode == "bf16_storage":
+        x = round_bf16(x)
+    r = moe_layer(x, w_router, w1, w3, w2, k, residual=hs, logit_bias=logit_bias, mode=mode)
+    r["x_norm"] = x
+    return r

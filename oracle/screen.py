@@ -29,21 +29,23 @@ def min_gap(logits: np.ndarray, k: int) -> np.ndarray:
 
 
 def screen_margin(x: torch.Tensor, w_router, logit_bias, k: int, redraw,
-                  margin: float = 1e-2, max_attempts: int = 64):
+                  margin: float = 1e-2, max_attempts: int = 64, prep=None):
     """Return (x, attempts [T] int64, near_tie_rows [n] int64).
 
     ``redraw(rows, attempt)`` returns bf16 rows [len(rows), H] for attempt number
-    ``attempt`` of the given row indices.
+    ``attempt`` of the given row indices. ``prep``, if given, maps rows of x to what the
+    router actually sees (for instance the normed activations).
     """
+    prep = prep or (lambda rows: rows)
     x = x.clone()
     attempts = torch.zeros(x.shape[0], dtype=torch.int64)
-    bad = np.nonzero(min_gap(router_logits(x, w_router, logit_bias), k) < margin)[0]
+    bad = np.nonzero(min_gap(router_logits(prep(x), w_router, logit_bias), k) < margin)[0]
     attempt = 0
     while bad.size and attempt < max_attempts:
         attempt += 1
         rows = torch.from_numpy(bad.astype(np.int64))
         x[rows] = redraw(rows, attempt).to(x.dtype)
         attempts[rows] = attempt
-        gaps = min_gap(router_logits(x[rows], w_router, logit_bias), k)
+        gaps = min_gap(router_logits(prep(x[rows]), w_router, logit_bias), k)
         bad = bad[gaps < margin]
     return x, attempts, torch.from_numpy(bad.astype(np.int64))

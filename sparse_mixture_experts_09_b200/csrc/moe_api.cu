@@ -46,7 +46,7 @@ inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 // Workspace regions, in order; each starts on a 1024-byte boundary.
 struct Layout {
   size_t status, topk_idx, topk_w, block_base, counts, offsets, row_of, token_of_row, x_perm, h,
-      y, end;
+      y, rnorm, end;
   size_t x_in, res_in, out_st, end_host;  // staging of moe_forward_host
 };
 
@@ -66,6 +66,7 @@ Layout layout(const Shape& s) {
   L.x_perm = o; o += up(rmax * s.H * 2);
   L.h = o; o += up(rmax * s.I * 2);
   L.y = o; o += up(rmax * s.H * 4);
+  L.rnorm = o; o += up((size_t)s.T * 4);
   L.end = o;
   L.x_in = o; o += up((size_t)s.T * s.H * 2);
   L.res_in = o; o += up((size_t)s.T * s.H * 2);
@@ -135,15 +136,17 @@ constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per wait
 
 moe_status_t run_forward(const Shape& s, const uint16_t* x, const uint16_t* wr, const float* bias,
                          const uint16_t* w1, const uint16_t* w3, const uint16_t* w2,
-                         const uint16_t* res, uint16_t* out, void* ws, cudaStream_t st) {
+                         const uint16_t* res, uint16_t* out, void* ws, cudaStream_t st,
+                         const uint16_t* norm_w = nullptr, float eps = 0.f) {
   const Layout L = layout(s);
+  float* rnorm = norm_w ? at<float>(ws, L.rnorm) : nullptr;
   cudaError_t e = launch_router(s, x, wr, bias, at<int32_t>(ws, L.topk_idx), at<float>(ws, L.topk_w),
-                                nullptr, st);
+                                nullptr, st, norm_w, eps, rnorm);
   if (e != cudaSuccess) return cuda_fail(e, "router launch");
   e = launch_permute(s, at<int32_t>(ws, L.topk_idx), x, at<int32_t>(ws, L.counts),
                      at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.row_of),
                      at<int32_t>(ws, L.token_of_row), at<uint16_t>(ws, L.x_perm),
-                     at<int32_t>(ws, L.block_base), st);
+                     at<int32_t>(ws, L.block_base), st, norm_w, rnorm);
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   GemmArgs g;
   g.a = at<uint16_t>(ws, L.x_perm);
@@ -354,6 +357,28 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_bf16_t* x, const mo
   MOE_TRY(check_ws(ws, ws_bytes, layout(s).end));
   return run_forward(s, x, w_router, logit_bias, w1, w3, w2, residual, out, ws,
                      (cudaStream_t)stream);
+}
+
+moe_status_t moe_forward_rmsnorm(const moe_shape_t* shape, const moe_bf16_t* h,
+                                 const moe_bf16_t* norm_weight, float eps,
+                                 const moe_bf16_t* w_router, const float* logit_bias,
+                                 const moe_bf16_t* w1, const moe_bf16_t* w3, const moe_bf16_t* w2,
+                                 moe_bf16_t* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(h, "h"));
+  MOE_TRY(check_ptr(norm_weight, "norm_weight"));
+  if (!(eps >= 0.f) || eps > 1.f) return fail(MOE_ERR_INVALID_ARG, "eps must be in [0, 1]");
+  MOE_TRY(check_ptr(w_router, "w_router"));
+  MOE_TRY(check_ptr(logit_bias, "logit_bias", true));
+  MOE_TRY(check_ptr(w1, "w1"));
+  MOE_TRY(check_ptr(w3, "w3"));
+  MOE_TRY(check_ptr(w2, "w2"));
+  MOE_TRY(check_ptr(out, "out"));
+  MOE_TRY(check_ws(ws, ws_bytes, layout(s).end));
+  return run_forward(s, h, w_router, logit_bias, w1, w3, w2, h, out, ws, (cudaStream_t)stream,
+                     norm_weight, eps);
 }
 
 moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_bf16_t* x_host,

@@ -33,14 +33,18 @@ inline int64_t num_token_blocks(const Shape& s) {
 
 // ---- launchers (each returns the launch's cudaError_t) ----
 
+// norm_w (nullable): RMSNorm gain [H]; the router then routes the normed rows and
+// writes 1/rms per token to rnorm, and the gather writes the normed rows.
 cudaError_t launch_router(const Shape& s, const uint16_t* x, const uint16_t* w_router,
                           const float* logit_bias, int32_t* topk_idx, float* topk_w,
-                          float* logits, cudaStream_t st);
+                          float* logits, cudaStream_t st, const uint16_t* norm_w = nullptr,
+                          float eps = 0.f, float* rnorm = nullptr);
 
 cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16_t* x,
                            int32_t* counts, int32_t* offsets, int32_t* row_of,
                            int32_t* token_of_row, uint16_t* x_perm, int32_t* block_base,
-                           cudaStream_t st);
+                           cudaStream_t st, const uint16_t* norm_w = nullptr,
+                           const float* rnorm = nullptr);
 
 struct GemmArgs {
   const uint16_t* a;        // x_perm [Rmax, K1] (GEMM1) or h [Rmax, I] (GEMM2)

@@ -25,6 +25,26 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   return r;
 }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Eight normed activations: bf16((x * r) * g), two float roundings then one bf16
+// rounding; the router and the gather both use exactly this.
+__device__ __forceinline__ uint4 norm8(uint4 xv, uint4 gv, float r) {
+  const uint32_t xq[4] = {xv.x, xv.y, xv.z, xv.w}, gq[4] = {gv.x, gv.y, gv.z, gv.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __fmul_rn(__fmul_rn(bf16_lo(xq[i]), r), bf16_lo(gq[i]));
+    const float hi = __fmul_rn(__fmul_rn(bf16_hi(xq[i]), r), bf16_hi(gq[i]));
+    o[i] = pack_bf16x2(lo, hi);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // Router and scoring. S warps cooperate on one token (S = 1, 2, 4 or 8; S > 1 when
 // there are too few tokens to keep the GPU busy): warp w of a token takes the w-th
 // of S equal slices of x[t] and of every router row. Each lane accumulates its
@@ -32,18 +52,26 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 // partial logits, and one thread adds the S partials in warp order, adds the bias,
 // and scores: float32 softmax over all E, the k largest logits (ties to the lower
 // expert index, slot 0 the largest), weights renormalised to sum to one.
-template <int EMAX, int S>
+//
+// With NORM the router first norms its token (the block's RMSNorm before the
+// mixture): r = 1 / sqrt(mean(x^2) + eps) over the whole row, then routes
+// xn = bf16((x * r) * g) instead of x, and stores r for the gather, which forms the
+// same xn with the same float operations.
+template <int EMAX, int S, bool NORM>
 __global__ void __launch_bounds__(256) k_router(const uint16_t* __restrict__ x,
                                                 const uint16_t* __restrict__ wr,
                                                 const float* __restrict__ bias, int64_t T,
                                                 int H, int E, int k,
                                                 int32_t* __restrict__ idx_out,
                                                 float* __restrict__ w_out,
-                                                float* __restrict__ logits_out) {
+                                                float* __restrict__ logits_out,
+                                                const uint16_t* __restrict__ norm_w, float eps,
+                                                float* __restrict__ rnorm_out) {
   pdl_trigger();
   pdl_wait();
   constexpr int TOK_PER_CTA = 8 / S;
   __shared__ float part[8][EMAX];
+  __shared__ float part_ss[8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slot = warp / S, sub = warp % S;
   const int per = (H >> 3) / S;  // 8-element chunks per warp; H % 128 == 0 keeps it whole
@@ -53,14 +81,44 @@ __global__ void __launch_bounds__(256) k_router(const uint16_t* __restrict__ x,
     float acc[EMAX];
 #pragma unroll
     for (int e = 0; e < EMAX; ++e) acc[e] = 0.f;
+    float rn = 1.f;
+    if (NORM) {
+      float ss = 0.f;
+      if (t < T) {
+        const uint4* xr = reinterpret_cast<const uint4*>(x + t * H) + sub * per;
+        for (int c = lane; c < per; c += 32) {
+          const uint4 xv = __ldg(xr + c);
+          const uint32_t q[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float a = bf16_lo(q[i]), b = bf16_hi(q[i]);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+          }
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      if (S > 1) {
+        if (lane == 0) part_ss[warp] = ss;
+        __syncthreads();
+        ss = part_ss[slot * S];
+#pragma unroll
+        for (int w = 1; w < S; ++w) ss += part_ss[slot * S + w];
+      }
+      rn = rsqrtf(ss / (float)H + eps);
+      if (sub == 0 && lane == 0 && t < T) rnorm_out[t] = rn;
+    }
     if (t < T) {
       const uint4* xr = reinterpret_cast<const uint4*>(x + t * H) + sub * per;
       const uint4* wrow = reinterpret_cast<const uint4*>(wr) + sub * per;
+      const uint4* grow = reinterpret_cast<const uint4*>(norm_w) + sub * per;
       const int rstride = H >> 3;
       // router rows in groups of 8: all loads of a group are issued before any use
       // (rows past E read row E-1 and are discarded), so they overlap in flight
       for (int c = lane; c < per; c += 32) {
-        const uint4 xv = ld_stream(xr + c);
+        uint4 xv = NORM ? __ldg(xr + c) : ld_stream(xr + c);
+        if (NORM) xv = norm8(xv, __ldg(grow + c), rn);
         const float x0 = bf16_lo(xv.x), x1 = bf16_hi(xv.x), x2 = bf16_lo(xv.y), x3 = bf16_hi(xv.y);
         const float x4 = bf16_lo(xv.z), x5 = bf16_hi(xv.z), x6 = bf16_lo(xv.w), x7 = bf16_hi(xv.w);
 #pragma unroll
@@ -329,11 +387,14 @@ __global__ void __launch_bounds__(1024) k_plan_small(const int32_t* __restrict__
 
 // One warp per row of x_perm below R_pad: copies x[token] or, on pad rows, writes
 // zeros and token -1.
+template <bool NORM>
 __global__ void __launch_bounds__(256) k_gather(const uint16_t* __restrict__ x, int H, int E,
                                                 const int32_t* __restrict__ counts,
                                                 const int32_t* __restrict__ offsets,
                                                 int32_t* __restrict__ token_of_row,
-                                                uint16_t* __restrict__ x_perm) {
+                                                uint16_t* __restrict__ x_perm,
+                                                const uint16_t* __restrict__ norm_w,
+                                                const float* __restrict__ rnorm) {
   pdl_trigger();
   pdl_wait();
   __shared__ int32_t s_off[65], s_cnt[64];
@@ -355,6 +416,12 @@ __global__ void __launch_bounds__(256) k_gather(const uint16_t* __restrict__ x, 
     if (pad) {
       if (lane == 0) token_of_row[r] = -1;
       for (int c = lane; c < chunks; c += 32) dst[c] = make_uint4(0, 0, 0, 0);
+    } else if (NORM) {
+      const int64_t t = token_of_row[r];
+      const uint4* src = reinterpret_cast<const uint4*>(x + t * H);
+      const uint4* g = reinterpret_cast<const uint4*>(norm_w);
+      const float rn = rnorm[t];
+      for (int c = lane; c < chunks; c += 32) dst[c] = norm8(__ldg(src + c), __ldg(g + c), rn);
     } else {
       const int64_t t = token_of_row[r];
       const uint4* src = reinterpret_cast<const uint4*>(x + t * H);
@@ -376,7 +443,8 @@ __global__ void __launch_bounds__(256) k_gather(const uint16_t* __restrict__ x, 
 
 cudaError_t launch_router(const Shape& s, const uint16_t* x, const uint16_t* w_router,
                           const float* logit_bias, int32_t* topk_idx, float* topk_w,
-                          float* logits, cudaStream_t st) {
+                          float* logits, cudaStream_t st, const uint16_t* norm_w, float eps,
+                          float* rnorm) {
   // enough warps to cover the GPU: split each token over S warps when T is small
   const int64_t want_warps = (int64_t)num_sms() * 32;
   int S = 1;
@@ -386,9 +454,13 @@ cudaError_t launch_router(const Shape& s, const uint16_t* x, const uint16_t* w_r
   const int64_t cap = (int64_t)num_sms() * 8;
   if (blocks > cap) blocks = cap;
   cudaError_t err = cudaSuccess;
-#define MOE_ROUTER(EM, SS)                                                                  \
-  err = launch_pdl(k_router<EM, SS>, dim3((unsigned)blocks), dim3(256), 0, st, x, w_router,   \
-                   logit_bias, s.T, s.H, s.E, s.k, topk_idx, topk_w, logits)
+#define MOE_ROUTER(EM, SS)                                                                    \
+  err = norm_w ? launch_pdl(k_router<EM, SS, true>, dim3((unsigned)blocks), dim3(256), 0, st, x,  \
+                            w_router, logit_bias, s.T, s.H, s.E, s.k, topk_idx, topk_w, logits, \
+                            norm_w, eps, rnorm)                                                 \
+               : launch_pdl(k_router<EM, SS, false>, dim3((unsigned)blocks), dim3(256), 0, st, x, \
+                            w_router, logit_bias, s.T, s.H, s.E, s.k, topk_idx, topk_w, logits, \
+                            norm_w, eps, rnorm)
 #define MOE_ROUTER_E(EM)           \
   switch (S) {                     \
     case 1: MOE_ROUTER(EM, 1); break; \
@@ -408,7 +480,7 @@ cudaError_t launch_router(const Shape& s, const uint16_t* x, const uint16_t* w_r
 cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16_t* x,
                            int32_t* counts, int32_t* offsets, int32_t* row_of,
                            int32_t* token_of_row, uint16_t* x_perm, int32_t* block_base,
-                           cudaStream_t st) {
+                           cudaStream_t st, const uint16_t* norm_w, const float* rnorm) {
   const int64_t nb = num_token_blocks(s);
   cudaError_t e;
   if (nb <= 32) {
@@ -430,8 +502,11 @@ cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16
   int64_t gblocks = (max_padded_rows(s) + 7) / 8;
   const int64_t cap = (int64_t)num_sms() * 8;
   if (gblocks > cap) gblocks = cap;
-  return launch_pdl(k_gather, dim3((unsigned)gblocks), dim3(256), 0, st, x, s.H, s.E, counts,
-                    offsets, token_of_row, x_perm);
+  if (norm_w)
+    return launch_pdl(k_gather<true>, dim3((unsigned)gblocks), dim3(256), 0, st, x, s.H, s.E,
+                      counts, offsets, token_of_row, x_perm, norm_w, rnorm);
+  return launch_pdl(k_gather<false>, dim3((unsigned)gblocks), dim3(256), 0, st, x, s.H, s.E, counts,
+                    offsets, token_of_row, x_perm, norm_w, rnorm);
 }
 
 }  // namespace moe

@@ -25,7 +25,7 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_size_host", "moe_max_padded_rows
            "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_expert_gate_up",
            "moe_expert_down", "moe_combine", "moe_forward",
            "moe_forward_host", "moe_device_status", "moe_last_error", "moe_permute_static",
-           "moe_selftest_wait_timeout")
+           "moe_selftest_wait_timeout", "moe_forward_rmsnorm")
 
 
 class MoeError(RuntimeError):
@@ -75,6 +75,9 @@ def lib() -> ctypes.CDLL:
         L.moe_combine.restype = st
         L.moe_forward.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
         L.moe_forward.restype = st
+        L.moe_forward_rmsnorm.argtypes = [sp, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P, _P, _P,
+                                          _SZ, _P]
+        L.moe_forward_rmsnorm.restype = st
         L.moe_forward_host.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
         L.moe_forward_host.restype = st
         L.moe_device_status.argtypes = [_P, _SZ, _P]
@@ -272,6 +275,26 @@ def forward(x, w_router, w1, w3, w2, k: int, residual=None, logit_bias=None, ws=
                              _dev(w2, "w2", torch.bfloat16),
                              _dev(residual, "residual", torch.bfloat16, True), _dev(out, "out"),
                              _dev(ws, "ws"), ws.numel(), _stream(stream)))
+    return out
+
+
+def forward_rmsnorm(h, norm_weight, eps: float, w_router, w1, w3, w2, k: int, logit_bias=None,
+                    ws=None, out=None, stream=None):
+    """out = h + moe(rms_norm(h)) on device tensors (the mixture half of the block)."""
+    t, hd = h.shape
+    e, i, _ = w1.shape
+    shape = make_shape(t, hd, i, e, k)
+    if ws is None:
+        ws = make_workspace(shape, h.device)
+    if out is None:
+        out = torch.empty((t, hd), dtype=torch.bfloat16, device=h.device)
+    _check(lib().moe_forward_rmsnorm(ctypes.byref(shape), _dev(h, "h", torch.bfloat16),
+                                     _dev(norm_weight, "norm_weight", torch.bfloat16), float(eps),
+                                     _dev(w_router, "w_router", torch.bfloat16),
+                                     _dev(logit_bias, "logit_bias", torch.float32, True),
+                                     _dev(w1, "w1", torch.bfloat16), _dev(w3, "w3", torch.bfloat16),
+                                     _dev(w2, "w2", torch.bfloat16), _dev(out, "out"),
+                                     _dev(ws, "ws"), ws.numel(), _stream(stream)))
     return out
 
 

@@ -22,7 +22,8 @@ import torch
 from . import synth
 
 # tensor ids of the generator streams
-X_ID, ROUTER_ID, W1_ID, W3_ID, W2_ID, RESIDUAL_ID = range(6)
+X_ID, ROUTER_ID, W1_ID, W3_ID, W2_ID, RESIDUAL_ID, NORM_ID = range(7)
+RMS_NORM_EPS = 1e-5  # rms_norm_eps of every Mixtral checkpoint
 
 
 @dataclass(frozen=True)
@@ -126,3 +127,9 @@ def draw(w: Workload, device="cpu") -> LayerInputs:
     if w.logit_bias is not None:
         bias = torch.tensor(w.logit_bias, dtype=torch.float32, device=device)
     return LayerInputs(draw_x(w, device), wr, w1, w3, w2, res, bias)
+
+
+def draw_norm_weight(w: Workload, device="cpu") -> torch.Tensor:
+    """RMSNorm gain [H] bf16: 1 + 0.1 N(0, 1) (a trained gain sits near one)."""
+    z = synth.normal((w.hidden_size,), 0.1, w.seed, NORM_ID, 0, device, dtype=torch.float64)
+    return (1.0 + z).to(torch.bfloat16)

@@ -287,3 +287,31 @@ def test_parameter_count_reconciles_45b_and_47b():
     total = experts + attn + router + embed
     assert round(experts / 1e9) == g["params_total_billion_doc"]
     assert round(total / 1e9) == g["params_total_billion_card"]
+
+
+# ---------------------------------------------------------------- RMSNorm (the block's norm)
+
+def test_rms_norm_matches_torch_and_closed_form():
+    rng = np.random.default_rng(10)
+    h = rng.standard_normal((50, 64)) * 3
+    g = 1 + 0.1 * rng.standard_normal(64)
+    want = F.rms_norm(torch.from_numpy(h), (64,), torch.from_numpy(g), eps=1e-5).numpy()
+    assert np.allclose(O.rms_norm(h, g, 1e-5), want, rtol=1e-13, atol=1e-14)
+    # a constant row c: c / sqrt(c^2 + eps) * g
+    c = -2.5
+    got = O.rms_norm(np.full((1, 8), c), np.arange(1.0, 9.0), 1e-5)
+    assert np.allclose(got, c / math.sqrt(c * c + 1e-5) * np.arange(1.0, 9.0), rtol=1e-15)
+    # scale invariance with eps = 0
+    assert np.allclose(O.rms_norm(7.0 * h, g, 0.0), O.rms_norm(h, g, 0.0), rtol=1e-13)
+
+
+def test_block_is_residual_plus_layer_on_normed_input():
+    x, wr, w1, w3, w2, res = _tiny_layer(11)
+    g = 1 + 0.1 * np.random.default_rng(3).standard_normal(x.shape[1])
+    blk = O.moe_block(res, g, 1e-5, wr, w1, w3, w2, 2, mode="exact")
+    xn = O.rms_norm(res, g, 1e-5)
+    lay = O.moe_layer(xn, wr, w1, w3, w2, 2, mode="exact")
+    assert np.allclose(blk["out"], res + lay["routed"], rtol=1e-14, atol=1e-14)
+    sub = O.moe_block(res, g, 1e-5, wr, w1, w3, w2, 2, mode="bf16_storage", tokens=[1, 4])
+    full = O.moe_block(res, g, 1e-5, wr, w1, w3, w2, 2, mode="bf16_storage")
+    assert np.array_equal(sub["out"], full["out"][[1, 4]])
