@@ -35,9 +35,14 @@ METRIC = "MoE-layer tokens/s and % of roofline (BF16 tensor peak / HBM BW) at 1 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 GEMM_SOURCE = os.path.join(ROOT, "sparse_mixture_experts_09_b200", "csrc", "gemm_sm100.cu")
-# kernels one moe_forward launches: router, 4 permutation kernels (histogram, scan,
-# rank, gather), the two expert GEMMs and the combine
-KERNELS_PER_FORWARD = 8
+
+
+def kernels_per_forward(num_tokens: int) -> int:
+    """Kernels one moe_forward launches: router, the permutation (one planning kernel
+    up to 1024 tokens, else histogram + scan + rank; then the gather), the two expert
+    GEMMs and the combine."""
+    plan = 1 if (num_tokens + 31) // 32 <= 32 else 3
+    return 1 + plan + 1 + 2 + 1
 
 
 def parse_args():
@@ -298,12 +303,20 @@ def run_ours(args):
     w = W.WORKLOADS[args.workload]
     inp = W.draw(w, dev)
     k = w.num_experts_per_tok
-    shape = moe.make_shape(*w.shape)
+    # the expert weights live in the library's blocked layout, converted once at load
+    # time (not timed); a row-major loop is timed alongside for comparison
+    bw1, bw3, bw2 = moe.pack_weights(inp.w1, inp.w3, inp.w2)
+    layout = moe.BLOCKED
+    shape = moe.make_shape(*w.shape, layout)
     ws = moe.make_workspace(shape, dev)
     out = torch.empty((w.num_tokens, w.hidden_size), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
+        moe.forward(inp.x, inp.w_router, bw1, bw3, bw2, k, residual=inp.residual,
+                    logit_bias=inp.logit_bias, ws=ws, out=out, weight_layout=layout)
+
+    def step_row_major():
         moe.forward(inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, k, residual=inp.residual,
                     logit_bias=inp.logit_bias, ws=ws, out=out)
 
@@ -333,10 +346,10 @@ def run_ours(args):
                                  p(perm["row_of"]), p(perm["token_of_row"]), p(perm["x_perm"]),
                                  p(ws), ws.numel(), st))
         ev[2].record(stream)
-        moe._check(L.moe_expert_gate_up(sp, p(perm["x_perm"]), p(perm["offsets"]), p(inp.w1),
-                                        p(inp.w3), p(hbuf), p(ws), ws.numel(), st))
+        moe._check(L.moe_expert_gate_up(sp, p(perm["x_perm"]), p(perm["offsets"]), p(bw1),
+                                        p(bw3), p(hbuf), p(ws), ws.numel(), st))
         ev[3].record(stream)
-        moe._check(L.moe_expert_down(sp, p(hbuf), p(perm["offsets"]), p(inp.w2), p(ybuf), p(ws),
+        moe._check(L.moe_expert_down(sp, p(hbuf), p(perm["offsets"]), p(bw2), p(ybuf), p(ws),
                                      ws.numel(), st))
         ev[4].record(stream)
         moe._check(L.moe_combine(sp, p(ybuf), p(perm["row_of"]), p(wt), p(inp.residual), p(out), st))
@@ -348,12 +361,13 @@ def run_ours(args):
     wsh = moe.make_workspace(shape, dev, host=True)
 
     def host_step():
-        moe.forward_host(xh, inp.w_router, inp.w1, inp.w3, inp.w2, k, residual_host=rh,
-                         logit_bias=inp.logit_bias, ws=wsh, out_host=oh)
+        moe.forward_host(xh, inp.w_router, bw1, bw3, bw2, k, residual_host=rh,
+                         logit_bias=inp.logit_bias, ws=wsh, out_host=oh, weight_layout=layout)
 
     K, Wm = args.steps, max(3, args.warmup)
     for _ in range(Wm):
         step()
+        step_row_major()
     scratch = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
     for _ in range(3):
         split_step(scratch)
@@ -394,6 +408,18 @@ def run_ours(args):
     stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
                 for j, n in enumerate(names)}
 
+    # (2b) the same layer with row-major expert weights
+    barrier()
+    torch.cuda.synchronize(dev)
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r0.record(stream)
+    for _ in range(K):
+        step_row_major()
+    r1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    rm_ms = r0.elapsed_time(r1) / K
+
     # (3) end to end from pinned host memory
     barrier()
     torch.cuda.synchronize(dev)
@@ -410,6 +436,7 @@ def run_ours(args):
     moe.device_status(wsh)
 
     ms, e2e_ms = slowest_rank(ms, e2e_ms, world, dev)
+    rm_ms, _ = slowest_rank(rm_ms, rm_ms, world, dev)
 
     counts = perm["counts"].cpu().tolist()
     peaks, peak_kind = load_peaks()
@@ -425,14 +452,17 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic: seeded SplitMix64/Box-Muller draws, weights ~N(0,1/fan_in), x rows RMS 1",
             "config": dict(workload_config(w), parallelism=f"replicas x{world}",
+                           weight_layout="blocked (moe_pack_weights once at load, untimed)",
                            l2=("no flush: each step streams %.2f GB of expert weights, more than "
                                "the 126 MB L2" % (roof["active_experts"] * w.expert_bytes() / 1e9))),
             "roofline": roof,
             "kernels_ms": stage_ms,
+            "row_major_weights": {"ms_per_step": rm_ms,
+                                  "value": job_throughput(w.num_tokens, world, rm_ms)},
             "e2e": {"value": job_throughput(w.num_tokens, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": 2 * bytes_io, "d2h_bytes_per_step": bytes_io,
                     "api": "moe_forward_host"},
-            "gpu_launches": KERNELS_PER_FORWARD * K,
+            "gpu_launches": kernels_per_forward(w.num_tokens) * K,
             "clocks": clk,
             "expert_counts": counts,
         }

@@ -20,7 +20,8 @@
  *   returns without synchronising (moe_forward_host excepted).
  * - bf16 tensors are raw IEEE bfloat16 bit patterns (moe_bf16_t), row-major,
  *   contiguous. Weights use nn.Linear [out, in] form stacked over experts:
- *   w_router [E, H]; w1 (gate) and w3 (up) [E, I, H]; w2 (down) [E, H, I].
+ *   w_router [E, H]; w1 (gate) and w3 (up) [E, I, H]; w2 (down) [E, H, I]; the
+ *   expert weights may instead be in the blocked layout (shape->weight_layout).
  * - Requirements (else MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED): num_tokens >= 1,
  *   1 <= num_experts_per_tok <= num_experts <= 64, num_experts_per_tok <= 8,
  *   hidden_size and intermediate_size positive multiples of 128, every pointer
@@ -60,15 +61,24 @@ typedef enum {
   MOE_ERR_TIMEOUT = 5
 } moe_status_t;
 
+/* Layouts of the stacked expert weights w1, w3 [E, I, H] and w2 [E, H, I]:
+ * ROW_MAJOR is nn.Linear's [out, in]; BLOCKED stores each [rows, K] matrix (rows =
+ * E*I or E*H) as [rows/128][K/64][128][64], so every 128 x 64 tile the kernels read
+ * is one contiguous 16 KiB run (moe_pack_weights converts once, at load time). */
+#define MOE_WEIGHTS_ROW_MAJOR 0
+#define MOE_WEIGHTS_BLOCKED 1
+
 /* The layer's sizes, named as in MixtralConfig (Hugging Face "Mixtral" doc):
  * hidden_size, intermediate_size, num_local_experts (here num_experts) and
- * num_experts_per_tok. num_tokens = batch * sequence length. */
+ * num_experts_per_tok. num_tokens = batch * sequence length. weight_layout is one of
+ * the MOE_WEIGHTS_* values (a zero-initialised shape means row-major). */
 typedef struct {
   int64_t num_tokens;
   int32_t hidden_size;
   int32_t intermediate_size;
   int32_t num_experts;
   int32_t num_experts_per_tok;
+  int32_t weight_layout;
 } moe_shape_t;
 
 /* Bytes of device workspace every workspace-taking entry point needs for `shape`;
@@ -211,6 +221,14 @@ moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_bf16_t* x_host
                               const moe_bf16_t* w2, const moe_bf16_t* residual_host,
                               moe_bf16_t* out_host, void* ws, size_t ws_bytes,
                               moe_stream_t stream);
+
+/* Convert row-major expert weights to MOE_WEIGHTS_BLOCKED: w1, w3 [E, I, H] and w2
+ * [E, H, I] in, the same-sized w1_blocked, w3_blocked, w2_blocked out (caller-owned,
+ * distinct from the inputs). Asynchronous on `stream`. */
+moe_status_t moe_pack_weights(const moe_shape_t* shape, const moe_bf16_t* w1,
+                              const moe_bf16_t* w3, const moe_bf16_t* w2,
+                              moe_bf16_t* w1_blocked, moe_bf16_t* w3_blocked,
+                              moe_bf16_t* w2_blocked, moe_stream_t stream);
 
 /* Waits for `stream`, then reads and clears the device status word in `ws`:
  * MOE_OK, or MOE_ERR_TIMEOUT if a kernel gave up a bounded wait since the last

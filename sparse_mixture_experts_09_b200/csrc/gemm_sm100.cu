@@ -66,6 +66,7 @@ struct KParams {
   int k_blocks;
   int n_tiles;
   int b_rows;  // rows of the B tensor per expert
+  int blocked;  // weights in the blocked layout (MOE_WEIGHTS_BLOCKED)
   unsigned long long timeout_ns;
 };
 
@@ -195,6 +196,20 @@ __device__ __noinline__ void drain_phase(uint32_t bar, uint32_t parity,
   const unsigned long long t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer() - t0 > timeout_ns) return;
+  }
+}
+
+// Tensor-map coordinates (x, y) of weight row `row`, k-block `kb`. Row-major weights
+// are a [rows, K] map; blocked weights ([rows/128][K/64][128][64], each 128 x 64 block
+// one contiguous 16 KiB run) are a [rows * K/64, 64] map, so every TMA box of up to
+// 128 rows reads contiguous memory.
+__device__ __forceinline__ void wcoord(int kb, int row, int k_blocks, int blocked, int& x, int& y) {
+  if (blocked) {
+    x = 0;
+    y = ((row >> 7) * k_blocks + kb) * 128 + (row & 127);
+  } else {
+    x = kb * BK;
+    y = row;
   }
 }
 
@@ -334,21 +349,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sb = sa + C::A_BYTES;
           mbar_expect_tx(full_bar(s), bytes);
           tma_load_2d(sa, &mapA, kb * BK, a_row, full_bar(s));
+          int wx, wy;
           if (pieces == 1) {
+            wcoord(kb, b_row, p.k_blocks, p.blocked, wx, wy);
             if (MODE == kSwiGLU) {
-              tma_load_2d(sb, &mapB0, kb * BK, b_row, full_bar(s));
-              tma_load_2d(sb + 128 * BK * 2, &mapB1, kb * BK, b_row, full_bar(s));
+              tma_load_2d(sb, &mapB0, wx, wy, full_bar(s));
+              tma_load_2d(sb + 128 * BK * 2, &mapB1, wx, wy, full_bar(s));
             } else {
-              tma_load_2d(sb, &mapB0, kb * BK, b_row, full_bar(s));
-              if (BN == 256) tma_load_2d(sb + 128 * BK * 2, &mapB0, kb * BK, b_row + 128, full_bar(s));
+              tma_load_2d(sb, &mapB0, wx, wy, full_bar(s));
+              if (BN == 256) {
+                wcoord(kb, b_row + 128, p.k_blocks, p.blocked, wx, wy);
+                tma_load_2d(sb + 128 * BK * 2, &mapB0, wx, wy, full_bar(s));
+              }
             }
           } else {
             // 32-row boxes; gate (or down) rows first, then the up rows
-            for (int j = 0; j < rp; j += 32)
-              tma_load_2d(sb + j * BK * 2, &mapB0s, kb * BK, b_row + j, full_bar(s));
+            for (int j = 0; j < rp; j += 32) {
+              wcoord(kb, b_row + j, p.k_blocks, p.blocked, wx, wy);
+              tma_load_2d(sb + j * BK * 2, &mapB0s, wx, wy, full_bar(s));
+            }
             if (MODE == kSwiGLU)
-              for (int j = 0; j < rp; j += 32)
-                tma_load_2d(sb + (rp + j) * BK * 2, &mapB1s, kb * BK, b_row + j, full_bar(s));
+              for (int j = 0; j < rp; j += 32) {
+                wcoord(kb, b_row + j, p.k_blocks, p.blocked, wx, wy);
+                tma_load_2d(sb + (rp + j) * BK * 2, &mapB1s, wx, wy, full_bar(s));
+              }
           }
         }
       }
@@ -677,7 +701,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (rank == 0) mbar_expect_tx(full_bar(s), 2 * C::STAGE_BYTES);
           const uint32_t fb = mapa_shared(full_bar(s), 0);
           tma_load_2d_pair(sa, &mapA, kb * BK, a_row, fb);
-          tma_load_2d_pair(sa + C::A_BYTES, mb, kb * BK, b_row, fb);
+          int wx, wy;
+          wcoord(kb, b_row, p.k_blocks, p.blocked, wx, wy);
+          tma_load_2d_pair(sa + C::A_BYTES, mb, wx, wy, fb);
         }
       }
       if (!ok && rank == 0) {
@@ -817,6 +843,22 @@ __global__ void k_wait_selftest(int32_t* status, unsigned long long timeout_ns) 
     wait_phase(smem_u32(&bar), 0, reinterpret_cast<volatile int*>(&abort_flag), status, timeout_ns);
 }
 
+// ---------------------------------------------------------------- weight packing
+// w [rows, cols] row-major -> [rows/128][cols/64][128][64]; one thread per 16 bytes.
+__global__ void __launch_bounds__(256) k_pack_blocked(const uint4* __restrict__ w,
+                                                      uint4* __restrict__ wp, int64_t rows,
+                                                      int64_t cols) {
+  const int64_t kb_n = cols / BK, n = rows * cols / 8;
+  for (int64_t o = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; o < n;
+       o += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c = o & 7;              // 16-byte chunk within a 64-wide row
+    const int64_t rr = (o >> 3) & 127;    // row within the block
+    const int64_t blk = o >> 10;          // (row block, k block)
+    const int64_t rb = blk / kb_n, kb = blk - rb * kb_n;
+    wp[o] = w[((rb * 128 + rr) * cols + kb * BK) / 8 + c];
+  }
+}
+
 // ---------------------------------------------------------------- host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -944,9 +986,10 @@ bool use_pair(const Shape& s) { return MOE_PAIR_GEMM && s.T * s.k >= (int64_t)10
 cudaError_t launch_gate_up(const Shape& s, const GemmArgs& g, cudaStream_t st, const char** why) {
   CUtensorMap mx, mw1, mw3, mw1s, mw3s;
   const uint64_t EI = (uint64_t)s.E * s.I;
-  if (!make_map(&mx, g.a, s.H, g.rmax, 128) || !make_map(&mw1, g.w1, s.H, EI, 128) ||
-      !make_map(&mw3, g.w3, s.H, EI, 128) || !make_map(&mw1s, g.w1, s.H, EI, 32) ||
-      !make_map(&mw3s, g.w3, s.H, EI, 32)) {
+  const uint64_t wi = s.blocked ? BK : s.H, wr = s.blocked ? EI * s.H / BK : EI;
+  if (!make_map(&mx, g.a, s.H, g.rmax, 128) || !make_map(&mw1, g.w1, wi, wr, 128) ||
+      !make_map(&mw3, g.w3, wi, wr, 128) || !make_map(&mw1s, g.w1, wi, wr, 32) ||
+      !make_map(&mw3s, g.w3, wi, wr, 32)) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad tensor)";
     return cudaErrorInvalidValue;
   }
@@ -959,6 +1002,7 @@ cudaError_t launch_gate_up(const Shape& s, const GemmArgs& g, cudaStream_t st, c
   p.k_blocks = s.H / BK;
   p.n_tiles = s.I / 128;
   p.b_rows = s.I;
+  p.blocked = s.blocked;
   p.timeout_ns = g.timeout_ns;
   cudaError_t e =
       launch_one<kSwiGLU, 256>(mx, mw1, mw3, mw1s, mw3s, p, (g.rmax / BM) * p.n_tiles, st);
@@ -969,8 +1013,9 @@ cudaError_t launch_gate_up(const Shape& s, const GemmArgs& g, cudaStream_t st, c
 cudaError_t launch_down(const Shape& s, const GemmArgs& g, cudaStream_t st, const char** why) {
   CUtensorMap mh, mw2, mw2s;
   const uint64_t EH = (uint64_t)s.E * s.H;
-  if (!make_map(&mh, g.h, s.I, g.rmax, 128) || !make_map(&mw2, g.w2, s.I, EH, 128) ||
-      !make_map(&mw2s, g.w2, s.I, EH, 32)) {
+  const uint64_t wi = s.blocked ? BK : s.I, wr = s.blocked ? EH * s.I / BK : EH;
+  if (!make_map(&mh, g.h, s.I, g.rmax, 128) || !make_map(&mw2, g.w2, wi, wr, 128) ||
+      !make_map(&mw2s, g.w2, wi, wr, 32)) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad tensor)";
     return cudaErrorInvalidValue;
   }
@@ -982,6 +1027,7 @@ cudaError_t launch_down(const Shape& s, const GemmArgs& g, cudaStream_t st, cons
   p.E = s.E;
   p.k_blocks = s.I / BK;
   p.b_rows = s.H;
+  p.blocked = s.blocked;
   p.timeout_ns = g.timeout_ns;
   cudaError_t e;
   if (s.H % 256 == 0 && use_pair(s)) {
@@ -996,6 +1042,16 @@ cudaError_t launch_down(const Shape& s, const GemmArgs& g, cudaStream_t st, cons
   }
   if (e != cudaSuccess) *why = "down GEMM launch failed";
   return e;
+}
+
+cudaError_t launch_pack_blocked(const uint16_t* w, uint16_t* wp, int64_t rows, int64_t cols,
+                                cudaStream_t st) {
+  int64_t blocks = (rows * cols / 8 + 255) / 256;
+  const int64_t cap = (int64_t)num_sms() * 16;
+  if (blocks > cap) blocks = cap;
+  k_pack_blocked<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(w),
+                                                   reinterpret_cast<uint4*>(wp), rows, cols);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_wait_selftest(int32_t* status, unsigned long long timeout_ns, cudaStream_t st) {

@@ -93,11 +93,15 @@ moe_status_t check_shape(const moe_shape_t* sh, Shape* out) {
   if (sh->num_tokens * sh->num_experts_per_tok > (int64_t)1 << 30)
     return fail(MOE_ERR_UNSUPPORTED, "num_tokens * num_experts_per_tok must be <= 2^30 (got %lld)",
                 (long long)(sh->num_tokens * sh->num_experts_per_tok));
+  if (sh->weight_layout != MOE_WEIGHTS_ROW_MAJOR && sh->weight_layout != MOE_WEIGHTS_BLOCKED)
+    return fail(MOE_ERR_INVALID_ARG, "weight_layout must be MOE_WEIGHTS_ROW_MAJOR or MOE_WEIGHTS_BLOCKED (got %d)",
+                sh->weight_layout);
   out->T = sh->num_tokens;
   out->H = sh->hidden_size;
   out->I = sh->intermediate_size;
   out->E = sh->num_experts;
   out->k = sh->num_experts_per_tok;
+  out->blocked = sh->weight_layout == MOE_WEIGHTS_BLOCKED;
   const int64_t rmax = max_padded_rows(*out);
   if ((rmax / 128) * (int64_t)(out->I / 128) > INT32_MAX || (int64_t)out->E * out->I > INT32_MAX)
     return fail(MOE_ERR_UNSUPPORTED, "shape too large for 32-bit tile indices");
@@ -425,6 +429,26 @@ moe_status_t moe_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t timeo
     return fail(MOE_ERR_INVALID_ARG, "timeout_ns must be in (0, 10 s]");
   cudaError_t e = launch_wait_selftest(at<int32_t>(ws, 0), timeout_ns, (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "self-test launch");
+}
+
+moe_status_t moe_pack_weights(const moe_shape_t* shape, const moe_bf16_t* w1, const moe_bf16_t* w3,
+                              const moe_bf16_t* w2, moe_bf16_t* w1_blocked, moe_bf16_t* w3_blocked,
+                              moe_bf16_t* w2_blocked, moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(w1, "w1"));
+  MOE_TRY(check_ptr(w3, "w3"));
+  MOE_TRY(check_ptr(w2, "w2"));
+  MOE_TRY(check_ptr(w1_blocked, "w1_blocked"));
+  MOE_TRY(check_ptr(w3_blocked, "w3_blocked"));
+  MOE_TRY(check_ptr(w2_blocked, "w2_blocked"));
+  cudaStream_t st = (cudaStream_t)stream;
+  const int64_t ei = (int64_t)s.E * s.I, eh = (int64_t)s.E * s.H;
+  cudaError_t e = launch_pack_blocked(w1, w1_blocked, ei, s.H, st);
+  if (e == cudaSuccess) e = launch_pack_blocked(w3, w3_blocked, ei, s.H, st);
+  if (e == cudaSuccess) e = launch_pack_blocked(w2, w2_blocked, eh, s.I, st);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "weight packing launch");
 }
 
 moe_status_t moe_device_status(void* ws, size_t ws_bytes, moe_stream_t stream) {

@@ -20,6 +20,7 @@ constexpr int32_t kStatusTimeout = 1;
 struct Shape {
   int64_t T;
   int H, I, E, k;
+  int blocked;  // expert weights in the blocked layout
 };
 
 inline int64_t max_padded_rows(const Shape& s) {
@@ -64,6 +65,11 @@ cudaError_t launch_gate_up(const Shape& s, const GemmArgs& g, cudaStream_t st, c
 cudaError_t launch_down(const Shape& s, const GemmArgs& g, cudaStream_t st, const char** why);
 cudaError_t launch_grouped_swiglu(const Shape& s, const GemmArgs& g, cudaStream_t st,
                                   const char** why);
+
+// w [rows, cols] -> blocked layout [rows/128][cols/64][128][64] (rows % 128 == 0,
+// cols % 64 == 0).
+cudaError_t launch_pack_blocked(const uint16_t* w, uint16_t* wp, int64_t rows, int64_t cols,
+                                cudaStream_t st);
 
 // One thread's bounded wait on a barrier nothing arrives on (checks timeout reporting).
 cudaError_t launch_wait_selftest(int32_t* status, unsigned long long timeout_ns, cudaStream_t st);

@@ -25,7 +25,7 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_size_host", "moe_max_padded_rows
            "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_expert_gate_up",
            "moe_expert_down", "moe_combine", "moe_forward",
            "moe_forward_host", "moe_device_status", "moe_last_error", "moe_permute_static",
-           "moe_selftest_wait_timeout", "moe_forward_rmsnorm")
+           "moe_selftest_wait_timeout", "moe_forward_rmsnorm", "moe_pack_weights")
 
 
 class MoeError(RuntimeError):
@@ -34,10 +34,13 @@ class MoeError(RuntimeError):
         self.status = status
 
 
+ROW_MAJOR, BLOCKED = 0, 1  # MOE_WEIGHTS_* layouts of the expert weights
+
+
 class Shape(ctypes.Structure):
     _fields_ = [("num_tokens", ctypes.c_int64), ("hidden_size", ctypes.c_int32),
                 ("intermediate_size", ctypes.c_int32), ("num_experts", ctypes.c_int32),
-                ("num_experts_per_tok", ctypes.c_int32)]
+                ("num_experts_per_tok", ctypes.c_int32), ("weight_layout", ctypes.c_int32)]
 
 
 _lib = None
@@ -78,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_rmsnorm.argtypes = [sp, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P, _P, _P,
                                           _SZ, _P]
         L.moe_forward_rmsnorm.restype = st
+        L.moe_pack_weights.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P]
+        L.moe_pack_weights.restype = st
         L.moe_forward_host.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
         L.moe_forward_host.restype = st
         L.moe_device_status.argtypes = [_P, _SZ, _P]
@@ -98,9 +103,9 @@ def _check(status: int) -> None:
 
 
 def make_shape(num_tokens: int, hidden_size: int, intermediate_size: int, num_experts: int,
-               num_experts_per_tok: int) -> Shape:
+               num_experts_per_tok: int, weight_layout: int = ROW_MAJOR) -> Shape:
     return Shape(int(num_tokens), int(hidden_size), int(intermediate_size), int(num_experts),
-                 int(num_experts_per_tok))
+                 int(num_experts_per_tok), int(weight_layout))
 
 
 def _dev(t: Optional[torch.Tensor], name: str, dtype=None, nullable=False) -> Optional[int]:
@@ -204,10 +209,11 @@ def permute_static(topk_idx, x, num_experts: int, intermediate_size: int, stream
     return out
 
 
-def grouped_swiglu(x_perm, offsets, w1, w3, w2, num_tokens: int, k: int, ws, stream=None):
+def grouped_swiglu(x_perm, offsets, w1, w3, w2, num_tokens: int, k: int, ws, stream=None,
+                   weight_layout: int = ROW_MAJOR):
     """y_perm [R_max, H] fp32 = w2[e] (silu(w1[e] x) * w3[e] x) per routed row."""
     e, i, h = w1.shape
-    shape = make_shape(num_tokens, h, i, e, k)
+    shape = make_shape(num_tokens, h, i, e, k, weight_layout)
     y = torch.zeros((max_padded_rows(shape), h), dtype=torch.float32, device=x_perm.device)
     _check(lib().moe_grouped_swiglu(ctypes.byref(shape), _dev(x_perm, "x_perm", torch.bfloat16),
                                     _dev(offsets, "offsets", torch.int32),
@@ -217,10 +223,11 @@ def grouped_swiglu(x_perm, offsets, w1, w3, w2, num_tokens: int, k: int, ws, str
     return y
 
 
-def expert_gate_up(x_perm, offsets, w1, w3, num_tokens: int, k: int, ws, h=None, stream=None):
+def expert_gate_up(x_perm, offsets, w1, w3, num_tokens: int, k: int, ws, h=None, stream=None,
+                   weight_layout: int = ROW_MAJOR):
     """h [R_max, I] bf16 = bf16(silu(x_perm w1[e]^T) * (x_perm w3[e]^T)) (GEMM1 alone)."""
     e, i, hd = w1.shape
-    shape = make_shape(num_tokens, hd, i, e, k)
+    shape = make_shape(num_tokens, hd, i, e, k, weight_layout)
     if h is None:
         h = torch.zeros((max_padded_rows(shape), i), dtype=torch.bfloat16, device=x_perm.device)
     _check(lib().moe_expert_gate_up(ctypes.byref(shape), _dev(x_perm, "x_perm", torch.bfloat16),
@@ -231,10 +238,11 @@ def expert_gate_up(x_perm, offsets, w1, w3, num_tokens: int, k: int, ws, h=None,
     return h
 
 
-def expert_down(h, offsets, w2, num_tokens: int, k: int, ws, y=None, stream=None):
+def expert_down(h, offsets, w2, num_tokens: int, k: int, ws, y=None, stream=None,
+                weight_layout: int = ROW_MAJOR):
     """y_perm [R_max, H] fp32 = h w2[e]^T (GEMM2 alone)."""
     e, hd, i = w2.shape
-    shape = make_shape(num_tokens, hd, i, e, k)
+    shape = make_shape(num_tokens, hd, i, e, k, weight_layout)
     if y is None:
         y = torch.zeros((max_padded_rows(shape), hd), dtype=torch.float32, device=h.device)
     _check(lib().moe_expert_down(ctypes.byref(shape), _dev(h, "h", torch.bfloat16),
@@ -259,11 +267,11 @@ def combine(y_perm, row_of, topk_w, residual=None, num_experts: int = 8, interme
 
 
 def forward(x, w_router, w1, w3, w2, k: int, residual=None, logit_bias=None, ws=None, out=None,
-            stream=None):
+            stream=None, weight_layout: int = ROW_MAJOR):
     """The whole layer on device tensors; returns out [T,H] bf16."""
     t, h = x.shape
     e, i, _ = w1.shape
-    shape = make_shape(t, h, i, e, k)
+    shape = make_shape(t, h, i, e, k, weight_layout)
     if ws is None:
         ws = make_workspace(shape, x.device)
     if out is None:
@@ -279,11 +287,11 @@ def forward(x, w_router, w1, w3, w2, k: int, residual=None, logit_bias=None, ws=
 
 
 def forward_rmsnorm(h, norm_weight, eps: float, w_router, w1, w3, w2, k: int, logit_bias=None,
-                    ws=None, out=None, stream=None):
+                    ws=None, out=None, stream=None, weight_layout: int = ROW_MAJOR):
     """out = h + moe(rms_norm(h)) on device tensors (the mixture half of the block)."""
     t, hd = h.shape
     e, i, _ = w1.shape
-    shape = make_shape(t, hd, i, e, k)
+    shape = make_shape(t, hd, i, e, k, weight_layout)
     if ws is None:
         ws = make_workspace(shape, h.device)
     if out is None:
@@ -299,11 +307,11 @@ def forward_rmsnorm(h, norm_weight, eps: float, w_router, w1, w3, w2, k: int, lo
 
 
 def forward_host(x_host, w_router, w1, w3, w2, k: int, residual_host=None, logit_bias=None,
-                 ws=None, out_host=None, stream=None):
+                 ws=None, out_host=None, stream=None, weight_layout: int = ROW_MAJOR):
     """The layer with host (ideally pinned) activations; returns out_host (synchronous)."""
     t, h = x_host.shape
     e, i, _ = w1.shape
-    shape = make_shape(t, h, i, e, k)
+    shape = make_shape(t, h, i, e, k, weight_layout)
     for name, a in (("x_host", x_host), ("residual_host", residual_host)):
         if a is not None and (a.is_cuda or a.dtype != torch.bfloat16 or not a.is_contiguous()):
             raise ValueError(f"{name} must be a contiguous bf16 host tensor")
@@ -325,6 +333,19 @@ def selftest_wait_timeout(ws, timeout_ns: int, stream=None) -> None:
     """Launch the bounded-wait check: a wait that nothing completes gives up after
     ``timeout_ns`` and records MOE_ERR_TIMEOUT in ``ws``'s status word."""
     _check(lib().moe_selftest_wait_timeout(_dev(ws, "ws"), ws.numel(), int(timeout_ns), _stream(stream)))
+
+
+def pack_weights(w1, w3, w2, stream=None):
+    """Row-major expert weights -> the blocked layout (new tensors of the same shapes);
+    pass weight_layout=BLOCKED with them."""
+    e, i, h = w1.shape
+    shape = make_shape(1, h, i, e, 1)
+    out = [torch.empty_like(t) for t in (w1, w3, w2)]
+    _check(lib().moe_pack_weights(ctypes.byref(shape), _dev(w1, "w1", torch.bfloat16),
+                                  _dev(w3, "w3", torch.bfloat16), _dev(w2, "w2", torch.bfloat16),
+                                  _dev(out[0], "w1_blocked"), _dev(out[1], "w3_blocked"),
+                                  _dev(out[2], "w2_blocked"), _stream(stream)))
+    return tuple(out)
 
 
 def device_status(ws, stream=None) -> None:

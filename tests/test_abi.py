@@ -37,8 +37,8 @@ def test_library_exports_every_declared_symbol(L):
         assert hasattr(L, name), name
 
 
-def shape(t=64, h=128, i=256, e=8, k=2):
-    return M.make_shape(t, h, i, e, k)
+def shape(t=64, h=128, i=256, e=8, k=2, layout=0):
+    return M.make_shape(t, h, i, e, k, layout)
 
 
 def test_workspace_and_padded_rows(L):
@@ -53,7 +53,8 @@ def test_workspace_and_padded_rows(L):
 
 
 @pytest.mark.parametrize("bad", [dict(t=0), dict(h=100), dict(i=200), dict(e=0), dict(e=65),
-                                 dict(k=0), dict(k=9, e=16), dict(k=3, e=2)])
+                                 dict(k=0), dict(k=9, e=16), dict(k=3, e=2), dict(layout=2),
+                                 dict(layout=-1)])
 def test_invalid_shapes_are_rejected(L, bad):
     s = shape(**bad)
     assert M.workspace_size(s) == 0
