@@ -71,7 +71,11 @@ typedef enum {
 /* The layer's sizes, named as in MixtralConfig (Hugging Face "Mixtral" doc):
  * hidden_size, intermediate_size, num_local_experts (here num_experts) and
  * num_experts_per_tok. num_tokens = batch * sequence length. weight_layout is one of
- * the MOE_WEIGHTS_* values (a zero-initialised shape means row-major). */
+ * the MOE_WEIGHTS_* values (a zero-initialised shape means row-major).
+ * router_bf16_logits: 0 keeps the router logits in fp32; 1 rounds each logit to bf16
+ * before scoring, as a bf16 load of the model does (its router's F.linear returns bf16
+ * logits that are then cast to float32 for the softmax: nnterp "Mixtral", "The router
+ * renormalizes its top 2, in float32"). Equal rounded logits go to the lower expert. */
 typedef struct {
   int64_t num_tokens;
   int32_t hidden_size;
@@ -79,6 +83,7 @@ typedef struct {
   int32_t num_experts;
   int32_t num_experts_per_tok;
   int32_t weight_layout;
+  int32_t router_bf16_logits;
 } moe_shape_t;
 
 /* Bytes of device workspace every workspace-taking entry point needs for `shape`;

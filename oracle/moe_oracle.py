@@ -76,13 +76,17 @@ def silu(g: np.ndarray) -> np.ndarray:
         return g / (1.0 + np.exp(-g))
 
 
-def router_logits(x, w_router, logit_bias=None) -> np.ndarray:
+def router_logits(x, w_router, logit_bias=None, bf16_logits: bool = False) -> np.ndarray:
     """[T, E] fp64 logits l[t, e] = sum_h x[t, h] * W_r[e, h] (+ logit_bias[e] if given).
 
     ``logit_bias`` is not part of Mixtral; the benchmark's imbalanced workload uses it
-    to skew routing.
+    to skew routing. With ``bf16_logits`` each logit is rounded to bf16 first, as in a
+    bf16 load, whose router returns bf16 logits that the scoring casts to float32
+    ("The router renormalizes its top 2, in float32").
     """
     logits = to_f64(x) @ to_f64(w_router).T
+    if bf16_logits:
+        logits = round_bf16(logits)
     if logit_bias is not None:
         logits = logits + to_f64(logit_bias)[None, :]
     return logits
@@ -154,7 +158,7 @@ def swiglu_expert(x_rows: np.ndarray, w1_e, w3_e, w2_e, h_bf16: bool = False) ->
 
 
 def moe_layer(x, w_router, w1, w3, w2, k: int, residual=None, logit_bias=None,
-              mode: str = "exact", tokens=None) -> dict:
+              mode: str = "exact", tokens=None, bf16_logits: bool = False) -> dict:
     """The layer on tokens ``tokens`` (all tokens when None).
 
     Returns a dict of fp64 arrays over the chosen tokens: ``logits`` [n, E], ``idx``
@@ -170,7 +174,7 @@ def moe_layer(x, w_router, w1, w3, w2, k: int, residual=None, logit_bias=None,
         tokens = np.asarray(tokens, dtype=np.int64)
         xs = xs[tokens]
     n, hidden = xs.shape
-    logits = router_logits(xs, w_router, logit_bias)
+    logits = router_logits(xs, w_router, logit_bias, bf16_logits)
     idx, weights, _ = route_topk(logits, k)
     num_experts = logits.shape[1]
     y = np.zeros((n, k, hidden), dtype=np.float64)

@@ -102,6 +102,10 @@ moe_status_t check_shape(const moe_shape_t* sh, Shape* out) {
   out->E = sh->num_experts;
   out->k = sh->num_experts_per_tok;
   out->blocked = sh->weight_layout == MOE_WEIGHTS_BLOCKED;
+  if (sh->router_bf16_logits != 0 && sh->router_bf16_logits != 1)
+    return fail(MOE_ERR_INVALID_ARG, "router_bf16_logits must be 0 or 1 (got %d)",
+                sh->router_bf16_logits);
+  out->bf16_logits = sh->router_bf16_logits;
   const int64_t rmax = max_padded_rows(*out);
   if ((rmax / 128) * (int64_t)(out->I / 128) > INT32_MAX || (int64_t)out->E * out->I > INT32_MAX)
     return fail(MOE_ERR_UNSUPPORTED, "shape too large for 32-bit tile indices");

@@ -21,6 +21,7 @@ struct Shape {
   int64_t T;
   int H, I, E, k;
   int blocked;  // expert weights in the blocked layout
+  int bf16_logits;  // router logits rounded to bf16 before scoring
 };
 
 inline int64_t max_padded_rows(const Shape& s) {

@@ -7,6 +7,7 @@
 // them by their sum, slot 0 the larger ("The router renormalizes its top 2, in
 // float32"). The expert-contiguous row order is this library's own: stable on
 // (expert, token, slot), groups padded to 128 rows.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -66,7 +67,7 @@ __global__ void __launch_bounds__(256) k_router(const uint16_t* __restrict__ x,
                                                 float* __restrict__ w_out,
                                                 float* __restrict__ logits_out,
                                                 const uint16_t* __restrict__ norm_w, float eps,
-                                                float* __restrict__ rnorm_out) {
+                                                float* __restrict__ rnorm_out, int bf16_logits) {
   pdl_trigger();
   pdl_wait();
   constexpr int TOK_PER_CTA = 8 / S;
@@ -171,6 +172,7 @@ __global__ void __launch_bounds__(256) k_router(const uint16_t* __restrict__ x,
 #pragma unroll
             for (int w = 1; w < S; ++w) v += part[slot * S + w][e];
           }
+          if (bf16_logits) v = __bfloat162float(__float2bfloat16_rn(v));
           l[e] = v + (bias ? bias[e] : 0.f);
           mx = fmaxf(mx, l[e]);
           if (logits_out) logits_out[t * E + e] = l[e];
@@ -457,10 +459,10 @@ cudaError_t launch_router(const Shape& s, const uint16_t* x, const uint16_t* w_r
 #define MOE_ROUTER(EM, SS)                                                                    \
   err = norm_w ? launch_pdl(k_router<EM, SS, true>, dim3((unsigned)blocks), dim3(256), 0, st, x,  \
                             w_router, logit_bias, s.T, s.H, s.E, s.k, topk_idx, topk_w, logits, \
-                            norm_w, eps, rnorm)                                                 \
+                            norm_w, eps, rnorm, s.bf16_logits)                                  \
                : launch_pdl(k_router<EM, SS, false>, dim3((unsigned)blocks), dim3(256), 0, st, x, \
                             w_router, logit_bias, s.T, s.H, s.E, s.k, topk_idx, topk_w, logits, \
-                            norm_w, eps, rnorm)
+                            norm_w, eps, rnorm, s.bf16_logits)
 #define MOE_ROUTER_E(EM)           \
   switch (S) {                     \
     case 1: MOE_ROUTER(EM, 1); break; \

@@ -40,7 +40,8 @@ ROW_MAJOR, BLOCKED = 0, 1  # MOE_WEIGHTS_* layouts of the expert weights
 class Shape(ctypes.Structure):
     _fields_ = [("num_tokens", ctypes.c_int64), ("hidden_size", ctypes.c_int32),
                 ("intermediate_size", ctypes.c_int32), ("num_experts", ctypes.c_int32),
-                ("num_experts_per_tok", ctypes.c_int32), ("weight_layout", ctypes.c_int32)]
+                ("num_experts_per_tok", ctypes.c_int32), ("weight_layout", ctypes.c_int32),
+                ("router_bf16_logits", ctypes.c_int32)]
 
 
 _lib = None
@@ -103,9 +104,10 @@ def _check(status: int) -> None:
 
 
 def make_shape(num_tokens: int, hidden_size: int, intermediate_size: int, num_experts: int,
-               num_experts_per_tok: int, weight_layout: int = ROW_MAJOR) -> Shape:
+               num_experts_per_tok: int, weight_layout: int = ROW_MAJOR,
+               router_bf16_logits: bool = False) -> Shape:
     return Shape(int(num_tokens), int(hidden_size), int(intermediate_size), int(num_experts),
-                 int(num_experts_per_tok), int(weight_layout))
+                 int(num_experts_per_tok), int(weight_layout), int(bool(router_bf16_logits)))
 
 
 def _dev(t: Optional[torch.Tensor], name: str, dtype=None, nullable=False) -> Optional[int]:
@@ -147,11 +149,12 @@ def make_workspace(shape: Shape, device="cuda", host: bool = False) -> torch.Ten
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
-def router_topk(x, w_router, k: int, logit_bias=None, return_logits=False, stream=None):
+def router_topk(x, w_router, k: int, logit_bias=None, return_logits=False, stream=None,
+                router_bf16_logits: bool = False):
     """(topk_idx [T,k] int32, topk_w [T,k] fp32[, logits [T,E] fp32])."""
     t, h = x.shape
     e = w_router.shape[0]
-    shape = make_shape(t, h, ROW_PAD, e, k)
+    shape = make_shape(t, h, ROW_PAD, e, k, router_bf16_logits=router_bf16_logits)
     idx = torch.empty((t, k), dtype=torch.int32, device=x.device)
     w = torch.empty((t, k), dtype=torch.float32, device=x.device)
     logits = torch.empty((t, e), dtype=torch.float32, device=x.device) if return_logits else None
@@ -267,11 +270,11 @@ def combine(y_perm, row_of, topk_w, residual=None, num_experts: int = 8, interme
 
 
 def forward(x, w_router, w1, w3, w2, k: int, residual=None, logit_bias=None, ws=None, out=None,
-            stream=None, weight_layout: int = ROW_MAJOR):
+            stream=None, weight_layout: int = ROW_MAJOR, router_bf16_logits: bool = False):
     """The whole layer on device tensors; returns out [T,H] bf16."""
     t, h = x.shape
     e, i, _ = w1.shape
-    shape = make_shape(t, h, i, e, k, weight_layout)
+    shape = make_shape(t, h, i, e, k, weight_layout, router_bf16_logits)
     if ws is None:
         ws = make_workspace(shape, x.device)
     if out is None:

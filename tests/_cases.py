@@ -62,3 +62,48 @@ def sample_tokens(t_count: int, n: int = 256, seed: int = 1234) -> np.ndarray:
 
 def bf16_np(t: torch.Tensor) -> np.ndarray:
     return O.to_f64(t)
+
+
+def bf16_midpoint_distance(v: np.ndarray) -> np.ndarray:
+    """Distance of each fp64 value to the nearest half-way point between bf16 values."""
+    _, e = np.frexp(v)
+    q = np.ldexp(1.0, np.maximum(e, -125) - 8)
+    u = v / q
+    return np.abs((u - np.floor(u)) - 0.5) * q
+
+
+def decision_window(exact: np.ndarray, k: int) -> np.ndarray:
+    """Logits that can decide a bf16-logit top-k: the k largest and any within two bf16
+    steps below the k-th (the renormalised weights depend on the selected logits only)."""
+    kth = -np.sort(-exact, axis=1)[:, k - 1:k]
+    _, e = np.frexp(kth)
+    step = np.ldexp(1.0, np.maximum(e, -125) - 8)
+    return exact >= kth - 2 * step
+
+
+def screened_bf16_logits(w: W.Workload, device="cuda", max_attempts: int = 64):
+    """Inputs whose router logits all sit far enough from bf16 rounding half-way points
+    that the GPU's fp32 sum and the exact sum round to the same bf16 value (redrawing
+    x rows that do not). Returns (LayerInputs on device, rows still failing)."""
+    wr, w1, w3, w2 = W.draw_weights(w, device)
+    wr_c = wr.cpu()
+    x = W.draw_x(w, "cpu")
+    absw = np.abs(O.to_f64(wr_c)).T
+
+    def bad_rows(xs):
+        exact = O.to_f64(xs) @ O.to_f64(wr_c).T
+        bound = 1e-5 * (np.abs(O.to_f64(xs)) @ absw) + 1e-6
+        near = bf16_midpoint_distance(exact) <= bound
+        return np.nonzero((near & decision_window(exact, w.num_experts_per_tok)).any(axis=1))[0]
+
+    bad = bad_rows(x)
+    attempt = 0
+    while bad.size and attempt < max_attempts:
+        attempt += 1
+        rows = torch.from_numpy(bad.astype(np.int64))
+        x[rows] = W.redraw_x_rows(w, rows, attempt)
+        still = bad_rows(x[rows])
+        bad = bad[still]
+    res = W.synth.normal_rows_unit_rms(w.num_tokens, w.hidden_size, w.seed, W.RESIDUAL_ID, 0, "cpu")
+    inp = W.LayerInputs(x.to(device), wr, w1, w3, w2, res.to(device), None)
+    return inp, torch.from_numpy(bad.astype(np.int64))

@@ -315,3 +315,16 @@ def test_block_is_residual_plus_layer_on_normed_input():
     sub = O.moe_block(res, g, 1e-5, wr, w1, w3, w2, 2, mode="bf16_storage", tokens=[1, 4])
     full = O.moe_block(res, g, 1e-5, wr, w1, w3, w2, 2, mode="bf16_storage")
     assert np.array_equal(sub["out"], full["out"][[1, 4]])
+
+
+def test_bf16_logits_round_before_scoring_and_ties_go_low():
+    # exact logits 1.001, 1.003, 0.5: as bf16 (spacing 2^-7 at 1) the first two are both
+    # 1.0, a tie that goes to the lower expert with equal weights; in fp32 expert 1 wins
+    x = np.array([[1.0, 0.0, 0.0]])
+    wr = np.array([[1.001, 0, 0], [1.003, 0, 0], [0.5, 0, 0]]).astype(np.float64)
+    lb = O.router_logits(x, wr, bf16_logits=True)
+    assert lb.tolist() == [[1.0, 1.0, 0.5]]
+    idx, w, _ = O.route_topk(lb, 2)
+    assert idx.tolist() == [[0, 1]] and np.allclose(w, [[0.5, 0.5]], rtol=0, atol=0)
+    idx32, _, _ = O.route_topk(O.router_logits(x, wr), 2)
+    assert idx32.tolist() == [[1, 0]]
