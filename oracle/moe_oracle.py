@@ -45,7 +45,7 @@ import numpy as np
 
 __all__ = [
     "to_f64", "round_bf16", "silu", "router_logits", "route_topk", "stable_permute",
-    "swiglu_expert", "moe_layer", "rms_norm", "moe_block",
+    "swiglu_expert", "moe_layer", "rms_norm", "moe_block", "quantize_int8_rows",
 ]
 
 
@@ -229,3 +229,23 @@ def moe_block(h, norm_weight, eps: float, w_router, w1, w3, w2, k: int, logit_bi
     r = moe_layer(x, w_router, w1, w3, w2, k, residual=hs, logit_bias=logit_bias, mode=mode)
     r["x_norm"] = x
     return r
+
+
+def quantize_int8_rows(w):
+    """Symmetric per-row int8 codes of a weight matrix (or a stack of them).
+
+    The pages load Mixtral in int8 or 4 bits to shrink its ~90 GB of bf16 weights
+    (Hugging Face "Mixtral" doc, "Shrinking down Mixtral using quantization"; "Welcome
+    Mixtral", "Quantizing Mixtral") but leave the scheme to the quantisation library.
+    This is the plain weight-only scheme: for every output row (channel), scale s =
+    max|w| / 127 and code q = round-half-even(w / s), so w ~ q * s with |w - q s| <= s/2.
+    The code is an integer that floating point decides, so it is decided in float32 (s
+    and w / s correctly rounded in float32, as the kernel does); an all-zero row has
+    s = 1 and q = 0. Returns (q int8 array, s float32 array [..., rows]).
+    """
+    w = np.asarray(to_f64(w), dtype=np.float32)
+    amax = np.abs(w).max(axis=-1)
+    s = np.where(amax > 0, amax / np.float32(127.0), np.float32(1.0)).astype(np.float32)
+    q = np.rint(w / s[..., None]).astype(np.float32)
+    q = np.clip(q, -127, 127).astype(np.int8)
+    return q, s

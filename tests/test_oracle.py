@@ -328,3 +328,34 @@ def test_bf16_logits_round_before_scoring_and_ties_go_low():
     assert idx.tolist() == [[0, 1]] and np.allclose(w, [[0.5, 0.5]], rtol=0, atol=0)
     idx32, _, _ = O.route_topk(O.router_logits(x, wr), 2)
     assert idx32.tolist() == [[1, 0]]
+
+
+# ---------------------------------------------------------------- int8 weight-only codes
+
+def test_int8_rows_bounds_and_extremes():
+    rng = np.random.default_rng(12)
+    w = O.round_bf16(rng.standard_normal((3, 40, 64)) / 8)
+    w[1, 5] = 0.0                                   # an all-zero row
+    q, s = O.quantize_int8_rows(w)
+    assert q.dtype == np.int8 and s.dtype == np.float32 and s.shape == (3, 40)
+    assert q.min() >= -127 and q.max() <= 127
+    deq = q.astype(np.float64) * s[..., None].astype(np.float64)
+    # |w - q s| <= s / 2, plus the float32 rounding of w / s (<= 127 * 2^-24 of s)
+    assert np.all(np.abs(w - deq) <= s[..., None] * (0.5 + 127 * 2.0 ** -23))
+    # the largest |w| of every non-zero row maps to +-127
+    amax_idx = np.abs(w).argmax(-1)
+    top = np.take_along_axis(q, amax_idx[..., None], -1)[..., 0]
+    nz = np.abs(w).max(-1) > 0
+    assert np.all(np.abs(top[nz]) == 127)
+    assert np.all(q[1, 5] == 0) and s[1, 5] == 1.0
+
+
+def test_int8_codes_match_torch_float32_arithmetic():
+    # same decision in float32 with torch's own ops: amax / 127, w / s, round half even
+    rng = np.random.default_rng(13)
+    w = O.round_bf16(rng.standard_normal((64, 96)) * 0.05)
+    q, s = O.quantize_int8_rows(w)
+    wt = torch.from_numpy(w).float()
+    st = wt.abs().amax(-1) / 127.0
+    qt = torch.round(wt / st[:, None]).clamp(-127, 127).to(torch.int8)
+    assert np.array_equal(s, st.numpy()) and np.array_equal(q, qt.numpy())
