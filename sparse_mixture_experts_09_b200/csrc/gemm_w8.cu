@@ -1,0 +1,699 @@
+// Weight-only int8 experts (W8A16): the grouped GEMMs with int8 weight codes and one
+// fp32 scale per output channel.
+//
+// Mixtral is loaded weight-only quantised to shrink it (Hugging Face "Mixtral" doc,
+// "Shrinking down Mixtral using quantization"; ZeroModels "Mixtral", "Lower memory":
+// int8 weights with bf16 activations). At decode the layer streams every active
+// expert's weights, so halving their bytes can halve the time.
+// Scheme (the pages do not fix one): per output row (channel) r, s[r] = max|w[r, :]| /
+// 127 and q = rint(w / s), decided in float32; w ~ q * s. Every int8 value is exactly a
+// bf16 value, so the tensor cores multiply the bf16 activations by the codes widened
+// to bf16 (exact), and the scale, constant along K, multiplies the fp32 accumulator in
+// the epilogue: sum_k x[k] q[r,k] s[r] = s[r] * sum_k x[k] q[r,k].
+//
+// Kernel: the bf16 kernel's persistent tile loop with a widening stage. Warp roles:
+//   warp 0      streams the int8 tiles (bulk copies: in the blocked code layout each
+//               128-row x 64-code tile is one contiguous 8 KiB run) into a code ring;
+//   warp 6      loads the activation tiles (TMA, 128-byte swizzle) into the main ring;
+//   warps 7..   widen each code tile to bf16 and store it, 128-byte swizzled, as the
+//               B operand of the main ring;
+//   warp 1      issues tcgen05.mma into a double-buffered TMEM accumulator;
+//   warps 2-5   scale, activate and store (epilogue).
+// Every wait is bounded (timeout -> status word, abort flag, drained copies).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128, BK = 64;
+#ifndef MOE_W8_A_STAGES
+#define MOE_W8_A_STAGES 4
+#endif
+#ifndef MOE_W8_B_STAGES
+#define MOE_W8_B_STAGES 3
+#endif
+#ifndef MOE_W8_CODE_STAGES
+#define MOE_W8_CODE_STAGES 4
+#endif
+#ifndef MOE_W8_CONV_WARPS
+#define MOE_W8_CONV_WARPS 8
+#endif
+// Three rings: activation tiles (TMA -> MMA), int8 code tiles (TMA -> converters) and
+// widened weight tiles (converters -> MMA). The activation ring is deep enough to hide
+// its L2 latency on its own; the widened ring only decouples widening from the MMA.
+constexpr int kAStages = MOE_W8_A_STAGES;
+constexpr int kBStages = MOE_W8_B_STAGES;
+constexpr int kCodeStages = MOE_W8_CODE_STAGES;
+constexpr int kConvWarps = MOE_W8_CONV_WARPS;
+#ifndef MOE_W8_SUSPEND_NS
+#define MOE_W8_SUSPEND_NS 20000
+#endif
+// Suspend limit of one try_wait in the waiting loop: a waiting warp issues no
+// instructions while it sleeps, leaving the issue slots to the converters. The abort
+// flag and the timeout are checked every 64 tries, i.e. at least every 64 limits.
+constexpr uint32_t kSuspendNs = MOE_W8_SUSPEND_NS;
+// warp 0: code TMA, 1: MMA, 2-5: epilogue, 6: activation TMA, 7..: converters
+constexpr int kConvWarp0 = 7;
+constexpr int kThreadsW8 = 32 * (kConvWarp0 + kConvWarps);
+constexpr int A_BYTES = BM * BK * 2;  // 16 KiB
+constexpr int kSwiGLU = 0, kPlain = 1;
+constexpr int kNumBars = 2 * (kAStages + kBStages + kCodeStages) + 5;
+
+// Per-BN shared-memory plan: [A ring][B ring][code ring][barriers, TMEM address, row tiles]
+template <int BN>
+struct TileW8 {
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int Q_BYTES = BN * BK;
+  static constexpr int B_OFF = kAStages * A_BYTES;
+  static constexpr int Q_OFF = B_OFF + kBStages * B_BYTES;
+  static constexpr int BAR_OFF = Q_OFF + kCodeStages * Q_BYTES;
+  static constexpr int SMEM = 1024 + BAR_OFF + kNumBars * 8 + 8 + 65 * 4;
+  static constexpr int CHUNKS = BN * BK / 16 / (32 * kConvWarps);  // code chunks per thread
+  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
+                                    ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+  static_assert(SMEM <= 232448, "shared memory plan exceeds 227 KiB");
+  static_assert(CHUNKS * 32 * kConvWarps * 16 == BN * BK, "converter split");
+};
+
+struct W8Params {
+  const int8_t* q0;      // blocked codes of the first weight (w1 or w2)
+  const int8_t* q1;      // blocked codes of w3 (gate/up only)
+  const int32_t* offsets;
+  const float* scale_a;  // per-row scales of the first weight (w1 or w2) [E * rows]
+  const float* scale_b;  // per-row scales of w3 (gate/up only)
+  int32_t* status;
+  void* out;
+  int64_t out_ld;
+  int E, k_blocks, n_tiles, b_rows;
+  unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// try_wait with an explicit suspend-time limit: a thread whose phase is not complete
+// sleeps in hardware until the phase completes or `ns` elapse, instead of re-polling.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+// Contiguous global -> shared copy of `bytes` (multiple of 16, both ends 16-byte aligned),
+// completing on the mbarrier's transaction count.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Bounded wait on an mbarrier phase (see the bf16 kernel): false after the CTA aborted
+// or after timeout_ns, which it records as kStatusTimeout.
+__device__ __noinline__ bool wait_w8(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                     int32_t* status, unsigned long long timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+    if ((n & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > timeout_ns) {
+        *abort_flag = 1;
+        atomicOr(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// The same wait executed by all 32 lanes of a warp (they stay converged): an inline
+// first test, then the bounded loop.
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int32_t* status, unsigned long long timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_w8(bar, parity, abort_flag, status, timeout_ns);
+}
+
+__device__ __noinline__ void drain_w8(uint32_t bar, uint32_t parity, unsigned long long timeout_ns) {
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > timeout_ns) return;
+  }
+}
+
+__device__ __forceinline__ void tile_coords_w8(int L, const int* row_tiles, int E, int n_tiles,
+                                               int& e, int& m, int& n) {
+  const int mrow = L / n_tiles;
+  e = 0;
+  while (e + 1 < E && row_tiles[e + 1] <= mrow) ++e;
+  const int cnt = row_tiles[e + 1] - row_tiles[e];
+  const int local = L - row_tiles[e] * n_tiles;
+  n = local / cnt;
+  m = row_tiles[e] + local % cnt;
+}
+
+// y coordinate of weight row `row` (multiple of 128), k-block kb, in the blocked code map
+__device__ __forceinline__ int code_y(int row, int kb, int k_blocks) {
+  return ((row >> 7) * k_blocks + kb) * 128;
+}
+
+// Two int8 codes (bytes a, b of a 32-bit word, placed in the low bytes of the two
+// 16-bit halves by a byte permute) -> bf16x2, exactly. With l = the code's low 7 bits
+// and t = its sign bit, the bf16 bit pattern 0x4300 | l is 128 + l and 0x4300 | t << 7
+// is 128 (t = 0) or 256 (t = 1); their difference is l - 128 t, the two's-complement
+// value, an integer in [-128, 127] and so exact in bf16.
+__device__ __forceinline__ uint32_t codes_to_bf16x2(uint32_t w, uint32_t sel) {
+  const uint32_t p = __byte_perm(w, 0u, sel);
+  const uint32_t x = (p & 0x007F007Fu) | 0x43004300u;
+  const uint32_t c = (p & 0x00800080u) | 0x43004300u;
+  uint32_t r;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(c));
+  return r;
+}
+
+// 16 codes (one uint4, columns 16v .. 16v+15) -> two 16-byte chunks of bf16
+__device__ __forceinline__ void widen16(const uint4 w4, uint4& lo8, uint4& hi8) {
+  lo8 = make_uint4(codes_to_bf16x2(w4.x, 0x4140u), codes_to_bf16x2(w4.x, 0x4342u),
+                   codes_to_bf16x2(w4.y, 0x4140u), codes_to_bf16x2(w4.y, 0x4342u));
+  hi8 = make_uint4(codes_to_bf16x2(w4.z, 0x4140u), codes_to_bf16x2(w4.z, 0x4342u),
+                   codes_to_bf16x2(w4.w, 0x4140u), codes_to_bf16x2(w4.w, 0x4342u));
+}
+
+// MODE kSwiGLU: A = x_perm [rows, H], weight tile = 128 rows of w1 then 128 rows of w3
+//   (BN = 256), h = bf16(silu(s1 * gate) * (s3 * up)).
+// MODE kPlain:  A = h [rows, I], weight tile = BN rows of w2, y = s2 * acc (fp32).
+template <int MODE, int BN>
+__global__ void __launch_bounds__(kThreadsW8, 1)
+    k_grouped_gemm_w8(const __grid_constant__ CUtensorMap mapA, const W8Params p) {
+  using TL = TileW8<BN>;
+  static_assert(MODE == kPlain || BN == 256, "gate/up tiles hold 128 gate + 128 up columns");
+  constexpr uint32_t kTmemCols = 2 * BN;  // two accumulators
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint8_t* bbase = smem + TL::B_OFF;
+  uint8_t* qbase = smem + TL::Q_OFF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TL::BAR_OFF);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* row_tiles = reinterpret_cast<int*>(tmem_holder + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // barriers: a_full, a_empty [kAStages]; b_full, b_empty [kBStages]; q_full, q_empty
+  // [kCodeStages]; tfull, tempty [2]; final
+  const uint32_t bar0 = smem_u32(bars);
+  constexpr int kB0 = 2 * kAStages, kQ0 = kB0 + 2 * kBStages, kT0 = kQ0 + 2 * kCodeStages;
+  auto a_full = [&](int s) { return bar0 + 8u * s; };
+  auto a_empty = [&](int s) { return bar0 + 8u * (kAStages + s); };
+  auto b_full = [&](int s) { return bar0 + 8u * (kB0 + s); };
+  auto b_empty = [&](int s) { return bar0 + 8u * (kB0 + kBStages + s); };
+  auto q_full = [&](int q) { return bar0 + 8u * (kQ0 + q); };
+  auto q_empty = [&](int q) { return bar0 + 8u * (kQ0 + kCodeStages + q); };
+  auto tfull = [&](int a) { return bar0 + 8u * (kT0 + a); };
+  auto tempty = [&](int a) { return bar0 + 8u * (kT0 + 2 + a); };
+  const uint32_t final_bar = bar0 + 8u * (kT0 + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(a_full(s), 1);
+      mbar_init(a_empty(s), 1);
+    }
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(b_full(s), kConvWarps);
+      mbar_init(b_empty(s), 1);
+    }
+    for (int q = 0; q < kCodeStages; ++q) {
+      mbar_init(q_full(q), 1);
+      mbar_init(q_empty(q), kConvWarps);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull(a), 1);
+      mbar_init(tempty(a), 4);
+    }
+    mbar_init(final_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  pdl_trigger();
+  pdl_wait();
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) row_tiles[i] = p.offsets[i] / BM;
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int total = row_tiles[p.E] * p.n_tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- int8 code stream: BN/128 boxes of 128 rows x 64 codes
+      int it = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        int e, m, n;
+        tile_coords_w8(L, row_tiles, p.E, p.n_tiles, e, m, n);
+        const int row0 = MODE == kSwiGLU ? e * p.b_rows + n * 128 : e * p.b_rows + n * BN;
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int q = it % kCodeStages;
+          const uint32_t ph = (uint32_t)(it / kCodeStages) & 1u;
+          if (!wait_w8(q_empty(q), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dq = smem_u32(qbase + q * TL::Q_BYTES);
+          mbar_expect_tx(q_full(q), TL::Q_BYTES);
+          if (MODE == kSwiGLU) {
+            const size_t off = (size_t)code_y(row0, kb, p.k_blocks) * BK;
+            bulk_load(dq, p.q0 + off, 128 * BK, q_full(q));
+            bulk_load(dq + 128 * BK, p.q1 + off, 128 * BK, q_full(q));
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 128; ++j)
+              bulk_load(dq + j * 128 * BK,
+                        p.q0 + (size_t)code_y(row0 + 128 * j, kb, p.k_blocks) * BK, 128 * BK,
+                        q_full(q));
+          }
+        }
+      }
+      if (!ok) {
+        const int first = it > kCodeStages ? it - kCodeStages : 0;
+        for (int i = first; i < it; ++i)
+          drain_w8(q_full(i % kCodeStages), (uint32_t)(i / kCodeStages) & 1u, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      int it = 0, tc = 0;
+      bool ok = true, issued = false;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tc) {
+        const int a = tc & 1;
+        const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
+        if (!wait_w8(tempty(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
+        fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(a * BN);
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int sa = it % kAStages, sb = it % kBStages;
+          if (!wait_w8(a_full(sa), (uint32_t)(it / kAStages) & 1u, abort_flag, p.status,
+                       p.timeout_ns) ||
+              !wait_w8(b_full(sb), (uint32_t)(it / kBStages) & 1u, abort_flag, p.status,
+                       p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          const uint32_t da = smem_u32(smem + sa * A_BYTES);
+          const uint32_t db = smem_u32(bbase + sb * TL::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_bf16(d, sdesc(da + kk * 32), sdesc(db + kk * 32), TL::IDESC, (kb | kk) ? 1u : 0u);
+          mma_commit(a_empty(sa));
+          mma_commit(b_empty(sb));
+          issued = true;
+        }
+        if (ok) mma_commit(tfull(a));
+      }
+      if (issued) {
+        mma_commit(final_bar);
+        drain_w8(final_bar, 0, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    if (lane == 0) {
+      // ---------------- activation tiles (bf16, 128-byte swizzle by the TMA)
+      int it = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        int e, m, n;
+        tile_coords_w8(L, row_tiles, p.E, p.n_tiles, e, m, n);
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int sa = it % kAStages;
+          const uint32_t ph = (uint32_t)(it / kAStages) & 1u;
+          if (!wait_w8(a_empty(sa), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(a_full(sa), A_BYTES);
+          tma_load_2d(smem_u32(smem + sa * A_BYTES), &mapA, kb * BK, m * BM, a_full(sa));
+        }
+      }
+      if (!ok) {
+        const int first = it > kAStages ? it - kAStages : 0;
+        for (int i = first; i < it; ++i)
+          drain_w8(a_full(i % kAStages), (uint32_t)(i / kAStages) & 1u, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= kConvWarp0) {
+    // ---------------- converters: int8 code tile -> bf16 B tile in the 128-byte
+    // swizzled K-major layout (row r: 128 bytes at r * 128, 16-byte chunk c stored at
+    // chunk position c ^ (r & 7)). Thread ct widens the 16-byte code chunks
+    // j = ct + 32 kConvWarps i (row j / 4, columns 16 (j % 4) ..): consecutive threads
+    // read consecutive chunks, and the 8 stores of a quarter-warp land in distinct
+    // banks.
+    const int ct = threadIdx.x - kConvWarp0 * 32;
+    int it = 0;
+    bool ok = true;
+    for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+      for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+        const int q = it % kCodeStages, sb = it % kBStages;
+        if (!wait_warp(q_full(q), (uint32_t)(it / kCodeStages) & 1u, abort_flag, p.status,
+                       p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        const uint4* qs = reinterpret_cast<const uint4*>(qbase + q * TL::Q_BYTES);
+        uint4 v[TL::CHUNKS];
+#pragma unroll
+        for (int i = 0; i < TL::CHUNKS; ++i) v[i] = qs[ct + 32 * kConvWarps * i];
+        if (!wait_warp(b_empty(sb), ((uint32_t)(it / kBStages) & 1u) ^ 1u, abort_flag, p.status,
+                       p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        uint8_t* bs = bbase + sb * TL::B_BYTES;
+#pragma unroll
+        for (int i = 0; i < TL::CHUNKS; ++i) {
+          const int j = ct + 32 * kConvWarps * i;
+          const int r = j >> 2, c = (j & 3) * 2;
+          uint4 lo8, hi8;
+          widen16(v[i], lo8, hi8);
+          uint8_t* row = bs + r * 128;
+          *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = lo8;
+          *reinterpret_cast<uint4*>(row + (((c + 1) ^ (r & 7)) << 4)) = hi8;
+        }
+        // make the generic-proxy stores visible to the tensor cores (async proxy)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        // The code stage is released only now: the stores consumed every loaded chunk,
+        // so no read of it is still in flight when the next TMA load overwrites it.
+        if (lane == 0) {
+          mbar_arrive(b_full(sb));
+          mbar_arrive(q_empty(q));
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5, TMEM lanes 32 (warp % 4) ..
+    const int qd = warp & 3;
+    const int row_in_tile = qd * 32 + lane;
+    int tc = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x, ++tc) {
+      int e, m, n;
+      tile_coords_w8(L, row_tiles, p.E, p.n_tiles, e, m, n);
+      const int a = tc & 1;
+      const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
+      if (!wait_warp(tfull(a), aph, abort_flag, p.status, p.timeout_ns)) break;
+      fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(qd * 32) << 16) + (uint32_t)(a * BN);
+      const int64_t row = (int64_t)m * BM + row_in_tile;
+      if (MODE == kSwiGLU) {
+        const float* sg = p.scale_a + (size_t)e * p.b_rows + n * 128;
+        const float* su = p.scale_b + (size_t)e * p.b_rows + n * 128;
+        uint16_t* h = reinterpret_cast<uint16_t*>(p.out) + row * p.out_ld + (int64_t)n * 128;
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 16) {
+          uint32_t g[16], u[16];
+          tmem_ld16(taddr + c, g);
+          tmem_ld16(taddr + 128 + c, u);
+          tmem_wait_ld();
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float g0 = __uint_as_float(g[2 * i]) * __ldg(sg + c + 2 * i);
+            const float g1 = __uint_as_float(g[2 * i + 1]) * __ldg(sg + c + 2 * i + 1);
+            const float u0 = __uint_as_float(u[2 * i]) * __ldg(su + c + 2 * i);
+            const float u1 = __uint_as_float(u[2 * i + 1]) * __ldg(su + c + 2 * i + 1);
+            pk[i] = pack_bf16x2_rn(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(h + c);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+      } else {
+        const float* sc = p.scale_a + (size_t)e * p.b_rows + n * BN;
+        float* y = reinterpret_cast<float*>(p.out) + row * p.out_ld + (int64_t)n * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(taddr + c, v);
+          tmem_wait_ld();
+          float4* dst = reinterpret_cast<float4*>(y + c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_float4(__uint_as_float(v[4 * i]) * __ldg(sc + c + 4 * i),
+                                 __uint_as_float(v[4 * i + 1]) * __ldg(sc + c + 4 * i + 1),
+                                 __uint_as_float(v[4 * i + 2]) * __ldg(sc + c + 4 * i + 2),
+                                 __uint_as_float(v[4 * i + 3]) * __ldg(sc + c + 4 * i + 3));
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty(a));
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// One warp per weight row: s = max|w| / 127, q = rint(w / s) in float32, written in
+// the blocked code layout [rows/128][K/64][128][64].
+__global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__ w,
+                                                    int8_t* __restrict__ q, float* __restrict__ s,
+                                                    int64_t rows, int K) {
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int kbn = K / BK;
+  for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
+       r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    const uint16_t* wr = w + r * K;
+    float amax = 0.f;
+    for (int c = lane; c < K; c += 32) amax = fmaxf(amax, fabsf(__uint_as_float((uint32_t)wr[c] << 16)));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const float sc = amax > 0.f ? __fdiv_rn(amax, 127.f) : 1.f;
+    if (lane == 0) s[r] = sc;
+    const int64_t rb = r >> 7, rr = r & 127;
+    for (int c = lane; c < K; c += 32) {
+      const float v = __uint_as_float((uint32_t)wr[c] << 16);
+      int qi = __float2int_rn(__fdiv_rn(v, sc));
+      qi = qi > 127 ? 127 : (qi < -127 ? -127 : qi);
+      const int64_t kb = c / BK, cc = c % BK;
+      q[((rb * kbn + kb) * 128 + rr) * BK + cc] = (int8_t)qi;
+    }
+  }
+}
+
+typedef CUresult (*EncodeTiledFnW8)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFnW8 encode_w8() {
+  static EncodeTiledFnW8 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                         &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFnW8>(f);
+  }
+  return fn;
+}
+
+// bf16 activations [rows, inner], box 64 x 128, 128-byte swizzle
+bool map_act(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
+  EncodeTiledFnW8 fn = encode_w8();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE, int BN>
+cudaError_t launch_w8(const CUtensorMap& a, const W8Params& p, int64_t max_tiles,
+                      cudaStream_t st) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm_w8<MODE, BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         TileW8<BN>::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  int64_t grid = num_sms();
+  if (grid > max_tiles) grid = max_tiles;
+  if (grid < 1) grid = 1;
+  return launch_pdl(k_grouped_gemm_w8<MODE, BN>, dim3((unsigned)grid), dim3(kThreadsW8),
+                    (size_t)TileW8<BN>::SMEM, st, a, p);
+}
+
+}  // namespace
+
+cudaError_t launch_quant_rows(const uint16_t* w, int8_t* q, float* s, int64_t rows, int K,
+                              cudaStream_t st) {
+  int64_t blocks = (rows + 7) / 8;
+  const int64_t cap = (int64_t)num_sms() * 16;
+  if (blocks > cap) blocks = cap;
+  return launch_pdl(k_quant_rows, dim3((unsigned)blocks), dim3(256), 0, st, w, q, s, rows, K);
+}
+
+cudaError_t launch_grouped_swiglu_w8(const Shape& s, const GemmArgsW8& g, cudaStream_t st,
+                                     const char** why) {
+  CUtensorMap mx, mh;
+  if (!map_act(&mx, g.a, s.H, g.rmax) || !map_act(&mh, g.h, s.I, g.rmax)) {
+    *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad tensor)";
+    return cudaErrorInvalidValue;
+  }
+  const int64_t mt_max = g.rmax / BM;
+  W8Params p1;
+  p1.q0 = g.q1;
+  p1.q1 = g.q3;
+  p1.offsets = g.offsets;
+  p1.scale_a = g.s1;
+  p1.scale_b = g.s3;
+  p1.status = g.status;
+  p1.out = g.h;
+  p1.out_ld = s.I;
+  p1.E = s.E;
+  p1.k_blocks = s.H / BK;
+  p1.n_tiles = s.I / 128;
+  p1.b_rows = s.I;
+  p1.timeout_ns = g.timeout_ns;
+  cudaError_t e = launch_w8<kSwiGLU, 256>(mx, p1, mt_max * p1.n_tiles, st);
+  if (e != cudaSuccess) {
+    *why = "int8 gate/up GEMM launch failed";
+    return e;
+  }
+  W8Params p2 = p1;
+  p2.q0 = g.q2;
+  p2.q1 = nullptr;
+  p2.scale_a = g.s2;
+  p2.scale_b = nullptr;
+  p2.out = g.y;
+  p2.out_ld = s.H;
+  p2.k_blocks = s.I / BK;
+  p2.b_rows = s.H;
+  if (s.H % 256 == 0) {
+    p2.n_tiles = s.H / 256;
+    e = launch_w8<kPlain, 256>(mh, p2, mt_max * p2.n_tiles, st);
+  } else {
+    p2.n_tiles = s.H / 128;
+    e = launch_w8<kPlain, 128>(mh, p2, mt_max * p2.n_tiles, st);
+  }
+  if (e != cudaSuccess) *why = "int8 down GEMM launch failed";
+  return e;
+}
+
+}  // namespace moe

@@ -142,10 +142,75 @@ T* at(void* ws, size_t off) {
 
 constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per wait
 
+// Expert weights of one layer: bf16 (w1, w3, w2), or int8 codes with per-row scales
+// (q1 non-null).
+struct Experts {
+  const uint16_t *w1, *w3, *w2;
+  const int8_t *q1, *q3, *q2;
+  const float *s1, *s3, *s2;
+};
+
+Experts bf16_experts(const uint16_t* w1, const uint16_t* w3, const uint16_t* w2) {
+  Experts x = {};
+  x.w1 = w1;
+  x.w3 = w3;
+  x.w2 = w2;
+  return x;
+}
+
+Experts int8_experts(const int8_t* q1, const int8_t* q3, const int8_t* q2, const float* s1,
+                     const float* s3, const float* s2) {
+  Experts x = {};
+  x.q1 = q1;
+  x.q3 = q3;
+  x.q2 = q2;
+  x.s1 = s1;
+  x.s3 = s3;
+  x.s2 = s2;
+  return x;
+}
+
+moe_status_t run_experts(const Shape& s, const uint16_t* x_perm, const int32_t* offsets,
+                         const Experts& w, uint16_t* h, float* y, int32_t* status,
+                         cudaStream_t st) {
+  const char* why = "";
+  cudaError_t e;
+  if (w.q1) {
+    GemmArgsW8 g;
+    g.a = x_perm;
+    g.offsets = offsets;
+    g.q1 = w.q1;
+    g.q3 = w.q3;
+    g.q2 = w.q2;
+    g.s1 = w.s1;
+    g.s3 = w.s3;
+    g.s2 = w.s2;
+    g.h = h;
+    g.y = y;
+    g.status = status;
+    g.rmax = max_padded_rows(s);
+    g.timeout_ns = kTimeoutNs;
+    e = launch_grouped_swiglu_w8(s, g, st, &why);
+  } else {
+    GemmArgs g;
+    g.a = x_perm;
+    g.offsets = offsets;
+    g.w1 = w.w1;
+    g.w3 = w.w3;
+    g.w2 = w.w2;
+    g.h = h;
+    g.y = y;
+    g.status = status;
+    g.rmax = max_padded_rows(s);
+    g.timeout_ns = kTimeoutNs;
+    e = launch_grouped_swiglu(s, g, st, &why);
+  }
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, why);
+}
+
 moe_status_t run_forward(const Shape& s, const uint16_t* x, const uint16_t* wr, const float* bias,
-                         const uint16_t* w1, const uint16_t* w3, const uint16_t* w2,
-                         const uint16_t* res, uint16_t* out, void* ws, cudaStream_t st,
-                         const uint16_t* norm_w = nullptr, float eps = 0.f) {
+                         const Experts& w, const uint16_t* res, uint16_t* out, void* ws,
+                         cudaStream_t st, const uint16_t* norm_w = nullptr, float eps = 0.f) {
   const Layout L = layout(s);
   float* rnorm = norm_w ? at<float>(ws, L.rnorm) : nullptr;
   cudaError_t e = launch_router(s, x, wr, bias, at<int32_t>(ws, L.topk_idx), at<float>(ws, L.topk_w),
@@ -156,20 +221,8 @@ moe_status_t run_forward(const Shape& s, const uint16_t* x, const uint16_t* wr, 
                      at<int32_t>(ws, L.token_of_row), at<uint16_t>(ws, L.x_perm),
                      at<int32_t>(ws, L.block_base), st, norm_w, rnorm);
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
-  GemmArgs g;
-  g.a = at<uint16_t>(ws, L.x_perm);
-  g.offsets = at<int32_t>(ws, L.offsets);
-  g.w1 = w1;
-  g.w3 = w3;
-  g.w2 = w2;
-  g.h = at<uint16_t>(ws, L.h);
-  g.y = at<float>(ws, L.y);
-  g.status = at<int32_t>(ws, L.status);
-  g.rmax = max_padded_rows(s);
-  g.timeout_ns = kTimeoutNs;
-  const char* why = "";
-  e = launch_grouped_swiglu(s, g, st, &why);
-  if (e != cudaSuccess) return cuda_fail(e, why);
+  MOE_TRY(run_experts(s, at<uint16_t>(ws, L.x_perm), at<int32_t>(ws, L.offsets), w,
+                      at<uint16_t>(ws, L.h), at<float>(ws, L.y), at<int32_t>(ws, L.status), st));
   e = launch_combine(s, at<float>(ws, L.y), at<int32_t>(ws, L.row_of), at<float>(ws, L.topk_w), res,
                      out, st);
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
@@ -263,20 +316,8 @@ moe_status_t moe_grouped_swiglu(const moe_shape_t* shape, const moe_bf16_t* x_pe
   MOE_TRY(check_ptr(y_perm, "y_perm"));
   const Layout L = layout(s);
   MOE_TRY(check_ws(ws, ws_bytes, L.end));
-  GemmArgs g;
-  g.a = x_perm;
-  g.offsets = expert_offsets;
-  g.w1 = w1;
-  g.w3 = w3;
-  g.w2 = w2;
-  g.h = at<uint16_t>(ws, L.h);
-  g.y = y_perm;
-  g.status = at<int32_t>(ws, L.status);
-  g.rmax = max_padded_rows(s);
-  g.timeout_ns = kTimeoutNs;
-  const char* why = "";
-  cudaError_t e = launch_grouped_swiglu(s, g, (cudaStream_t)stream, &why);
-  return e == cudaSuccess ? MOE_OK : cuda_fail(e, why);
+  return run_experts(s, x_perm, expert_offsets, bf16_experts(w1, w3, w2), at<uint16_t>(ws, L.h),
+                     y_perm, at<int32_t>(ws, L.status), (cudaStream_t)stream);
 }
 
 moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* x_perm,
@@ -363,7 +404,7 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_bf16_t* x, const mo
   MOE_TRY(check_ptr(residual, "residual", true));
   MOE_TRY(check_ptr(out, "out"));
   MOE_TRY(check_ws(ws, ws_bytes, layout(s).end));
-  return run_forward(s, x, w_router, logit_bias, w1, w3, w2, residual, out, ws,
+  return run_forward(s, x, w_router, logit_bias, bf16_experts(w1, w3, w2), residual, out, ws,
                      (cudaStream_t)stream);
 }
 
@@ -385,8 +426,8 @@ moe_status_t moe_forward_rmsnorm(const moe_shape_t* shape, const moe_bf16_t* h,
   MOE_TRY(check_ptr(w2, "w2"));
   MOE_TRY(check_ptr(out, "out"));
   MOE_TRY(check_ws(ws, ws_bytes, layout(s).end));
-  return run_forward(s, h, w_router, logit_bias, w1, w3, w2, h, out, ws, (cudaStream_t)stream,
-                     norm_weight, eps);
+  return run_forward(s, h, w_router, logit_bias, bf16_experts(w1, w3, w2), h, out, ws,
+                     (cudaStream_t)stream, norm_weight, eps);
 }
 
 moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_bf16_t* x_host,
@@ -417,7 +458,7 @@ moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_bf16_t* x_host
     e = cudaMemcpyAsync(rd, residual_host, bytes, cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(e, "copy of residual to the device");
   }
-  MOE_TRY(run_forward(s, xd, w_router, logit_bias, w1, w3, w2, rd, od, ws, st));
+  MOE_TRY(run_forward(s, xd, w_router, logit_bias, bf16_experts(w1, w3, w2), rd, od, ws, st));
   e = cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, st);
   if (e != cudaSuccess) return cuda_fail(e, "copy of out to the host");
   e = cudaStreamSynchronize(st);
@@ -471,6 +512,77 @@ moe_status_t moe_device_status(void* ws, size_t ws_bytes, moe_stream_t stream) {
     return fail(MOE_ERR_TIMEOUT, "a kernel gave up a bounded wait (device status 0x%x)",
                 (unsigned)word);
   return fail(MOE_ERR_CUDA, "unknown device status 0x%x", (unsigned)word);
+}
+
+moe_status_t moe_quantize_int8(const moe_shape_t* shape, const moe_bf16_t* w1,
+                               const moe_bf16_t* w3, const moe_bf16_t* w2, int8_t* q1, int8_t* q3,
+                               int8_t* q2, float* s1, float* s3, float* s2, moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(w1, "w1"));
+  MOE_TRY(check_ptr(w3, "w3"));
+  MOE_TRY(check_ptr(w2, "w2"));
+  MOE_TRY(check_ptr(q1, "q1"));
+  MOE_TRY(check_ptr(q3, "q3"));
+  MOE_TRY(check_ptr(q2, "q2"));
+  MOE_TRY(check_ptr(s1, "s1"));
+  MOE_TRY(check_ptr(s3, "s3"));
+  MOE_TRY(check_ptr(s2, "s2"));
+  cudaStream_t st = (cudaStream_t)stream;
+  const int64_t ei = (int64_t)s.E * s.I, eh = (int64_t)s.E * s.H;
+  cudaError_t e = launch_quant_rows(w1, q1, s1, ei, s.H, st);
+  if (e == cudaSuccess) e = launch_quant_rows(w3, q3, s3, ei, s.H, st);
+  if (e == cudaSuccess) e = launch_quant_rows(w2, q2, s2, eh, s.I, st);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "int8 quantiser launch");
+}
+
+moe_status_t moe_grouped_swiglu_w8(const moe_shape_t* shape, const moe_bf16_t* x_perm,
+                                   const int32_t* expert_offsets, const int8_t* q1,
+                                   const int8_t* q3, const int8_t* q2, const float* s1,
+                                   const float* s3, const float* s2, float* y_perm, void* ws,
+                                   size_t ws_bytes, moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(x_perm, "x_perm"));
+  MOE_TRY(check_ptr(expert_offsets, "expert_offsets"));
+  MOE_TRY(check_ptr(q1, "q1"));
+  MOE_TRY(check_ptr(q3, "q3"));
+  MOE_TRY(check_ptr(q2, "q2"));
+  MOE_TRY(check_ptr(s1, "s1"));
+  MOE_TRY(check_ptr(s3, "s3"));
+  MOE_TRY(check_ptr(s2, "s2"));
+  MOE_TRY(check_ptr(y_perm, "y_perm"));
+  const Layout L = layout(s);
+  MOE_TRY(check_ws(ws, ws_bytes, L.end));
+  return run_experts(s, x_perm, expert_offsets, int8_experts(q1, q3, q2, s1, s3, s2),
+                     at<uint16_t>(ws, L.h), y_perm, at<int32_t>(ws, L.status),
+                     (cudaStream_t)stream);
+}
+
+moe_status_t moe_forward_w8(const moe_shape_t* shape, const moe_bf16_t* x,
+                            const moe_bf16_t* w_router, const float* logit_bias, const int8_t* q1,
+                            const int8_t* q3, const int8_t* q2, const float* s1, const float* s3,
+                            const float* s2, const moe_bf16_t* residual, moe_bf16_t* out,
+                            void* ws, size_t ws_bytes, moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(x, "x"));
+  MOE_TRY(check_ptr(w_router, "w_router"));
+  MOE_TRY(check_ptr(logit_bias, "logit_bias", true));
+  MOE_TRY(check_ptr(q1, "q1"));
+  MOE_TRY(check_ptr(q3, "q3"));
+  MOE_TRY(check_ptr(q2, "q2"));
+  MOE_TRY(check_ptr(s1, "s1"));
+  MOE_TRY(check_ptr(s3, "s3"));
+  MOE_TRY(check_ptr(s2, "s2"));
+  MOE_TRY(check_ptr(residual, "residual", true));
+  MOE_TRY(check_ptr(out, "out"));
+  MOE_TRY(check_ws(ws, ws_bytes, layout(s).end));
+  return run_forward(s, x, w_router, logit_bias, int8_experts(q1, q3, q2, s1, s3, s2), residual,
+                     out, ws, (cudaStream_t)stream);
 }
 
 }  // extern "C"

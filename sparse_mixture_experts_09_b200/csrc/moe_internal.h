@@ -67,6 +67,33 @@ cudaError_t launch_down(const Shape& s, const GemmArgs& g, cudaStream_t st, cons
 cudaError_t launch_grouped_swiglu(const Shape& s, const GemmArgs& g, cudaStream_t st,
                                   const char** why);
 
+// ---- weight-only int8 experts ----
+// Per output row r of w [rows, K] (bf16): s[r] = max|w[r,:]| / 127 (1 for a zero row),
+// q = rint(w / s) clamped to [-127, 127], both in float32; q is written in the blocked
+// layout [rows/128][K/64][128][64] (rows % 128 == 0, K % 64 == 0).
+cudaError_t launch_quant_rows(const uint16_t* w, int8_t* q, float* s, int64_t rows, int K,
+                              cudaStream_t st);
+
+struct GemmArgsW8 {
+  const uint16_t* a;       // x_perm [Rmax, H]
+  const int32_t* offsets;  // [E+1], multiples of 128
+  const int8_t* q1;        // blocked codes of w1 [E*I/128][H/64][128][64]
+  const int8_t* q3;        // same for w3
+  const int8_t* q2;        // blocked codes of w2 [E*H/128][I/64][128][64]
+  const float* s1;         // [E*I]
+  const float* s3;         // [E*I]
+  const float* s2;         // [E*H]
+  uint16_t* h;             // [Rmax, I]
+  float* y;                // [Rmax, H]
+  int32_t* status;
+  int64_t rmax;
+  unsigned long long timeout_ns;
+};
+
+// GEMM1 (int8 gate/up + SwiGLU -> h) then GEMM2 (h q2^T * s2 -> y).
+cudaError_t launch_grouped_swiglu_w8(const Shape& s, const GemmArgsW8& g, cudaStream_t st,
+                                     const char** why);
+
 // w [rows, cols] -> blocked layout [rows/128][cols/64][128][64] (rows % 128 == 0,
 // cols % 64 == 0).
 cudaError_t launch_pack_blocked(const uint16_t* w, uint16_t* wp, int64_t rows, int64_t cols,

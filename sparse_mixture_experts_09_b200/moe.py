@@ -9,6 +9,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+from dataclasses import dataclass
 from typing import Optional
 
 import torch
@@ -25,7 +26,26 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_size_host", "moe_max_padded_rows
            "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_expert_gate_up",
            "moe_expert_down", "moe_combine", "moe_forward",
            "moe_forward_host", "moe_device_status", "moe_last_error", "moe_permute_static",
-           "moe_selftest_wait_timeout", "moe_forward_rmsnorm", "moe_pack_weights")
+           "moe_selftest_wait_timeout", "moe_forward_rmsnorm", "moe_pack_weights",
+           "moe_quantize_int8", "moe_grouped_swiglu_w8", "moe_forward_w8")
+
+
+@dataclass
+class Int8Experts:
+    """Weight-only int8 experts as written by quantize_int8: codes q1, q3 [E, I, H] and
+    q2 [E, H, I] int8 in the blocked layout [rows/128][K/64][128][64] (same number of
+    elements), per-row scales s1, s3 [E, I] and s2 [E, H] fp32."""
+    q1: torch.Tensor
+    q3: torch.Tensor
+    q2: torch.Tensor
+    s1: torch.Tensor
+    s3: torch.Tensor
+    s2: torch.Tensor
+
+    def pointers(self):
+        return [_dev(self.q1, "q1", torch.int8), _dev(self.q3, "q3", torch.int8),
+                _dev(self.q2, "q2", torch.int8), _dev(self.s1, "s1", torch.float32),
+                _dev(self.s3, "s3", torch.float32), _dev(self.s2, "s2", torch.float32)]
 
 
 class MoeError(RuntimeError):
@@ -92,6 +112,12 @@ def lib() -> ctypes.CDLL:
         L.moe_permute_static.restype = st
         L.moe_selftest_wait_timeout.argtypes = [_P, _SZ, ctypes.c_uint64, _P]
         L.moe_selftest_wait_timeout.restype = st
+        L.moe_quantize_int8.argtypes = [sp] + [_P] * 10
+        L.moe_quantize_int8.restype = st
+        L.moe_grouped_swiglu_w8.argtypes = [sp] + [_P] * 10 + [_SZ, _P]
+        L.moe_grouped_swiglu_w8.restype = st
+        L.moe_forward_w8.argtypes = [sp] + [_P] * 12 + [_SZ, _P]
+        L.moe_forward_w8.restype = st
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         _lib = L
@@ -354,3 +380,51 @@ def pack_weights(w1, w3, w2, stream=None):
 def device_status(ws, stream=None) -> None:
     """Raise MoeError(MOE_ERR_TIMEOUT) if a kernel gave up a bounded wait since last checked."""
     _check(lib().moe_device_status(_dev(ws, "ws"), ws.numel(), _stream(stream)))
+
+
+def quantize_int8(w1, w3, w2, stream=None) -> Int8Experts:
+    """Row-major bf16 expert weights -> Int8Experts (per-row symmetric int8)."""
+    e, i, h = w1.shape
+    shape = make_shape(1, h, i, e, 1)
+    dev = w1.device
+    q = [torch.empty(t.shape, dtype=torch.int8, device=dev) for t in (w1, w3, w2)]
+    sc = [torch.empty((e, i), dtype=torch.float32, device=dev),
+          torch.empty((e, i), dtype=torch.float32, device=dev),
+          torch.empty((e, h), dtype=torch.float32, device=dev)]
+    out = Int8Experts(q[0], q[1], q[2], sc[0], sc[1], sc[2])
+    _check(lib().moe_quantize_int8(ctypes.byref(shape), _dev(w1, "w1", torch.bfloat16),
+                                   _dev(w3, "w3", torch.bfloat16), _dev(w2, "w2", torch.bfloat16),
+                                   *out.pointers(), _stream(stream)))
+    return out
+
+
+def grouped_swiglu_w8(x_perm, offsets, experts: Int8Experts, num_tokens: int, k: int, ws,
+                      stream=None):
+    """grouped_swiglu with int8 expert weights: y_perm [R_max, H] fp32."""
+    e, i, h = experts.q1.shape
+    shape = make_shape(num_tokens, h, i, e, k)
+    y = torch.zeros((max_padded_rows(shape), h), dtype=torch.float32, device=x_perm.device)
+    _check(lib().moe_grouped_swiglu_w8(ctypes.byref(shape), _dev(x_perm, "x_perm", torch.bfloat16),
+                                       _dev(offsets, "offsets", torch.int32), *experts.pointers(),
+                                       _dev(y, "y_perm"), _dev(ws, "ws"), ws.numel(),
+                                       _stream(stream)))
+    return y
+
+
+def forward_w8(x, w_router, experts: Int8Experts, k: int, residual=None, logit_bias=None,
+               ws=None, out=None, stream=None, router_bf16_logits: bool = False):
+    """The whole layer with int8 expert weights; returns out [T,H] bf16."""
+    t, h = x.shape
+    e, i, _ = experts.q1.shape
+    shape = make_shape(t, h, i, e, k, ROW_MAJOR, router_bf16_logits)
+    if ws is None:
+        ws = make_workspace(shape, x.device)
+    if out is None:
+        out = torch.empty((t, h), dtype=torch.bfloat16, device=x.device)
+    _check(lib().moe_forward_w8(ctypes.byref(shape), _dev(x, "x", torch.bfloat16),
+                                _dev(w_router, "w_router", torch.bfloat16),
+                                _dev(logit_bias, "logit_bias", torch.float32, True),
+                                *experts.pointers(),
+                                _dev(residual, "residual", torch.bfloat16, True), _dev(out, "out"),
+                                _dev(ws, "ws"), ws.numel(), _stream(stream)))
+    return out
