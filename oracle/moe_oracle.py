@@ -44,7 +44,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "to_f64", "round_bf16", "silu", "router_logits", "route_topk", "stable_permute",
+    "to_f64", "round_bf16", "round_f16", "silu", "router_logits", "route_topk", "stable_permute",
     "swiglu_expert", "moe_layer", "rms_norm", "moe_block", "quantize_int8_rows",
 ]
 
@@ -68,6 +68,22 @@ def round_bf16(a) -> np.ndarray:
     _, e = np.frexp(a)
     quantum = np.ldexp(1.0, np.maximum(e, -125) - 8)
     return np.rint(a / quantum) * quantum
+
+
+def round_f16(a) -> np.ndarray:
+    """Nearest IEEE half-precision (float16) value of each fp64 element, ties to even,
+    returned as fp64; magnitudes that round past the largest finite value 65504 become
+    infinite.
+
+    float16 keeps 11 significant bits; its smallest normal is 2**-14 and its subnormal
+    spacing 2**-24. For |a| = m * 2**e with 0.5 <= m < 1 the spacing near a is
+    2**(e - 11), floored at 2**-24.
+    """
+    a = np.asarray(a, dtype=np.float64)
+    _, e = np.frexp(a)
+    quantum = np.ldexp(1.0, np.maximum(e, -13) - 11)
+    r = np.rint(a / quantum) * quantum
+    return np.where(np.abs(r) > 65504.0, np.copysign(np.inf, a), r)
 
 
 def silu(g: np.ndarray) -> np.ndarray:
@@ -161,14 +177,21 @@ def moe_layer(x, w_router, w1, w3, w2, k: int, residual=None, logit_bias=None,
               mode: str = "exact", tokens=None, bf16_logits: bool = False) -> dict:
     """The layer on tokens ``tokens`` (all tokens when None).
 
+    ``mode``: ``exact`` rounds nothing; ``bf16_storage`` rounds h and the output to
+    bf16 (a bf16 load); ``f16_experts`` is a half-precision expert path, as a float16
+    load computes it (Hugging Face "Mixtral" doc, "Shrinking down Mixtral using
+    quantization": the model in half precision, float16): the experts read x rounded
+    to float16 and store h as float16, the router and the combine are as in
+    ``bf16_storage``.
+
     Returns a dict of fp64 arrays over the chosen tokens: ``logits`` [n, E], ``idx``
     [n, k], ``weights`` [n, k], ``y`` [n, k, H] (unweighted expert outputs),
     ``expert_outputs`` [n, k, H] (weighted), ``routed`` [n, H] and ``out`` [n, H]
     (residual + routed; rounded to bf16 in ``bf16_storage`` mode).
     """
-    if mode not in ("exact", "bf16_storage"):
+    if mode not in ("exact", "bf16_storage", "f16_experts"):
         raise ValueError(mode)
-    storage = mode == "bf16_storage"
+    storage = mode != "exact"
     xs = to_f64(x)
     if tokens is not None:
         tokens = np.asarray(tokens, dtype=np.int64)
@@ -177,12 +200,18 @@ def moe_layer(x, w_router, w1, w3, w2, k: int, residual=None, logit_bias=None,
     logits = router_logits(xs, w_router, logit_bias, bf16_logits)
     idx, weights, _ = route_topk(logits, k)
     num_experts = logits.shape[1]
+    # f16_experts: the experts read x as float16 and store h as float16
+    x_experts = round_f16(xs) if mode == "f16_experts" else xs
     y = np.zeros((n, k, hidden), dtype=np.float64)
     for e in range(num_experts):
         tok, slot = np.nonzero(idx == e)
         if tok.size == 0:
             continue
-        y[tok, slot] = swiglu_expert(xs[tok], w1[e], w3[e], w2[e], h_bf16=storage)
+        if mode == "f16_experts":
+            h = silu(x_experts[tok] @ to_f64(w1[e]).T) * (x_experts[tok] @ to_f64(w3[e]).T)
+            y[tok, slot] = round_f16(h) @ to_f64(w2[e]).T
+        else:
+            y[tok, slot] = swiglu_expert(xs[tok], w1[e], w3[e], w2[e], h_bf16=storage)
     expert_outputs = weights[:, :, None] * y
     routed = np.zeros((n, hidden), dtype=np.float64)
     for j in range(k):

@@ -359,3 +359,60 @@ def test_int8_codes_match_torch_float32_arithmetic():
     st = wt.abs().amax(-1) / 127.0
     qt = torch.round(wt / st[:, None]).clamp(-127, 127).to(torch.int8)
     assert np.array_equal(s, st.numpy()) and np.array_equal(q, qt.numpy())
+
+
+def test_round_f16_closed_forms():
+    # IEEE binary16: 11 significant bits, smallest normal 2**-14, subnormal step 2**-24,
+    # largest finite 65504; ties go to the even significand
+    for v in (0.0, 1.0, -2.5, 65504.0, 2.0 ** -14, 2.0 ** -24, 1 + 2.0 ** -10):
+        assert O.round_f16(v) == v
+    assert O.round_f16(1 + 2.0 ** -11) == 1.0                      # tie, to even
+    assert O.round_f16(1 + 3 * 2.0 ** -11) == 1 + 2.0 ** -9        # tie, to even
+    assert O.round_f16(2049.0) == 2048.0 and O.round_f16(2051.0) == 2052.0
+    assert O.round_f16(2.0 ** -25) == 0.0                          # subnormal tie
+    assert O.round_f16(3 * 2.0 ** -25) == 2.0 ** -23
+    assert O.round_f16(65519.0) == 65504.0
+    assert np.isinf(O.round_f16(65520.0)) and O.round_f16(-1e6) == -np.inf
+
+
+def test_round_f16_matches_numpy_half_cast():
+    g = np.random.default_rng(3)
+    a = np.concatenate([g.standard_normal(4000) * 10.0 ** g.integers(-9, 6, 4000),
+                        g.standard_normal(100) * 1e-7, [7e4, -7e4, 65519.9, 65520.0]])
+    with np.errstate(over="ignore"):
+        want = a.astype(np.float16).astype(np.float64)
+    assert np.array_equal(O.round_f16(a), want)
+
+
+def test_bf16_values_in_f16_normal_range_are_exact_in_f16():
+    # 8 significant bits fit in 11: the half-precision expert path reads bf16 inputs
+    # unchanged when 2**-14 <= |x| <= 65504
+    g = np.random.default_rng(4)
+    x = O.round_bf16(g.standard_normal(5000) * 10.0 ** g.integers(-4, 4, 5000))
+    x = x[(np.abs(x) >= 2.0 ** -14) & (np.abs(x) <= 65504)]
+    assert np.array_equal(O.round_f16(x), x)
+
+
+def test_f16_expert_mode_differs_from_exact_by_f16_rounding_of_h():
+    # with inputs exact in float16, the f16 expert mode equals the exact layer up to
+    # the float16 rounding of h (and the final bf16 rounding)
+    g = torch.Generator().manual_seed(9)
+    t, hd, i, e, k = 24, 32, 48, 4, 2
+    x = (torch.randn(t, hd, generator=g)).to(torch.bfloat16)
+    wr = (torch.randn(e, hd, generator=g) * 0.2).to(torch.bfloat16)
+    w1 = (torch.randn(e, i, hd, generator=g) * 0.2).to(torch.bfloat16)
+    w3 = (torch.randn(e, i, hd, generator=g) * 0.2).to(torch.bfloat16)
+    w2 = (torch.randn(e, hd, i, generator=g) * 0.2).to(torch.bfloat16)
+    ex = O.moe_layer(x, wr, w1, w3, w2, k, mode="exact")
+    f16 = O.moe_layer(x, wr, w1, w3, w2, k, mode="f16_experts")
+    assert np.array_equal(ex["idx"], f16["idx"])
+    # h relative rounding <= 2**-11, so each y moves by at most that times sum |w2| |h|
+    xs = O.to_f64(x)
+    for tt in range(t):
+        for j in range(k):
+            ee = ex["idx"][tt, j]
+            h = O.silu(xs[tt] @ O.to_f64(w1[ee]).T) * (xs[tt] @ O.to_f64(w3[ee]).T)
+            bound = 2.0 ** -11 * (np.abs(O.to_f64(w2[ee])) @ np.abs(h)) + 1e-12
+            assert np.all(np.abs(f16["y"][tt, j] - ex["y"][tt, j]) <= bound)
+    assert not np.array_equal(f16["y"], ex["y"])
+    assert np.array_equal(f16["out"], O.round_bf16(f16["routed"]))
