@@ -316,6 +316,14 @@ def run_ours(args):
         moe.forward(inp.x, inp.w_router, bw1, bw3, bw2, k, residual=inp.residual,
                     logit_bias=inp.logit_bias, ws=ws, out=out, weight_layout=layout)
 
+    # weight-only int8 experts, quantised once at load time (not timed)
+    w8 = moe.quantize_int8(inp.w1, inp.w3, inp.w2)
+    ws8 = moe.make_workspace(moe.make_shape(*w.shape), dev)
+
+    def step_w8():
+        moe.forward_w8(inp.x, inp.w_router, w8, k, residual=inp.residual,
+                       logit_bias=inp.logit_bias, ws=ws8, out=out)
+
     def step_row_major():
         moe.forward(inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, k, residual=inp.residual,
                     logit_bias=inp.logit_bias, ws=ws, out=out)
@@ -368,6 +376,7 @@ def run_ours(args):
     for _ in range(Wm):
         step()
         step_row_major()
+        step_w8()
     scratch = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
     for _ in range(3):
         split_step(scratch)
@@ -431,12 +440,26 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = h0.elapsed_time(h1) / K
+
+    # (4) the same layer with weight-only int8 experts
+    barrier()
+    torch.cuda.synchronize(dev)
+    q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    q0.record(stream)
+    for _ in range(K):
+        step_w8()
+    q1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    w8_ms = q0.elapsed_time(q1) / K
     clk = clocks.stop()
     moe.device_status(ws)
     moe.device_status(wsh)
+    moe.device_status(ws8)
 
     ms, e2e_ms = slowest_rank(ms, e2e_ms, world, dev)
     rm_ms, _ = slowest_rank(rm_ms, rm_ms, world, dev)
+    w8_ms, _ = slowest_rank(w8_ms, w8_ms, world, dev)
 
     counts = perm["counts"].cpu().tolist()
     peaks, peak_kind = load_peaks()
@@ -459,6 +482,12 @@ def run_ours(args):
             "kernels_ms": stage_ms,
             "row_major_weights": {"ms_per_step": rm_ms,
                                   "value": job_throughput(w.num_tokens, world, rm_ms)},
+            "int8_experts": {"ms_per_step": w8_ms,
+                             "value": job_throughput(w.num_tokens, world, w8_ms),
+                             "api": "moe_forward_w8",
+                             "weight_gb_per_step": roof["active_experts"] * w.expert_bytes() / 2e9,
+                             "note": "weight-only int8 experts, half-precision expert math, "
+                                     "quantised once at load (untimed); not the headline"},
             "e2e": {"value": job_throughput(w.num_tokens, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": 2 * bytes_io, "d2h_bytes_per_step": bytes_io,
                     "api": "moe_forward_host"},

@@ -235,44 +235,56 @@ moe_status_t moe_pack_weights(const moe_shape_t* shape, const moe_bf16_t* w1,
                               moe_bf16_t* w1_blocked, moe_bf16_t* w3_blocked,
                               moe_bf16_t* w2_blocked, moe_stream_t stream);
 
-/* ---- Weight-only int8 experts (W8A16) ----
+/* ---- Weight-only int8 experts ----
  * The pages load Mixtral weight-only quantised to shrink it (Hugging Face "Mixtral",
  * "Shrinking down Mixtral using quantization"; ZeroModels "Mixtral", "Lower memory":
- * int8 weights with bf16 activations). They do not fix the scheme; this library uses
- * symmetric int8 with one fp32 scale per output row (channel) of each expert matrix:
+ * int8 weights). They do not fix the scheme; this library uses symmetric int8 with
+ * one fp32 scale per output row (channel) of each expert matrix:
  *   s[r] = max_c |w[r, c]| / 127   (1 for an all-zero row),
  *   q[r, c] = clamp(rint(w[r, c] / s[r]), -127, 127),   w[r, c] ~ q[r, c] * s[r],
  * the divisions and the rounding (to nearest, ties to even) in float32.
- * Codes are stored in the blocked layout [rows/128][K/64][128][64] (int8), where a
- * matrix of `rows` rows and K columns is w1/w3 of all experts (rows = E*I, K = H) or
- * w2 (rows = E*H, K = I); scales are [rows] fp32, row e*I + i (or e*H + j).
- * The shape's weight_layout field is ignored by these entry points.
+ * Codes are stored offset-binary, u = q + 128 (uint8, 1 .. 255), tiled: a matrix of
+ * `rows` rows and K columns (w1 or w3 of all experts: rows = E*I, K = H; w2: rows =
+ * E*H, K = I) is cut into 128 x 64 tiles, tile (row / 128, col / 64) being the 8 KiB
+ * block number (row / 128) * (K / 64) + col / 64; inside a tile, with r = row % 128
+ * and c = col % 64, the code is at byte (c / 16) * 2048 + r * 16 + c % 16.
+ * Scales are [rows] fp32, row e*I + i (or e*H + j). The shape's weight_layout field
+ * is ignored by these entry points.
+ *
+ * Precision. The int8 experts compute in IEEE half precision, as a float16 load of
+ * the model does (Hugging Face "Mixtral": the model in half precision, float16): the
+ * routed rows are converted bf16 -> half (exact for magnitudes in [2^-14, 65504];
+ * smaller ones are rounded to half's subnormal grid, larger ones overflow to
+ * infinity), each code widens exactly to a half, products accumulate in fp32, and the
+ * hidden activation is stored as half:
+ *   h = half(silu(s1 * (x_perm q1[e]^T)) * (s3 * (x_perm q3[e]^T))),
+ *   y_perm = s2 * (h q2[e]^T)  (fp32).
+ * Routing and the combine are the bf16 layer's.
  *
  * moe_quantize_int8: w1, w3 [E, I, H] and w2 [E, H, I] bf16 row-major in (device);
- * q1, q3 [E*I*H], q2 [E*H*I] int8 and s1, s3 [E*I], s2 [E*H] fp32 out (device,
+ * q1, q3 [E*I*H], q2 [E*H*I] codes and s1, s3 [E*I], s2 [E*H] fp32 out (device,
  * caller-owned). Asynchronous on `stream`. */
 moe_status_t moe_quantize_int8(const moe_shape_t* shape, const moe_bf16_t* w1,
-                               const moe_bf16_t* w3, const moe_bf16_t* w2, int8_t* q1,
-                               int8_t* q3, int8_t* q2, float* s1, float* s3, float* s2,
+                               const moe_bf16_t* w3, const moe_bf16_t* w2, uint8_t* q1,
+                               uint8_t* q3, uint8_t* q2, float* s1, float* s3, float* s2,
                                moe_stream_t stream);
 
 /* moe_grouped_swiglu with int8 expert weights (codes and scales as written by
- * moe_quantize_int8): the tensor cores multiply the bf16 rows by the codes (exact
- * in bf16) with fp32 accumulation; the epilogues apply the scales:
- *   h = bf16(silu(s1 * (x_perm q1[e]^T)) * (s3 * (x_perm q3[e]^T))),
- *   y_perm = s2 * (h q2[e]^T)  (fp32).
- * Other arguments and errors as for moe_grouped_swiglu. */
+ * moe_quantize_int8), computed as described above. x_perm is bf16 as moe_permute
+ * writes it (converted to half into ws); other arguments and errors as for
+ * moe_grouped_swiglu. */
 moe_status_t moe_grouped_swiglu_w8(const moe_shape_t* shape, const moe_bf16_t* x_perm,
-                                   const int32_t* expert_offsets, const int8_t* q1,
-                                   const int8_t* q3, const int8_t* q2, const float* s1,
+                                   const int32_t* expert_offsets, const uint8_t* q1,
+                                   const uint8_t* q3, const uint8_t* q2, const float* s1,
                                    const float* s3, const float* s2, float* y_perm, void* ws,
                                    size_t ws_bytes, moe_stream_t stream);
 
 /* moe_forward with int8 expert weights: router, permutation and combine as in
- * moe_forward, experts as in moe_grouped_swiglu_w8. */
+ * moe_forward (the gather writes the routed rows as half), experts as in
+ * moe_grouped_swiglu_w8. */
 moe_status_t moe_forward_w8(const moe_shape_t* shape, const moe_bf16_t* x,
                             const moe_bf16_t* w_router, const float* logit_bias,
-                            const int8_t* q1, const int8_t* q3, const int8_t* q2,
+                            const uint8_t* q1, const uint8_t* q3, const uint8_t* q2,
                             const float* s1, const float* s3, const float* s2,
                             const moe_bf16_t* residual, moe_bf16_t* out, void* ws,
                             size_t ws_bytes, moe_stream_t stream);

@@ -3,20 +3,24 @@
 //
 // Mixtral is loaded weight-only quantised to shrink it (Hugging Face "Mixtral" doc,
 // "Shrinking down Mixtral using quantization"; ZeroModels "Mixtral", "Lower memory":
-// int8 weights with bf16 activations). At decode the layer streams every active
-// expert's weights, so halving their bytes can halve the time.
+// int8 weights). At decode the layer streams every active expert's weights, so halving
+// their bytes can halve the time.
 // Scheme (the pages do not fix one): per output row (channel) r, s[r] = max|w[r, :]| /
-// 127 and q = rint(w / s), decided in float32; w ~ q * s. Every int8 value is exactly a
-// bf16 value, so the tensor cores multiply the bf16 activations by the codes widened
-// to bf16 (exact), and the scale, constant along K, multiplies the fp32 accumulator in
-// the epilogue: sum_k x[k] q[r,k] s[r] = s[r] * sum_k x[k] q[r,k].
+// 127 and q = rint(w / s), decided in float32; w ~ q * s. The experts compute in half
+// precision, as a float16 load of the model does (Hugging Face "Mixtral" doc: the model
+// in half precision, float16): the activations arrive as IEEE half, every code widens
+// exactly to a half, the tensor cores accumulate in fp32, and the scale, constant along
+// K, multiplies the accumulator in the epilogue: sum_k x[k] q[r,k] s[r] = s[r] sum_k
+// x[k] q[r,k]. Half, not bf16, because an 8-bit code fits a half's 10-bit mantissa in
+// one binade, so widening costs one byte permute and one packed subtraction per two
+// codes; a bf16 has 7 mantissa bits and needs twice the integer work.
 //
-// Kernel: the bf16 kernel's persistent tile loop with a widening stage. Warp roles:
-//   warp 0      streams the int8 tiles (bulk copies: in the blocked code layout each
-//               128-row x 64-code tile is one contiguous 8 KiB run) into a code ring;
-//   warp 6      loads the activation tiles (TMA, 128-byte swizzle) into the main ring;
-//   warps 7..   widen each code tile to bf16 and store it, 128-byte swizzled, as the
-//               B operand of the main ring;
+// Kernel k_grouped_gemm_w8: the bf16 GEMM's persistent tile loop with a widening
+// stage. Warp roles:
+//   warp 0      streams the code tiles (bulk copies: each 128-row x 64-code tile is one
+//               contiguous 8 KiB run) into a code ring;
+//   warp 6      loads the activation tiles (TMA, 128-byte swizzle) into their ring;
+//   warps 7..   widen each code tile and store it, 128-byte swizzled, as the B operand;
 //   warp 1      issues tcgen05.mma into a double-buffered TMEM accumulator;
 //   warps 2-5   scale, activate and store (epilogue).
 // Every wait is bounded (timeout -> status word, abort flag, drained copies).
@@ -49,14 +53,7 @@ constexpr int kAStages = MOE_W8_A_STAGES;
 constexpr int kBStages = MOE_W8_B_STAGES;
 constexpr int kCodeStages = MOE_W8_CODE_STAGES;
 constexpr int kConvWarps = MOE_W8_CONV_WARPS;
-#ifndef MOE_W8_SUSPEND_NS
-#define MOE_W8_SUSPEND_NS 20000
-#endif
-// Suspend limit of one try_wait in the waiting loop: a waiting warp issues no
-// instructions while it sleeps, leaving the issue slots to the converters. The abort
-// flag and the timeout are checked every 64 tries, i.e. at least every 64 limits.
-constexpr uint32_t kSuspendNs = MOE_W8_SUSPEND_NS;
-// warp 0: code TMA, 1: MMA, 2-5: epilogue, 6: activation TMA, 7..: converters
+// warp 0: code copies, 1: MMA, 2-5: epilogue, 6: activation TMA, 7..: converters
 constexpr int kConvWarp0 = 7;
 constexpr int kThreadsW8 = 32 * (kConvWarp0 + kConvWarps);
 constexpr int A_BYTES = BM * BK * 2;  // 16 KiB
@@ -73,15 +70,16 @@ struct TileW8 {
   static constexpr int BAR_OFF = Q_OFF + kCodeStages * Q_BYTES;
   static constexpr int SMEM = 1024 + BAR_OFF + kNumBars * 8 + 8 + 65 * 4;
   static constexpr int CHUNKS = BN * BK / 16 / (32 * kConvWarps);  // code chunks per thread
-  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
-                                    ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+  // D f32, A and B f16 (format 0), both K-major
+  static constexpr uint32_t IDESC =
+      (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
   static_assert(SMEM <= 232448, "shared memory plan exceeds 227 KiB");
   static_assert(CHUNKS * 32 * kConvWarps * 16 == BN * BK, "converter split");
 };
 
 struct W8Params {
-  const int8_t* q0;      // blocked codes of the first weight (w1 or w2)
-  const int8_t* q1;      // blocked codes of w3 (gate/up only)
+  const uint8_t* q0;     // tiled codes of the first weight (w1 or w2)
+  const uint8_t* q1;     // tiled codes of w3 (gate/up only)
   const int32_t* offsets;
   const float* scale_a;  // per-row scales of the first weight (w1 or w2) [E * rows]
   const float* scale_b;  // per-row scales of w3 (gate/up only)
@@ -89,6 +87,7 @@ struct W8Params {
   void* out;
   int64_t out_ld;
   int E, k_blocks, n_tiles, b_rows;
+  int n_cols;  // small-batch kernel: token columns N (multiple of 16, at most 64)
   unsigned long long timeout_ns;
 };
 
@@ -111,19 +110,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// try_wait with an explicit suspend-time limit: a thread whose phase is not complete
-// sleeps in hardware until the phase completes or `ns` elapse, instead of re-polling.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(ns)
       : "memory");
   return ok != 0;
 }
@@ -162,7 +148,7 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
   return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
          (2ull << 61);
 }
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                          uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -188,20 +174,15 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
 
-// Bounded wait on an mbarrier phase (see the bf16 kernel): false after the CTA aborted
+// Bounded wait on an mbarrier phase (as in the bf16 GEMM): false after the CTA aborted
 // or after timeout_ns, which it records as kStatusTimeout.
 __device__ __noinline__ bool wait_w8(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                      int32_t* status, unsigned long long timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if ((n & 63u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > timeout_ns) {
@@ -244,30 +225,45 @@ __device__ __forceinline__ int code_y(int row, int kb, int k_blocks) {
   return ((row >> 7) * k_blocks + kb) * 128;
 }
 
-// Two int8 codes (bytes a, b of a 32-bit word, placed in the low bytes of the two
-// 16-bit halves by a byte permute) -> bf16x2, exactly. With l = the code's low 7 bits
-// and t = its sign bit, the bf16 bit pattern 0x4300 | l is 128 + l and 0x4300 | t << 7
-// is 128 (t = 0) or 256 (t = 1); their difference is l - 128 t, the two's-complement
-// value, an integer in [-128, 127] and so exact in bf16.
-__device__ __forceinline__ uint32_t codes_to_bf16x2(uint32_t w, uint32_t sel) {
-  const uint32_t p = __byte_perm(w, 0u, sel);
-  const uint32_t x = (p & 0x007F007Fu) | 0x43004300u;
-  const uint32_t c = (p & 0x00800080u) | 0x43004300u;
+// ---- code layout and widening ----
+// Codes are stored offset-binary, u = q + 128 in [1, 255]. A 128-row x 64-column tile
+// is one contiguous 8 KiB block: four 2 KiB column chunks (columns 16v .. 16v+15),
+// each holding the 128 rows' 16 codes in row order, so a thread that owns a row (or
+// consecutive threads that own consecutive rows) read without bank conflicts.
+//
+// Widening to IEEE half: the half whose high byte is 0x64 and low byte u is 1024 + u
+// (exponent 2^10, 10 mantissa bits); subtracting 1152 leaves u - 128 = q exactly. One
+// byte permute builds two such halves, one packed subtraction (on the FMA pipe) finishes
+// them: half an integer-pipe instruction per code.
+__device__ __forceinline__ uint32_t codes_to_f16x2(uint32_t w, uint32_t sel) {
+  const uint32_t x = __byte_perm(w, 0x64646464u, sel);
   uint32_t r;
-  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(c));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(0x64806480u));
   return r;
 }
 
-// 16 codes (one uint4, columns 16v .. 16v+15) -> two 16-byte chunks of bf16
-__device__ __forceinline__ void widen16(const uint4 w4, uint4& lo8, uint4& hi8) {
-  lo8 = make_uint4(codes_to_bf16x2(w4.x, 0x4140u), codes_to_bf16x2(w4.x, 0x4342u),
-                   codes_to_bf16x2(w4.y, 0x4140u), codes_to_bf16x2(w4.y, 0x4342u));
-  hi8 = make_uint4(codes_to_bf16x2(w4.z, 0x4140u), codes_to_bf16x2(w4.z, 0x4342u),
-                   codes_to_bf16x2(w4.w, 0x4140u), codes_to_bf16x2(w4.w, 0x4342u));
+// One word (columns 4m .. 4m+3) -> half pairs (4m, 4m+1) and (4m+2, 4m+3)
+__device__ __forceinline__ void widen_word(uint32_t w, uint32_t& p01, uint32_t& p23) {
+  p01 = codes_to_f16x2(w, 0x4140u);
+  p23 = codes_to_f16x2(w, 0x4342u);
 }
 
-// MODE kSwiGLU: A = x_perm [rows, H], weight tile = 128 rows of w1 then 128 rows of w3
-//   (BN = 256), h = bf16(silu(s1 * gate) * (s3 * up)).
+// 16 codes (one chunk) -> two 16-byte runs of halves, columns 16v .. 16v+7 and +8 .. +15
+__device__ __forceinline__ void widen16(const uint4 w4, uint4& lo8, uint4& hi8) {
+  widen_word(w4.x, lo8.x, lo8.y);
+  widen_word(w4.y, lo8.z, lo8.w);
+  widen_word(w4.z, hi8.x, hi8.y);
+  widen_word(w4.w, hi8.z, hi8.w);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// MODE kSwiGLU: A = x_perm [rows, H] (half), weight tile = 128 rows of w1 then 128 rows
+//   of w3 (BN = 256), h = half(silu(s1 * gate) * (s3 * up)).
 // MODE kPlain:  A = h [rows, I], weight tile = BN rows of w2, y = s2 * acc (fp32).
 template <int MODE, int BN>
 __global__ void __launch_bounds__(kThreadsW8, 1)
@@ -401,7 +397,7 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
           const uint32_t db = smem_u32(bbase + sb * TL::B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            mma_bf16(d, sdesc(da + kk * 32), sdesc(db + kk * 32), TL::IDESC, (kb | kk) ? 1u : 0u);
+            mma_f16(d, sdesc(da + kk * 32), sdesc(db + kk * 32), TL::IDESC, (kb | kk) ? 1u : 0u);
           mma_commit(a_empty(sa));
           mma_commit(b_empty(sb));
           issued = true;
@@ -416,7 +412,7 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
     __syncwarp();
   } else if (warp == 6) {
     if (lane == 0) {
-      // ---------------- activation tiles (bf16, 128-byte swizzle by the TMA)
+      // ---------------- activation tiles (half, 128-byte swizzle by the TMA)
       int it = 0;
       bool ok = true;
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
@@ -441,12 +437,12 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
     }
     __syncwarp();
   } else if (warp >= kConvWarp0) {
-    // ---------------- converters: int8 code tile -> bf16 B tile in the 128-byte
+    // ---------------- converters: code tile -> half B tile in the 128-byte
     // swizzled K-major layout (row r: 128 bytes at r * 128, 16-byte chunk c stored at
     // chunk position c ^ (r & 7)). Thread ct widens the 16-byte code chunks
-    // j = ct + 32 kConvWarps i (row j / 4, columns 16 (j % 4) ..): consecutive threads
-    // read consecutive chunks, and the 8 stores of a quarter-warp land in distinct
-    // banks.
+    // j = ct + 32 kConvWarps i of the stage (128-row tile j / 512, column chunk
+    // (j / 128) % 4, row j % 128): consecutive threads read consecutive chunks, and the
+    // 8 stores of a quarter-warp (8 consecutive rows) land in distinct banks.
     const int ct = threadIdx.x - kConvWarp0 * 32;
     int it = 0;
     bool ok = true;
@@ -471,7 +467,7 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
 #pragma unroll
         for (int i = 0; i < TL::CHUNKS; ++i) {
           const int j = ct + 32 * kConvWarps * i;
-          const int r = j >> 2, c = (j & 3) * 2;
+          const int r = (j >> 9) * 128 + (j & 127), c = ((j >> 7) & 3) * 2;
           uint4 lo8, hi8;
           widen16(v[i], lo8, hi8);
           uint8_t* row = bs + r * 128;
@@ -520,7 +516,7 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
             const float g1 = __uint_as_float(g[2 * i + 1]) * __ldg(sg + c + 2 * i + 1);
             const float u0 = __uint_as_float(u[2 * i]) * __ldg(su + c + 2 * i);
             const float u1 = __uint_as_float(u[2 * i + 1]) * __ldg(su + c + 2 * i + 1);
-            pk[i] = pack_bf16x2_rn(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1);
+            pk[i] = pack_f16x2_rn(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1);
           }
           uint4* dst = reinterpret_cast<uint4*>(h + c);
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -559,10 +555,28 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
   }
 }
 
+// bf16 rows -> IEEE half rows (round to nearest even), 8 values per thread-step
+__global__ void __launch_bounds__(256) k_rows_to_f16(const uint4* __restrict__ src,
+                                                     uint4* __restrict__ dst, int64_t n8) {
+  pdl_trigger();
+  pdl_wait();
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = __ldg(src + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      o[j] = pack_f16x2_rn(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
+    dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 // One warp per weight row: s = max|w| / 127, q = rint(w / s) in float32, written in
-// the blocked code layout [rows/128][K/64][128][64].
+// the tiled code layout: tile (row / 128, column / 64) is the 8 KiB block number
+// (row / 128) * (K / 64) + column / 64, arranged inside as described above.
 __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__ w,
-                                                    int8_t* __restrict__ q, float* __restrict__ s,
+                                                    uint8_t* __restrict__ q, float* __restrict__ s,
                                                     int64_t rows, int K) {
   pdl_trigger();
   pdl_wait();
@@ -583,7 +597,9 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
       int qi = __float2int_rn(__fdiv_rn(v, sc));
       qi = qi > 127 ? 127 : (qi < -127 ? -127 : qi);
       const int64_t kb = c / BK, cc = c % BK;
-      q[((rb * kbn + kb) * 128 + rr) * BK + cc] = (int8_t)qi;
+      // byte of column cc in the tile: chunk cc / 16, row rr, column cc % 16
+      const int64_t in_tile = (cc >> 4) * 2048 + rr * 16 + (cc & 15);
+      q[(rb * kbn + kb) * (128 * BK) + in_tile] = (uint8_t)(qi + 128);
     }
   }
 }
@@ -606,7 +622,7 @@ EncodeTiledFnW8 encode_w8() {
   return fn;
 }
 
-// bf16 activations [rows, inner], box 64 x 128, 128-byte swizzle
+// half activations [rows, inner], box 64 x 128, 128-byte swizzle
 bool map_act(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
   EncodeTiledFnW8 fn = encode_w8();
   if (!fn) return false;
@@ -614,7 +630,7 @@ bool map_act(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
   const cuuint64_t strides[1] = {inner * 2};
   const cuuint32_t box[2] = {(cuuint32_t)BK, 128};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -641,7 +657,18 @@ cudaError_t launch_w8(const CUtensorMap& a, const W8Params& p, int64_t max_tiles
 
 }  // namespace
 
-cudaError_t launch_quant_rows(const uint16_t* w, int8_t* q, float* s, int64_t rows, int K,
+cudaError_t launch_rows_to_f16(const uint16_t* src, uint16_t* dst, int64_t rows, int H,
+                               cudaStream_t st) {
+  const int64_t n8 = rows * H / 8;
+  int64_t blocks = (n8 + 255) / 256;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return launch_pdl(k_rows_to_f16, dim3((unsigned)blocks), dim3(256), 0, st,
+                    reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(dst), n8);
+}
+
+cudaError_t launch_quant_rows(const uint16_t* w, uint8_t* q, float* s, int64_t rows, int K,
                               cudaStream_t st) {
   int64_t blocks = (rows + 7) / 8;
   const int64_t cap = (int64_t)num_sms() * 16;
@@ -657,7 +684,7 @@ cudaError_t launch_grouped_swiglu_w8(const Shape& s, const GemmArgsW8& g, cudaSt
     return cudaErrorInvalidValue;
   }
   const int64_t mt_max = g.rmax / BM;
-  W8Params p1;
+  W8Params p1 = {};
   p1.q0 = g.q1;
   p1.q1 = g.q3;
   p1.offsets = g.offsets;

@@ -143,10 +143,10 @@ T* at(void* ws, size_t off) {
 constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per wait
 
 // Expert weights of one layer: bf16 (w1, w3, w2), or int8 codes with per-row scales
-// (q1 non-null).
+// (q1 non-null; then x_perm and h are IEEE half).
 struct Experts {
   const uint16_t *w1, *w3, *w2;
-  const int8_t *q1, *q3, *q2;
+  const uint8_t *q1, *q3, *q2;
   const float *s1, *s3, *s2;
 };
 
@@ -158,7 +158,7 @@ Experts bf16_experts(const uint16_t* w1, const uint16_t* w3, const uint16_t* w2)
   return x;
 }
 
-Experts int8_experts(const int8_t* q1, const int8_t* q3, const int8_t* q2, const float* s1,
+Experts int8_experts(const uint8_t* q1, const uint8_t* q3, const uint8_t* q2, const float* s1,
                      const float* s3, const float* s2) {
   Experts x = {};
   x.q1 = q1;
@@ -219,7 +219,7 @@ moe_status_t run_forward(const Shape& s, const uint16_t* x, const uint16_t* wr, 
   e = launch_permute(s, at<int32_t>(ws, L.topk_idx), x, at<int32_t>(ws, L.counts),
                      at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.row_of),
                      at<int32_t>(ws, L.token_of_row), at<uint16_t>(ws, L.x_perm),
-                     at<int32_t>(ws, L.block_base), st, norm_w, rnorm);
+                     at<int32_t>(ws, L.block_base), st, norm_w, rnorm, w.q1 != nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   MOE_TRY(run_experts(s, at<uint16_t>(ws, L.x_perm), at<int32_t>(ws, L.offsets), w,
                       at<uint16_t>(ws, L.h), at<float>(ws, L.y), at<int32_t>(ws, L.status), st));
@@ -515,8 +515,9 @@ moe_status_t moe_device_status(void* ws, size_t ws_bytes, moe_stream_t stream) {
 }
 
 moe_status_t moe_quantize_int8(const moe_shape_t* shape, const moe_bf16_t* w1,
-                               const moe_bf16_t* w3, const moe_bf16_t* w2, int8_t* q1, int8_t* q3,
-                               int8_t* q2, float* s1, float* s3, float* s2, moe_stream_t stream) {
+                               const moe_bf16_t* w3, const moe_bf16_t* w2, uint8_t* q1,
+                               uint8_t* q3, uint8_t* q2, float* s1, float* s3, float* s2,
+                               moe_stream_t stream) {
   g_err[0] = 0;
   Shape s;
   MOE_TRY(check_shape(shape, &s));
@@ -538,8 +539,8 @@ moe_status_t moe_quantize_int8(const moe_shape_t* shape, const moe_bf16_t* w1,
 }
 
 moe_status_t moe_grouped_swiglu_w8(const moe_shape_t* shape, const moe_bf16_t* x_perm,
-                                   const int32_t* expert_offsets, const int8_t* q1,
-                                   const int8_t* q3, const int8_t* q2, const float* s1,
+                                   const int32_t* expert_offsets, const uint8_t* q1,
+                                   const uint8_t* q3, const uint8_t* q2, const float* s1,
                                    const float* s3, const float* s2, float* y_perm, void* ws,
                                    size_t ws_bytes, moe_stream_t stream) {
   g_err[0] = 0;
@@ -556,14 +557,19 @@ moe_status_t moe_grouped_swiglu_w8(const moe_shape_t* shape, const moe_bf16_t* x
   MOE_TRY(check_ptr(y_perm, "y_perm"));
   const Layout L = layout(s);
   MOE_TRY(check_ws(ws, ws_bytes, L.end));
-  return run_experts(s, x_perm, expert_offsets, int8_experts(q1, q3, q2, s1, s3, s2),
+  // the int8 experts read half activations: convert the caller's rows into ws
+  uint16_t* xh = at<uint16_t>(ws, L.x_perm);
+  cudaError_t e = launch_rows_to_f16(x_perm, xh, max_padded_rows(s), s.H, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "x_perm conversion launch");
+  return run_experts(s, xh, expert_offsets, int8_experts(q1, q3, q2, s1, s3, s2),
                      at<uint16_t>(ws, L.h), y_perm, at<int32_t>(ws, L.status),
                      (cudaStream_t)stream);
 }
 
 moe_status_t moe_forward_w8(const moe_shape_t* shape, const moe_bf16_t* x,
-                            const moe_bf16_t* w_router, const float* logit_bias, const int8_t* q1,
-                            const int8_t* q3, const int8_t* q2, const float* s1, const float* s3,
+                            const moe_bf16_t* w_router, const float* logit_bias,
+                            const uint8_t* q1, const uint8_t* q3, const uint8_t* q2,
+                            const float* s1, const float* s3,
                             const float* s2, const moe_bf16_t* residual, moe_bf16_t* out,
                             void* ws, size_t ws_bytes, moe_stream_t stream) {
   g_err[0] = 0;

@@ -46,7 +46,11 @@ cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16
                            int32_t* counts, int32_t* offsets, int32_t* row_of,
                            int32_t* token_of_row, uint16_t* x_perm, int32_t* block_base,
                            cudaStream_t st, const uint16_t* norm_w = nullptr,
-                           const float* rnorm = nullptr);
+                           const float* rnorm = nullptr, bool f16_out = false);
+
+// x_perm rows [0, rows) of width H: bf16 -> IEEE half (the int8 experts' input).
+cudaError_t launch_rows_to_f16(const uint16_t* src, uint16_t* dst, int64_t rows, int H,
+                               cudaStream_t st);
 
 struct GemmArgs {
   const uint16_t* a;        // x_perm [Rmax, K1] (GEMM1) or h [Rmax, I] (GEMM2)
@@ -69,28 +73,28 @@ cudaError_t launch_grouped_swiglu(const Shape& s, const GemmArgs& g, cudaStream_
 
 // ---- weight-only int8 experts ----
 // Per output row r of w [rows, K] (bf16): s[r] = max|w[r,:]| / 127 (1 for a zero row),
-// q = rint(w / s) clamped to [-127, 127], both in float32; q is written in the blocked
-// layout [rows/128][K/64][128][64] (rows % 128 == 0, K % 64 == 0).
-cudaError_t launch_quant_rows(const uint16_t* w, int8_t* q, float* s, int64_t rows, int K,
+// q = rint(w / s) clamped to [-127, 127], both in float32; q + 128 is written in the
+// tiled code layout (rows % 128 == 0, K % 64 == 0).
+cudaError_t launch_quant_rows(const uint16_t* w, uint8_t* q, float* s, int64_t rows, int K,
                               cudaStream_t st);
 
 struct GemmArgsW8 {
-  const uint16_t* a;       // x_perm [Rmax, H]
+  const uint16_t* a;       // x_perm [Rmax, H], IEEE half
   const int32_t* offsets;  // [E+1], multiples of 128
-  const int8_t* q1;        // blocked codes of w1 [E*I/128][H/64][128][64]
-  const int8_t* q3;        // same for w3
-  const int8_t* q2;        // blocked codes of w2 [E*H/128][I/64][128][64]
+  const uint8_t* q1;       // tiled offset-binary codes of w1 (rows E*I, K = H)
+  const uint8_t* q3;       // same for w3
+  const uint8_t* q2;       // tiled codes of w2 (rows E*H, K = I)
   const float* s1;         // [E*I]
   const float* s3;         // [E*I]
   const float* s2;         // [E*H]
-  uint16_t* h;             // [Rmax, I]
+  uint16_t* h;             // [Rmax, I], IEEE half
   float* y;                // [Rmax, H]
   int32_t* status;
   int64_t rmax;
   unsigned long long timeout_ns;
 };
 
-// GEMM1 (int8 gate/up + SwiGLU -> h) then GEMM2 (h q2^T * s2 -> y).
+// GEMM1 (int8 gate/up + SwiGLU -> h) then GEMM2 (h q2^T * s2 -> y), in float16.
 cudaError_t launch_grouped_swiglu_w8(const Shape& s, const GemmArgsW8& g, cudaStream_t st,
                                      const char** why);
 

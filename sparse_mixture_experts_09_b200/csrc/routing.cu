@@ -387,9 +387,22 @@ __global__ void __launch_bounds__(1024) k_plan_small(const int32_t* __restrict__
   }
 }
 
-// One warp per row of x_perm below R_pad: copies x[token] or, on pad rows, writes
-// zeros and token -1.
-template <bool NORM>
+// 8 bf16 values -> 8 IEEE half values (round to nearest even; exact for magnitudes in
+// [2^-14, 65504], larger ones become infinite).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint4 to_f16x8(uint4 v) {
+  return make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
+                    bf16x2_to_f16x2(v.w));
+}
+
+// One warp per row of x_perm below R_pad: copies x[token] (as bf16, or converted to
+// float16 when F16) or, on pad rows, writes zeros and token -1.
+template <bool NORM, bool F16>
 __global__ void __launch_bounds__(256) k_gather(const uint16_t* __restrict__ x, int H, int E,
                                                 const int32_t* __restrict__ counts,
                                                 const int32_t* __restrict__ offsets,
@@ -423,7 +436,14 @@ __global__ void __launch_bounds__(256) k_gather(const uint16_t* __restrict__ x, 
       const uint4* src = reinterpret_cast<const uint4*>(x + t * H);
       const uint4* g = reinterpret_cast<const uint4*>(norm_w);
       const float rn = rnorm[t];
-      for (int c = lane; c < chunks; c += 32) dst[c] = norm8(__ldg(src + c), __ldg(g + c), rn);
+      for (int c = lane; c < chunks; c += 32) {
+        const uint4 v = norm8(__ldg(src + c), __ldg(g + c), rn);
+        dst[c] = F16 ? to_f16x8(v) : v;
+      }
+    } else if (F16) {
+      const int64_t t = token_of_row[r];
+      const uint4* src = reinterpret_cast<const uint4*>(x + t * H);
+      for (int c = lane; c < chunks; c += 32) dst[c] = to_f16x8(__ldg(src + c));
     } else {
       const int64_t t = token_of_row[r];
       const uint4* src = reinterpret_cast<const uint4*>(x + t * H);
@@ -482,7 +502,8 @@ cudaError_t launch_router(const Shape& s, const uint16_t* x, const uint16_t* w_r
 cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16_t* x,
                            int32_t* counts, int32_t* offsets, int32_t* row_of,
                            int32_t* token_of_row, uint16_t* x_perm, int32_t* block_base,
-                           cudaStream_t st, const uint16_t* norm_w, const float* rnorm) {
+                           cudaStream_t st, const uint16_t* norm_w, const float* rnorm,
+                           bool f16_out) {
   const int64_t nb = num_token_blocks(s);
   cudaError_t e;
   if (nb <= 32) {
@@ -504,11 +525,12 @@ cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16
   int64_t gblocks = (max_padded_rows(s) + 7) / 8;
   const int64_t cap = (int64_t)num_sms() * 8;
   if (gblocks > cap) gblocks = cap;
-  if (norm_w)
-    return launch_pdl(k_gather<true>, dim3((unsigned)gblocks), dim3(256), 0, st, x, s.H, s.E,
-                      counts, offsets, token_of_row, x_perm, norm_w, rnorm);
-  return launch_pdl(k_gather<false>, dim3((unsigned)gblocks), dim3(256), 0, st, x, s.H, s.E, counts,
-                    offsets, token_of_row, x_perm, norm_w, rnorm);
+#define MOE_GATHER(NM, FH)                                                                   \
+  launch_pdl(k_gather<NM, FH>, dim3((unsigned)gblocks), dim3(256), 0, st, x, s.H, s.E, counts, \
+             offsets, token_of_row, x_perm, norm_w, rnorm)
+  if (norm_w) return f16_out ? MOE_GATHER(true, true) : MOE_GATHER(true, false);
+  return f16_out ? MOE_GATHER(false, true) : MOE_GATHER(false, false);
+#undef MOE_GATHER
 }
 
 }  // namespace moe

@@ -33,8 +33,9 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_size_host", "moe_max_padded_rows
 @dataclass
 class Int8Experts:
     """Weight-only int8 experts as written by quantize_int8: codes q1, q3 [E, I, H] and
-    q2 [E, H, I] int8 in the blocked layout [rows/128][K/64][128][64] (same number of
-    elements), per-row scales s1, s3 [E, I] and s2 [E, H] fp32."""
+    q2 [E, H, I] (uint8, offset-binary q + 128, in the library's tiled code layout of
+    include/moe.h; same number of elements), per-row scales s1, s3 [E, I] and s2 [E, H]
+    fp32."""
     q1: torch.Tensor
     q3: torch.Tensor
     q2: torch.Tensor
@@ -43,8 +44,8 @@ class Int8Experts:
     s2: torch.Tensor
 
     def pointers(self):
-        return [_dev(self.q1, "q1", torch.int8), _dev(self.q3, "q3", torch.int8),
-                _dev(self.q2, "q2", torch.int8), _dev(self.s1, "s1", torch.float32),
+        return [_dev(self.q1, "q1", torch.uint8), _dev(self.q3, "q3", torch.uint8),
+                _dev(self.q2, "q2", torch.uint8), _dev(self.s1, "s1", torch.float32),
                 _dev(self.s3, "s3", torch.float32), _dev(self.s2, "s2", torch.float32)]
 
 
@@ -387,7 +388,7 @@ def quantize_int8(w1, w3, w2, stream=None) -> Int8Experts:
     e, i, h = w1.shape
     shape = make_shape(1, h, i, e, 1)
     dev = w1.device
-    q = [torch.empty(t.shape, dtype=torch.int8, device=dev) for t in (w1, w3, w2)]
+    q = [torch.empty(t.shape, dtype=torch.uint8, device=dev) for t in (w1, w3, w2)]
     sc = [torch.empty((e, i), dtype=torch.float32, device=dev),
           torch.empty((e, i), dtype=torch.float32, device=dev),
           torch.empty((e, h), dtype=torch.float32, device=dev)]

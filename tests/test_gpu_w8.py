@@ -1,6 +1,6 @@
-"""Weight-only int8 experts (W8A16): the quantiser's codes and scales equal the
-oracle's bit for bit, and the int8 grouped GEMMs and the whole int8 layer match the
-oracle's layer run on the dequantised weights q * s."""
+"""Weight-only int8 experts: the quantiser's codes and scales equal the oracle's bit
+for bit, and the int8 grouped GEMMs and the whole int8 layer match the oracle's
+half-precision expert mode run on the dequantised weights q * s."""
 import numpy as np
 import pytest
 import torch
@@ -16,9 +16,11 @@ pytestmark = pytest.mark.gpu
 
 
 def _unblock(q):
-    # blocked codes [E*R/128][K/64][128][64] -> row-major [E, R, K]
+    """Tiled offset-binary codes -> row-major int8 [E, R, K]. Tile (row tile, column
+    tile) is 8 KiB: [column chunk v (16 columns)][row][16 columns]."""
     e, r, k = q.shape
-    return q.reshape(e * r // 128, k // 64, 128, 64).permute(0, 2, 1, 3).reshape(e, r, k)
+    t = q.reshape(e * r // 128, k // 64, 4, 128, 16).permute(0, 3, 1, 2, 4).reshape(e, r, k)
+    return (t.to(torch.int16) - 128).to(torch.int8)
 
 
 def _oracle_experts(c):
@@ -54,17 +56,30 @@ def test_quantize_matches_oracle(name):
         q, s = O.quantize_int8_rows(src.cpu())
         assert np.array_equal(_unblock(q_gpu).cpu().numpy(), q)
         assert np.array_equal(s_gpu.cpu().numpy().view(np.uint32), s.view(np.uint32))
-    assert float(ex.s1[0, 5]) == 1.0 and int(ex.q1.reshape(-1).abs().max()) == 127
+    codes = _unblock(ex.q1)
+    assert float(ex.s1[0, 5]) == 1.0 and int(codes[0, 5].abs().max()) == 0
+    assert int(codes.to(torch.int16).abs().max()) == 127
 
 
-@pytest.mark.parametrize("name", list(SMALL))
+# Few tokens (one row tile per expert, mostly padding): an odd token count, many
+# experts with k = 8, a hidden size that is not a multiple of 256, k = 1.
+SMALL_BATCH = {
+    "ts_t33": W.Workload("ts_t33", 33, 256, 384, 8, 2, seed=31),
+    "ts_e64k8": W.Workload("ts_e64k8", 50, 256, 256, 64, 8, seed=32),
+    "ts_h640": W.Workload("ts_h640", 48, 640, 512, 16, 4, seed=33),
+    "ts_k1": W.Workload("ts_k1", 7, 128, 1024, 4, 1, seed=34),
+}
+CASES = {**SMALL, **SMALL_BATCH}
+
+
+@pytest.mark.parametrize("name", list(CASES))
 def test_grouped_swiglu_w8_matches_oracle(name):
-    w = SMALL[name]
+    w = CASES[name]
     inp, _ = screened(w)
     c = to_cpu(inp)
     k = w.num_experts_per_tok
     (q1, _, d1), (q3, _, d3), (q2, _, d2) = _oracle_experts(c)
-    ref = O.moe_layer(c.x, c.w_router, d1, d3, d2, k, logit_bias=c.logit_bias, mode="bf16_storage")
+    ref = O.moe_layer(c.x, c.w_router, d1, d3, d2, k, logit_bias=c.logit_bias, mode="f16_experts")
     ex = M.quantize_int8(inp.w1, inp.w3, inp.w2)
     shape = M.make_shape(*w.shape)
     ws = M.make_workspace(shape)
@@ -79,9 +94,10 @@ def test_grouped_swiglu_w8_matches_oracle(name):
     assert np.all(y.cpu().numpy()[: tok.size][tok < 0] == 0)
 
 
-@pytest.mark.parametrize("name", ["tiny", "ragged", "e5k3", "one_token", "skewed", "bn128_split"])
+@pytest.mark.parametrize("name", ["tiny", "ragged", "e5k3", "one_token", "skewed", "bn128_split",
+                                  "ts_t33", "ts_e64k8", "ts_h640"])
 def test_forward_w8_matches_oracle(name):
-    w = SMALL[name]
+    w = CASES[name]
     inp, near = screened(w)
     assert near.numel() == 0
     c = to_cpu(inp)
@@ -95,7 +111,7 @@ def test_forward_w8_matches_oracle(name):
         M.device_status(ws)
         ref = O.moe_layer(c.x, c.w_router, d1, d3, d2, k,
                           residual=None if residual is None else c.residual,
-                          logit_bias=c.logit_bias, mode="bf16_storage")
+                          logit_bias=c.logit_bias, mode="f16_experts")
         assert_layer_close(O.to_f64(out.cpu()), ref["out"], name)
 
 
@@ -115,9 +131,9 @@ def test_forward_w8_full_size_against_oracle(name):
     tokens = sample_tokens(w.num_tokens)
     c = to_cpu(inp)
     deq = [_Dequantised(t) for t in (c.w1, c.w3, c.w2)]
-    ref = O.moe_layer(c.x, c.w_router, deq[0], deq[1], deq[2], 2, mode="bf16_storage", tokens=tokens)
+    ref = O.moe_layer(c.x, c.w_router, deq[0], deq[1], deq[2], 2, mode="f16_experts", tokens=tokens)
     assert_layer_close(O.to_f64(out.cpu())[tokens], ref["out"], name)
-    # the int8 layer stays close to the bf16 layer (quantisation error only)
+    # the int8 layer stays close to the bf16 layer (quantisation and half rounding)
     out_bf16 = M.forward(inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, 2)
     rel = (out.double() - out_bf16.double()).norm() / out_bf16.double().norm()
     assert float(rel) < 4e-2
