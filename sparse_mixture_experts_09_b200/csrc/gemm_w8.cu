@@ -16,7 +16,8 @@
 // codes; a bf16 has 7 mantissa bits and needs twice the integer work.
 //
 // Kernel k_grouped_gemm_w8: the bf16 GEMM's persistent tile loop with a widening
-// stage. Warp roles:
+// stage, on 128-row tiles, or on 64-row tiles (tcgen05 M = 64) when the batch has at
+// most 64 tokens. Warp roles:
 //   warp 0      streams the code tiles (bulk copies: each 128-row x 64-code tile is one
 //               contiguous 8 KiB run) into a code ring;
 //   warp 6      loads the activation tiles (TMA, 128-byte swizzle) into their ring;
@@ -43,36 +44,49 @@ constexpr int BM = 128, BK = 64;
 #ifndef MOE_W8_CODE_STAGES
 #define MOE_W8_CODE_STAGES 4
 #endif
+#ifndef MOE_W8_CODE_STAGES_M64
+#define MOE_W8_CODE_STAGES_M64 6
+#endif
+#ifndef MOE_W8_A_STAGES_M64
+#define MOE_W8_A_STAGES_M64 4
+#endif
 #ifndef MOE_W8_CONV_WARPS
 #define MOE_W8_CONV_WARPS 8
 #endif
-// Three rings: activation tiles (TMA -> MMA), int8 code tiles (TMA -> converters) and
-// widened weight tiles (converters -> MMA). The activation ring is deep enough to hide
-// its L2 latency on its own; the widened ring only decouples widening from the MMA.
-constexpr int kAStages = MOE_W8_A_STAGES;
-constexpr int kBStages = MOE_W8_B_STAGES;
-constexpr int kCodeStages = MOE_W8_CODE_STAGES;
 constexpr int kConvWarps = MOE_W8_CONV_WARPS;
 // warp 0: code copies, 1: MMA, 2-5: epilogue, 6: activation TMA, 7..: converters
 constexpr int kConvWarp0 = 7;
 constexpr int kThreadsW8 = 32 * (kConvWarp0 + kConvWarps);
-constexpr int A_BYTES = BM * BK * 2;  // 16 KiB
 constexpr int kSwiGLU = 0, kPlain = 1;
-constexpr int kNumBars = 2 * (kAStages + kBStages + kCodeStages) + 5;
+#ifndef MOE_W8_HALF_TILES
+#define MOE_W8_HALF_TILES 1
+#endif
+constexpr bool kUseHalfTiles = MOE_W8_HALF_TILES != 0;
 
-// Per-BN shared-memory plan: [A ring][B ring][code ring][barriers, TMEM address, row tiles]
-template <int BN>
+// Shared-memory plan for an MT x BN tile: [A ring][B ring][code ring][barriers, TMEM
+// address, row tiles]. Three rings: activation tiles (TMA -> MMA), code tiles (bulk
+// copy -> converters) and widened weight tiles (converters -> MMA). MT = 128 rows, or
+// 64 when every expert has at most 64 routed rows (the tile's first 64 rows hold all
+// of them): then the tensor core does half the work per k-block, and the 8 KiB saved
+// per activation stage buys deeper code prefetch.
+template <int BN, int MT>
 struct TileW8 {
+  static constexpr int A_ST = MT == 64 ? MOE_W8_A_STAGES_M64 : MOE_W8_A_STAGES;
+  static constexpr int B_ST = MOE_W8_B_STAGES;
+  static constexpr int Q_ST = MT == 64 ? MOE_W8_CODE_STAGES_M64 : MOE_W8_CODE_STAGES;
+  static constexpr int A_BYTES = MT * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int Q_BYTES = BN * BK;
-  static constexpr int B_OFF = kAStages * A_BYTES;
-  static constexpr int Q_OFF = B_OFF + kBStages * B_BYTES;
-  static constexpr int BAR_OFF = Q_OFF + kCodeStages * Q_BYTES;
-  static constexpr int SMEM = 1024 + BAR_OFF + kNumBars * 8 + 8 + 65 * 4;
+  static constexpr int B_OFF = A_ST * A_BYTES;
+  static constexpr int Q_OFF = B_OFF + B_ST * B_BYTES;
+  static constexpr int BAR_OFF = Q_OFF + Q_ST * Q_BYTES;
+  static constexpr int NUM_BARS = 2 * (A_ST + B_ST + Q_ST) + 5;
+  static constexpr int SMEM = 1024 + BAR_OFF + NUM_BARS * 8 + 8 + 65 * 4;
   static constexpr int CHUNKS = BN * BK / 16 / (32 * kConvWarps);  // code chunks per thread
-  // D f32, A and B f16 (format 0), both K-major
+  // D f32, A and B f16 (format 0), both K-major, M = MT, N = BN
   static constexpr uint32_t IDESC =
-      (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+      (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(MT >> 4) << 24);
+  static_assert(MT == 64 || MT == 128, "tile rows");
   static_assert(SMEM <= 232448, "shared memory plan exceeds 227 KiB");
   static_assert(CHUNKS * 32 * kConvWarps * 16 == BN * BK, "converter split");
 };
@@ -265,10 +279,12 @@ __device__ __forceinline__ uint32_t pack_f16x2_rn(float lo, float hi) {
 // MODE kSwiGLU: A = x_perm [rows, H] (half), weight tile = 128 rows of w1 then 128 rows
 //   of w3 (BN = 256), h = half(silu(s1 * gate) * (s3 * up)).
 // MODE kPlain:  A = h [rows, I], weight tile = BN rows of w2, y = s2 * acc (fp32).
-template <int MODE, int BN>
+template <int MODE, int BN, int MT>
 __global__ void __launch_bounds__(kThreadsW8, 1)
     k_grouped_gemm_w8(const __grid_constant__ CUtensorMap mapA, const W8Params p) {
-  using TL = TileW8<BN>;
+  using TL = TileW8<BN, MT>;
+  constexpr int kAStages = TL::A_ST, kBStages = TL::B_ST, kCodeStages = TL::Q_ST;
+  constexpr int A_BYTES = TL::A_BYTES;
   static_assert(MODE == kPlain || BN == 256, "gate/up tiles hold 128 gate + 128 up columns");
   constexpr uint32_t kTmemCols = 2 * BN;  // two accumulators
   extern __shared__ uint8_t smem_raw[];
@@ -277,7 +293,7 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
   uint8_t* bbase = smem + TL::B_OFF;
   uint8_t* qbase = smem + TL::Q_OFF;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TL::BAR_OFF);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + TL::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* row_tiles = reinterpret_cast<int*>(tmem_holder + 2);
 
@@ -486,9 +502,11 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
       }
     }
   } else {
-    // ---------------- epilogue: warps 2..5, TMEM lanes 32 (warp % 4) ..
+    // ---------------- epilogue: warps 2..5, TMEM lanes 32 (warp % 4) ..; with MT = 64
+    // rows 16 q .. 16 q + 15 sit in the first 16 lanes of quarter q
     const int qd = warp & 3;
-    const int row_in_tile = qd * 32 + lane;
+    const int row_in_tile = MT == 128 ? qd * 32 + lane : qd * 16 + lane;
+    const bool row_valid = MT == 128 || lane < 16;
     int tc = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x, ++tc) {
       int e, m, n;
@@ -518,9 +536,11 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
             const float u1 = __uint_as_float(u[2 * i + 1]) * __ldg(su + c + 2 * i + 1);
             pk[i] = pack_f16x2_rn(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1);
           }
-          uint4* dst = reinterpret_cast<uint4*>(h + c);
-          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          if (row_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(h + c);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
         }
       } else {
         const float* sc = p.scale_a + (size_t)e * p.b_rows + n * BN;
@@ -532,7 +552,7 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
           tmem_wait_ld();
           float4* dst = reinterpret_cast<float4*>(y + c);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
+          for (int i = 0; i < 4 && row_valid; ++i)
             dst[i] = make_float4(__uint_as_float(v[4 * i]) * __ldg(sc + c + 4 * i),
                                  __uint_as_float(v[4 * i + 1]) * __ldg(sc + c + 4 * i + 1),
                                  __uint_as_float(v[4 * i + 2]) * __ldg(sc + c + 4 * i + 2),
@@ -622,37 +642,37 @@ EncodeTiledFnW8 encode_w8() {
   return fn;
 }
 
-// half activations [rows, inner], box 64 x 128, 128-byte swizzle
-bool map_act(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
+// half activations [rows, inner], box 64 x box_rows, 128-byte swizzle
+bool map_act(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
   EncodeTiledFnW8 fn = encode_w8();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, rows};
   const cuuint64_t strides[1] = {inner * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)BK, 128};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, int MT>
 cudaError_t launch_w8(const CUtensorMap& a, const W8Params& p, int64_t max_tiles,
                       cudaStream_t st) {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm_w8<MODE, BN>,
+    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm_w8<MODE, BN, MT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         TileW8<BN>::SMEM);
+                                         TileW8<BN, MT>::SMEM);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   int64_t grid = num_sms();
   if (grid > max_tiles) grid = max_tiles;
   if (grid < 1) grid = 1;
-  return launch_pdl(k_grouped_gemm_w8<MODE, BN>, dim3((unsigned)grid), dim3(kThreadsW8),
-                    (size_t)TileW8<BN>::SMEM, st, a, p);
+  return launch_pdl(k_grouped_gemm_w8<MODE, BN, MT>, dim3((unsigned)grid), dim3(kThreadsW8),
+                    (size_t)TileW8<BN, MT>::SMEM, st, a, p);
 }
 
 }  // namespace
@@ -676,10 +696,14 @@ cudaError_t launch_quant_rows(const uint16_t* w, uint8_t* q, float* s, int64_t r
   return launch_pdl(k_quant_rows, dim3((unsigned)blocks), dim3(256), 0, st, w, q, s, rows, K);
 }
 
-cudaError_t launch_grouped_swiglu_w8(const Shape& s, const GemmArgsW8& g, cudaStream_t st,
-                                     const char** why) {
+namespace {
+
+// Both GEMMs with MT-row tiles (see TileW8)
+template <int MT>
+cudaError_t launch_swiglu_w8_tiles(const Shape& s, const GemmArgsW8& g, cudaStream_t st,
+                                   const char** why) {
   CUtensorMap mx, mh;
-  if (!map_act(&mx, g.a, s.H, g.rmax) || !map_act(&mh, g.h, s.I, g.rmax)) {
+  if (!map_act(&mx, g.a, s.H, g.rmax, MT) || !map_act(&mh, g.h, s.I, g.rmax, MT)) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad tensor)";
     return cudaErrorInvalidValue;
   }
@@ -698,7 +722,7 @@ cudaError_t launch_grouped_swiglu_w8(const Shape& s, const GemmArgsW8& g, cudaSt
   p1.n_tiles = s.I / 128;
   p1.b_rows = s.I;
   p1.timeout_ns = g.timeout_ns;
-  cudaError_t e = launch_w8<kSwiGLU, 256>(mx, p1, mt_max * p1.n_tiles, st);
+  cudaError_t e = launch_w8<kSwiGLU, 256, MT>(mx, p1, mt_max * p1.n_tiles, st);
   if (e != cudaSuccess) {
     *why = "int8 gate/up GEMM launch failed";
     return e;
@@ -714,13 +738,23 @@ cudaError_t launch_grouped_swiglu_w8(const Shape& s, const GemmArgsW8& g, cudaSt
   p2.b_rows = s.H;
   if (s.H % 256 == 0) {
     p2.n_tiles = s.H / 256;
-    e = launch_w8<kPlain, 256>(mh, p2, mt_max * p2.n_tiles, st);
+    e = launch_w8<kPlain, 256, MT>(mh, p2, mt_max * p2.n_tiles, st);
   } else {
     p2.n_tiles = s.H / 128;
-    e = launch_w8<kPlain, 128>(mh, p2, mt_max * p2.n_tiles, st);
+    e = launch_w8<kPlain, 128, MT>(mh, p2, mt_max * p2.n_tiles, st);
   }
   if (e != cudaSuccess) *why = "int8 down GEMM launch failed";
   return e;
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_swiglu_w8(const Shape& s, const GemmArgsW8& g, cudaStream_t st,
+                                     const char** why) {
+  // a token is routed to an expert at most once, so with at most 64 tokens every expert
+  // has at most 64 rows, all in the first half of its 128-row tile
+  if (s.T <= 64 && kUseHalfTiles) return launch_swiglu_w8_tiles<64>(s, g, st, why);
+  return launch_swiglu_w8_tiles<128>(s, g, st, why);
 }
 
 }  // namespace moe
