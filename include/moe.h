@@ -162,7 +162,8 @@ moe_status_t moe_permute_static(const moe_shape_t* shape, const int32_t* topk_id
  *   GEMM2: y_perm = h w2[e]^T, fp32.
  *   x_perm [R_pad, H] bf16 and expert_offsets [E+1] int32 as written by moe_permute;
  *   w1, w3 [E, I, H] bf16; w2 [E, H, I] bf16;
- *   y_perm [moe_max_padded_rows, H] fp32 out (rows past R_pad untouched). */
+ *   y_perm [moe_max_padded_rows, H] fp32 out for the routed rows (pad rows hold zero
+ *     or are left untouched; rows past R_pad untouched). */
 moe_status_t moe_grouped_swiglu(const moe_shape_t* shape, const moe_bf16_t* x_perm,
                                 const int32_t* expert_offsets, const moe_bf16_t* w1,
                                 const moe_bf16_t* w3, const moe_bf16_t* w2,
@@ -172,7 +173,7 @@ moe_status_t moe_grouped_swiglu(const moe_shape_t* shape, const moe_bf16_t* x_pe
 /* The two halves of moe_grouped_swiglu, for callers that keep h themselves or time
  * the GEMMs apart. `ws` as for moe_grouped_swiglu (ws_bytes >= moe_workspace_size).
  *   moe_expert_gate_up: h [moe_max_padded_rows, I] bf16 out = bf16(silu(x_perm
- *     w1[e]^T) * (x_perm w3[e]^T)) for the rows below R_pad;
+ *     w1[e]^T) * (x_perm w3[e]^T)) for the routed rows (pad rows zero or untouched);
  *   moe_expert_down: y_perm [moe_max_padded_rows, H] fp32 out = h w2[e]^T. */
 moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* x_perm,
                                 const int32_t* expert_offsets, const moe_bf16_t* w1,
