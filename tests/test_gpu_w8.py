@@ -61,13 +61,18 @@ def test_quantize_matches_oracle(name):
     assert int(codes.to(torch.int16).abs().max()) == 127
 
 
-# Few tokens (one row tile per expert, mostly padding): an odd token count, many
-# experts with k = 8, a hidden size that is not a multiple of 256, k = 1.
+# Few tokens (one row tile per expert, mostly padding; at most 64 tokens run on 64-row
+# tiles): an odd token count, many experts with k = 8, a hidden size that is not a
+# multiple of 256, k = 1, and both sides of the 64-token switch with every token on
+# both of 2 experts (64 and 65 rows per expert).
 SMALL_BATCH = {
     "ts_t33": W.Workload("ts_t33", 33, 256, 384, 8, 2, seed=31),
     "ts_e64k8": W.Workload("ts_e64k8", 50, 256, 256, 64, 8, seed=32),
     "ts_h640": W.Workload("ts_h640", 48, 640, 512, 16, 4, seed=33),
     "ts_k1": W.Workload("ts_k1", 7, 128, 1024, 4, 1, seed=34),
+    # 64 tokens is the last batch on 64-row tiles; 65 takes the 128-row tiles
+    "t64_edge": W.Workload("t64_edge", 64, 256, 256, 2, 2, seed=35),
+    "t65_edge": W.Workload("t65_edge", 65, 256, 256, 2, 2, seed=36),
 }
 CASES = {**SMALL, **SMALL_BATCH}
 
@@ -95,7 +100,7 @@ def test_grouped_swiglu_w8_matches_oracle(name):
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged", "e5k3", "one_token", "skewed", "bn128_split",
-                                  "ts_t33", "ts_e64k8", "ts_h640"])
+                                  "ts_t33", "ts_e64k8", "ts_h640", "t64_edge", "t65_edge"])
 def test_forward_w8_matches_oracle(name):
     w = CASES[name]
     inp, near = screened(w)
