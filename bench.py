@@ -178,7 +178,7 @@ def run_reference(args):
         return 0
     import torch
     from sparse_mixture_experts_09_b200 import workloads as W
-    w = W.WORKLOADS[args.workload]
+    w = W.workload(args.workload)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = W.draw(w, dev)
     inp = W.LayerInputs(*(None if t is None else t.cpu() for t in
@@ -300,7 +300,7 @@ def run_ours(args):
             dist.barrier()
 
     moe.lib()  # fail loudly if the library is missing
-    w = W.WORKLOADS[args.workload]
+    w = W.workload(args.workload)
     inp = W.draw(w, dev)
     k = w.num_experts_per_tok
     # the expert weights live in the library's blocked layout, converted once at load

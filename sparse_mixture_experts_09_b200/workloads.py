@@ -84,6 +84,16 @@ def decode_sweep():
     return [WORKLOADS["larger"].with_tokens(t, f"larger_decode_T{t}") for t in DECODE_SWEEP_TOKENS]
 
 
+def workload(name: str) -> "Workload":
+    """A named workload, or one of the decode sweep's (larger_decode_T<t>)."""
+    if name in WORKLOADS:
+        return WORKLOADS[name]
+    sweep = {w.name: w for w in decode_sweep()}
+    if name in sweep:
+        return sweep[name]
+    raise KeyError(f"unknown workload {name!r}: one of {sorted(WORKLOADS) + sorted(sweep)}")
+
+
 @dataclass
 class LayerInputs:
     """bf16 tensors of one layer: x [T,H], w_router [E,H], w1/w3 [E,I,H], w2 [E,H,I],
