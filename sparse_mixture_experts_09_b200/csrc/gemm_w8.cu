@@ -101,7 +101,6 @@ struct W8Params {
   void* out;
   int64_t out_ld;
   int E, k_blocks, n_tiles, b_rows;
-  int n_cols;  // small-batch kernel: token columns N (multiple of 16, at most 64)
   unsigned long long timeout_ns;
 };
 
@@ -234,7 +233,8 @@ __device__ __forceinline__ void tile_coords_w8(int L, const int* row_tiles, int 
   m = row_tiles[e] + local % cnt;
 }
 
-// y coordinate of weight row `row` (multiple of 128), k-block kb, in the blocked code map
+// Tile number (times 128) of weight rows row .. row+127 (row a multiple of 128) and
+// k-block kb in the tiled code layout; times 64 bytes it is the tile's byte offset
 __device__ __forceinline__ int code_y(int row, int kb, int k_blocks) {
   return ((row >> 7) * k_blocks + kb) * 128;
 }
