@@ -290,6 +290,19 @@ moe_status_t moe_forward_w8(const moe_shape_t* shape, const moe_bf16_t* x,
                             const moe_bf16_t* residual, moe_bf16_t* out, void* ws,
                             size_t ws_bytes, moe_stream_t stream);
 
+/* Row gather for the expert-parallel layer (this library's own step; the pages say
+ * only that experts may be spread over devices, Hugging Face "Mixtral", MixtralConfig
+ * num_local_experts): dst[i, :] = src[index[i], :] for 0 <= i < n_rows. A rank
+ * regroups the rows it received from its peers (ordered by source rank, then expert)
+ * into expert-contiguous groups with it, and restores the order after the experts.
+ *   src [src_rows, row_bytes] and dst [n_rows, row_bytes] device buffers, row_bytes a
+ *   positive multiple of 16, 16-byte aligned; index [n_rows] int64 device array. An
+ *   index outside [0, src_rows) writes a zero row (so pad rows can be produced and no
+ *   read leaves src). n_rows = 0 is a no-op. src and dst must not overlap. */
+moe_status_t moe_gather_rows(const void* src, int64_t src_rows, const int64_t* index,
+                             int64_t n_rows, int64_t row_bytes, void* dst,
+                             moe_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the device status word in `ws`:
  * MOE_OK, or MOE_ERR_TIMEOUT if a kernel gave up a bounded wait since the last
  * call. */

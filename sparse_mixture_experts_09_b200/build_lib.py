@@ -17,7 +17,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoe.so")
-SOURCES = ["moe_api.cu", "routing.cu", "gemm_sm100.cu", "gemm_w8.cu", "combine.cu", "moe_noalloc.cu"]
+SOURCES = ["moe_api.cu", "routing.cu", "gemm_sm100.cu", "gemm_w8.cu", "combine.cu", "moe_noalloc.cu",
+           "gather_rows.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

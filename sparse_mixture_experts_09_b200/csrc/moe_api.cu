@@ -591,4 +591,20 @@ moe_status_t moe_forward_w8(const moe_shape_t* shape, const moe_bf16_t* x,
                      out, ws, (cudaStream_t)stream);
 }
 
+moe_status_t moe_gather_rows(const void* src, int64_t src_rows, const int64_t* index,
+                             int64_t n_rows, int64_t row_bytes, void* dst, moe_stream_t stream) {
+  g_err[0] = 0;
+  if (n_rows < 0 || src_rows < 0) return fail(MOE_ERR_INVALID_ARG, "row counts must be >= 0");
+  if (row_bytes <= 0 || row_bytes % 16)
+    return fail(MOE_ERR_INVALID_ARG, "row_bytes must be a positive multiple of 16 (got %lld)",
+                (long long)row_bytes);
+  if (n_rows == 0) return MOE_OK;
+  MOE_TRY(check_ptr(src, "src", src_rows == 0));
+  MOE_TRY(check_ptr(index, "index"));
+  MOE_TRY(check_ptr(dst, "dst"));
+  cudaError_t e = launch_gather_rows(src, dst, index, n_rows, src_rows, row_bytes,
+                                     (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "row gather launch");
+}
+
 }  // extern "C"

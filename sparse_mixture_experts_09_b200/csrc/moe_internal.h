@@ -110,6 +110,11 @@ cudaError_t launch_combine(const Shape& s, const float* y, const int32_t* row_of
                            const float* topk_w, const uint16_t* residual, uint16_t* out,
                            cudaStream_t st);
 
+// dst[i] = src[index[i]] for i < n_rows, rows of row_bytes (a multiple of 16) bytes;
+// an index outside [0, src_rows) writes a zero row.
+cudaError_t launch_gather_rows(const void* src, void* dst, const int64_t* index, int64_t n_rows,
+                               int64_t src_rows, int64_t row_bytes, cudaStream_t st);
+
 int num_sms();
 
 // Host helpers of the C ABI (moe_api.cu): shape validation returning a moe_status_t

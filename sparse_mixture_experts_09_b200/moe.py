@@ -27,7 +27,7 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_size_host", "moe_max_padded_rows
            "moe_expert_down", "moe_combine", "moe_forward",
            "moe_forward_host", "moe_device_status", "moe_last_error", "moe_permute_static",
            "moe_selftest_wait_timeout", "moe_forward_rmsnorm", "moe_pack_weights",
-           "moe_quantize_int8", "moe_grouped_swiglu_w8", "moe_forward_w8")
+           "moe_quantize_int8", "moe_grouped_swiglu_w8", "moe_forward_w8", "moe_gather_rows")
 
 
 @dataclass
@@ -119,6 +119,8 @@ def lib() -> ctypes.CDLL:
         L.moe_grouped_swiglu_w8.restype = st
         L.moe_forward_w8.argtypes = [sp] + [_P] * 12 + [_SZ, _P]
         L.moe_forward_w8.restype = st
+        L.moe_gather_rows.argtypes = [_P, ctypes.c_int64, _P, ctypes.c_int64, ctypes.c_int64, _P, _P]
+        L.moe_gather_rows.restype = st
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         _lib = L
@@ -428,4 +430,18 @@ def forward_w8(x, w_router, experts: Int8Experts, k: int, residual=None, logit_b
                                 *experts.pointers(),
                                 _dev(residual, "residual", torch.bfloat16, True), _dev(out, "out"),
                                 _dev(ws, "ws"), ws.numel(), _stream(stream)))
+    return out
+
+
+def gather_rows(src, index, stream=None):
+    """out[i] = src[index[i]] (a zero row where index[i] is outside [0, len(src))); src is
+    a 2-D CUDA tensor whose rows are a multiple of 16 bytes, index an int64 CUDA tensor."""
+    if src.dim() != 2:
+        raise ValueError("src must be 2-D")
+    n = index.numel()
+    out = torch.empty((n, src.shape[1]), dtype=src.dtype, device=src.device)
+    row_bytes = src.shape[1] * src.element_size()
+    _check(lib().moe_gather_rows(_dev(src, "src") if src.shape[0] else None, src.shape[0],
+                                 _dev(index, "index", torch.int64) if n else None, n, row_bytes,
+                                 _dev(out, "dst") if n else None, _stream(stream)))
     return out

@@ -1,0 +1,153 @@
+"""Expert parallelism on CPU with gloo ranks: the exchange plan, and the whole
+expert-parallel layer with oracle stand-ins for the compute steps, against the
+single-process oracle layer (experts split over 2 and 4 ranks, uneven token counts,
+ranks that own no routed rows)."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+from sparse_mixture_experts_09_b200 import ep
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+class OracleOps:
+    """The layer's steps from the fp64 oracle on CPU tensors (test infrastructure)."""
+
+    def __init__(self):
+        from oracle import moe_oracle as O
+        self.O = O
+
+    def router_topk(self, x, w_router, k, logit_bias):
+        O = self.O
+        idx, w, _ = O.route_topk(O.router_logits(x, w_router, logit_bias), k)
+        return torch.from_numpy(idx), torch.from_numpy(w)
+
+    def permute(self, idx, x, num_experts, intermediate_size):
+        O = self.O
+        count, offset, row_of, tok = O.stable_permute(idx.numpy(), num_experts)
+        # rows keep x's dtype (exact copies), as the library's gather does
+        x_perm = torch.zeros((int(offset[-1]), x.shape[1]), dtype=x.dtype)
+        real = torch.from_numpy(tok >= 0)
+        x_perm[real] = x[torch.from_numpy(tok)[real]]
+        return {"counts": torch.from_numpy(count), "offsets": torch.from_numpy(offset),
+                "row_of": torch.from_numpy(row_of), "x_perm": x_perm}
+
+    def gather_rows(self, src, index):
+        out = torch.zeros((index.numel(), src.shape[1]), dtype=src.dtype)
+        ok = (index >= 0) & (index < src.shape[0])
+        out[ok] = src[index[ok]]
+        return out
+
+    def grouped_swiglu(self, x_groups, offsets, w1, w3, w2, rows):
+        y = torch.zeros((x_groups.shape[0], w2.shape[1]), dtype=torch.float64)
+        off = offsets.tolist()
+        for e in range(w1.shape[0]):
+            a, b = off[e], off[e + 1]
+            if b > a:
+                rows_e = self.O.to_f64(x_groups[a:b])
+                y[a:b] = torch.from_numpy(self.O.swiglu_expert(rows_e, w1[e], w3[e], w2[e]))
+        return y
+
+    def combine(self, y_perm, row_of, topk_w, residual, num_experts, intermediate_size):
+        out = torch.zeros((row_of.shape[0], y_perm.shape[1]), dtype=torch.float64)
+        for j in range(row_of.shape[1]):
+            out += topk_w[:, j:j + 1] * y_perm[row_of[:, j]]
+        if residual is not None:
+            out += residual.double()
+        return out
+
+    def padded_rows(self, rows, num_experts):
+        return (max(rows, 1) + 127) // 128 * 128 + 128 * num_experts
+
+
+def _layer_inputs(t_total, hd, inter, e, seed):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(t_total, hd, generator=g).to(torch.bfloat16)
+    wr = (torch.randn(e, hd, generator=g) / hd ** 0.5).to(torch.bfloat16)
+    w1 = (torch.randn(e, inter, hd, generator=g) / hd ** 0.5).to(torch.bfloat16)
+    w3 = (torch.randn(e, inter, hd, generator=g) / hd ** 0.5).to(torch.bfloat16)
+    w2 = (torch.randn(e, hd, inter, generator=g) / inter ** 0.5).to(torch.bfloat16)
+    res = torch.randn(t_total, hd, generator=g).to(torch.bfloat16)
+    return x, wr, w1, w3, w2, res
+
+
+def _rank(rank, world, port, q, tokens, e, k, bias):
+    import datetime
+    import sys
+    import torch.distributed as dist
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from sparse_mixture_experts_09_b200 import ep as EP
+    from tests.test_ep import OracleOps, _layer_inputs
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    x, wr, w1, w3, w2, res = _layer_inputs(sum(tokens), 32, 48, e, seed=7)
+    lo = sum(tokens[:rank])
+    mine = slice(lo, lo + tokens[rank])
+    l1, l3, l2 = EP.shard_experts(w1, w3, w2, rank, world)
+    b = None if bias is None else torch.tensor(bias, dtype=torch.float64)
+    out = EP.forward_ep(x[mine], wr, l1, l3, l2, k, e, residual=res[mine], logit_bias=b,
+                        ops=OracleOps())
+    q.put((rank, out.double().numpy()))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def _run(world, tokens, e, k, bias=None):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, world, port, q, tokens, e, k, bias))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    return np.concatenate([got[r] for r in range(world)])
+
+
+@pytest.mark.parametrize("world,tokens,e,k,bias", [
+    (2, [5, 9], 4, 2, None),
+    (4, [3, 0, 11, 6], 8, 2, None),
+    # all tokens go to experts 0 and 1 (rank 0): the other ranks receive nothing
+    (2, [7, 4], 4, 2, [30.0, 30.0, -30.0, -30.0]),
+    (2, [6, 6], 2, 1, None),
+])
+def test_expert_parallel_layer_equals_single_process_layer(world, tokens, e, k, bias):
+    from oracle import moe_oracle as O
+    got = _run(world, tokens, e, k, bias)
+    x, wr, w1, w3, w2, res = _layer_inputs(sum(tokens), 32, 48, e, seed=7)
+    b = None if bias is None else np.asarray(bias)
+    ref = O.moe_layer(x, wr, w1, w3, w2, k, residual=res, logit_bias=b, mode="exact")
+    np.testing.assert_allclose(got, ref["out"], rtol=1e-12, atol=1e-12)
+
+
+def test_exchange_plan_regroups_by_expert_and_inverts():
+    # rank with 2 local experts (E = 4 over 2 ranks); padded offsets of its own tokens
+    offsets = [0, 128, 384, 384, 512]
+    recv = [[128, 0], [256, 128]]          # from rank 0, from rank 1
+    send, recv_rows, local_off, to_local, to_recv = ep.exchange_plan(offsets, 2, recv)
+    assert send == [384, 128] and recv_rows == [128, 384]
+    # expert 0: source 0 rows 0..127, then source 1 rows 128..383; expert 1: 384..511
+    assert local_off == [0, 384, 512]
+    assert to_local == list(range(0, 128)) + list(range(128, 384)) + list(range(384, 512))
+    assert all(to_local[to_recv[i]] == i for i in range(512))
+    # a permutation when a source sends several experts' rows
+    send, recv_rows, local_off, to_local, to_recv = ep.exchange_plan(offsets, 2, [[128, 256],
+                                                                                  [128, 0]])
+    assert local_off == [0, 256, 512]
+    assert to_local[:256] == list(range(0, 128)) + list(range(384, 512))
+    assert sorted(to_local) == list(range(512))
+    assert all(to_local[to_recv[i]] == i for i in range(512))
