@@ -382,6 +382,13 @@ def run_ours(args):
         split_step(scratch)
         host_step()
     torch.cuda.synchronize(dev)
+    # the same forward captured once in a CUDA graph (replayed in loop 5)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize(dev)
     moe.device_status(ws)
     barrier()
 
@@ -452,6 +459,18 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     barrier()
     w8_ms = q0.elapsed_time(q1) / K
+
+    # (5) the default forward replayed from a CUDA graph
+    barrier()
+    torch.cuda.synchronize(dev)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(K):
+        graph.replay()
+    g1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    graph_ms = g0.elapsed_time(g1) / K
     clk = clocks.stop()
     moe.device_status(ws)
     moe.device_status(wsh)
@@ -460,6 +479,7 @@ def run_ours(args):
     ms, e2e_ms = slowest_rank(ms, e2e_ms, world, dev)
     rm_ms, _ = slowest_rank(rm_ms, rm_ms, world, dev)
     w8_ms, _ = slowest_rank(w8_ms, w8_ms, world, dev)
+    graph_ms, _ = slowest_rank(graph_ms, graph_ms, world, dev)
 
     counts = perm["counts"].cpu().tolist()
     peaks, peak_kind = load_peaks()
@@ -482,6 +502,9 @@ def run_ours(args):
             "kernels_ms": stage_ms,
             "row_major_weights": {"ms_per_step": rm_ms,
                                   "value": job_throughput(w.num_tokens, world, rm_ms)},
+            "cuda_graph": {"ms_per_step": graph_ms,
+                           "value": job_throughput(w.num_tokens, world, graph_ms),
+                           "note": "the default forward captured once, replayed"},
             "int8_experts": {"ms_per_step": w8_ms,
                              "value": job_throughput(w.num_tokens, world, w8_ms),
                              "api": "moe_forward_w8",
