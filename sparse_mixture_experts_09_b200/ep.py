@@ -9,16 +9,18 @@ only their weights; every rank keeps the router and routes its own tokens. One l
 1. route and permute this rank's tokens (the library's router and permutation): rows
    grouped by expert, each group padded to 128 rows, so the rows bound for rank r are
    one contiguous block;
-2. exchange per-expert padded row counts (all_to_all of E/W integers per peer);
-3. exchange the rows themselves (all_to_all_single, uneven splits): rank r receives,
-   from every source rank in turn, the padded groups of its own experts;
-4. regroup the received rows expert-contiguously (the library's row gather), run the
-   grouped SwiGLU experts on them, and restore the received order (row gather);
+2. exchange per-expert routed row counts (all_to_all of E/W integers per peer);
+3. exchange the rows themselves, without pad rows (a row gather packs them;
+   all_to_all_single, uneven splits): rank r receives, from every source rank in turn,
+   the rows of its own experts;
+4. regroup the received rows into expert groups padded to 128 rows (row gather), run
+   the grouped SwiGLU experts on them, and restore the received order (row gather);
 5. send every expert output back to the rank its token came from (all_to_all_single,
-   the splits of step 3 reversed), then combine into the residual there.
+   the splits of step 3 reversed), put it back in the permuted order (row gather) and
+   combine into the residual there.
 
 Every arithmetic step runs in the library's kernels; this module only plans the
-exchange on the host (it reads the E+1 group offsets back, one synchronisation) and
+exchange on the host (it reads the group offsets and counts back, one synchronisation) and
 calls torch.distributed, whose collectives are NCCL on GPUs. The compute steps are
 reached through an ``ops`` object (``CudaOps`` by default), so the same plan can be
 exercised with other implementations of the steps.
@@ -68,41 +70,62 @@ class CudaOps:
         return self.moe.max_padded_rows(shape)
 
 
-def exchange_plan(offsets, world: int, recv_counts):
-    """Host-side plan of one exchange.
+def _pad(n: int) -> int:
+    return (n + 127) // 128 * 128
 
-    offsets: this rank's padded group offsets [E+1] (E = world * E_loc experts);
-    recv_counts: [world, E_loc] padded rows this rank receives for each of its experts
-    from each source rank.
-    Returns (send_rows [world], recv_rows [world], local_offsets [E_loc+1],
-    to_local [n_recv], to_recv [n_recv]): rows sent to / received from each rank; the
-    expert-contiguous layout of the received rows (expert e's rows from source 0, then
-    source 1, ...); and the two row maps, local row -> received row and back.
+
+def exchange_plan(offsets, counts, world: int, recv_counts):
+    """Host-side plan of one exchange. Only real rows cross between ranks; groups are
+    padded to 128 rows where they are computed.
+
+    offsets: this rank's padded group offsets [E+1]; counts: its routed rows per expert
+    [E] (E = world * E_loc); recv_counts: [world, E_loc] rows this rank receives for each
+    of its experts from each source rank.
+    Returns a dict:
+      send_index [n_send]: rows of this rank's x_perm to send, grouped by owner rank
+        (expert order), without pad rows;
+      send_rows [world], recv_rows [world]: rows sent to / received from each rank;
+      local_offsets [E_loc+1]: expert groups of the received rows, each padded to 128;
+      to_local [local_offsets[-1]]: received row of each local row (-1 on pad rows);
+      to_recv [n_recv]: local row of each received row;
+      back_index [offsets[-1]]: position in the returned rows of each x_perm row (-1 on
+        pad rows).
     """
     offsets = [int(v) for v in offsets]
-    e_total = len(offsets) - 1
+    counts = [int(v) for v in counts]
+    e_total = len(counts)
     e_loc = e_total // world
-    send_rows = [offsets[(r + 1) * e_loc] - offsets[r * e_loc] for r in range(world)]
-    counts = [[int(c) for c in row] for row in recv_counts]
-    recv_rows = [sum(row) for row in counts]
+    send_index, back_index = [], [-1] * offsets[-1]
+    for e in range(e_total):
+        for j in range(counts[e]):
+            back_index[offsets[e] + j] = len(send_index)
+            send_index.append(offsets[e] + j)
+    send_rows = [sum(counts[r * e_loc:(r + 1) * e_loc]) for r in range(world)]
+    rc = [[int(c) for c in row] for row in recv_counts]
+    recv_rows = [sum(row) for row in rc]
     # start of the (source s, expert e) segment in the received buffer
     seg = [[0] * e_loc for _ in range(world)]
     pos = 0
     for s in range(world):
         for e in range(e_loc):
             seg[s][e] = pos
-            pos += counts[s][e]
+            pos += rc[s][e]
     n_recv = pos
     local_offsets = [0]
     to_local = []
     for e in range(e_loc):
         for s in range(world):
-            to_local.extend(range(seg[s][e], seg[s][e] + counts[s][e]))
+            to_local.extend(range(seg[s][e], seg[s][e] + rc[s][e]))
+        to_local.extend([-1] * (_pad(len(to_local) - local_offsets[-1]) -
+                                (len(to_local) - local_offsets[-1])))
         local_offsets.append(len(to_local))
     to_recv = [0] * n_recv
     for dst, src in enumerate(to_local):
-        to_recv[src] = dst
-    return send_rows, recv_rows, local_offsets, to_local, to_recv
+        if src >= 0:
+            to_recv[src] = dst
+    return {"send_index": send_index, "send_rows": send_rows, "recv_rows": recv_rows,
+            "local_offsets": local_offsets, "to_local": to_local, "to_recv": to_recv,
+            "back_index": back_index}
 
 
 def forward_ep(x, w_router, w1_local, w3_local, w2_local, k: int, num_experts: int,
@@ -112,7 +135,7 @@ def forward_ep(x, w_router, w1_local, w3_local, w2_local, k: int, num_experts: i
     full router w_router [E, H]. Returns out [T, H] = residual + routed output.
 
     Every rank of ``group`` must call it (the collectives are collective); T may differ
-    between ranks. E must be a multiple of the group size.
+    between ranks, and may be 0. E must be a multiple of the group size.
     """
     ops = ops or CudaOps()
     world = dist.get_world_size(group)
@@ -122,6 +145,7 @@ def forward_ep(x, w_router, w1_local, w3_local, w2_local, k: int, num_experts: i
     if w1_local.shape[0] != e_loc:
         raise ValueError(f"this rank must hold {e_loc} experts, got {w1_local.shape[0]}")
     inter = w1_local.shape[1]
+    hidden = x.shape[1]
     dev = x.device
 
     # 1. route and permute this rank's tokens (a rank without tokens sends nothing but
@@ -129,43 +153,43 @@ def forward_ep(x, w_router, w1_local, w3_local, w2_local, k: int, num_experts: i
     if x.shape[0] == 0:
         wt = None
         perm = {"offsets": torch.zeros(num_experts + 1, dtype=torch.int64),
-                "x_perm": torch.empty((0, x.shape[1]), dtype=x.dtype, device=dev)}
+                "counts": torch.zeros(num_experts, dtype=torch.int64),
+                "x_perm": torch.empty((0, hidden), dtype=x.dtype, device=dev)}
     else:
         idx, wt = ops.router_topk(x, w_router, k, logit_bias)
         perm = ops.permute(idx, x, num_experts, inter)
     offsets = perm["offsets"].to("cpu", torch.int64)
-    r_pad = int(offsets[-1])
+    counts = perm["counts"].to("cpu", torch.int64)
 
-    # 2. padded rows per expert, E/W to each owner
-    padded = (offsets[1:] - offsets[:-1]).to(dev)
+    # 2. routed rows per expert, E/W to each owner
     recv_counts = torch.empty(world * e_loc, dtype=torch.int64, device=dev)
-    dist.all_to_all_single(recv_counts, padded, group=group)
-    recv_counts = recv_counts.view(world, e_loc).cpu()
-    send_rows, recv_rows, local_offsets, to_local, to_recv = exchange_plan(offsets, world,
-                                                                          recv_counts)
+    dist.all_to_all_single(recv_counts, counts.to(dev), group=group)
+    plan = exchange_plan(offsets, counts, world, recv_counts.view(world, e_loc).cpu())
 
-    # 3. the rows
-    x_perm = perm["x_perm"][:r_pad].contiguous()
-    x_recv = torch.empty((sum(recv_rows), x.shape[1]), dtype=x_perm.dtype, device=dev)
-    dist.all_to_all_single(x_recv, x_perm, recv_rows, send_rows, group=group)
+    # 3. the rows, without padding
+    def rows_index(values):
+        return torch.tensor(values, dtype=torch.int64).to(dev)
 
-    # 4. regroup by local expert (padded to the grouped GEMM's buffer size), the experts,
-    #    and back to the received order
-    n_local = len(to_local)
+    x_send = ops.gather_rows(perm["x_perm"], rows_index(plan["send_index"]))
+    x_recv = torch.empty((sum(plan["recv_rows"]), hidden), dtype=x_send.dtype, device=dev)
+    dist.all_to_all_single(x_recv, x_send, plan["recv_rows"], plan["send_rows"], group=group)
+
+    # 4. expert groups padded to 128 rows (to the grouped GEMM's buffer size), the
+    #    experts, and back to the received order
+    n_local = len(plan["to_local"])
     rows_buf = ops.padded_rows(n_local, e_loc)
-    index = torch.full((rows_buf,), -1, dtype=torch.int64)
-    index[:n_local] = torch.tensor(to_local, dtype=torch.int64)
-    x_local = ops.gather_rows(x_recv, index.to(dev))
-    loc_off = torch.tensor(local_offsets, dtype=torch.int32, device=dev)
+    x_local = ops.gather_rows(x_recv, rows_index(plan["to_local"] + [-1] * (rows_buf - n_local)))
+    loc_off = torch.tensor(plan["local_offsets"], dtype=torch.int32, device=dev)
     y_local = ops.grouped_swiglu(x_local, loc_off, w1_local, w3_local, w2_local, n_local)
-    y_recv = ops.gather_rows(y_local, torch.tensor(to_recv, dtype=torch.int64, device=dev))
+    y_recv = ops.gather_rows(y_local, rows_index(plan["to_recv"]))
 
-    # 5. outputs back to their tokens' ranks, then the combine
-    y_back = torch.empty((max(r_pad, 1), x.shape[1]), dtype=y_recv.dtype, device=dev)
-    dist.all_to_all_single(y_back[:r_pad], y_recv, send_rows, recv_rows, group=group)
+    # 5. outputs back to their tokens' ranks, into the permuted order, then the combine
+    y_back = torch.empty((sum(plan["send_rows"]), hidden), dtype=y_recv.dtype, device=dev)
+    dist.all_to_all_single(y_back, y_recv, plan["send_rows"], plan["recv_rows"], group=group)
     if x.shape[0] == 0:
-        return torch.empty((0, x.shape[1]), dtype=x.dtype, device=dev)
-    return ops.combine(y_back, perm["row_of"], wt, residual, num_experts, inter)
+        return torch.empty((0, hidden), dtype=x.dtype, device=dev)
+    y_perm = ops.gather_rows(y_back, rows_index(plan["back_index"]))
+    return ops.combine(y_perm, perm["row_of"], wt, residual, num_experts, inter)
 
 
 def shard_experts(w1, w3, w2, rank: int, world: int):

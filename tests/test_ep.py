@@ -134,20 +134,28 @@ def test_expert_parallel_layer_equals_single_process_layer(world, tokens, e, k, 
     np.testing.assert_allclose(got, ref["out"], rtol=1e-12, atol=1e-12)
 
 
-def test_exchange_plan_regroups_by_expert_and_inverts():
-    # rank with 2 local experts (E = 4 over 2 ranks); padded offsets of its own tokens
+def test_exchange_plan_sends_real_rows_and_pads_per_expert():
+    # E = 4 over 2 ranks; this rank routed 3, 130, 0, 5 rows (padded offsets below) and
+    # receives, for its experts 0 and 1, 3 and 0 rows from rank 0, 7 and 2 from rank 1
     offsets = [0, 128, 384, 384, 512]
-    recv = [[128, 0], [256, 128]]          # from rank 0, from rank 1
-    send, recv_rows, local_off, to_local, to_recv = ep.exchange_plan(offsets, 2, recv)
-    assert send == [384, 128] and recv_rows == [128, 384]
-    # expert 0: source 0 rows 0..127, then source 1 rows 128..383; expert 1: 384..511
-    assert local_off == [0, 384, 512]
-    assert to_local == list(range(0, 128)) + list(range(128, 384)) + list(range(384, 512))
-    assert all(to_local[to_recv[i]] == i for i in range(512))
-    # a permutation when a source sends several experts' rows
-    send, recv_rows, local_off, to_local, to_recv = ep.exchange_plan(offsets, 2, [[128, 256],
-                                                                                  [128, 0]])
-    assert local_off == [0, 256, 512]
-    assert to_local[:256] == list(range(0, 128)) + list(range(384, 512))
-    assert sorted(to_local) == list(range(512))
-    assert all(to_local[to_recv[i]] == i for i in range(512))
+    counts = [3, 130, 0, 5]
+    p = ep.exchange_plan(offsets, counts, 2, [[3, 0], [7, 2]])
+    assert p["send_rows"] == [133, 5] and p["recv_rows"] == [3, 9]
+    assert p["send_index"] == [0, 1, 2] + list(range(128, 258)) + [384, 385, 386, 387, 388]
+    # every x_perm row maps to its place in the packed rows, pad rows to -1
+    back = p["back_index"]
+    assert len(back) == 512 and sum(b >= 0 for b in back) == 138
+    assert all(p["send_index"][back[r]] == r for r in range(512) if back[r] >= 0)
+    # local expert 0: source 0 rows 0..2, source 1 rows 3..9, padded to 128; expert 1:
+    # source 1 rows 10..11, padded
+    assert p["local_offsets"] == [0, 128, 256]
+    tl = p["to_local"]
+    assert tl[:10] == list(range(10)) and tl[10:128] == [-1] * 118
+    assert tl[128:130] == [10, 11] and tl[130:] == [-1] * 126
+    assert all(tl[p["to_recv"][i]] == i for i in range(12))
+
+
+def test_exchange_plan_empty_rank():
+    p = ep.exchange_plan([0, 0, 0, 0, 0], [0, 0, 0, 0], 2, [[0, 0], [4, 0]])
+    assert p["send_rows"] == [0, 0] and p["send_index"] == [] and p["back_index"] == []
+    assert p["local_offsets"] == [0, 128, 128] and p["to_recv"] == [0, 1, 2, 3]
