@@ -119,3 +119,42 @@ def test_forward_decode_sweep(t):
     assert near.numel() == 0
     got, ref, _ = _forward_and_check(w, inp, residual=False)
     assert_layer_close(got, ref["out"], w.name)
+
+
+# Every token on experts 0 and 1 (bias +30): two experts with 3000 rows each (24 row
+# tiles), six empty experts; the routing margin between the two is still screened.
+ALL_ON_TWO = W.Workload("all_on_two", 3000, 256, 512, 8, 2, seed=41,
+                        logit_bias=(30.0, 30.0, 0, 0, 0, 0, 0, 0))
+# 100k tokens: the multi-block histogram / scan / rank path with 3125 token blocks
+MANY_TOKENS = W.Workload("many_tokens", 100_000, 128, 128, 8, 2, seed=42)
+
+
+@pytest.mark.parametrize("w", [ALL_ON_TWO, MANY_TOKENS], ids=lambda w: w.name)
+def test_forward_extreme_batches(w):
+    inp, near = screened(w)
+    assert near.numel() == 0
+    tokens = sample_tokens(w.num_tokens, 512)
+    got, ref, out = _forward_and_check(w, inp, tokens=tokens, residual=False)
+    assert_layer_close(got, ref["out"], w.name)
+    idx, _ = M.router_topk(inp.x, inp.w_router, 2, inp.logit_bias)
+    counts = torch.bincount(idx.reshape(-1).long(), minlength=w.num_experts).cpu()
+    if w is ALL_ON_TWO:
+        assert counts[:2].tolist() == [w.num_tokens] * 2 and int(counts[2:].sum()) == 0
+    assert int(counts.sum()) == 2 * w.num_tokens
+
+
+def test_int8_extreme_imbalance():
+    w = ALL_ON_TWO
+    inp, _ = screened(w)
+    q = M.quantize_int8(inp.w1, inp.w3, inp.w2)
+    out = M.forward_w8(inp.x, inp.w_router, q, 2, logit_bias=inp.logit_bias)
+    torch.cuda.synchronize()
+    c = to_cpu(inp)
+    deq = []
+    for full in (c.w1, c.w3, c.w2):
+        qq, s = O.quantize_int8_rows(full)
+        deq.append(qq.astype(np.float64) * s.astype(np.float64)[..., None])
+    tokens = sample_tokens(w.num_tokens, 512)
+    ref = O.moe_layer(c.x, c.w_router, deq[0], deq[1], deq[2], 2, logit_bias=c.logit_bias,
+                      mode="f16_experts", tokens=tokens)
+    assert_layer_close(O.to_f64(out.cpu())[tokens], ref["out"], "int8 all_on_two")
