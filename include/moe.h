@@ -228,6 +228,20 @@ moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_bf16_t* x_host
                               moe_bf16_t* out_host, void* ws, size_t ws_bytes,
                               moe_stream_t stream);
 
+/* moe_forward_host without the final wait: enqueues the copies in, the layer and the
+ * copy out on `stream` and returns. out_host holds the result, and x_host and
+ * residual_host may be reused, once the stream has reached this point (for example
+ * after cudaStreamSynchronize). Calls on one stream with one ws are ordered by the
+ * stream, so a serving loop can enqueue step after step and wait once; calls that may
+ * overlap on different streams need separate workspaces. Host buffers must be pinned
+ * for the copies to be asynchronous. */
+moe_status_t moe_forward_host_async(const moe_shape_t* shape, const moe_bf16_t* x_host,
+                                    const moe_bf16_t* w_router, const float* logit_bias,
+                                    const moe_bf16_t* w1, const moe_bf16_t* w3,
+                                    const moe_bf16_t* w2, const moe_bf16_t* residual_host,
+                                    moe_bf16_t* out_host, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream);
+
 /* Convert row-major expert weights to MOE_WEIGHTS_BLOCKED: w1, w3 [E, I, H] and w2
  * [E, H, I] in, the same-sized w1_blocked, w3_blocked, w2_blocked out (caller-owned,
  * distinct from the inputs). Asynchronous on `stream`. */

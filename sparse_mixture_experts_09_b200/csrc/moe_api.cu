@@ -229,6 +229,38 @@ moe_status_t run_forward(const Shape& s, const uint16_t* x, const uint16_t* wr, 
   return MOE_OK;
 }
 
+moe_status_t forward_host_enqueue(const moe_shape_t* shape, const moe_bf16_t* x_host,
+                                  const moe_bf16_t* w_router, const float* logit_bias,
+                                  const moe_bf16_t* w1, const moe_bf16_t* w3, const moe_bf16_t* w2,
+                                  const moe_bf16_t* residual_host, moe_bf16_t* out_host, void* ws,
+                                  size_t ws_bytes, cudaStream_t st) {
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  if (!x_host) return fail(MOE_ERR_INVALID_ARG, "x_host is NULL");
+  if (!out_host) return fail(MOE_ERR_INVALID_ARG, "out_host is NULL");
+  MOE_TRY(check_ptr(w_router, "w_router"));
+  MOE_TRY(check_ptr(logit_bias, "logit_bias", true));
+  MOE_TRY(check_ptr(w1, "w1"));
+  MOE_TRY(check_ptr(w3, "w3"));
+  MOE_TRY(check_ptr(w2, "w2"));
+  const Layout L = layout(s);
+  MOE_TRY(check_ws(ws, ws_bytes, L.end_host));
+  const size_t bytes = (size_t)s.T * s.H * 2;
+  uint16_t* xd = at<uint16_t>(ws, L.x_in);
+  uint16_t* rd = residual_host ? at<uint16_t>(ws, L.res_in) : nullptr;
+  uint16_t* od = at<uint16_t>(ws, L.out_st);
+  cudaError_t e = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e, "copy of x to the device");
+  if (rd) {
+    e = cudaMemcpyAsync(rd, residual_host, bytes, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "copy of residual to the device");
+  }
+  MOE_TRY(run_forward(s, xd, w_router, logit_bias, bf16_experts(w1, w3, w2), rd, od, ws, st));
+  e = cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e, "copy of out to the host");
+  return MOE_OK;
+}
+
 }  // namespace
 
 int validate_shape(const moe_shape_t* shape, Shape* out) { return (int)check_shape(shape, out); }
@@ -436,34 +468,23 @@ moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_bf16_t* x_host
                               const moe_bf16_t* residual_host, moe_bf16_t* out_host, void* ws,
                               size_t ws_bytes, moe_stream_t stream) {
   g_err[0] = 0;
-  Shape s;
-  MOE_TRY(check_shape(shape, &s));
-  if (!x_host) return fail(MOE_ERR_INVALID_ARG, "x_host is NULL");
-  if (!out_host) return fail(MOE_ERR_INVALID_ARG, "out_host is NULL");
-  MOE_TRY(check_ptr(w_router, "w_router"));
-  MOE_TRY(check_ptr(logit_bias, "logit_bias", true));
-  MOE_TRY(check_ptr(w1, "w1"));
-  MOE_TRY(check_ptr(w3, "w3"));
-  MOE_TRY(check_ptr(w2, "w2"));
-  const Layout L = layout(s);
-  MOE_TRY(check_ws(ws, ws_bytes, L.end_host));
   cudaStream_t st = (cudaStream_t)stream;
-  const size_t bytes = (size_t)s.T * s.H * 2;
-  uint16_t* xd = at<uint16_t>(ws, L.x_in);
-  uint16_t* rd = residual_host ? at<uint16_t>(ws, L.res_in) : nullptr;
-  uint16_t* od = at<uint16_t>(ws, L.out_st);
-  cudaError_t e = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, st);
-  if (e != cudaSuccess) return cuda_fail(e, "copy of x to the device");
-  if (rd) {
-    e = cudaMemcpyAsync(rd, residual_host, bytes, cudaMemcpyHostToDevice, st);
-    if (e != cudaSuccess) return cuda_fail(e, "copy of residual to the device");
-  }
-  MOE_TRY(run_forward(s, xd, w_router, logit_bias, bf16_experts(w1, w3, w2), rd, od, ws, st));
-  e = cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, st);
-  if (e != cudaSuccess) return cuda_fail(e, "copy of out to the host");
-  e = cudaStreamSynchronize(st);
+  MOE_TRY(forward_host_enqueue(shape, x_host, w_router, logit_bias, w1, w3, w2, residual_host,
+                               out_host, ws, ws_bytes, st));
+  cudaError_t e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
   return MOE_OK;
+}
+
+moe_status_t moe_forward_host_async(const moe_shape_t* shape, const moe_bf16_t* x_host,
+                                    const moe_bf16_t* w_router, const float* logit_bias,
+                                    const moe_bf16_t* w1, const moe_bf16_t* w3,
+                                    const moe_bf16_t* w2, const moe_bf16_t* residual_host,
+                                    moe_bf16_t* out_host, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream) {
+  g_err[0] = 0;
+  return forward_host_enqueue(shape, x_host, w_router, logit_bias, w1, w3, w2, residual_host,
+                              out_host, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 moe_status_t moe_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t timeout_ns,

@@ -27,7 +27,8 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_size_host", "moe_max_padded_rows
            "moe_expert_down", "moe_combine", "moe_forward",
            "moe_forward_host", "moe_device_status", "moe_last_error", "moe_permute_static",
            "moe_selftest_wait_timeout", "moe_forward_rmsnorm", "moe_pack_weights",
-           "moe_quantize_int8", "moe_grouped_swiglu_w8", "moe_forward_w8", "moe_gather_rows")
+           "moe_quantize_int8", "moe_grouped_swiglu_w8", "moe_forward_w8", "moe_gather_rows",
+           "moe_forward_host_async")
 
 
 @dataclass
@@ -106,6 +107,8 @@ def lib() -> ctypes.CDLL:
         L.moe_pack_weights.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P]
         L.moe_pack_weights.restype = st
         L.moe_forward_host.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.moe_forward_host_async.argtypes = [sp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.moe_forward_host_async.restype = st
         L.moe_forward_host.restype = st
         L.moe_device_status.argtypes = [_P, _SZ, _P]
         L.moe_device_status.restype = st
@@ -339,8 +342,11 @@ def forward_rmsnorm(h, norm_weight, eps: float, w_router, w1, w3, w2, k: int, lo
 
 
 def forward_host(x_host, w_router, w1, w3, w2, k: int, residual_host=None, logit_bias=None,
-                 ws=None, out_host=None, stream=None, weight_layout: int = ROW_MAJOR):
-    """The layer with host (ideally pinned) activations; returns out_host (synchronous)."""
+                 ws=None, out_host=None, stream=None, weight_layout: int = ROW_MAJOR,
+                 wait: bool = True):
+    """The layer with host (ideally pinned) activations; returns out_host. With
+    wait=False the call only enqueues (moe_forward_host_async): out_host is ready once
+    the stream has been synchronised."""
     t, h = x_host.shape
     e, i, _ = w1.shape
     shape = make_shape(t, h, i, e, k, weight_layout)
@@ -351,7 +357,8 @@ def forward_host(x_host, w_router, w1, w3, w2, k: int, residual_host=None, logit
         ws = make_workspace(shape, w1.device, host=True)
     if out_host is None:
         out_host = torch.empty((t, h), dtype=torch.bfloat16, pin_memory=True)
-    _check(lib().moe_forward_host(ctypes.byref(shape), x_host.data_ptr(),
+    fn = lib().moe_forward_host if wait else lib().moe_forward_host_async
+    _check(fn(ctypes.byref(shape), x_host.data_ptr(),
                                   _dev(w_router, "w_router", torch.bfloat16),
                                   _dev(logit_bias, "logit_bias", torch.float32, True),
                                   _dev(w1, "w1", torch.bfloat16), _dev(w3, "w3", torch.bfloat16),

@@ -158,3 +158,23 @@ def test_int8_extreme_imbalance():
     ref = O.moe_layer(c.x, c.w_router, deq[0], deq[1], deq[2], 2, logit_bias=c.logit_bias,
                       mode="f16_experts", tokens=tokens)
     assert_layer_close(O.to_f64(out.cpu())[tokens], ref["out"], "int8 all_on_two")
+
+
+def test_forward_host_async_steps_queue_on_one_stream():
+    # three steps with different activations enqueued back to back on one stream and
+    # one workspace, one wait at the end: each equals the device-resident forward
+    w = SMALL["ragged"]
+    inp, _ = screened(w)
+    shape = M.make_shape(*w.shape)
+    ws = M.make_workspace(shape, "cuda", host=True)
+    xs = [W.redraw_x_rows(w, torch.arange(w.num_tokens), a).pin_memory() for a in (1, 2, 3)]
+    rh = inp.residual.cpu().pin_memory()
+    outs = [torch.empty_like(x).pin_memory() for x in xs]
+    for x, o in zip(xs, outs):
+        M.forward_host(x, inp.w_router, inp.w1, inp.w3, inp.w2, w.num_experts_per_tok,
+                       residual_host=rh, ws=ws, out_host=o, wait=False)
+    torch.cuda.synchronize()
+    for x, o in zip(xs, outs):
+        want = M.forward(x.cuda(), inp.w_router, inp.w1, inp.w3, inp.w2, w.num_experts_per_tok,
+                         residual=inp.residual)
+        assert torch.equal(o, want.cpu())
