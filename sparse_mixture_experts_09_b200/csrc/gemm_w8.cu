@@ -3,8 +3,9 @@
 //
 // Mixtral is loaded weight-only quantised to shrink it (Hugging Face "Mixtral" doc,
 // "Shrinking down Mixtral using quantization"; ZeroModels "Mixtral", "Lower memory":
-// int8 weights). At decode the layer streams every active expert's weights, so halving
-// their bytes can halve the time.
+// int8 weights): half the weight memory of bf16. (At decode this kernel streams half
+// the bytes but is not faster than the bf16 one: its per-stage pipeline of copy,
+// widening and MMA handoffs, not HBM, sets its pace.)
 // Scheme (the pages do not fix one): per output row (channel) r, s[r] = max|w[r, :]| /
 // 127 and q = rint(w / s), decided in float32; w ~ q * s. The experts compute in half
 // precision, as a float16 load of the model does (Hugging Face "Mixtral" doc: the model
@@ -67,8 +68,8 @@ constexpr bool kUseHalfTiles = MOE_W8_HALF_TILES != 0;
 // address, row tiles]. Three rings: activation tiles (TMA -> MMA), code tiles (bulk
 // copy -> converters) and widened weight tiles (converters -> MMA). MT = 128 rows, or
 // 64 when every expert has at most 64 routed rows (the tile's first 64 rows hold all
-// of them): then the tensor core does half the work per k-block, and the 8 KiB saved
-// per activation stage buys deeper code prefetch.
+// of them): the MMAs then cover only those rows, and the 8 KiB saved per activation
+// stage buys deeper code prefetch.
 template <int BN, int MT>
 struct TileW8 {
   static constexpr int A_ST = MT == 64 ? MOE_W8_A_STAGES_M64 : MOE_W8_A_STAGES;
