@@ -384,8 +384,9 @@ def run_ours(args):
         host_step()
     torch.cuda.synchronize(dev)
     # the same forward captured once in a CUDA graph (replayed in loop 5)
+    # thread-local capture: other threads (a process group's watchdog) may use CUDA
     graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
         step()
     for _ in range(3):
         graph.replay()
