@@ -6,6 +6,10 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "../../include/moe.h"
 #include "moe_internal.h"
 
@@ -47,7 +51,7 @@ inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 struct Layout {
   size_t status, topk_idx, topk_w, block_base, counts, offsets, row_of, token_of_row, x_perm, h,
       y, rnorm, end;
-  size_t x_in, res_in, out_st, end_host;  // staging of moe_forward_host
+  size_t x_in[2], res_in[2], out_st, end_host;  // staging of the host entry points
 };
 
 Layout layout(const Shape& s) {
@@ -68,8 +72,10 @@ Layout layout(const Shape& s) {
   L.y = o; o += up(rmax * s.H * 4);
   L.rnorm = o; o += up((size_t)s.T * 4);
   L.end = o;
-  L.x_in = o; o += up((size_t)s.T * s.H * 2);
-  L.res_in = o; o += up((size_t)s.T * s.H * 2);
+  for (int b = 0; b < 2; ++b) {
+    L.x_in[b] = o; o += up((size_t)s.T * s.H * 2);
+    L.res_in[b] = o; o += up((size_t)s.T * s.H * 2);
+  }
   L.out_st = o; o += up((size_t)s.T * s.H * 2);
   L.end_host = o;
   return L;
@@ -229,6 +235,37 @@ moe_status_t run_forward(const Shape& s, const uint16_t* x, const uint16_t* wr, 
   return MOE_OK;
 }
 
+// Host-path overlap. The copies in of a host call run on a copy stream of the library's
+// own, into one of two staging slots of the workspace, so they overlap the previous
+// call's layer; the caller's stream waits for them (event `ready`) before the layer, and
+// a slot is refilled only after the layer two calls back has read it (event `freed`).
+struct HostPath {
+  cudaStream_t copy = nullptr;
+  cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
+  bool freed_recorded[2] = {false, false};
+  unsigned calls = 0;
+};
+
+std::mutex g_host_mutex;
+std::map<std::pair<int, void*>, HostPath> g_host_paths;  // (device, workspace)
+
+cudaError_t host_path(void* ws, HostPath** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  HostPath& h = g_host_paths[std::make_pair(dev, ws)];
+  if (!h.copy) {
+    e = cudaStreamCreateWithFlags(&h.copy, cudaStreamNonBlocking);
+    for (int b = 0; b < 2 && e == cudaSuccess; ++b) {
+      e = cudaEventCreateWithFlags(&h.ready[b], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h.freed[b], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) return e;
+  }
+  *out = &h;
+  return cudaSuccess;
+}
+
 moe_status_t forward_host_enqueue(const moe_shape_t* shape, const moe_bf16_t* x_host,
                                   const moe_bf16_t* w_router, const float* logit_bias,
                                   const moe_bf16_t* w1, const moe_bf16_t* w3, const moe_bf16_t* w2,
@@ -245,17 +282,34 @@ moe_status_t forward_host_enqueue(const moe_shape_t* shape, const moe_bf16_t* x_
   MOE_TRY(check_ptr(w2, "w2"));
   const Layout L = layout(s);
   MOE_TRY(check_ws(ws, ws_bytes, L.end_host));
+  std::lock_guard<std::mutex> lock(g_host_mutex);
+  HostPath* hp = nullptr;
+  cudaError_t e = host_path(ws, &hp);
+  if (e != cudaSuccess) return cuda_fail(e, "host-path stream or event creation");
+  const int b = (int)(hp->calls++ & 1u);
   const size_t bytes = (size_t)s.T * s.H * 2;
-  uint16_t* xd = at<uint16_t>(ws, L.x_in);
-  uint16_t* rd = residual_host ? at<uint16_t>(ws, L.res_in) : nullptr;
+  uint16_t* xd = at<uint16_t>(ws, L.x_in[b]);
+  uint16_t* rd = residual_host ? at<uint16_t>(ws, L.res_in[b]) : nullptr;
   uint16_t* od = at<uint16_t>(ws, L.out_st);
-  cudaError_t e = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, st);
+  // copies in, on the copy stream, once the layer two calls back has read this slot
+  if (hp->freed_recorded[b]) {
+    e = cudaStreamWaitEvent(hp->copy, hp->freed[b], 0);
+    if (e != cudaSuccess) return cuda_fail(e, "copy-stream wait");
+  }
+  e = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, hp->copy);
   if (e != cudaSuccess) return cuda_fail(e, "copy of x to the device");
   if (rd) {
-    e = cudaMemcpyAsync(rd, residual_host, bytes, cudaMemcpyHostToDevice, st);
+    e = cudaMemcpyAsync(rd, residual_host, bytes, cudaMemcpyHostToDevice, hp->copy);
     if (e != cudaSuccess) return cuda_fail(e, "copy of residual to the device");
   }
+  e = cudaEventRecord(hp->ready[b], hp->copy);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, hp->ready[b], 0);
+  if (e != cudaSuccess) return cuda_fail(e, "copy-in event");
+  // the layer and the copy out, on the caller's stream
   MOE_TRY(run_forward(s, xd, w_router, logit_bias, bf16_experts(w1, w3, w2), rd, od, ws, st));
+  e = cudaEventRecord(hp->freed[b], st);
+  if (e != cudaSuccess) return cuda_fail(e, "slot event");
+  hp->freed_recorded[b] = true;
   e = cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, st);
   if (e != cudaSuccess) return cuda_fail(e, "copy of out to the host");
   return MOE_OK;
