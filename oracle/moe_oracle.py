@@ -46,6 +46,7 @@ import numpy as np
 __all__ = [
     "to_f64", "round_bf16", "round_f16", "silu", "router_logits", "route_topk", "stable_permute",
     "swiglu_expert", "moe_layer", "rms_norm", "moe_block", "quantize_int8_rows",
+    "quantize_int4_groups", "dequantize_int4_groups",
 ]
 
 
@@ -278,3 +279,40 @@ def quantize_int8_rows(w):
     q = np.rint(w / s[..., None]).astype(np.float32)
     q = np.clip(q, -127, 127).astype(np.int8)
     return q, s
+
+
+def quantize_int4_groups(w, group: int = 64):
+    """Symmetric 4-bit codes with one half-precision scale per ``group`` columns of a row.
+
+    The pages also load Mixtral in 4 bits (Hugging Face "Mixtral" doc, "Shrinking down
+    Mixtral using quantization"; "Welcome Mixtral", "Quantizing Mixtral") and leave the
+    format to the quantisation library. Fifteen levels cannot cover a whole row well, so
+    the scale is per run of ``group`` consecutive columns of a row (a group), in the
+    manner of block-wise 4-bit schemes: for each group, s = max|w| / 7 in float32, then
+    rounded to the nearest IEEE half (s16; a group whose s16 is zero, all zeros or too
+    small for a half, takes s16 = 1); code q = round-half-even(w / s16) in float32,
+    clamped to [-7, 7]. The code is decided in float32 as the kernel decides it.
+    Returns (q int8 [..., rows, K], s16 float16 [..., rows, K / group]).
+    """
+    w = np.asarray(to_f64(w), dtype=np.float32)
+    k = w.shape[-1]
+    if k % group:
+        raise ValueError(f"row length {k} is not a multiple of the group {group}")
+    g = w.reshape(*w.shape[:-1], k // group, group)
+    amax = np.abs(g).max(axis=-1)
+    s = (amax / np.float32(7.0)).astype(np.float32)
+    s16 = round_f16(s.astype(np.float64))
+    s16 = np.where(s16 == 0, 1.0, s16).astype(np.float16)
+    q = np.rint(g / s16.astype(np.float32)[..., None])
+    q = np.clip(q, -7, 7).astype(np.int8).reshape(w.shape)
+    return q, s16
+
+
+def dequantize_int4_groups(q, s16, group: int = 64) -> np.ndarray:
+    """The weight a 4-bit expert multiplies: q * s16 rounded once to the nearest half
+    (the product of a code and a half scale, formed in half precision), as fp64."""
+    q = np.asarray(q)
+    k = q.shape[-1]
+    prod = (q.astype(np.float64).reshape(*q.shape[:-1], k // group, group)
+            * np.asarray(s16, dtype=np.float64)[..., None])
+    return round_f16(prod).reshape(q.shape)

@@ -361,6 +361,74 @@ def test_int8_codes_match_torch_float32_arithmetic():
     assert np.array_equal(s, st.numpy()) and np.array_equal(q, qt.numpy())
 
 
+# ---------------------------------------------------------------- 4-bit group codes
+
+def test_int4_groups_closed_form():
+    # every group holds integer multiples k * 2**-6 with k in [-7, 7] and reaches |k| = 7:
+    # s = 7 * 2**-6 / 7 = 2**-6 exactly, so the codes are the k and the weights come back
+    rng = np.random.default_rng(21)
+    k = rng.integers(-7, 8, size=(2, 5, 192))
+    k[..., ::64] = 7 * np.where(rng.random((2, 5, 3)) < 0.5, -1, 1)
+    w = k * 2.0 ** -6
+    q, s16 = O.quantize_int4_groups(w)
+    assert q.dtype == np.int8 and s16.dtype == np.float16 and s16.shape == (2, 5, 3)
+    assert np.all(s16 == np.float16(2.0 ** -6)) and np.array_equal(q, k)
+    assert np.array_equal(O.dequantize_int4_groups(q, s16), w)
+
+
+def test_int4_groups_nearest_code_brute_force():
+    # each code is, of the 15 levels q * s16, the one nearest to w (clamped at +-7)
+    rng = np.random.default_rng(22)
+    w = O.round_bf16(rng.standard_normal((6, 128)) * 0.02)
+    w[2, 70] = 0.5                                    # one outlier in a group
+    q, s16 = O.quantize_int4_groups(w)
+    s = np.repeat(s16.astype(np.float64), 64, axis=-1)
+    levels = np.arange(-7, 8, dtype=np.float64)
+    err = np.abs(w[..., None] - levels * s[..., None])
+    best = err.min(axis=-1)
+    mine = np.abs(w - q.astype(np.float64) * s)
+    assert np.all(mine <= best + s * 2.0 ** -20)
+    # the group's largest magnitude takes code +-7 (its scale is within a half's rounding)
+    g = np.abs(w).reshape(6, 2, 64)
+    top = np.take_along_axis(q.reshape(6, 2, 64), g.argmax(-1)[..., None], -1)[..., 0]
+    assert np.all(np.abs(top) == 7)
+
+
+def test_int4_groups_degenerate_groups_and_bound():
+    rng = np.random.default_rng(23)
+    w = O.round_bf16(rng.standard_normal((4, 256)) * 0.05)
+    w[0, 64:128] = 0.0                   # all zeros: scale 1, codes 0
+    w[1, :64] = 0.0
+    w[1, 10] = 2.0 ** -30                # amax / 7 underflows a half: scale 1, codes 0
+    q, s16 = O.quantize_int4_groups(w)
+    assert s16[0, 1] == 1.0 and np.all(q[0, 64:128] == 0)
+    assert s16[1, 0] == 1.0 and np.all(q[1, :64] == 0)
+    deq = O.dequantize_int4_groups(q, s16)
+    s = np.repeat(s16.astype(np.float64), 64, axis=-1)
+    # |w - f16(q s16)| <= s16 / 2 (nearest level; no clamping when s16 >= amax / 7) plus
+    # the half rounding of the product (2**-11 relative)
+    unclamped = np.repeat(s16.astype(np.float64) * 7 >= np.abs(w).reshape(4, 4, 64).max(-1), 64, -1)
+    bound = s / 2 + np.abs(deq) * 2.0 ** -11
+    assert np.all((np.abs(w - deq) <= bound)[unclamped])
+    # a clamped level sits at most one half-rounding of the scale further out
+    assert np.all(np.abs(w - deq) <= s / 2 + 7 * s * 2.0 ** -10 + np.abs(deq) * 2.0 ** -11)
+
+
+def test_int4_groups_match_torch_arithmetic():
+    # the same decisions with torch's float32 and half ops: amax / 7, rounded to half;
+    # w / s, round half even, clamp; the product q * s formed in half precision
+    rng = np.random.default_rng(24)
+    w = O.round_bf16(rng.standard_normal((32, 192)) * 0.03)
+    q, s16 = O.quantize_int4_groups(w)
+    wt = torch.from_numpy(w).float().reshape(32, 3, 64)
+    st = (wt.abs().amax(-1) / 7.0).half()
+    st = torch.where(st == 0, torch.ones_like(st), st)
+    qt = torch.round(wt / st.float()[..., None]).clamp(-7, 7)
+    assert np.array_equal(s16, st.numpy()) and np.array_equal(q, qt.reshape(32, 192).to(torch.int8).numpy())
+    dt = (qt.half() * st[..., None]).reshape(32, 192).double().numpy()
+    assert np.array_equal(O.dequantize_int4_groups(q, s16), dt)
+
+
 def test_round_f16_closed_forms():
     # IEEE binary16: 11 significant bits, smallest normal 2**-14, subnormal step 2**-24,
     # largest finite 65504; ties go to the even significand
