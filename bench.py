@@ -324,6 +324,14 @@ def run_ours(args):
         moe.forward_w8(inp.x, inp.w_router, w8, k, residual=inp.residual,
                        logit_bias=inp.logit_bias, ws=ws8, out=out)
 
+    # weight-only 4-bit experts (a half scale per 64-column group), quantised once
+    w4 = moe.quantize_int4(inp.w1, inp.w3, inp.w2)
+    ws4 = moe.make_workspace(moe.make_shape(*w.shape), dev)
+
+    def step_w4():
+        moe.forward_w4(inp.x, inp.w_router, w4, k, residual=inp.residual,
+                       logit_bias=inp.logit_bias, ws=ws4, out=out)
+
     def step_row_major():
         moe.forward(inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, k, residual=inp.residual,
                     logit_bias=inp.logit_bias, ws=ws, out=out)
@@ -378,6 +386,7 @@ def run_ours(args):
         step()
         step_row_major()
         step_w8()
+        step_w4()
     scratch = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
     for _ in range(3):
         split_step(scratch)
@@ -475,6 +484,18 @@ def run_ours(args):
     barrier()
     w8_ms = q0.elapsed_time(q1) / K
 
+    # (4b) the same layer with weight-only 4-bit experts
+    barrier()
+    torch.cuda.synchronize(dev)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(K):
+        step_w4()
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    w4_ms = f0.elapsed_time(f1) / K
+
     # (5) the default forward replayed from a CUDA graph
     barrier()
     torch.cuda.synchronize(dev)
@@ -490,11 +511,13 @@ def run_ours(args):
     moe.device_status(ws)
     moe.device_status(wsh)
     moe.device_status(ws8)
+    moe.device_status(ws4)
 
     ms, e2e_ms = slowest_rank(ms, e2e_ms, world, dev)
     e2e_sync_ms, _ = slowest_rank(e2e_sync_ms, e2e_sync_ms, world, dev)
     rm_ms, _ = slowest_rank(rm_ms, rm_ms, world, dev)
     w8_ms, _ = slowest_rank(w8_ms, w8_ms, world, dev)
+    w4_ms, _ = slowest_rank(w4_ms, w4_ms, world, dev)
     graph_ms, _ = slowest_rank(graph_ms, graph_ms, world, dev)
 
     counts = perm["counts"].cpu().tolist()
@@ -527,6 +550,14 @@ def run_ours(args):
                              "weight_gb_per_step": roof["active_experts"] * w.expert_bytes() / 2e9,
                              "note": "weight-only int8 experts, half-precision expert math, "
                                      "quantised once at load (untimed); not the headline"},
+            "int4_experts": {"ms_per_step": w4_ms,
+                             "value": job_throughput(w.num_tokens, world, w4_ms),
+                             "api": "moe_forward_w4",
+                             "weight_gb_per_step": (roof["active_experts"] * w.expert_bytes()
+                                                    * (1 / 4 + 1 / 64) / 1e9),
+                             "note": "weight-only 4-bit experts (a half scale per 64-column "
+                                     "group), half-precision expert math, quantised once at "
+                                     "load (untimed); not the headline"},
             "e2e": {"value": job_throughput(w.num_tokens, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": 2 * bytes_io, "d2h_bytes_per_step": bytes_io,
                     "api": "moe_forward_host_async, steps enqueued back to back, one wait",

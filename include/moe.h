@@ -306,6 +306,56 @@ moe_status_t moe_forward_w8(const moe_shape_t* shape, const moe_bf16_t* x,
                             const moe_bf16_t* residual, moe_bf16_t* out, void* ws,
                             size_t ws_bytes, moe_stream_t stream);
 
+/* ---- Weight-only 4-bit experts ----
+ * The pages also load Mixtral in 4 bits (Hugging Face "Mixtral", "Shrinking down
+ * Mixtral using quantization"; "Welcome Mixtral", "Quantizing Mixtral") and leave the
+ * format to the quantisation library. This library uses symmetric 4-bit codes with one
+ * IEEE-half scale per group of 64 consecutive columns of a row (one K tile):
+ *   s = half(max |w| over the group / 7)   (1 when that is zero in half),
+ *   q[r, c] = clamp(rint(w[r, c] / s), -7, 7),
+ * the division and the rounding (to nearest, ties to even) in float32; the experts
+ * multiply the weight half(q * s), one rounding of the product to half.
+ * Codes are stored offset-binary, u = q + 8 (1 .. 15), two to a byte, tiled like the
+ * int8 codes: tile (row / 128, col / 64) is the 4 KiB block number (row / 128) * (K /
+ * 64) + col / 64; inside it, with r = row % 128 and c = col % 64, the code sits in the
+ * 32-bit word at byte (c / 32) * 2048 + r * 16 + ((c % 32) / 8) * 4, nibble n (bits 4n
+ * .. 4n+3) with n = (c % 8) / 2 for even c and 4 + (c % 8) / 2 for odd c.
+ * Scales are IEEE half bit patterns in the same tile order: the scale of row `row`,
+ * group g = col / 64, is element ((row / 128) * (K / 64) + g) * 128 + row % 128.
+ * Buffers: q1, q3 [E*I*H/2] and q2 [E*H*I/2] bytes; s1, s3 [E*I*H/64] and s2
+ * [E*H*I/64] halves. The shape's weight_layout field is ignored by these entry points.
+ *
+ * Precision: as the int8 experts (half activations and h, fp32 accumulation), with
+ * the scales inside the weight instead of the epilogue:
+ *   h = half(silu(x_perm W1q[e]^T) * (x_perm W3q[e]^T)),  y_perm = h W2q[e]^T (fp32),
+ * where Wq = half(q * s).
+ *
+ * moe_quantize_int4: w1, w3 [E, I, H] and w2 [E, H, I] bf16 row-major in (device);
+ * codes and scales out (device, caller-owned). Asynchronous on `stream`. */
+moe_status_t moe_quantize_int4(const moe_shape_t* shape, const moe_bf16_t* w1,
+                               const moe_bf16_t* w3, const moe_bf16_t* w2, uint8_t* q1,
+                               uint8_t* q3, uint8_t* q2, uint16_t* s1, uint16_t* s3,
+                               uint16_t* s2, moe_stream_t stream);
+
+/* moe_grouped_swiglu with 4-bit expert weights (codes and scales as written by
+ * moe_quantize_int4). x_perm is bf16 as moe_permute writes it (converted to half into
+ * ws); other arguments and errors as for moe_grouped_swiglu. */
+moe_status_t moe_grouped_swiglu_w4(const moe_shape_t* shape, const moe_bf16_t* x_perm,
+                                   const int32_t* expert_offsets, const uint8_t* q1,
+                                   const uint8_t* q3, const uint8_t* q2, const uint16_t* s1,
+                                   const uint16_t* s3, const uint16_t* s2, float* y_perm,
+                                   void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward with 4-bit expert weights: router, permutation and combine as in
+ * moe_forward (the gather writes the routed rows as half), experts as in
+ * moe_grouped_swiglu_w4. */
+moe_status_t moe_forward_w4(const moe_shape_t* shape, const moe_bf16_t* x,
+                            const moe_bf16_t* w_router, const float* logit_bias,
+                            const uint8_t* q1, const uint8_t* q3, const uint8_t* q2,
+                            const uint16_t* s1, const uint16_t* s3, const uint16_t* s2,
+                            const moe_bf16_t* residual, moe_bf16_t* out, void* ws,
+                            size_t ws_bytes, moe_stream_t stream);
+
 /* Row gather for the expert-parallel layer (this library's own step; the pages say
  * only that experts may be spread over devices, Hugging Face "Mixtral", MixtralConfig
  * num_local_experts): dst[i, :] = src[index[i], :] for 0 <= i < n_rows. A rank

@@ -1,5 +1,6 @@
 // Weight-only int8 experts (W8A16): the grouped GEMMs with int8 weight codes and one
-// fp32 scale per output channel.
+// fp32 scale per output channel; and 4-bit experts (W4A16): 4-bit codes with one half
+// scale per 64-column group of a row, applied while widening.
 //
 // Mixtral is loaded weight-only quantised to shrink it (Hugging Face "Mixtral" doc,
 // "Shrinking down Mixtral using quantization"; ZeroModels "Mixtral", "Lower memory":
@@ -25,6 +26,9 @@
 //   warps 7..   widen each code tile and store it, 128-byte swizzled, as the B operand;
 //   warp 1      issues tcgen05.mma into a double-buffered TMEM accumulator;
 //   warps 2-5   scale, activate and store (epilogue).
+// The 4-bit kernel (BITS = 4) is the same pipeline: a code tile is 4 KiB plus its 128
+// half scales, and the converters widen each code to a half and multiply it by its
+// group's scale (the scale varies along K, so it cannot wait for the epilogue).
 // Every wait is bounded (timeout -> status word, abort flag, drained copies).
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -51,6 +55,12 @@ constexpr int BM = 128, BK = 64;
 #ifndef MOE_W8_A_STAGES_M64
 #define MOE_W8_A_STAGES_M64 4
 #endif
+#ifndef MOE_W4_CODE_STAGES
+#define MOE_W4_CODE_STAGES 7
+#endif
+#ifndef MOE_W4_CODE_STAGES_M64
+#define MOE_W4_CODE_STAGES_M64 10
+#endif
 #ifndef MOE_W8_CONV_WARPS
 #define MOE_W8_CONV_WARPS 8
 #endif
@@ -70,34 +80,44 @@ constexpr bool kUseHalfTiles = MOE_W8_HALF_TILES != 0;
 // 64 when every expert has at most 64 routed rows (the tile's first 64 rows hold all
 // of them): the MMAs then cover only those rows, and the 8 KiB saved per activation
 // stage buys deeper code prefetch.
-template <int BN, int MT>
+// With BITS = 4 a code stage holds BN/128 boxes of 4 KiB codes, then BN half scales
+// (stage row r's scale at element r), and more stages fit.
+template <int BN, int MT, int BITS>
 struct TileW8 {
   static constexpr int A_ST = MT == 64 ? MOE_W8_A_STAGES_M64 : MOE_W8_A_STAGES;
   static constexpr int B_ST = MOE_W8_B_STAGES;
-  static constexpr int Q_ST = MT == 64 ? MOE_W8_CODE_STAGES_M64 : MOE_W8_CODE_STAGES;
+  static constexpr int Q_ST = BITS == 8
+                                  ? (MT == 64 ? MOE_W8_CODE_STAGES_M64 : MOE_W8_CODE_STAGES)
+                                  : (MT == 64 ? MOE_W4_CODE_STAGES_M64 : MOE_W4_CODE_STAGES);
   static constexpr int A_BYTES = MT * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int Q_BYTES = BN * BK;
+  static constexpr int BOX_CODE = 128 * BK * BITS / 8;  // code bytes of a 128-row box
+  static constexpr int Q_CODE = BN * BK * BITS / 8;     // code bytes of a stage
+  static constexpr int Q_BYTES = Q_CODE + (BITS == 4 ? BN * 2 : 0);
   static constexpr int B_OFF = A_ST * A_BYTES;
   static constexpr int Q_OFF = B_OFF + B_ST * B_BYTES;
   static constexpr int BAR_OFF = Q_OFF + Q_ST * Q_BYTES;
   static constexpr int NUM_BARS = 2 * (A_ST + B_ST + Q_ST) + 5;
   static constexpr int SMEM = 1024 + BAR_OFF + NUM_BARS * 8 + 8 + 65 * 4;
-  static constexpr int CHUNKS = BN * BK / 16 / (32 * kConvWarps);  // code chunks per thread
+  static constexpr int CHUNKS = Q_CODE / 16 / (32 * kConvWarps);  // 16-byte code chunks per thread
   // D f32, A and B f16 (format 0), both K-major, M = MT, N = BN
   static constexpr uint32_t IDESC =
       (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(MT >> 4) << 24);
   static_assert(MT == 64 || MT == 128, "tile rows");
+  static_assert(BITS == 8 || BITS == 4, "code width");
+  static_assert(Q_BYTES % 16 == 0, "bulk copies need 16-byte stage boundaries");
   static_assert(SMEM <= 232448, "shared memory plan exceeds 227 KiB");
-  static_assert(CHUNKS * 32 * kConvWarps * 16 == BN * BK, "converter split");
+  static_assert(CHUNKS * 32 * kConvWarps * 16 == Q_CODE, "converter split");
 };
 
 struct W8Params {
   const uint8_t* q0;     // tiled codes of the first weight (w1 or w2)
   const uint8_t* q1;     // tiled codes of w3 (gate/up only)
   const int32_t* offsets;
-  const float* scale_a;  // per-row scales of the first weight (w1 or w2) [E * rows]
-  const float* scale_b;  // per-row scales of w3 (gate/up only)
+  const float* scale_a;  // int8: per-row scales of the first weight (w1 or w2) [E * rows]
+  const float* scale_b;  // int8: per-row scales of w3 (gate/up only)
+  const uint16_t* gscale_a;  // 4-bit: half group scales of the first weight, tile order
+  const uint16_t* gscale_b;  // 4-bit: of w3 (gate/up only)
   int32_t* status;
   void* out;
   int64_t out_ld;
@@ -271,6 +291,33 @@ __device__ __forceinline__ void widen16(const uint4 w4, uint4& lo8, uint4& hi8) 
   widen_word(w4.w, hi8.z, hi8.w);
 }
 
+// 4-bit codes, offset-binary u = q + 8, eight to a 32-bit word: column 2j of the word's
+// 8 columns sits in nibble j and column 2j + 1 in nibble j + 4 (j = 0..3), so one
+// shift and mask bring a column pair into the low bits of the word's two halves.
+// OR-ing in 0x6400 makes the halves 1024 + u (exponent 2^10, exact), subtracting 1032
+// leaves q exactly, and one packed multiply forms half(q * s), rounded once.
+__device__ __forceinline__ uint32_t nibbles_to_f16x2(uint32_t w, int j, uint32_t s2) {
+  const uint32_t x = ((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
+  uint32_t d, r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(x), "r"(0x64086408u));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(d), "r"(s2));
+  return r;
+}
+
+// One word (8 columns) -> one 16-byte run of 8 halves, each times the scale pair s2
+__device__ __forceinline__ uint4 widen_word4(uint32_t w, uint32_t s2) {
+  return make_uint4(nibbles_to_f16x2(w, 0, s2), nibbles_to_f16x2(w, 1, s2),
+                    nibbles_to_f16x2(w, 2, s2), nibbles_to_f16x2(w, 3, s2));
+}
+
+// Per-channel scale of the int8 codes, applied to the fp32 accumulator; the 4-bit
+// weights carry their scales already (a factor of 1, exact)
+template <int BITS>
+__device__ __forceinline__ float chan_scale(const float* s, int i) {
+  if constexpr (BITS == 8) return __ldg(s + i);
+  else return 1.f;
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2_rn(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -280,10 +327,10 @@ __device__ __forceinline__ uint32_t pack_f16x2_rn(float lo, float hi) {
 // MODE kSwiGLU: A = x_perm [rows, H] (half), weight tile = 128 rows of w1 then 128 rows
 //   of w3 (BN = 256), h = half(silu(s1 * gate) * (s3 * up)).
 // MODE kPlain:  A = h [rows, I], weight tile = BN rows of w2, y = s2 * acc (fp32).
-template <int MODE, int BN, int MT>
+template <int MODE, int BN, int MT, int BITS>
 __global__ void __launch_bounds__(kThreadsW8, 1)
     k_grouped_gemm_w8(const __grid_constant__ CUtensorMap mapA, const W8Params p) {
-  using TL = TileW8<BN, MT>;
+  using TL = TileW8<BN, MT, BITS>;
   constexpr int kAStages = TL::A_ST, kBStages = TL::B_ST, kCodeStages = TL::Q_ST;
   constexpr int A_BYTES = TL::A_BYTES;
   static_assert(MODE == kPlain || BN == 256, "gate/up tiles hold 128 gate + 128 up columns");
@@ -369,16 +416,26 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
           }
           const uint32_t dq = smem_u32(qbase + q * TL::Q_BYTES);
           mbar_expect_tx(q_full(q), TL::Q_BYTES);
+          // code_y / 128 is the tile number: its codes start at byte tile * BOX_CODE
+          // and (4-bit) its 128 scales at element tile * 128 = code_y
+          constexpr int kBox = TL::BOX_CODE;
           if (MODE == kSwiGLU) {
-            const size_t off = (size_t)code_y(row0, kb, p.k_blocks) * BK;
-            bulk_load(dq, p.q0 + off, 128 * BK, q_full(q));
-            bulk_load(dq + 128 * BK, p.q1 + off, 128 * BK, q_full(q));
+            const int cy = code_y(row0, kb, p.k_blocks);
+            const size_t off = (size_t)cy * (kBox / 128);
+            bulk_load(dq, p.q0 + off, kBox, q_full(q));
+            bulk_load(dq + kBox, p.q1 + off, kBox, q_full(q));
+            if constexpr (BITS == 4) {
+              bulk_load(dq + TL::Q_CODE, p.gscale_a + cy, 256, q_full(q));
+              bulk_load(dq + TL::Q_CODE + 256, p.gscale_b + cy, 256, q_full(q));
+            }
           } else {
 #pragma unroll
-            for (int j = 0; j < BN / 128; ++j)
-              bulk_load(dq + j * 128 * BK,
-                        p.q0 + (size_t)code_y(row0 + 128 * j, kb, p.k_blocks) * BK, 128 * BK,
-                        q_full(q));
+            for (int j = 0; j < BN / 128; ++j) {
+              const int cy = code_y(row0 + 128 * j, kb, p.k_blocks);
+              bulk_load(dq + j * kBox, p.q0 + (size_t)cy * (kBox / 128), kBox, q_full(q));
+              if constexpr (BITS == 4)
+                bulk_load(dq + TL::Q_CODE + j * 256, p.gscale_a + cy, 256, q_full(q));
+            }
           }
         }
       }
@@ -473,8 +530,21 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
         }
         const uint4* qs = reinterpret_cast<const uint4*>(qbase + q * TL::Q_BYTES);
         uint4 v[TL::CHUNKS];
+        uint32_t sc2[TL::CHUNKS];
 #pragma unroll
-        for (int i = 0; i < TL::CHUNKS; ++i) v[i] = qs[ct + 32 * kConvWarps * i];
+        for (int i = 0; i < TL::CHUNKS; ++i) {
+          const int j = ct + 32 * kConvWarps * i;
+          v[i] = qs[j];
+          if constexpr (BITS == 4) {
+            // 4-bit chunk j: box j / 256, column half (j / 128) % 2, row j % 128; the
+            // scale of stage row (j / 256) * 128 + j % 128, as a pair
+            const uint16_t* ss =
+                reinterpret_cast<const uint16_t*>(qbase + q * TL::Q_BYTES + TL::Q_CODE);
+            sc2[i] = (uint32_t)ss[(j >> 8) * 128 + (j & 127)] * 0x10001u;
+          } else {
+            sc2[i] = 0u;
+          }
+        }
         if (!wait_warp(b_empty(sb), ((uint32_t)(it / kBStages) & 1u) ^ 1u, abort_flag, p.status,
                        p.timeout_ns)) {
           ok = false;
@@ -484,12 +554,23 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
 #pragma unroll
         for (int i = 0; i < TL::CHUNKS; ++i) {
           const int j = ct + 32 * kConvWarps * i;
-          const int r = (j >> 9) * 128 + (j & 127), c = ((j >> 7) & 3) * 2;
-          uint4 lo8, hi8;
-          widen16(v[i], lo8, hi8);
-          uint8_t* row = bs + r * 128;
-          *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = lo8;
-          *reinterpret_cast<uint4*>(row + (((c + 1) ^ (r & 7)) << 4)) = hi8;
+          if constexpr (BITS == 8) {
+            const int r = (j >> 9) * 128 + (j & 127), c = ((j >> 7) & 3) * 2;
+            uint4 lo8, hi8;
+            widen16(v[i], lo8, hi8);
+            uint8_t* row = bs + r * 128;
+            *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = lo8;
+            *reinterpret_cast<uint4*>(row + (((c + 1) ^ (r & 7)) << 4)) = hi8;
+          } else {
+            // 32 codes of row r, columns 32 (c / 4) .. + 31: four 16-byte runs of halves
+            const int r = (j >> 8) * 128 + (j & 127), c = ((j >> 7) & 1) * 4;
+            uint8_t* row = bs + r * 128;
+            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+            for (int mw = 0; mw < 4; ++mw)
+              *reinterpret_cast<uint4*>(row + (((c + mw) ^ (r & 7)) << 4)) =
+                  widen_word4(w[mw], sc2[i]);
+          }
         }
         // make the generic-proxy stores visible to the tensor cores (async proxy)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -519,8 +600,8 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
       const uint32_t taddr = tmem_base + ((uint32_t)(qd * 32) << 16) + (uint32_t)(a * BN);
       const int64_t row = (int64_t)m * BM + row_in_tile;
       if (MODE == kSwiGLU) {
-        const float* sg = p.scale_a + (size_t)e * p.b_rows + n * 128;
-        const float* su = p.scale_b + (size_t)e * p.b_rows + n * 128;
+        const float* sg = BITS == 8 ? p.scale_a + (size_t)e * p.b_rows + n * 128 : nullptr;
+        const float* su = BITS == 8 ? p.scale_b + (size_t)e * p.b_rows + n * 128 : nullptr;
         uint16_t* h = reinterpret_cast<uint16_t*>(p.out) + row * p.out_ld + (int64_t)n * 128;
 #pragma unroll 1
         for (int c = 0; c < 128; c += 16) {
@@ -531,10 +612,10 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
           uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float g0 = __uint_as_float(g[2 * i]) * __ldg(sg + c + 2 * i);
-            const float g1 = __uint_as_float(g[2 * i + 1]) * __ldg(sg + c + 2 * i + 1);
-            const float u0 = __uint_as_float(u[2 * i]) * __ldg(su + c + 2 * i);
-            const float u1 = __uint_as_float(u[2 * i + 1]) * __ldg(su + c + 2 * i + 1);
+            const float g0 = __uint_as_float(g[2 * i]) * chan_scale<BITS>(sg, c + 2 * i);
+            const float g1 = __uint_as_float(g[2 * i + 1]) * chan_scale<BITS>(sg, c + 2 * i + 1);
+            const float u0 = __uint_as_float(u[2 * i]) * chan_scale<BITS>(su, c + 2 * i);
+            const float u1 = __uint_as_float(u[2 * i + 1]) * chan_scale<BITS>(su, c + 2 * i + 1);
             pk[i] = pack_f16x2_rn(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1);
           }
           if (row_valid) {
@@ -544,7 +625,7 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
           }
         }
       } else {
-        const float* sc = p.scale_a + (size_t)e * p.b_rows + n * BN;
+        const float* sc = BITS == 8 ? p.scale_a + (size_t)e * p.b_rows + n * BN : nullptr;
         float* y = reinterpret_cast<float*>(p.out) + row * p.out_ld + (int64_t)n * BN;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 16) {
@@ -554,10 +635,10 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
           float4* dst = reinterpret_cast<float4*>(y + c);
 #pragma unroll
           for (int i = 0; i < 4 && row_valid; ++i)
-            dst[i] = make_float4(__uint_as_float(v[4 * i]) * __ldg(sc + c + 4 * i),
-                                 __uint_as_float(v[4 * i + 1]) * __ldg(sc + c + 4 * i + 1),
-                                 __uint_as_float(v[4 * i + 2]) * __ldg(sc + c + 4 * i + 2),
-                                 __uint_as_float(v[4 * i + 3]) * __ldg(sc + c + 4 * i + 3));
+            dst[i] = make_float4(__uint_as_float(v[4 * i]) * chan_scale<BITS>(sc, c + 4 * i),
+                                 __uint_as_float(v[4 * i + 1]) * chan_scale<BITS>(sc, c + 4 * i + 1),
+                                 __uint_as_float(v[4 * i + 2]) * chan_scale<BITS>(sc, c + 4 * i + 2),
+                                 __uint_as_float(v[4 * i + 3]) * chan_scale<BITS>(sc, c + 4 * i + 3));
         }
       }
       fence_before();
@@ -625,6 +706,76 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
   }
 }
 
+__device__ __forceinline__ uint16_t f32_to_f16_rn(float f) {
+  uint16_t h;
+  asm("cvt.rn.f16.f32 %0, %1;" : "=h"(h) : "f"(f));
+  return h;
+}
+__device__ __forceinline__ float f16_to_f32(uint16_t h) {
+  float f;
+  asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"(h));
+  return f;
+}
+
+// One warp per weight row, four 64-column groups per step (8 lanes to a group, 8
+// consecutive columns to a lane): s = half(max|w| / 7) (1 when that is zero), q =
+// rint(w / s) clamped to [-7, 7], in float32. A lane packs its 8 codes (plus 8) into
+// one word of the tiled 4-bit layout; the group's first lane writes the scale.
+__global__ void __launch_bounds__(256) k_quant_groups4(const uint16_t* __restrict__ w,
+                                                       uint8_t* __restrict__ q,
+                                                       uint16_t* __restrict__ s, int64_t rows,
+                                                       int K) {
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31, grp = lane >> 3, m8 = lane & 7;
+  const int kbn = K / BK;
+  for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
+       r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    const uint16_t* wr = w + r * K;
+    const int64_t rb = r >> 7, rr = r & 127;
+    for (int kb0 = 0; kb0 < kbn; kb0 += 4) {
+      const int kb = kb0 + grp;
+      const bool act = kb < kbn;
+      float v[8];
+      if (act) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(wr + kb * BK + 8 * m8));
+        const uint32_t ww[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          v[2 * t] = __uint_as_float(ww[t] << 16);
+          v[2 * t + 1] = __uint_as_float(ww[t] & 0xFFFF0000u);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.f;
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      uint16_t sh = f32_to_f16_rn(__fdiv_rn(amax, 7.f));
+      if ((sh & 0x7FFFu) == 0) sh = 0x3C00u;  // a zero scale (in half) becomes 1
+      const float sd = f16_to_f32(sh);
+      uint32_t word = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        int qi = __float2int_rn(__fdiv_rn(v[i], sd));
+        qi = qi > 7 ? 7 : (qi < -7 ? -7 : qi);
+        const int nib = (i & 1) ? 4 + (i >> 1) : (i >> 1);
+        word |= (uint32_t)(qi + 8) << (4 * nib);
+      }
+      if (act) {
+        const int64_t tile = rb * kbn + kb;
+        *reinterpret_cast<uint32_t*>(q + tile * (128 * BK / 2) + (m8 >> 2) * 2048 + rr * 16 +
+                                     (m8 & 3) * 4) = word;
+        if (m8 == 0) s[tile * 128 + rr] = sh;
+      }
+    }
+  }
+}
+
 typedef CUresult (*EncodeTiledFnW8)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                     const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                     const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -656,24 +807,24 @@ bool map_act(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, ui
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE, int BN, int MT>
+template <int MODE, int BN, int MT, int BITS>
 cudaError_t launch_w8(const CUtensorMap& a, const W8Params& p, int64_t max_tiles,
                       cudaStream_t st) {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm_w8<MODE, BN, MT>,
+    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm_w8<MODE, BN, MT, BITS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         TileW8<BN, MT>::SMEM);
+                                         TileW8<BN, MT, BITS>::SMEM);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   int64_t grid = num_sms();
   if (grid > max_tiles) grid = max_tiles;
   if (grid < 1) grid = 1;
-  return launch_pdl(k_grouped_gemm_w8<MODE, BN, MT>, dim3((unsigned)grid), dim3(kThreadsW8),
-                    (size_t)TileW8<BN, MT>::SMEM, st, a, p);
+  return launch_pdl(k_grouped_gemm_w8<MODE, BN, MT, BITS>, dim3((unsigned)grid), dim3(kThreadsW8),
+                    (size_t)TileW8<BN, MT, BITS>::SMEM, st, a, p);
 }
 
 }  // namespace
@@ -697,10 +848,18 @@ cudaError_t launch_quant_rows(const uint16_t* w, uint8_t* q, float* s, int64_t r
   return launch_pdl(k_quant_rows, dim3((unsigned)blocks), dim3(256), 0, st, w, q, s, rows, K);
 }
 
+cudaError_t launch_quant_groups4(const uint16_t* w, uint8_t* q, uint16_t* s, int64_t rows, int K,
+                                 cudaStream_t st) {
+  int64_t blocks = (rows + 7) / 8;
+  const int64_t cap = (int64_t)num_sms() * 16;
+  if (blocks > cap) blocks = cap;
+  return launch_pdl(k_quant_groups4, dim3((unsigned)blocks), dim3(256), 0, st, w, q, s, rows, K);
+}
+
 namespace {
 
-// Both GEMMs with MT-row tiles (see TileW8)
-template <int MT>
+// Both GEMMs with MT-row tiles (see TileW8), BITS-bit codes
+template <int MT, int BITS>
 cudaError_t launch_swiglu_w8_tiles(const Shape& s, const GemmArgsW8& g, cudaStream_t st,
                                    const char** why) {
   CUtensorMap mx, mh;
@@ -715,6 +874,8 @@ cudaError_t launch_swiglu_w8_tiles(const Shape& s, const GemmArgsW8& g, cudaStre
   p1.offsets = g.offsets;
   p1.scale_a = g.s1;
   p1.scale_b = g.s3;
+  p1.gscale_a = g.g1;
+  p1.gscale_b = g.g3;
   p1.status = g.status;
   p1.out = g.h;
   p1.out_ld = s.I;
@@ -723,9 +884,9 @@ cudaError_t launch_swiglu_w8_tiles(const Shape& s, const GemmArgsW8& g, cudaStre
   p1.n_tiles = s.I / 128;
   p1.b_rows = s.I;
   p1.timeout_ns = g.timeout_ns;
-  cudaError_t e = launch_w8<kSwiGLU, 256, MT>(mx, p1, mt_max * p1.n_tiles, st);
+  cudaError_t e = launch_w8<kSwiGLU, 256, MT, BITS>(mx, p1, mt_max * p1.n_tiles, st);
   if (e != cudaSuccess) {
-    *why = "int8 gate/up GEMM launch failed";
+    *why = BITS == 8 ? "int8 gate/up GEMM launch failed" : "4-bit gate/up GEMM launch failed";
     return e;
   }
   W8Params p2 = p1;
@@ -733,18 +894,21 @@ cudaError_t launch_swiglu_w8_tiles(const Shape& s, const GemmArgsW8& g, cudaStre
   p2.q1 = nullptr;
   p2.scale_a = g.s2;
   p2.scale_b = nullptr;
+  p2.gscale_a = g.g2;
+  p2.gscale_b = nullptr;
   p2.out = g.y;
   p2.out_ld = s.H;
   p2.k_blocks = s.I / BK;
   p2.b_rows = s.H;
   if (s.H % 256 == 0) {
     p2.n_tiles = s.H / 256;
-    e = launch_w8<kPlain, 256, MT>(mh, p2, mt_max * p2.n_tiles, st);
+    e = launch_w8<kPlain, 256, MT, BITS>(mh, p2, mt_max * p2.n_tiles, st);
   } else {
     p2.n_tiles = s.H / 128;
-    e = launch_w8<kPlain, 128, MT>(mh, p2, mt_max * p2.n_tiles, st);
+    e = launch_w8<kPlain, 128, MT, BITS>(mh, p2, mt_max * p2.n_tiles, st);
   }
-  if (e != cudaSuccess) *why = "int8 down GEMM launch failed";
+  if (e != cudaSuccess)
+    *why = BITS == 8 ? "int8 down GEMM launch failed" : "4-bit down GEMM launch failed";
   return e;
 }
 
@@ -754,8 +918,12 @@ cudaError_t launch_grouped_swiglu_w8(const Shape& s, const GemmArgsW8& g, cudaSt
                                      const char** why) {
   // a token is routed to an expert at most once, so with at most 64 tokens every expert
   // has at most 64 rows, all in the first half of its 128-row tile
-  if (s.T <= 64 && kUseHalfTiles) return launch_swiglu_w8_tiles<64>(s, g, st, why);
-  return launch_swiglu_w8_tiles<128>(s, g, st, why);
+  const bool half_tiles = s.T <= 64 && kUseHalfTiles;
+  if (g.bits == 4)
+    return half_tiles ? launch_swiglu_w8_tiles<64, 4>(s, g, st, why)
+                      : launch_swiglu_w8_tiles<128, 4>(s, g, st, why);
+  return half_tiles ? launch_swiglu_w8_tiles<64, 8>(s, g, st, why)
+                    : launch_swiglu_w8_tiles<128, 8>(s, g, st, why);
 }
 
 }  // namespace moe

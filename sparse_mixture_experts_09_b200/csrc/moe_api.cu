@@ -148,12 +148,14 @@ T* at(void* ws, size_t off) {
 
 constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per wait
 
-// Expert weights of one layer: bf16 (w1, w3, w2), or int8 codes with per-row scales
-// (q1 non-null; then x_perm and h are IEEE half).
+// Expert weights of one layer: bf16 (w1, w3, w2), int8 codes with per-row scales, or
+// 4-bit codes with half group scales (q1 non-null; then x_perm and h are IEEE half).
 struct Experts {
   const uint16_t *w1, *w3, *w2;
   const uint8_t *q1, *q3, *q2;
   const float *s1, *s3, *s2;
+  const uint16_t *g1, *g3, *g2;
+  int bits;
 };
 
 Experts bf16_experts(const uint16_t* w1, const uint16_t* w3, const uint16_t* w2) {
@@ -173,6 +175,20 @@ Experts int8_experts(const uint8_t* q1, const uint8_t* q3, const uint8_t* q2, co
   x.s1 = s1;
   x.s3 = s3;
   x.s2 = s2;
+  x.bits = 8;
+  return x;
+}
+
+Experts int4_experts(const uint8_t* q1, const uint8_t* q3, const uint8_t* q2, const uint16_t* g1,
+                     const uint16_t* g3, const uint16_t* g2) {
+  Experts x = {};
+  x.q1 = q1;
+  x.q3 = q3;
+  x.q2 = q2;
+  x.g1 = g1;
+  x.g3 = g3;
+  x.g2 = g2;
+  x.bits = 4;
   return x;
 }
 
@@ -191,6 +207,10 @@ moe_status_t run_experts(const Shape& s, const uint16_t* x_perm, const int32_t* 
     g.s1 = w.s1;
     g.s3 = w.s3;
     g.s2 = w.s2;
+    g.g1 = w.g1;
+    g.g3 = w.g3;
+    g.g2 = w.g2;
+    g.bits = w.bits == 4 ? 4 : 8;
     g.h = h;
     g.y = y;
     g.status = status;
@@ -663,6 +683,83 @@ moe_status_t moe_forward_w8(const moe_shape_t* shape, const moe_bf16_t* x,
   MOE_TRY(check_ptr(out, "out"));
   MOE_TRY(check_ws(ws, ws_bytes, layout(s).end));
   return run_forward(s, x, w_router, logit_bias, int8_experts(q1, q3, q2, s1, s3, s2), residual,
+                     out, ws, (cudaStream_t)stream);
+}
+
+moe_status_t moe_quantize_int4(const moe_shape_t* shape, const moe_bf16_t* w1,
+                               const moe_bf16_t* w3, const moe_bf16_t* w2, uint8_t* q1,
+                               uint8_t* q3, uint8_t* q2, uint16_t* s1, uint16_t* s3,
+                               uint16_t* s2, moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(w1, "w1"));
+  MOE_TRY(check_ptr(w3, "w3"));
+  MOE_TRY(check_ptr(w2, "w2"));
+  MOE_TRY(check_ptr(q1, "q1"));
+  MOE_TRY(check_ptr(q3, "q3"));
+  MOE_TRY(check_ptr(q2, "q2"));
+  MOE_TRY(check_ptr(s1, "s1"));
+  MOE_TRY(check_ptr(s3, "s3"));
+  MOE_TRY(check_ptr(s2, "s2"));
+  cudaStream_t st = (cudaStream_t)stream;
+  const int64_t ei = (int64_t)s.E * s.I, eh = (int64_t)s.E * s.H;
+  cudaError_t e = launch_quant_groups4(w1, q1, s1, ei, s.H, st);
+  if (e == cudaSuccess) e = launch_quant_groups4(w3, q3, s3, ei, s.H, st);
+  if (e == cudaSuccess) e = launch_quant_groups4(w2, q2, s2, eh, s.I, st);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "4-bit quantiser launch");
+}
+
+moe_status_t moe_grouped_swiglu_w4(const moe_shape_t* shape, const moe_bf16_t* x_perm,
+                                   const int32_t* expert_offsets, const uint8_t* q1,
+                                   const uint8_t* q3, const uint8_t* q2, const uint16_t* s1,
+                                   const uint16_t* s3, const uint16_t* s2, float* y_perm,
+                                   void* ws, size_t ws_bytes, moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(x_perm, "x_perm"));
+  MOE_TRY(check_ptr(expert_offsets, "expert_offsets"));
+  MOE_TRY(check_ptr(q1, "q1"));
+  MOE_TRY(check_ptr(q3, "q3"));
+  MOE_TRY(check_ptr(q2, "q2"));
+  MOE_TRY(check_ptr(s1, "s1"));
+  MOE_TRY(check_ptr(s3, "s3"));
+  MOE_TRY(check_ptr(s2, "s2"));
+  MOE_TRY(check_ptr(y_perm, "y_perm"));
+  const Layout L = layout(s);
+  MOE_TRY(check_ws(ws, ws_bytes, L.end));
+  // the 4-bit experts read half activations: convert the caller's rows into ws
+  uint16_t* xh = at<uint16_t>(ws, L.x_perm);
+  cudaError_t e = launch_rows_to_f16(x_perm, xh, max_padded_rows(s), s.H, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "x_perm conversion launch");
+  return run_experts(s, xh, expert_offsets, int4_experts(q1, q3, q2, s1, s3, s2),
+                     at<uint16_t>(ws, L.h), y_perm, at<int32_t>(ws, L.status),
+                     (cudaStream_t)stream);
+}
+
+moe_status_t moe_forward_w4(const moe_shape_t* shape, const moe_bf16_t* x,
+                            const moe_bf16_t* w_router, const float* logit_bias,
+                            const uint8_t* q1, const uint8_t* q3, const uint8_t* q2,
+                            const uint16_t* s1, const uint16_t* s3, const uint16_t* s2,
+                            const moe_bf16_t* residual, moe_bf16_t* out, void* ws,
+                            size_t ws_bytes, moe_stream_t stream) {
+  g_err[0] = 0;
+  Shape s;
+  MOE_TRY(check_shape(shape, &s));
+  MOE_TRY(check_ptr(x, "x"));
+  MOE_TRY(check_ptr(w_router, "w_router"));
+  MOE_TRY(check_ptr(logit_bias, "logit_bias", true));
+  MOE_TRY(check_ptr(q1, "q1"));
+  MOE_TRY(check_ptr(q3, "q3"));
+  MOE_TRY(check_ptr(q2, "q2"));
+  MOE_TRY(check_ptr(s1, "s1"));
+  MOE_TRY(check_ptr(s3, "s3"));
+  MOE_TRY(check_ptr(s2, "s2"));
+  MOE_TRY(check_ptr(residual, "residual", true));
+  MOE_TRY(check_ptr(out, "out"));
+  MOE_TRY(check_ws(ws, ws_bytes, layout(s).end));
+  return run_forward(s, x, w_router, logit_bias, int4_experts(q1, q3, q2, s1, s3, s2), residual,
                      out, ws, (cudaStream_t)stream);
 }
 

@@ -78,23 +78,34 @@ cudaError_t launch_grouped_swiglu(const Shape& s, const GemmArgs& g, cudaStream_
 cudaError_t launch_quant_rows(const uint16_t* w, uint8_t* q, float* s, int64_t rows, int K,
                               cudaStream_t st);
 
+// Per group of 64 columns of a row of w [rows, K] (bf16): s = half(max|w| / 7) (1 when
+// that is zero), q = rint(w / s) clamped to [-7, 7], in float32; q + 8 is written in
+// the tiled 4-bit layout and s, as IEEE half bits, in the same tile order (element
+// ((row / 128) * (K / 64) + col / 64) * 128 + row % 128).
+cudaError_t launch_quant_groups4(const uint16_t* w, uint8_t* q, uint16_t* s, int64_t rows, int K,
+                                 cudaStream_t st);
+
 struct GemmArgsW8 {
-  const uint16_t* a;       // x_perm [Rmax, H], IEEE half
-  const int32_t* offsets;  // [E+1], multiples of 128
-  const uint8_t* q1;       // tiled offset-binary codes of w1 (rows E*I, K = H)
-  const uint8_t* q3;       // same for w3
-  const uint8_t* q2;       // tiled codes of w2 (rows E*H, K = I)
-  const float* s1;         // [E*I]
-  const float* s3;         // [E*I]
-  const float* s2;         // [E*H]
-  uint16_t* h;             // [Rmax, I], IEEE half
-  float* y;                // [Rmax, H]
-  int32_t* status;
-  int64_t rmax;
-  unsigned long long timeout_ns;
+  const uint16_t* a = nullptr;        // x_perm [Rmax, H], IEEE half
+  const int32_t* offsets = nullptr;   // [E+1], multiples of 128
+  const uint8_t* q1 = nullptr;        // tiled offset-binary codes of w1 (rows E*I, K = H)
+  const uint8_t* q3 = nullptr;        // same for w3
+  const uint8_t* q2 = nullptr;        // tiled codes of w2 (rows E*H, K = I)
+  const float* s1 = nullptr;          // int8: per-row scales [E*I]
+  const float* s3 = nullptr;          // [E*I]
+  const float* s2 = nullptr;          // [E*H]
+  const uint16_t* g1 = nullptr;       // 4-bit: half group scales of w1, tile order
+  const uint16_t* g3 = nullptr;
+  const uint16_t* g2 = nullptr;
+  int bits = 8;                       // 8 or 4
+  uint16_t* h = nullptr;              // [Rmax, I], IEEE half
+  float* y = nullptr;                 // [Rmax, H]
+  int32_t* status = nullptr;
+  int64_t rmax = 0;
+  unsigned long long timeout_ns = 0;
 };
 
-// GEMM1 (int8 gate/up + SwiGLU -> h) then GEMM2 (h q2^T * s2 -> y), in float16.
+// GEMM1 (int8 or 4-bit gate/up + SwiGLU -> h) then GEMM2 (h q2^T -> y), in float16.
 cudaError_t launch_grouped_swiglu_w8(const Shape& s, const GemmArgsW8& g, cudaStream_t st,
                                      const char** why);
 

@@ -28,7 +28,7 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_size_host", "moe_max_padded_rows
            "moe_forward_host", "moe_device_status", "moe_last_error", "moe_permute_static",
            "moe_selftest_wait_timeout", "moe_forward_rmsnorm", "moe_pack_weights",
            "moe_quantize_int8", "moe_grouped_swiglu_w8", "moe_forward_w8", "moe_gather_rows",
-           "moe_forward_host_async")
+           "moe_forward_host_async", "moe_quantize_int4", "moe_grouped_swiglu_w4", "moe_forward_w4")
 
 
 @dataclass
@@ -48,6 +48,25 @@ class Int8Experts:
         return [_dev(self.q1, "q1", torch.uint8), _dev(self.q3, "q3", torch.uint8),
                 _dev(self.q2, "q2", torch.uint8), _dev(self.s1, "s1", torch.float32),
                 _dev(self.s3, "s3", torch.float32), _dev(self.s2, "s2", torch.float32)]
+
+
+@dataclass
+class Int4Experts:
+    """Weight-only 4-bit experts as written by quantize_int4: codes q1, q3 [E, I, H/2] and
+    q2 [E, H, I/2] (uint8, two offset-binary codes q + 8 to a byte, in the library's
+    tiled 4-bit layout of include/moe.h) and float16 scales, one per row and 64-column
+    group in tile order: s1, s3 [E, I/128, H/64, 128] and s2 [E, H/128, I/64, 128]."""
+    q1: torch.Tensor
+    q3: torch.Tensor
+    q2: torch.Tensor
+    s1: torch.Tensor
+    s3: torch.Tensor
+    s2: torch.Tensor
+
+    def pointers(self):
+        return [_dev(self.q1, "q1", torch.uint8), _dev(self.q3, "q3", torch.uint8),
+                _dev(self.q2, "q2", torch.uint8), _dev(self.s1, "s1", torch.float16),
+                _dev(self.s3, "s3", torch.float16), _dev(self.s2, "s2", torch.float16)]
 
 
 class MoeError(RuntimeError):
@@ -122,6 +141,12 @@ def lib() -> ctypes.CDLL:
         L.moe_grouped_swiglu_w8.restype = st
         L.moe_forward_w8.argtypes = [sp] + [_P] * 12 + [_SZ, _P]
         L.moe_forward_w8.restype = st
+        L.moe_quantize_int4.argtypes = [sp] + [_P] * 10
+        L.moe_quantize_int4.restype = st
+        L.moe_grouped_swiglu_w4.argtypes = [sp] + [_P] * 10 + [_SZ, _P]
+        L.moe_grouped_swiglu_w4.restype = st
+        L.moe_forward_w4.argtypes = [sp] + [_P] * 12 + [_SZ, _P]
+        L.moe_forward_w4.restype = st
         L.moe_gather_rows.argtypes = [_P, ctypes.c_int64, _P, ctypes.c_int64, ctypes.c_int64, _P, _P]
         L.moe_gather_rows.restype = st
         L.moe_last_error.argtypes = []
@@ -432,6 +457,57 @@ def forward_w8(x, w_router, experts: Int8Experts, k: int, residual=None, logit_b
     if out is None:
         out = torch.empty((t, h), dtype=torch.bfloat16, device=x.device)
     _check(lib().moe_forward_w8(ctypes.byref(shape), _dev(x, "x", torch.bfloat16),
+                                _dev(w_router, "w_router", torch.bfloat16),
+                                _dev(logit_bias, "logit_bias", torch.float32, True),
+                                *experts.pointers(),
+                                _dev(residual, "residual", torch.bfloat16, True), _dev(out, "out"),
+                                _dev(ws, "ws"), ws.numel(), _stream(stream)))
+    return out
+
+
+def quantize_int4(w1, w3, w2, stream=None) -> Int4Experts:
+    """Row-major bf16 expert weights -> Int4Experts (symmetric 4-bit, a half scale per
+    64-column group of a row)."""
+    e, i, h = w1.shape
+    shape = make_shape(1, h, i, e, 1)
+    dev = w1.device
+    q = [torch.empty((e, i, h // 2), dtype=torch.uint8, device=dev),
+         torch.empty((e, i, h // 2), dtype=torch.uint8, device=dev),
+         torch.empty((e, h, i // 2), dtype=torch.uint8, device=dev)]
+    sc = [torch.empty((e, i // 128, h // 64, 128), dtype=torch.float16, device=dev),
+          torch.empty((e, i // 128, h // 64, 128), dtype=torch.float16, device=dev),
+          torch.empty((e, h // 128, i // 64, 128), dtype=torch.float16, device=dev)]
+    out = Int4Experts(q[0], q[1], q[2], sc[0], sc[1], sc[2])
+    _check(lib().moe_quantize_int4(ctypes.byref(shape), _dev(w1, "w1", torch.bfloat16),
+                                   _dev(w3, "w3", torch.bfloat16), _dev(w2, "w2", torch.bfloat16),
+                                   *out.pointers(), _stream(stream)))
+    return out
+
+
+def grouped_swiglu_w4(x_perm, offsets, experts: Int4Experts, num_tokens: int, k: int, ws,
+                      stream=None):
+    """grouped_swiglu with 4-bit expert weights: y_perm [R_max, H] fp32."""
+    e, i, h2 = experts.q1.shape
+    shape = make_shape(num_tokens, 2 * h2, i, e, k)
+    y = torch.zeros((max_padded_rows(shape), 2 * h2), dtype=torch.float32, device=x_perm.device)
+    _check(lib().moe_grouped_swiglu_w4(ctypes.byref(shape), _dev(x_perm, "x_perm", torch.bfloat16),
+                                       _dev(offsets, "offsets", torch.int32), *experts.pointers(),
+                                       _dev(y, "y_perm"), _dev(ws, "ws"), ws.numel(),
+                                       _stream(stream)))
+    return y
+
+
+def forward_w4(x, w_router, experts: Int4Experts, k: int, residual=None, logit_bias=None,
+               ws=None, out=None, stream=None, router_bf16_logits: bool = False):
+    """The whole layer with 4-bit expert weights; returns out [T,H] bf16."""
+    t, h = x.shape
+    e, i, _ = experts.q1.shape
+    shape = make_shape(t, h, i, e, k, ROW_MAJOR, router_bf16_logits)
+    if ws is None:
+        ws = make_workspace(shape, x.device)
+    if out is None:
+        out = torch.empty((t, h), dtype=torch.bfloat16, device=x.device)
+    _check(lib().moe_forward_w4(ctypes.byref(shape), _dev(x, "x", torch.bfloat16),
                                 _dev(w_router, "w_router", torch.bfloat16),
                                 _dev(logit_bias, "logit_bias", torch.float32, True),
                                 *experts.pointers(),
