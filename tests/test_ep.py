@@ -159,3 +159,75 @@ def test_exchange_plan_empty_rank():
     p = ep.exchange_plan([0, 0, 0, 0, 0], [0, 0, 0, 0], 2, [[0, 0], [4, 0]])
     assert p["send_rows"] == [0, 0] and p["send_index"] == [] and p["back_index"] == []
     assert p["local_offsets"] == [0, 128, 128] and p["to_recv"] == [0, 1, 2, 3]
+
+
+def _simulate_world(counts):
+    """All ranks' plans of one exchange, run on the host: counts[r][e] rows routed by
+    rank r to global expert e. Rows are tagged (rank, expert, j); the all-to-all is
+    emulated as concatenation by source rank. Returns what every owner computes on and
+    what every source gets back."""
+    world, e_total = len(counts), len(counts[0])
+    e_loc = e_total // world
+    pad = lambda n: (n + 127) // 128 * 128
+    x_perm, plans = [], []
+    for r in range(world):
+        offs = [0]
+        rows = []
+        for e in range(e_total):
+            rows += [(r, e, j) for j in range(counts[r][e])]
+            rows += [None] * (pad(counts[r][e]) - counts[r][e])
+            offs.append(len(rows))
+        x_perm.append(rows)
+        recv = [[counts[s][r * e_loc + e] for e in range(e_loc)] for s in range(world)]
+        plans.append(ep.exchange_plan(offs, counts[r], world, recv))
+    sent = []
+    for r in range(world):
+        rows = [x_perm[r][i] for i in plans[r]["send_index"]]
+        pieces, at = [], 0
+        for s in range(world):
+            pieces.append(rows[at:at + plans[r]["send_rows"][s]])
+            at += plans[r]["send_rows"][s]
+        sent.append(pieces)
+    local, back = [], []
+    for s in range(world):
+        received = [row for r in range(world) for row in sent[r][s]]
+        assert len(received) == sum(plans[s]["recv_rows"])
+        local.append([received[i] if i >= 0 else None for i in plans[s]["to_local"]])
+        # the experts keep rows in place; the reply goes out in received order
+        reply = [local[s][i] for i in plans[s]["to_recv"]]
+        back.append(reply)
+    returned = []
+    for r in range(world):
+        rows, at = [], 0
+        for s in range(world):
+            # rank s replies to r with the segment it received from r, in order
+            start = sum(plans[s]["recv_rows"][:r])
+            rows += back[s][start:start + plans[s]["recv_rows"][r]]
+        returned.append([rows[i] if i >= 0 else None for i in plans[r]["back_index"]])
+    return x_perm, plans, local, returned
+
+
+def test_exchange_plan_random_worlds_round_trip():
+    rng = np.random.default_rng(41)
+    for trial in range(60):
+        world = int(rng.choice([1, 2, 4]))
+        e_loc = int(rng.integers(1, 4))
+        # mostly small groups, some past one or two 128-row tiles, some empty
+        counts = rng.choice([0, 1, 3, 17, 127, 128, 129, 260], size=(world, world * e_loc))
+        counts = counts.tolist()
+        x_perm, plans, local, returned = _simulate_world(counts)
+        for s in range(world):
+            lo = plans[s]["local_offsets"]
+            assert len(lo) == e_loc + 1 and all(v % 128 == 0 for v in lo)
+            for e in range(e_loc):
+                group = local[s][lo[e]:lo[e + 1]]
+                real = [g for g in group if g is not None]
+                # expert group e of owner s: every source's rows for it, by source, then j
+                want = [(r, s * e_loc + e, j) for r in range(world)
+                        for j in range(counts[r][s * e_loc + e])]
+                assert real == want and group[len(real):] == [None] * (len(group) - len(real))
+        for r in range(world):
+            # every row comes back to its own place; pad rows stay empty
+            assert returned[r] == x_perm[r]
+            for s in range(world):
+                assert plans[r]["send_rows"][s] == plans[s]["recv_rows"][r]
