@@ -181,6 +181,43 @@ def _dev(t: Optional[torch.Tensor], name: str, dtype=None, nullable=False) -> Op
     return t.data_ptr()
 
 
+def _sized(name: str, t: Optional[torch.Tensor], n: int, at_least: bool = False) -> None:
+    """The kernels index a buffer by the layer's shape alone (the C ABI takes bare
+    pointers), so one of the wrong size would be read or written out of bounds: refuse
+    it here, before any pointer is taken."""
+    if t is None:
+        return
+    if t.numel() < n or (t.numel() != n and not at_least):
+        need = f"at least {n}" if at_least else f"{n}"
+        raise ValueError(f"{name} has {t.numel()} elements; the layer's shape needs {need}")
+
+
+def _layer_sizes(t: int, h: int, e: int, i: int, w_router=None, logit_bias=None, residual=None,
+                 out=None, **weights) -> None:
+    """Element counts of the tensors of a whole-layer call: w_router [E, H], logit_bias
+    [E], residual and out [T, H], and each keyword ``name=(tensor, count)``."""
+    _sized("w_router", w_router, e * h)
+    _sized("logit_bias", logit_bias, e)
+    _sized("residual", residual, t * h)
+    _sized("out", out, t * h)
+    for name, (tensor, n) in weights.items():
+        # x_perm may be a larger buffer: the kernels read its first R_max rows
+        _sized(name, tensor, n, at_least=name == "x_perm")
+
+
+def _bf16_weights(e: int, i: int, h: int, w1, w3, w2) -> dict:
+    return {"w1": (w1, e * i * h), "w3": (w3, e * i * h), "w2": (w2, e * h * i)}
+
+
+def _quant_weights(e: int, i: int, h: int, ex, bits: int) -> dict:
+    """Codes and scales of Int8Experts (bits 8) or Int4Experts (bits 4)."""
+    per = (lambda n: n) if bits == 8 else (lambda n: n // 2)
+    sc = (lambda rows, k: rows) if bits == 8 else (lambda rows, k: rows * k // 64)
+    return {"q1": (ex.q1, per(e * i * h)), "q3": (ex.q3, per(e * i * h)),
+            "q2": (ex.q2, per(e * h * i)), "s1": (ex.s1, sc(e * i, h)),
+            "s3": (ex.s3, sc(e * i, h)), "s2": (ex.s2, sc(e * h, i))}
+
+
 def _stream(stream) -> Optional[int]:
     s = stream if stream is not None else torch.cuda.current_stream()
     return s.cuda_stream
@@ -274,6 +311,8 @@ def grouped_swiglu(x_perm, offsets, w1, w3, w2, num_tokens: int, k: int, ws, str
     """y_perm [R_max, H] fp32 = w2[e] (silu(w1[e] x) * w3[e] x) per routed row."""
     e, i, h = w1.shape
     shape = make_shape(num_tokens, h, i, e, k, weight_layout)
+    _layer_sizes(0, h, e, i, x_perm=(x_perm, max_padded_rows(shape) * h),
+                 offsets=(offsets, e + 1), **_bf16_weights(e, i, h, w1, w3, w2))
     y = torch.zeros((max_padded_rows(shape), h), dtype=torch.float32, device=x_perm.device)
     _check(lib().moe_grouped_swiglu(ctypes.byref(shape), _dev(x_perm, "x_perm", torch.bfloat16),
                                     _dev(offsets, "offsets", torch.int32),
@@ -332,6 +371,8 @@ def forward(x, w_router, w1, w3, w2, k: int, residual=None, logit_bias=None, ws=
     t, h = x.shape
     e, i, _ = w1.shape
     shape = make_shape(t, h, i, e, k, weight_layout, router_bf16_logits)
+    _layer_sizes(t, h, e, i, w_router, logit_bias, residual, out,
+                 **_bf16_weights(e, i, h, w1, w3, w2))
     if ws is None:
         ws = make_workspace(shape, x.device)
     if out is None:
@@ -352,6 +393,8 @@ def forward_rmsnorm(h, norm_weight, eps: float, w_router, w1, w3, w2, k: int, lo
     t, hd = h.shape
     e, i, _ = w1.shape
     shape = make_shape(t, hd, i, e, k, weight_layout)
+    _layer_sizes(t, hd, e, i, w_router, logit_bias, None, out, norm_weight=(norm_weight, hd),
+                 **_bf16_weights(e, i, hd, w1, w3, w2))
     if ws is None:
         ws = make_workspace(shape, h.device)
     if out is None:
@@ -375,7 +418,9 @@ def forward_host(x_host, w_router, w1, w3, w2, k: int, residual_host=None, logit
     t, h = x_host.shape
     e, i, _ = w1.shape
     shape = make_shape(t, h, i, e, k, weight_layout)
-    for name, a in (("x_host", x_host), ("residual_host", residual_host)):
+    _layer_sizes(t, h, e, i, w_router, logit_bias, residual_host=(residual_host, t * h),
+                 out_host=(out_host, t * h), **_bf16_weights(e, i, h, w1, w3, w2))
+    for name, a in (("x_host", x_host), ("residual_host", residual_host), ("out_host", out_host)):
         if a is not None and (a.is_cuda or a.dtype != torch.bfloat16 or not a.is_contiguous()):
             raise ValueError(f"{name} must be a contiguous bf16 host tensor")
     if ws is None:
@@ -438,6 +483,8 @@ def grouped_swiglu_w8(x_perm, offsets, experts: Int8Experts, num_tokens: int, k:
     """grouped_swiglu with int8 expert weights: y_perm [R_max, H] fp32."""
     e, i, h = experts.q1.shape
     shape = make_shape(num_tokens, h, i, e, k)
+    _layer_sizes(0, h, e, i, x_perm=(x_perm, max_padded_rows(shape) * h),
+                 offsets=(offsets, e + 1), **_quant_weights(e, i, h, experts, 8))
     y = torch.zeros((max_padded_rows(shape), h), dtype=torch.float32, device=x_perm.device)
     _check(lib().moe_grouped_swiglu_w8(ctypes.byref(shape), _dev(x_perm, "x_perm", torch.bfloat16),
                                        _dev(offsets, "offsets", torch.int32), *experts.pointers(),
@@ -452,6 +499,8 @@ def forward_w8(x, w_router, experts: Int8Experts, k: int, residual=None, logit_b
     t, h = x.shape
     e, i, _ = experts.q1.shape
     shape = make_shape(t, h, i, e, k, ROW_MAJOR, router_bf16_logits)
+    _layer_sizes(t, h, e, i, w_router, logit_bias, residual, out,
+                 **_quant_weights(e, i, h, experts, 8))
     if ws is None:
         ws = make_workspace(shape, x.device)
     if out is None:
@@ -489,6 +538,8 @@ def grouped_swiglu_w4(x_perm, offsets, experts: Int4Experts, num_tokens: int, k:
     """grouped_swiglu with 4-bit expert weights: y_perm [R_max, H] fp32."""
     e, i, h2 = experts.q1.shape
     shape = make_shape(num_tokens, 2 * h2, i, e, k)
+    _layer_sizes(0, 2 * h2, e, i, x_perm=(x_perm, max_padded_rows(shape) * 2 * h2),
+                 offsets=(offsets, e + 1), **_quant_weights(e, i, 2 * h2, experts, 4))
     y = torch.zeros((max_padded_rows(shape), 2 * h2), dtype=torch.float32, device=x_perm.device)
     _check(lib().moe_grouped_swiglu_w4(ctypes.byref(shape), _dev(x_perm, "x_perm", torch.bfloat16),
                                        _dev(offsets, "offsets", torch.int32), *experts.pointers(),
@@ -503,6 +554,8 @@ def forward_w4(x, w_router, experts: Int4Experts, k: int, residual=None, logit_b
     t, h = x.shape
     e, i, _ = experts.q1.shape
     shape = make_shape(t, h, i, e, k, ROW_MAJOR, router_bf16_logits)
+    _layer_sizes(t, h, e, i, w_router, logit_bias, residual, out,
+                 **_quant_weights(e, i, h, experts, 4))
     if ws is None:
         ws = make_workspace(shape, x.device)
     if out is None:
