@@ -249,6 +249,7 @@ def router_topk(x, w_router, k: int, logit_bias=None, return_logits=False, strea
     t, h = x.shape
     e = w_router.shape[0]
     shape = make_shape(t, h, ROW_PAD, e, k, router_bf16_logits=router_bf16_logits)
+    _layer_sizes(t, h, e, ROW_PAD, w_router, logit_bias)
     idx = torch.empty((t, k), dtype=torch.int32, device=x.device)
     w = torch.empty((t, k), dtype=torch.float32, device=x.device)
     logits = torch.empty((t, e), dtype=torch.float32, device=x.device) if return_logits else None
@@ -265,6 +266,7 @@ def permute(topk_idx, x, num_experts: int, intermediate_size: int, ws, stream=No
     t, k = topk_idx.shape
     h = x.shape[1]
     shape = make_shape(t, h, intermediate_size, num_experts, k)
+    _sized("x", x, t * h, at_least=True)      # the gather reads rows 0 .. T-1
     rmax = max_padded_rows(shape)
     dev = x.device
     out = {
@@ -289,6 +291,7 @@ def permute_static(topk_idx, x, num_experts: int, intermediate_size: int, stream
     t, k = topk_idx.shape
     h = x.shape[1]
     shape = make_shape(t, h, intermediate_size, num_experts, k)
+    _sized("x", x, t * h, at_least=True)      # the gather reads rows 0 .. T-1
     rmax = max_padded_rows(shape)
     dev = x.device
     out = {
@@ -357,6 +360,8 @@ def combine(y_perm, row_of, topk_w, residual=None, num_experts: int = 8, interme
     t, k = row_of.shape
     h = y_perm.shape[1]
     shape = make_shape(t, h, intermediate_size, max(num_experts, k), k)
+    _sized("topk_w", topk_w, t * k)
+    _sized("residual", residual, t * h)
     out = torch.empty((t, h), dtype=torch.bfloat16, device=y_perm.device)
     _check(lib().moe_combine(ctypes.byref(shape), _dev(y_perm, "y_perm", torch.float32),
                              _dev(row_of, "row_of", torch.int32), _dev(topk_w, "topk_w", torch.float32),

@@ -99,3 +99,27 @@ def test_mis_sized_quantised_experts_and_buffers_are_refused():
     with pytest.raises(ValueError, match="out_host"):
         M.forward_host(a["x"], a["w_router"], a["w1"], a["w3"], a["w2"], K,
                        out_host=_bf16(T - 1, H))
+
+
+def test_split_entry_points_check_sizes():
+    x = _bf16(T, H)
+    with pytest.raises(ValueError, match="CUDA"):
+        M.router_topk(x, _bf16(E, H), K, torch.zeros(E, dtype=torch.float32))
+    with pytest.raises(ValueError, match="w_router"):
+        M.router_topk(x, _bf16(E, H // 2), K)
+    with pytest.raises(ValueError, match="logit_bias"):
+        M.router_topk(x, _bf16(E, H), K, torch.zeros(E - 1, dtype=torch.float32))
+    idx = torch.zeros((T, K), dtype=torch.int32)
+    for fn, extra in ((M.permute, (torch.zeros(8),)), (M.permute_static, ())):
+        with pytest.raises(ValueError, match="CUDA"):
+            fn(idx, _bf16(T + 3, H), E, I, *extra)           # more rows than tokens is fine
+        with pytest.raises(ValueError, match="x has"):
+            fn(idx, _bf16(T - 1, H), E, I, *extra)
+    y = torch.zeros((40, H), dtype=torch.float32)           # rows as the caller's groups need
+    row_of = torch.zeros((T, K), dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        M.combine(y, row_of, torch.zeros((T, K)), _bf16(T, H), E, I)
+    with pytest.raises(ValueError, match="topk_w"):
+        M.combine(y, row_of, torch.zeros((T, K + 1)), None, E, I)
+    with pytest.raises(ValueError, match="residual"):
+        M.combine(y, row_of, torch.zeros((T, K)), _bf16(T, H + 128), E, I)
