@@ -4,9 +4,10 @@
 //
 // Mixtral is loaded weight-only quantised to shrink it (Hugging Face "Mixtral" doc,
 // "Shrinking down Mixtral using quantization"; ZeroModels "Mixtral", "Lower memory":
-// int8 weights): half the weight memory of bf16. (At decode this kernel streams half
-// the bytes but is not faster than the bf16 one: its per-stage pipeline of copy,
-// widening and MMA handoffs, not HBM, sets its pace.)
+// int8 weights): half the weight memory of bf16, a quarter with 4-bit codes. (At
+// decode the int8 kernel streams half the bytes and the 4-bit one a quarter, yet
+// neither is faster than the bf16 kernel: the per-stage pipeline of copy, widening and
+// MMA handoffs, not HBM, sets their pace.)
 // Scheme (the pages do not fix one): per output row (channel) r, s[r] = max|w[r, :]| /
 // 127 and q = rint(w / s), decided in float32; w ~ q * s. The experts compute in half
 // precision, as a float16 load of the model does (Hugging Face "Mixtral" doc: the model
