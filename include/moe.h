@@ -314,7 +314,9 @@ moe_status_t moe_forward_w8(const moe_shape_t* shape, const moe_bf16_t* x,
  *   s = half(max |w| over the group / 7)   (1 when that is zero in half),
  *   q[r, c] = clamp(rint(w[r, c] / s), -7, 7),
  * the division and the rounding (to nearest, ties to even) in float32; the experts
- * multiply the weight half(q * s), one rounding of the product to half.
+ * multiply the weight half(q * s), one rounding of the product to half. The format
+ * covers groups whose largest |w| is at most 7 * 65504 (beyond it the half scale is
+ * infinite and the group's weights are not finite).
  * Codes are stored offset-binary, u = q + 8 (1 .. 15), two to a byte, tiled like the
  * int8 codes: tile (row / 128, col / 64) is the 4 KiB block number (row / 128) * (K /
  * 64) + col / 64; inside it, with r = row % 128 and c = col % 64, the code sits in the

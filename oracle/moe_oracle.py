@@ -291,7 +291,9 @@ def quantize_int4_groups(w, group: int = 64):
     manner of block-wise 4-bit schemes: for each group, s = max|w| / 7 in float32, then
     rounded to the nearest IEEE half (s16; a group whose s16 is zero, all zeros or too
     small for a half, takes s16 = 1); code q = round-half-even(w / s16) in float32,
-    clamped to [-7, 7]. The code is decided in float32 as the kernel decides it.
+    clamped to [-7, 7]. The code is decided in float32 as the kernel decides it. A
+    group whose largest |w| exceeds 7 * 65504 has an infinite half scale (outside the
+    format: its weights dequantise to NaN).
     Returns (q int8 [..., rows, K], s16 float16 [..., rows, K / group]).
     """
     w = np.asarray(to_f64(w), dtype=np.float32)
