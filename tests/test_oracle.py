@@ -400,9 +400,16 @@ def test_int4_groups_degenerate_groups_and_bound():
     w[0, 64:128] = 0.0                   # all zeros: scale 1, codes 0
     w[1, :64] = 0.0
     w[1, 10] = 2.0 ** -30                # amax / 7 underflows a half: scale 1, codes 0
+    w[2, 128:192] = 0.0                  # a subnormal scale: amax / 7 = (10/7) 2**-24
+    w[2, 130] = 10 * 2.0 ** -24          # rounds to the half 2**-24, so w / s = 10: clamped
+    w[2, 131] = -3 * 2.0 ** -24
+    w[2, 132] = -9 * 2.0 ** -24          # clamped at -7, not -8
     q, s16 = O.quantize_int4_groups(w)
     assert s16[0, 1] == 1.0 and np.all(q[0, 64:128] == 0)
     assert s16[1, 0] == 1.0 and np.all(q[1, :64] == 0)
+    assert s16[2, 2] == np.float16(2.0 ** -24) and q[2, 130] == 7 and q[2, 131] == -3
+    assert q[2, 132] == -7
+    assert np.all(q[2, 128:130] == 0) and np.all(q[2, 133:192] == 0)
     deq = O.dequantize_int4_groups(q, s16)
     s = np.repeat(s16.astype(np.float64), 64, axis=-1)
     # |w - f16(q s16)| <= s16 / 2 (nearest level; no clamping when s16 >= amax / 7) plus
@@ -410,8 +417,11 @@ def test_int4_groups_degenerate_groups_and_bound():
     unclamped = np.repeat(s16.astype(np.float64) * 7 >= np.abs(w).reshape(4, 4, 64).max(-1), 64, -1)
     bound = s / 2 + np.abs(deq) * 2.0 ** -11
     assert np.all((np.abs(w - deq) <= bound)[unclamped])
-    # a clamped level sits at most one half-rounding of the scale further out
-    assert np.all(np.abs(w - deq) <= s / 2 + 7 * s * 2.0 ** -10 + np.abs(deq) * 2.0 ** -11)
+    # with a normal half scale (relative rounding 2**-11), a clamped level sits at most one
+    # half-rounding of the scale further out (the subnormal group above is checked exactly)
+    normal = s >= 2.0 ** -14
+    err_ok = np.abs(w - deq) <= s / 2 + 7 * s * 2.0 ** -10 + np.abs(deq) * 2.0 ** -11
+    assert np.all(err_ok[normal]) and not np.all(normal)
 
 
 def test_int4_groups_match_torch_arithmetic():
