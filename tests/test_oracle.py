@@ -136,6 +136,17 @@ def test_stable_permute_against_library_sort(t_count, e_count, k):
     assert np.unique(row_of).size == t_count * k
 
 
+def test_stable_permute_offsets_closed_form():
+    # groups of 0, 1, 128, 129 and 256 rows take 0, 128, 128, 256 and 256 padded rows:
+    # an empty expert takes none, an exact multiple of 128 takes no extra tile
+    counts = [0, 1, 128, 129, 256]
+    idx = np.concatenate([np.full(c, e, dtype=np.int32) for e, c in enumerate(counts)])[:, None]
+    count, offset, row_of, tok = O.stable_permute(idx, len(counts))
+    assert count.tolist() == counts
+    assert offset.tolist() == [0, 0, 128, 256, 512, 768]
+    assert tok.size == 768 and int((tok >= 0).sum()) == sum(counts)
+
+
 # ---------------------------------------------------------------- experts and layer
 
 def _tiny_layer(seed, t_count=24, h=16, i=32, e_count=4, k=2):
@@ -469,6 +480,27 @@ def test_bf16_values_in_f16_normal_range_are_exact_in_f16():
     x = O.round_bf16(g.standard_normal(5000) * 10.0 ** g.integers(-4, 4, 5000))
     x = x[(np.abs(x) >= 2.0 ** -14) & (np.abs(x) <= 65504)]
     assert np.array_equal(O.round_f16(x), x)
+
+
+def test_f16_expert_mode_reads_x_rounded_to_half():
+    # one expert, one unit: x = 2**-20 (1 + 2**-7) is a bf16 value below half's normal
+    # range, where half spacing is 2**-24, so the experts read x16 = 2**-20. With gate and
+    # up weights 2**20, g = u = 1 and h = silu(1), stored as the nearest half; the down
+    # weight 1 passes it through. Unrounded x would give g = u = 1 + 2**-7 instead.
+    x = torch.tensor([[2.0 ** -20 * (1 + 2.0 ** -7)]], dtype=torch.bfloat16)
+    one = torch.ones((1, 1), dtype=torch.bfloat16)
+    big = torch.full((1, 1, 1), 2.0 ** 20, dtype=torch.bfloat16)
+    r = O.moe_layer(x, one, big, big, torch.ones((1, 1, 1), dtype=torch.bfloat16), 1,
+                    mode="f16_experts")
+    assert r["y"][0, 0, 0] == float(np.float16(1.0 / (1.0 + np.exp(-1.0))))
+    # values beyond half's largest finite value overflow when the experts read them
+    xl = torch.tensor([[70000.0]], dtype=torch.bfloat16)
+    rl = O.moe_layer(xl, one, one.view(1, 1, 1), one.view(1, 1, 1),
+                     torch.ones((1, 1, 1), dtype=torch.bfloat16), 1, mode="f16_experts")
+    assert not np.isfinite(rl["y"][0, 0, 0])
+    assert np.isfinite(O.moe_layer(xl, one, one.view(1, 1, 1), one.view(1, 1, 1),
+                                   torch.ones((1, 1, 1), dtype=torch.bfloat16), 1,
+                                   mode="exact")["y"][0, 0, 0])
 
 
 def test_f16_expert_mode_differs_from_exact_by_f16_rounding_of_h():
