@@ -115,6 +115,21 @@ def test_route_ties_to_lower_index_and_k1():
     assert idx1.tolist() == [[1]] and w1.tolist() == [[1.0]]
 
 
+def test_route_topk_ranks_float32_logits_ties_low():
+    # the reading: the top-k decision is taken on the logits rounded to float32 and equal
+    # float32 logits go to the lower expert index. 1 and 1 + 2**-30 differ in fp64 but
+    # round to the same float32, so expert 0 wins; the weights still use fp64 logits.
+    logits = np.array([[1.0, 1.0 + 2.0 ** -30, 0.5]])
+    idx, w, p = O.route_topk(logits, 2)
+    assert idx.tolist() == [[0, 1]]
+    assert w[0, 0] < w[0, 1] and abs(w.sum() - 1.0) < 1e-15
+    idx1, _, _ = O.route_topk(logits, 1)
+    assert idx1.tolist() == [[0]]
+    # a difference float32 keeps decides the order as usual
+    idx2, _, _ = O.route_topk(np.array([[1.0, 1.0 + 2.0 ** -20, 0.5]]), 1)
+    assert idx2.tolist() == [[1]]
+
+
 # ---------------------------------------------------------------- permutation
 
 @pytest.mark.parametrize("t_count,e_count,k", [(37, 8, 2), (300, 5, 3), (1, 8, 2), (64, 1, 1)])
