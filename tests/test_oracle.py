@@ -242,6 +242,21 @@ def test_token_subset_matches_full_layer():
         assert np.array_equal(part[key], full[key][sub])
 
 
+def test_bf16_storage_mode_rounds_h_and_out_closed_form():
+    # one expert, one unit, x = gate = up = 1: h = silu(1) is stored as its nearest bf16;
+    # y = bf16(silu(1)) * w2 stays wide, and the output is y rounded once to bf16
+    # (nearest values from torch's bf16 conversion, not the oracle's rounding)
+    import math
+    bf = lambda v: float(torch.tensor(v, dtype=torch.float64).to(torch.bfloat16))
+    one = torch.ones((1, 1), dtype=torch.bfloat16)
+    w2 = torch.full((1, 1, 1), 1 + 2.0 ** -7, dtype=torch.bfloat16)
+    r = O.moe_layer(one, one, one.view(1, 1, 1), one.view(1, 1, 1), w2, 1, mode="bf16_storage")
+    h = bf(1.0 / (1.0 + math.exp(-1.0)))
+    assert h != 1.0 / (1.0 + math.exp(-1.0))
+    assert r["y"][0, 0, 0] == h * (1 + 2.0 ** -7)
+    assert r["out"][0, 0] == bf(h * (1 + 2.0 ** -7)) != r["routed"][0, 0]
+
+
 def test_storage_mode_differs_only_by_bf16_rounding():
     x, wr, w1, w3, w2, _ = _tiny_layer(9)
     ex = O.moe_layer(x, wr, w1, w3, w2, k=2, mode="exact")
