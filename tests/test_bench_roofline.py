@@ -1,0 +1,38 @@
+"""The benchmark's roofline arithmetic against closed forms: the algorithmic bytes and
+flops it divides by the measured kernel time, the bound it picks, and the fraction."""
+import bench
+from sparse_mixture_experts_09_b200 import workloads as W
+
+PEAKS = {"hbm_gbs": 6556.2, "bf16_tflops": 1613.7, "bf16_tflops_sustained": 1342.7}
+
+
+def test_decode_gate_up_bytes_and_hbm_bound():
+    w = W.WORKLOADS["decode"]            # T=16, H=4096, I=14336, E=8, k=2
+    stage_ms = {"router": 0.01, "permute": 0.01, "gate_up": 0.3, "down": 0.15, "combine": 0.01}
+    r = bench.kernel_roofline(w, stage_ms, [4] * 8, PEAKS, "measured", False)
+    per_expert = 2 * 14336 * 4096 * 2    # w1 + w3 rows of one expert: 234.9 MB
+    assert per_expert == 234_881_024
+    routed = 16 * 2
+    assert r["algorithmic_bytes"] == 8 * per_expert + routed * 4096 * 2 + routed * 14336 * 2
+    assert r["kernel"] == "gate_up" and r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["achieved"] - r["algorithmic_bytes"] / 0.3e-3 / 1e9) < 1e-6
+    assert abs(r["frac"] - r["achieved"] / 6556.2) < 1e-12
+    # only experts that received rows are streamed
+    r2 = bench.kernel_roofline(w, stage_ms, [16, 16, 0, 0, 0, 0, 0, 0], PEAKS, "measured", False)
+    assert r2["active_experts"] == 2
+    assert r2["algorithmic_bytes"] == 2 * per_expert + routed * 4096 * 2 + routed * 14336 * 2
+
+
+def test_prefill_flops_and_tensor_bound():
+    w = W.WORKLOADS["prefill"]           # T=4096: 8192 routed rows
+    stage_ms = {"router": 0.01, "permute": 0.02, "gate_up": 1.7, "down": 0.85, "combine": 0.03}
+    r = bench.kernel_roofline(w, stage_ms, [1024] * 8, PEAKS, "measured", False)
+    assert r["kernel"] == "gate_up" and r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["algorithmic_flops"] == 4 * 8192 * 4096 * 14336
+    assert r["peak"] == 1613.7 and r["peak_source"] == "measured burst"
+    # the whole layer's expert work, 6 R H I = 2.886 TFLOP
+    down = bench.kernel_roofline(w, {"down": 1.0}, [1024] * 8, PEAKS, "measured", False)
+    assert round((r["algorithmic_flops"] + down["algorithmic_flops"]) / 1e12, 3) == 2.886
+    # a long timed region takes the sustained tensor peak
+    r_long = bench.kernel_roofline(w, stage_ms, [1024] * 8, PEAKS, "measured", True)
+    assert r_long["peak"] == 1342.7 and r_long["peak_source"] == "measured sustained"
