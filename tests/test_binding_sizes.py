@@ -123,3 +123,15 @@ def test_split_entry_points_check_sizes():
         M.combine(y, row_of, torch.zeros((T, K + 1)), None, E, I)
     with pytest.raises(ValueError, match="residual"):
         M.combine(y, row_of, torch.zeros((T, K)), _bf16(T, H + 128), E, I)
+
+
+def test_profile_driver_parses_and_needs_a_gpu():
+    import pytest as _pt
+    from sparse_mixture_experts_09_b200 import profile_run
+    with _pt.raises(SystemExit) as e:
+        profile_run.main(["--help"])
+    assert e.value.code == 0
+    if not torch.cuda.is_available():
+        # no CPU fallback: drawing the inputs on a CUDA device fails loudly
+        with _pt.raises((RuntimeError, AssertionError)):
+            profile_run.main(["--path", "int4", "tiny"])
