@@ -70,3 +70,14 @@ def test_workload_shapes_follow_config(name):
     w = workloads.WORKLOADS[name]
     assert w.hidden_size % 128 == 0 and w.intermediate_size % 128 == 0
     assert w.num_experts == 8 and w.num_experts_per_tok == 2
+
+
+def test_workload_names_resolve():
+    import pytest as _pt
+    from sparse_mixture_experts_09_b200 import workloads as W
+    assert W.workload("decode") is W.WORKLOADS["decode"]
+    for t in (1, 4, 16, 64, 256):
+        w = W.workload(f"larger_decode_T{t}")
+        assert (w.num_tokens, w.hidden_size, w.intermediate_size) == (t, 6144, 16384)
+    with _pt.raises(KeyError):
+        W.workload("larger_decode_T3")
