@@ -36,3 +36,43 @@ def test_prefill_flops_and_tensor_bound():
     # a long timed region takes the sustained tensor peak
     r_long = bench.kernel_roofline(w, stage_ms, [1024] * 8, PEAKS, "measured", True)
     assert r_long["peak"] == 1342.7 and r_long["peak_source"] == "measured sustained"
+
+
+class _Proc:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+
+def _sampler_with(rows):
+    import tempfile
+    s = bench.ClockSampler()
+    s.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+    s.file.write("\n".join(rows) + "\n")
+    s.proc = _Proc()
+    return s
+
+
+def test_clock_sampler_reads_loaded_samples_and_reasons():
+    # index, bus, util %, sm MHz, max sm MHz, W, active mask, hw_slowdown,
+    # hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap
+    row = "0, 00000000:1B:00.0, {u}, {sm}, 1965, {w}, 0x4, Not Active, Not Active, Not Active, {cap}"
+    rows = [row.format(u=0, sm=345, w=120.0, cap="Not Active"),       # idle: ignored
+            row.format(u=100, sm=1845, w=700.5, cap="Active"),
+            row.format(u=97, sm=1800, w=690.0, cap="Not Active"),
+            row.format(u=100, sm=1900, w=707.2, cap="Active")]
+    c = _sampler_with(rows).stop()
+    assert c["sm_mhz"] == 1845.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"] and c["samples_under_load"] == 3
+    assert c["power_w_max"] == 707.2
+
+
+def test_clock_sampler_reports_slowdowns_and_tolerates_no_samples():
+    row = "0, 00000000:1B:00.0, 100, 1200, 1965, 600, 0x8, {hw}, Not Active, {sw}, Not Active"
+    c = _sampler_with([row.format(hw="Active", sw="Not Active"),
+                       row.format(hw="Not Active", sw="Active")]).stop()
+    assert c["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert _sampler_with(["garbage"]).stop() is None
+    assert bench.ClockSampler().stop() is None          # nvidia-smi never started
