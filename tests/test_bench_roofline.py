@@ -76,3 +76,12 @@ def test_clock_sampler_reports_slowdowns_and_tolerates_no_samples():
     assert c["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
     assert _sampler_with(["garbage"]).stop() is None
     assert bench.ClockSampler().stop() is None          # nvidia-smi never started
+
+
+def test_kernels_per_forward_matches_the_launch_lists():
+    # the ncu launch lists: 6 kernels per forward at decode (router, plan, gather, two
+    # GEMMs, combine); 8 above 1024 tokens (histogram, scan and rank replace the plan)
+    assert bench.kernels_per_forward(16) == 6
+    assert bench.kernels_per_forward(1024) == 6
+    assert bench.kernels_per_forward(1025) == 8
+    assert bench.kernels_per_forward(4096) == 8
