@@ -27,6 +27,8 @@ exercised with other implementations of the steps.
 """
 from __future__ import annotations
 
+import dataclasses
+
 import torch
 import torch.distributed as dist
 
@@ -59,6 +61,17 @@ class CudaOps:
         shape = self.moe.make_shape(rows, h, i, e, 1)
         ws = self.moe.make_workspace(shape, x_groups.device)
         return self.moe.grouped_swiglu(x_groups, offsets, w1, w3, w2, rows, 1, ws)
+
+    def grouped_swiglu_quantized(self, x_groups, offsets, experts, rows):
+        """The same with int8 (Int8Experts) or 4-bit (Int4Experts) expert weights."""
+        e, i, _ = experts.q1.shape
+        h = x_groups.shape[1]
+        rows = max(rows, 1)
+        shape = self.moe.make_shape(rows, h, i, e, 1)
+        ws = self.moe.make_workspace(shape, x_groups.device)
+        fn = (self.moe.grouped_swiglu_w4 if isinstance(experts, self.moe.Int4Experts)
+              else self.moe.grouped_swiglu_w8)
+        return fn(x_groups, offsets, experts, rows, 1, ws)
 
     def combine(self, y_perm, row_of, topk_w, residual, num_experts, intermediate_size):
         return self.moe.combine(y_perm, row_of, topk_w, residual, num_experts, intermediate_size)
@@ -138,13 +151,34 @@ def forward_ep(x, w_router, w1_local, w3_local, w2_local, k: int, num_experts: i
     between ranks, and may be 0. E must be a multiple of the group size.
     """
     ops = ops or CudaOps()
+    return _forward_ep(
+        x, w_router, k, num_experts, w1_local.shape[0], w1_local.shape[1],
+        lambda xl, off, n: ops.grouped_swiglu(xl, off, w1_local, w3_local, w2_local, n),
+        group, residual, logit_bias, ops)
+
+
+def forward_ep_quantized(x, w_router, experts_local, k: int, num_experts: int, group=None,
+                         residual=None, logit_bias=None, ops=None):
+    """forward_ep with this rank's experts as weight-only int8 or 4-bit codes
+    (moe.Int8Experts / moe.Int4Experts holding E/W experts, e.g. from shard_quantized).
+    Routing and the exchanges are the bf16 layer's; the experts compute as the
+    library's quantised grouped entry points do (half precision)."""
+    ops = ops or CudaOps()
+    e_loc, inter = experts_local.q1.shape[0], experts_local.q1.shape[1]
+    return _forward_ep(
+        x, w_router, k, num_experts, e_loc, inter,
+        lambda xl, off, n: ops.grouped_swiglu_quantized(xl, off, experts_local, n),
+        group, residual, logit_bias, ops)
+
+
+def _forward_ep(x, w_router, k, num_experts, held, inter, run_experts, group, residual,
+                logit_bias, ops):
     world = dist.get_world_size(group)
     if num_experts % world:
         raise ValueError(f"num_experts {num_experts} is not a multiple of the group size {world}")
     e_loc = num_experts // world
-    if w1_local.shape[0] != e_loc:
-        raise ValueError(f"this rank must hold {e_loc} experts, got {w1_local.shape[0]}")
-    inter = w1_local.shape[1]
+    if held != e_loc:
+        raise ValueError(f"this rank must hold {e_loc} experts, got {held}")
     hidden = x.shape[1]
     dev = x.device
 
@@ -180,7 +214,7 @@ def forward_ep(x, w_router, w1_local, w3_local, w2_local, k: int, num_experts: i
     rows_buf = ops.padded_rows(n_local, e_loc)
     x_local = ops.gather_rows(x_recv, rows_index(plan["to_local"] + [-1] * (rows_buf - n_local)))
     loc_off = torch.tensor(plan["local_offsets"], dtype=torch.int32, device=dev)
-    y_local = ops.grouped_swiglu(x_local, loc_off, w1_local, w3_local, w2_local, n_local)
+    y_local = run_experts(x_local, loc_off, n_local)
     y_recv = ops.gather_rows(y_local, rows_index(plan["to_recv"]))
 
     # 5. outputs back to their tokens' ranks, into the permuted order, then the combine
@@ -190,6 +224,18 @@ def forward_ep(x, w_router, w1_local, w3_local, w2_local, k: int, num_experts: i
         return torch.empty((0, hidden), dtype=x.dtype, device=dev)
     y_perm = ops.gather_rows(y_back, rows_index(plan["back_index"]))
     return ops.combine(y_perm, perm["row_of"], wt, residual, num_experts, inter)
+
+
+def shard_quantized(experts, rank: int, world: int):
+    """This rank's slice of quantised experts (Int8Experts or Int4Experts). Codes and
+    scales are stored expert after expert (an expert's rows fill whole 128-row tiles),
+    so a slice along the expert axis is itself a valid layout for E/W experts."""
+    e = experts.q1.shape[0]
+    if e % world:
+        raise ValueError(f"{e} experts do not split over {world} ranks")
+    lo, hi = rank * e // world, (rank + 1) * e // world
+    return dataclasses.replace(experts, **{f.name: getattr(experts, f.name)[lo:hi].contiguous()
+                                           for f in dataclasses.fields(experts)})
 
 
 def shard_experts(w1, w3, w2, rank: int, world: int):

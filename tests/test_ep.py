@@ -57,6 +57,21 @@ class OracleOps:
                 y[a:b] = torch.from_numpy(self.O.swiglu_expert(rows_e, w1[e], w3[e], w2[e]))
         return y
 
+    def grouped_swiglu_quantized(self, x_groups, offsets, experts, rows):
+        """Half-precision experts on dequantised weights (experts.deq = fp64 w1, w3, w2
+        of this rank's experts), as the oracle's f16_experts mode computes them."""
+        O = self.O
+        d1, d3, d2 = experts.deq
+        y = torch.zeros((x_groups.shape[0], d2.shape[1]), dtype=torch.float64)
+        off = offsets.tolist()
+        for e in range(d1.shape[0]):
+            a, b = off[e], off[e + 1]
+            if b > a:
+                x16 = O.round_f16(O.to_f64(x_groups[a:b]))
+                h = O.silu(x16 @ d1[e].T) * (x16 @ d3[e].T)
+                y[a:b] = torch.from_numpy(O.round_f16(h) @ d2[e].T)
+        return y
+
     def combine(self, y_perm, row_of, topk_w, residual, num_experts, intermediate_size):
         out = torch.zeros((row_of.shape[0], y_perm.shape[1]), dtype=torch.float64)
         for j in range(row_of.shape[1]):
@@ -80,7 +95,12 @@ def _layer_inputs(t_total, hd, inter, e, seed):
     return x, wr, w1, w3, w2, res
 
 
-def _rank(rank, world, port, q, tokens, e, k, bias):
+def _dequantised_4bit(w1, w3, w2):
+    from oracle import moe_oracle as O
+    return [O.dequantize_int4_groups(*O.quantize_int4_groups(w)) for w in (w1, w3, w2)]
+
+
+def _rank(rank, world, port, q, tokens, e, k, bias, quant=False):
     import datetime
     import sys
     import torch.distributed as dist
@@ -91,23 +111,34 @@ def _rank(rank, world, port, q, tokens, e, k, bias):
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
-    x, wr, w1, w3, w2, res = _layer_inputs(sum(tokens), 32, 48, e, seed=7)
+    hd, inter = (128, 128) if quant else (32, 48)
+    x, wr, w1, w3, w2, res = _layer_inputs(sum(tokens), hd, inter, e, seed=7)
     lo = sum(tokens[:rank])
     mine = slice(lo, lo + tokens[rank])
-    l1, l3, l2 = EP.shard_experts(w1, w3, w2, rank, world)
     b = None if bias is None else torch.tensor(bias, dtype=torch.float64)
-    out = EP.forward_ep(x[mine], wr, l1, l3, l2, k, e, residual=res[mine], logit_bias=b,
-                        ops=OracleOps())
+    if quant:
+        from types import SimpleNamespace
+        from tests.test_ep import _dequantised_4bit
+        d = _dequantised_4bit(w1, w3, w2)
+        el = e // world
+        part = [t[rank * el:(rank + 1) * el] for t in d]
+        local = SimpleNamespace(q1=torch.from_numpy(part[0]), deq=part)
+        out = EP.forward_ep_quantized(x[mine], wr, local, k, e, residual=res[mine], logit_bias=b,
+                                      ops=OracleOps())
+    else:
+        l1, l3, l2 = EP.shard_experts(w1, w3, w2, rank, world)
+        out = EP.forward_ep(x[mine], wr, l1, l3, l2, k, e, residual=res[mine], logit_bias=b,
+                            ops=OracleOps())
     q.put((rank, out.double().numpy()))
     dist.barrier()
     dist.destroy_process_group()
 
 
-def _run(world, tokens, e, k, bias=None):
+def _run(world, tokens, e, k, bias=None, quant=False):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, world, port, q, tokens, e, k, bias))
+    procs = [ctx.Process(target=_rank, args=(r, world, port, q, tokens, e, k, bias, quant))
              for r in range(world)]
     for p in procs:
         p.start()
@@ -231,3 +262,47 @@ def test_exchange_plan_random_worlds_round_trip():
             assert returned[r] == x_perm[r]
             for s in range(world):
                 assert plans[r]["send_rows"][s] == plans[s]["recv_rows"][r]
+
+
+def test_expert_parallel_4bit_layer_equals_single_process_layer():
+    # experts as 4-bit codes: each rank computes its experts in half precision on the
+    # dequantised weights; the result is the oracle's half-precision layer (before its
+    # output rounding) plus the residual
+    from oracle import moe_oracle as O
+    tokens, e, k = [6, 11], 4, 2
+    got = _run(2, tokens, e, k, quant=True)
+    x, wr, w1, w3, w2, res = _layer_inputs(sum(tokens), 128, 128, e, seed=7)
+    d1, d3, d2 = _dequantised_4bit(w1, w3, w2)
+    ref = O.moe_layer(x, wr, d1, d3, d2, k, mode="f16_experts")
+    np.testing.assert_allclose(got, O.to_f64(res) + ref["routed"], rtol=1e-12, atol=1e-12)
+
+
+def test_shard_quantized_slices_are_valid_layouts():
+    # 4-bit codes packed by the header's layout statement, sliced per rank, decode to
+    # exactly the codes and scales of that rank's experts
+    from oracle import moe_oracle as O
+    from sparse_mixture_experts_09_b200 import moe as M
+    from .test_gpu_w4 import unblock4
+    from .test_w4_layout import _pack_from_header, _scales_from_header
+    rng = np.random.default_rng(42)
+    e, i, h = 4, 256, 128
+    mats = {"1": (i, h), "3": (i, h), "2": (h, i)}
+    codes, fields = {}, {}
+    for name, (r, kk) in mats.items():
+        w = O.round_bf16(rng.standard_normal((e * r, kk)) * 0.05)
+        q, s16 = O.quantize_int4_groups(w)
+        codes[name] = (q, s16)
+        fields["q" + name] = torch.from_numpy(_pack_from_header(q, kk).copy()).reshape(e, r, kk // 2)
+        fields["s" + name] = torch.from_numpy(_scales_from_header(s16, e * r, kk)).reshape(
+            e, r // 128, kk // 64, 128)
+    ex = M.Int4Experts(**fields)
+    for rank in range(2):
+        part = ep.shard_quantized(ex, rank, 2)
+        lo, hi = rank * 2, rank * 2 + 2
+        for name, (r, kk) in mats.items():
+            got_q, got_s = unblock4(getattr(part, "q" + name), getattr(part, "s" + name))
+            q, s16 = codes[name]
+            assert np.array_equal(got_q.reshape(-1, kk), q[lo * r:hi * r])
+            assert np.array_equal(got_s.reshape(-1, kk // 64), s16[lo * r:hi * r])
+    with pytest.raises(ValueError):
+        ep.shard_quantized(ex, 0, 3)
