@@ -231,12 +231,12 @@ moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_bf16_t* x_host
 /* moe_forward_host without the final wait: enqueues the copies in, the layer and the
  * copy out and returns. The copies in run on a copy stream of the library's own, into
  * one of two staging slots of `ws`, so they overlap the previous call's layer; the
- * layer and the copy out run on `stream`, which waits for them. out_host holds the result, and x_host and
- * residual_host may be reused, once the stream has reached this point (for example
- * after cudaStreamSynchronize). Calls on one stream with one ws are ordered by the
- * stream, so a serving loop can enqueue step after step and wait once; calls that may
- * overlap on different streams need separate workspaces. Host buffers must be pinned
- * for the copies to be asynchronous. */
+ * layer and the copy out run on `stream`, which waits for them. out_host holds the
+ * result, and x_host and residual_host may be reused, once the stream has reached this
+ * point (for example after cudaStreamSynchronize). Calls on one stream with one ws are
+ * ordered by the stream, so a serving loop can enqueue step after step and wait once;
+ * calls that may overlap on different streams need separate workspaces. Host buffers
+ * must be pinned for the copies to be asynchronous. */
 moe_status_t moe_forward_host_async(const moe_shape_t* shape, const moe_bf16_t* x_host,
                                     const moe_bf16_t* w_router, const float* logit_bias,
                                     const moe_bf16_t* w1, const moe_bf16_t* w3,
