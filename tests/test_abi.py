@@ -90,3 +90,18 @@ def test_binding_refuses_cpu_tensors(L):
     x = torch.zeros(4, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         M.router_topk(x, torch.zeros(8, 128, dtype=torch.bfloat16), 2)
+
+
+@pytest.mark.parametrize("t,h,i,e,k", [(1, 128, 128, 1, 1), (16, 4096, 14336, 8, 2),
+                                       (777, 256, 256, 5, 3), (4096, 640, 512, 64, 8),
+                                       (100000, 4096, 14336, 8, 2)])
+def test_workspace_holds_every_region(L, t, h, i, e, k):
+    s = M.make_shape(t, h, i, e, k)
+    rmax = M.max_padded_rows(s)
+    assert rmax == (t * k + 127) // 128 * 128 + 128 * e
+    ws = M.workspace_size(s)
+    # routed-row buffers (x_perm and h as 2-byte values, y fp32) and the per-slot tables
+    assert ws >= rmax * (h * 2 + i * 2 + h * 4) + rmax * 4 + 3 * t * k * 4 + 256
+    # host entry points: two staging slots for x and the residual, one for the output
+    assert M.workspace_size_host(s) - ws >= 5 * t * h * 2
+    assert ws % 256 == 0 and M.workspace_size_host(s) % 256 == 0
