@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="leave out the prefill sub-record of the default line")
     return ap.parse_args()
 
 
@@ -67,11 +69,16 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def workload_config(w):
+def workload_config(w, world=1):
+    """The ``config`` object of the JSON line; both arms print the same one."""
+    routed_gb = w.num_experts_per_tok * w.expert_bytes() / 1e9
     return {"workload": w.name, "num_tokens": w.num_tokens, "hidden_size": w.hidden_size,
             "intermediate_size": w.intermediate_size, "num_experts": w.num_experts,
             "num_experts_per_tok": w.num_experts_per_tok,
-            "logit_bias": list(w.logit_bias) if w.logit_bias else None}
+            "logit_bias": list(w.logit_bias) if w.logit_bias else None,
+            "parallelism": f"replicas x{world}",
+            "l2": ("no flush: every step reads the weights of each routed expert, at least "
+                   "%.2f GB, more than the 126 MB L2" % routed_gb)}
 
 
 # ------------------------------------------------------------------ clocks
@@ -144,19 +151,25 @@ def blas_threads():
         return None
 
 
-def oracle_timing(inp_cpu, w, budget_s, max_runs=None, tokens=None):
-    """Run the oracle (as it stands) on the workload until ``budget_s`` of CPU time
-    has passed; returns (seconds per run, runs, tokens per run)."""
+def oracle_timing(inp_cpu, w, budget_s=0.0, max_runs=None, tokens=None, layer=None):
+    """Run the oracle (as it stands) on the workload: exactly ``max_runs`` times when it
+    is given, else until ``budget_s`` seconds have passed (at least once). Returns
+    (seconds per run, runs, tokens per run, torch threads)."""
     import torch
-    from oracle import moe_oracle as O
+    if layer is None:
+        from oracle import moe_oracle as O
+        layer = O.moe_layer
     runs, t0 = 0, time.perf_counter()
     while True:
-        O.moe_layer(inp_cpu.x, inp_cpu.w_router, inp_cpu.w1, inp_cpu.w3, inp_cpu.w2,
-                    w.num_experts_per_tok, residual=inp_cpu.residual, logit_bias=inp_cpu.logit_bias,
-                    mode="exact", tokens=tokens)
+        layer(inp_cpu.x, inp_cpu.w_router, inp_cpu.w1, inp_cpu.w3, inp_cpu.w2,
+              w.num_experts_per_tok, residual=inp_cpu.residual, logit_bias=inp_cpu.logit_bias,
+              mode="exact", tokens=tokens)
         runs += 1
         el = time.perf_counter() - t0
-        if el >= budget_s or (max_runs and runs >= max_runs):
+        if max_runs is not None:
+            if runs >= max_runs:
+                break
+        elif el >= budget_s:
             break
     n_tok = w.num_tokens if tokens is None else len(tokens)
     return el / runs, runs, n_tok, torch.get_num_threads()
@@ -184,23 +197,22 @@ def run_reference(args):
     inp = W.LayerInputs(*(None if t is None else t.cpu() for t in
                           (inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, inp.residual, inp.logit_bias)))
     tokens = cpu_sample_tokens(w)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     # probe one step, then size the run to a few minutes
-    per_step, _, n_tok, threads = oracle_timing(inp, w, 0.0, max_runs=1, tokens=tokens)
+    per_step, _, n_tok, threads = oracle_timing(inp, w, max_runs=1, tokens=tokens)
     budget = 150.0
     steps = max(1, min(args.steps, int((budget - per_step) / per_step) - args.warmup))
     warm = min(args.warmup, max(0, int(budget / per_step) - steps - 1))
     if warm:
-        oracle_timing(inp, w, 0.0, max_runs=warm, tokens=tokens)
-    t0 = time.perf_counter()
-    oracle_timing(inp, w, 0.0, max_runs=steps, tokens=tokens)
-    el = time.perf_counter() - t0
-    value = n_tok * steps / el
+        oracle_timing(inp, w, max_runs=warm, tokens=tokens)
+    per_step, steps, n_tok, threads = oracle_timing(inp, w, max_runs=steps, tokens=tokens)
+    value = n_tok / per_step
     sample = (f"{'all ' if tokens is None else ''}{n_tok} tokens of the {w.name} batch per step, "
               f"fp64 exact mode, {steps} timed steps after {warm} warm-up")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 0,
-            "steps": steps, "warmup": warm, "ms_per_step": 1e3 * el / steps, "higher_is_better": True,
+            "steps": steps, "warmup": warm, "ms_per_step": 1e3 * per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(w),
+            "config": workload_config(w, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads() or threads,
                              "kind": "oracle", "sample": sample, "host_cpus": os.cpu_count()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -278,6 +290,154 @@ def job_throughput(tokens_per_rank, world, ms):
     return tokens_per_rank * world / (ms * 1e-3)
 
 
+NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}   # B200 spec: HBM3e, dense bf16
+
+
+def layer_roofline(w, ms, counts, peaks, peak_kind, long_run):
+    """Whole-layer fraction of roofline: the layer's algorithmic bytes (decode) or expert
+    flops (prefill) over the step time, against the nominal B200 peaks (8 TB/s, 2.25
+    PFLOP/s dense bf16) and the measured ones."""
+    H, I, k, T, E = (w.hidden_size, w.intermediate_size, w.num_experts_per_tok, w.num_tokens,
+                     w.num_experts)
+    n_active = int(sum(1 for c in counts if c > 0))
+    bytes_ = n_active * w.expert_bytes() + 3 * T * H * 2 + E * H * 2 + T * k * 8
+    flops = w.routed_flops() + w.router_flops()
+    sec = ms * 1e-3
+    if flops / (NOMINAL["bf16_tflops"] * 1e12) > bytes_ / (NOMINAL["hbm_gbs"] * 1e9):
+        achieved = flops / sec / 1e12
+        meas = peaks["bf16_tflops_sustained" if long_run else "bf16_tflops"]
+        return {"bound": "tensor", "achieved": achieved, "unit": "TFLOP/s",
+                "nominal_peak": NOMINAL["bf16_tflops"], "frac_of_nominal": achieved / NOMINAL["bf16_tflops"],
+                "measured_peak": meas, "frac_of_measured": achieved / meas,
+                "measured_peak_source": peak_kind + (" sustained" if long_run else " burst"),
+                "algorithmic_flops": flops}
+    achieved = bytes_ / sec / 1e9
+    return {"bound": "hbm", "achieved": achieved, "unit": "GB/s",
+            "nominal_peak": NOMINAL["hbm_gbs"], "frac_of_nominal": achieved / NOMINAL["hbm_gbs"],
+            "measured_peak": peaks["hbm_gbs"], "frac_of_measured": achieved / peaks["hbm_gbs"],
+            "measured_peak_source": peak_kind, "algorithmic_bytes": bytes_}
+
+
+def near_tie_tokens(logits, k, margin=1e-2):
+    """Tokens whose float32 router logits have a gap below ``margin`` between any two
+    neighbours among their k + 1 largest (the ranks that decide the top-k and its slot
+    order). Reported only; the benchmark draws x without the parity tests' screen."""
+    import torch
+    top = torch.topk(logits, min(k + 1, logits.shape[1]), dim=1).values
+    gaps = top[:, :-1] - top[:, 1:]
+    return int((gaps < margin).any(dim=1).sum().item())
+
+
+def _time_loop(fn, K, stream, barrier, dev):
+    import torch
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    return e0.elapsed_time(e1) / K
+
+
+class Bf16Layer:
+    """The default (bf16, blocked weights) layer of one workload, ready to time: whole
+    forwards, and the split entry points with events between the stages."""
+
+    def __init__(self, w, dev, keep_row_major=False):
+        import torch
+        from sparse_mixture_experts_09_b200 import moe
+        from sparse_mixture_experts_09_b200 import workloads as W
+        self.w, self.dev, self.moe = w, dev, moe
+        inp = W.draw(w, dev)
+        self.inp = inp
+        # the expert weights live in the library's blocked layout, converted once at load
+        # time (not timed)
+        self.bw = moe.pack_weights(inp.w1, inp.w3, inp.w2)
+        if not keep_row_major:
+            inp.w1 = inp.w3 = inp.w2 = None
+            torch.cuda.empty_cache()
+        self.k = k = w.num_experts_per_tok
+        self.shape = moe.make_shape(*w.shape, moe.BLOCKED)
+        self.ws = moe.make_workspace(self.shape, dev)
+        self.out = torch.empty((w.num_tokens, w.hidden_size), dtype=torch.bfloat16, device=dev)
+        self.stream = torch.cuda.current_stream(dev)
+        rmax = moe.max_padded_rows(self.shape)
+        T, E = w.num_tokens, w.num_experts
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+        self.wt = torch.empty((T, k), dtype=torch.float32, device=dev)
+        self.logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+        self.perm = {"counts": torch.empty(E, dtype=torch.int32, device=dev),
+                     "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+                     "row_of": torch.empty((T, k), dtype=torch.int32, device=dev),
+                     "token_of_row": torch.empty(rmax, dtype=torch.int32, device=dev),
+                     "x_perm": torch.empty((rmax, w.hidden_size), dtype=torch.bfloat16, device=dev)}
+        self.hbuf = torch.empty((rmax, w.intermediate_size), dtype=torch.bfloat16, device=dev)
+        self.ybuf = torch.empty((rmax, w.hidden_size), dtype=torch.float32, device=dev)
+
+    def step(self):
+        i, (b1, b3, b2) = self.inp, self.bw
+        self.moe.forward(i.x, i.w_router, b1, b3, b2, self.k, residual=i.residual,
+                         logit_bias=i.logit_bias, ws=self.ws, out=self.out,
+                         weight_layout=self.moe.BLOCKED)
+
+    def split_step(self, ev, logits=False):
+        import ctypes
+        moe, L, i = self.moe, self.moe.lib(), self.inp
+        sp, st = ctypes.byref(self.shape), self.stream.cuda_stream
+        p = lambda t: t.data_ptr()  # noqa: E731
+        bias = None if i.logit_bias is None else p(i.logit_bias)
+        perm, ws = self.perm, self.ws
+        ev[0].record(self.stream)
+        moe._check(L.moe_router_topk(sp, p(i.x), p(i.w_router), bias, p(self.idx), p(self.wt),
+                                     p(self.logits) if logits else None, st))
+        ev[1].record(self.stream)
+        moe._check(L.moe_permute(sp, p(self.idx), p(i.x), p(perm["counts"]), p(perm["offsets"]),
+                                 p(perm["row_of"]), p(perm["token_of_row"]), p(perm["x_perm"]),
+                                 p(ws), ws.numel(), st))
+        ev[2].record(self.stream)
+        moe._check(L.moe_expert_gate_up(sp, p(perm["x_perm"]), p(perm["offsets"]), p(self.bw[0]),
+                                        p(self.bw[1]), p(self.hbuf), p(ws), ws.numel(), st))
+        ev[3].record(self.stream)
+        moe._check(L.moe_expert_down(sp, p(self.hbuf), p(perm["offsets"]), p(self.bw[2]),
+                                     p(self.ybuf), p(ws), ws.numel(), st))
+        ev[4].record(self.stream)
+        moe._check(L.moe_combine(sp, p(self.ybuf), p(perm["row_of"]), p(self.wt), p(i.residual),
+                                 p(self.out), st))
+        ev[5].record(self.stream)
+
+    def warm(self, n):
+        import torch
+        scratch = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        for _ in range(n):
+            self.step()
+        self.split_step(scratch, logits=True)
+        torch.cuda.synchronize(self.dev)
+        self.moe.device_status(self.ws)
+
+    def time_forward(self, K, barrier):
+        return _time_loop(self.step, K, self.stream, barrier, self.dev)
+
+    def time_stages(self, K):
+        import torch
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+        torch.cuda.synchronize(self.dev)
+        for i in range(K):
+            self.split_step(evs[i])
+        torch.cuda.synchronize(self.dev)
+        self.moe.device_status(self.ws)
+        names = ["router", "permute", "gate_up", "down", "combine"]
+        return {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
+                for j, n in enumerate(names)}
+
+    def routing_report(self):
+        """Expert counts and near-tie tokens of the last split step (untimed)."""
+        return (self.perm["counts"].cpu().tolist(),
+                near_tie_tokens(self.logits, self.k))
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -301,20 +461,11 @@ def run_ours(args):
 
     moe.lib()  # fail loudly if the library is missing
     w = W.workload(args.workload)
-    inp = W.draw(w, dev)
-    k = w.num_experts_per_tok
-    # the expert weights live in the library's blocked layout, converted once at load
-    # time (not timed); a row-major loop is timed alongside for comparison
-    bw1, bw3, bw2 = moe.pack_weights(inp.w1, inp.w3, inp.w2)
-    layout = moe.BLOCKED
-    shape = moe.make_shape(*w.shape, layout)
-    ws = moe.make_workspace(shape, dev)
-    out = torch.empty((w.num_tokens, w.hidden_size), dtype=torch.bfloat16, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    def step():
-        moe.forward(inp.x, inp.w_router, bw1, bw3, bw2, k, residual=inp.residual,
-                    logit_bias=inp.logit_bias, ws=ws, out=out, weight_layout=layout)
+    layer = Bf16Layer(w, dev, keep_row_major=True)
+    inp, k = layer.inp, layer.k
+    ws, out, stream = layer.ws, layer.out, layer.stream
+    bw1, bw3, bw2 = layer.bw
+    step = layer.step
 
     # weight-only int8 experts, quantised once at load time (not timed)
     w8 = moe.quantize_int8(inp.w1, inp.w3, inp.w2)
@@ -336,60 +487,31 @@ def run_ours(args):
         moe.forward(inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, k, residual=inp.residual,
                     logit_bias=inp.logit_bias, ws=ws, out=out)
 
-    # split-path buffers for the per-kernel breakdown
-    rmax = moe.max_padded_rows(shape)
-    idx = torch.empty((w.num_tokens, k), dtype=torch.int32, device=dev)
-    wt = torch.empty((w.num_tokens, k), dtype=torch.float32, device=dev)
-    perm = {"counts": torch.empty(w.num_experts, dtype=torch.int32, device=dev),
-            "offsets": torch.empty(w.num_experts + 1, dtype=torch.int32, device=dev),
-            "row_of": torch.empty((w.num_tokens, k), dtype=torch.int32, device=dev),
-            "token_of_row": torch.empty(rmax, dtype=torch.int32, device=dev),
-            "x_perm": torch.empty((rmax, w.hidden_size), dtype=torch.bfloat16, device=dev)}
-    hbuf = torch.empty((rmax, w.intermediate_size), dtype=torch.bfloat16, device=dev)
-    ybuf = torch.empty((rmax, w.hidden_size), dtype=torch.float32, device=dev)
-    L = moe.lib()
-    import ctypes
-    sp = ctypes.byref(shape)
-    st = stream.cuda_stream
-    p = lambda t: t.data_ptr()  # noqa: E731
-    bias = None if inp.logit_bias is None else p(inp.logit_bias)
-
-    def split_step(ev):
-        ev[0].record(stream)
-        moe._check(L.moe_router_topk(sp, p(inp.x), p(inp.w_router), bias, p(idx), p(wt), None, st))
-        ev[1].record(stream)
-        moe._check(L.moe_permute(sp, p(idx), p(inp.x), p(perm["counts"]), p(perm["offsets"]),
-                                 p(perm["row_of"]), p(perm["token_of_row"]), p(perm["x_perm"]),
-                                 p(ws), ws.numel(), st))
-        ev[2].record(stream)
-        moe._check(L.moe_expert_gate_up(sp, p(perm["x_perm"]), p(perm["offsets"]), p(bw1),
-                                        p(bw3), p(hbuf), p(ws), ws.numel(), st))
-        ev[3].record(stream)
-        moe._check(L.moe_expert_down(sp, p(hbuf), p(perm["offsets"]), p(bw2), p(ybuf), p(ws),
-                                     ws.numel(), st))
-        ev[4].record(stream)
-        moe._check(L.moe_combine(sp, p(ybuf), p(perm["row_of"]), p(wt), p(inp.residual), p(out), st))
-        ev[5].record(stream)
-
     xh = inp.x.cpu().pin_memory()
     rh = inp.residual.cpu().pin_memory()
     oh = torch.empty_like(xh).pin_memory()
-    wsh = moe.make_workspace(shape, dev, host=True)
+    wsh = moe.make_workspace(layer.shape, dev, host=True)
 
     def host_step(wait=True):
         moe.forward_host(xh, inp.w_router, bw1, bw3, bw2, k, residual_host=rh,
-                         logit_bias=inp.logit_bias, ws=wsh, out_host=oh, weight_layout=layout,
+                         logit_bias=inp.logit_bias, ws=wsh, out_host=oh, weight_layout=moe.BLOCKED,
                          wait=wait)
+
+    # the prefill layer rides along with the default (decode) line: the tensor-bound
+    # half of the metric
+    pre = None
+    if args.workload != "prefill" and not args.no_prefill:
+        pre = Bf16Layer(W.workload("prefill"), dev)
 
     K, Wm = args.steps, max(3, args.warmup)
     for _ in range(Wm):
-        step()
         step_row_major()
         step_w8()
         step_w4()
-    scratch = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    layer.warm(Wm)
+    if pre is not None:
+        pre.warm(Wm)
     for _ in range(3):
-        split_step(scratch)
         host_step()
     torch.cuda.synchronize(dev)
     # the same forward captured once in a CUDA graph (replayed in loop 5)
@@ -401,6 +523,7 @@ def run_ours(args):
         graph.replay()
     torch.cuda.synchronize(dev)
     moe.device_status(ws)
+    counts, near_ties = layer.routing_report()
     barrier()
 
     bus = None
@@ -414,104 +537,46 @@ def run_ours(args):
     time.sleep(0.3)
 
     # (1) value: K back-to-back moe_forward calls, inputs resident in HBM
-    barrier()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(K):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    ms = e0.elapsed_time(e1) / K
-
+    ms = layer.time_forward(K, barrier)
     # (2) per-kernel breakdown through the split entry points
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
-    torch.cuda.synchronize(dev)
-    for i in range(K):
-        split_step(evs[i])
-    torch.cuda.synchronize(dev)
-    names = ["router", "permute", "gate_up", "down", "combine"]
-    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
-                for j, n in enumerate(names)}
-
+    stage_ms = layer.time_stages(K)
     # (2b) the same layer with row-major expert weights
-    barrier()
-    torch.cuda.synchronize(dev)
-    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    r0.record(stream)
-    for _ in range(K):
-        step_row_major()
-    r1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    rm_ms = r0.elapsed_time(r1) / K
-
-    # (3) end to end from pinned host memory
-    barrier()
-    torch.cuda.synchronize(dev)
-    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    h0.record(stream)
-    for _ in range(K):
-        host_step()
-    h1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    e2e_sync_ms = h0.elapsed_time(h1) / K
-
+    rm_ms = _time_loop(step_row_major, K, stream, barrier, dev)
+    # (3) end to end from pinned host memory, waiting after every call
+    e2e_sync_ms = _time_loop(host_step, K, stream, barrier, dev)
     # (3b) the same host path as a serving loop runs it: every step enqueued back to back
     #      (moe_forward_host_async: copy in, layer, copy out), one wait at the end
-    barrier()
-    torch.cuda.synchronize(dev)
-    h2, h3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    h2.record(stream)
-    for _ in range(K):
-        host_step(wait=False)
-    h3.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    e2e_ms = h2.elapsed_time(h3) / K
-
-    # (4) the same layer with weight-only int8 experts
-    barrier()
-    torch.cuda.synchronize(dev)
-    q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    q0.record(stream)
-    for _ in range(K):
-        step_w8()
-    q1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    w8_ms = q0.elapsed_time(q1) / K
-
-    # (4b) the same layer with weight-only 4-bit experts
-    barrier()
-    torch.cuda.synchronize(dev)
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(K):
-        step_w4()
-    f1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    w4_ms = f0.elapsed_time(f1) / K
-
+    e2e_ms = _time_loop(lambda: host_step(wait=False), K, stream, barrier, dev)
+    # (4) the same layer with weight-only int8 experts, (4b) 4-bit experts
+    w8_ms = _time_loop(step_w8, K, stream, barrier, dev)
+    w4_ms = _time_loop(step_w4, K, stream, barrier, dev)
     # (5) the default forward replayed from a CUDA graph
-    barrier()
-    torch.cuda.synchronize(dev)
-    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    g0.record(stream)
-    for _ in range(K):
-        graph.replay()
-    g1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    graph_ms = g0.elapsed_time(g1) / K
+    graph_ms = _time_loop(graph.replay, K, stream, barrier, dev)
     clk = clocks.stop()
-    moe.device_status(ws)
-    moe.device_status(wsh)
-    moe.device_status(ws8)
-    moe.device_status(ws4)
+    for b in (ws, wsh, ws8, ws4):
+        moe.device_status(b)
+
+    # (6) the prefill layer: whole forwards, then the stage breakdown
+    pre_rec = None
+    if pre is not None:
+        pclk = ClockSampler(bus)
+        pclk.start()
+        time.sleep(0.3)
+        pms = pre.time_forward(K, barrier)
+        pstage = pre.time_stages(K)
+        pclocks = pclk.stop()
+        pms, _ = slowest_rank(pms, pms, world, dev)
+        pcounts, pnear = pre.routing_report()
+        peaks, peak_kind = load_peaks()
+        plong = pms * K > 1000.0
+        pre_rec = {"workload": pre.w.name, "config": workload_config(pre.w, world),
+                   "value": job_throughput(pre.w.num_tokens, world, pms), "unit": "tokens/s",
+                   "ms_per_step": pms, "steps": K,
+                   "layer_roofline": layer_roofline(pre.w, pms, pcounts, peaks, peak_kind, plong),
+                   "roofline": kernel_roofline(pre.w, pstage, pcounts, peaks, peak_kind, plong),
+                   "kernels_ms": pstage, "expert_counts": pcounts, "near_ties": pnear,
+                   "clocks": pclocks,
+                   "gpu_launches": kernels_per_forward(pre.w.num_tokens) * K}
 
     ms, e2e_ms = slowest_rank(ms, e2e_ms, world, dev)
     e2e_sync_ms, _ = slowest_rank(e2e_sync_ms, e2e_sync_ms, world, dev)
@@ -520,7 +585,6 @@ def run_ours(args):
     w4_ms, _ = slowest_rank(w4_ms, w4_ms, world, dev)
     graph_ms, _ = slowest_rank(graph_ms, graph_ms, world, dev)
 
-    counts = perm["counts"].cpu().tolist()
     peaks, peak_kind = load_peaks()
     long_run = ms * K > 1000.0
     roof = kernel_roofline(w, stage_ms, counts, peaks, peak_kind, long_run)
@@ -528,16 +592,16 @@ def run_ours(args):
     line = None
     if rank == 0:
         bytes_io = w.num_tokens * w.hidden_size * 2
+        n_active = roof["active_experts"]
         line = {
             "metric": METRIC, "value": job_throughput(w.num_tokens, world, ms), "unit": "tokens/s",
             "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic: seeded SplitMix64/Box-Muller draws, weights ~N(0,1/fan_in), x rows RMS 1",
-            "config": dict(workload_config(w), parallelism=f"replicas x{world}",
-                           weight_layout="blocked (moe_pack_weights once at load, untimed)",
-                           l2=("no flush: each step streams %.2f GB of expert weights, more than "
-                               "the 126 MB L2" % (roof["active_experts"] * w.expert_bytes() / 1e9))),
+            "config": workload_config(w, world),
+            "weight_layout": "blocked (moe_pack_weights once at load, untimed)",
             "roofline": roof,
+            "layer_roofline": layer_roofline(w, ms, counts, peaks, peak_kind, long_run),
             "kernels_ms": stage_ms,
             "row_major_weights": {"ms_per_step": rm_ms,
                                   "value": job_throughput(w.num_tokens, world, rm_ms)},
@@ -547,13 +611,13 @@ def run_ours(args):
             "int8_experts": {"ms_per_step": w8_ms,
                              "value": job_throughput(w.num_tokens, world, w8_ms),
                              "api": "moe_forward_w8",
-                             "weight_gb_per_step": roof["active_experts"] * w.expert_bytes() / 2e9,
+                             "weight_gb_per_step": n_active * w.expert_bytes() / 2e9,
                              "note": "weight-only int8 experts, half-precision expert math, "
                                      "quantised once at load (untimed); not the headline"},
             "int4_experts": {"ms_per_step": w4_ms,
                              "value": job_throughput(w.num_tokens, world, w4_ms),
                              "api": "moe_forward_w4",
-                             "weight_gb_per_step": (roof["active_experts"] * w.expert_bytes()
+                             "weight_gb_per_step": (n_active * w.expert_bytes()
                                                     * (1 / 4 + 1 / 64) / 1e9),
                              "note": "weight-only 4-bit experts (a half scale per 64-column "
                                      "group), half-precision expert math, quantised once at "
@@ -566,7 +630,13 @@ def run_ours(args):
             "gpu_launches": kernels_per_forward(w.num_tokens) * K,
             "clocks": clk,
             "expert_counts": counts,
+            "near_ties": {"tokens": near_ties, "margin": 1e-2,
+                          "rule": "float32 router logits, gap below the margin between neighbours "
+                                  "among the k+1 largest"},
         }
+        if pre_rec is not None:
+            line["prefill"] = pre_rec
+            line["gpu_launches"] += pre_rec["gpu_launches"]
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

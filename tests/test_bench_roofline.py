@@ -85,3 +85,58 @@ def test_kernels_per_forward_matches_the_launch_lists():
     assert bench.kernels_per_forward(1024) == 6
     assert bench.kernels_per_forward(1025) == 8
     assert bench.kernels_per_forward(4096) == 8
+
+
+class _Inputs:
+    x = w_router = w1 = w3 = w2 = residual = logit_bias = None
+
+
+def test_oracle_timing_runs_exactly_max_runs():
+    # the reference arm asks for a number of runs with no time budget: every one of
+    # them must run (a budget of 0 s must not stop the loop after the first)
+    calls = []
+    w = W.WORKLOADS["decode"]
+    per, runs, n_tok, _ = bench.oracle_timing(_Inputs(), w, budget_s=0.0, max_runs=3,
+                                              layer=lambda *a, **kw: calls.append(kw["mode"]))
+    assert calls == ["exact"] * 3 and runs == 3 and n_tok == 16
+    # with a budget and no run count, at least one run and then the budget decides
+    calls.clear()
+    bench.oracle_timing(_Inputs(), w, budget_s=0.0, layer=lambda *a, **kw: calls.append(1))
+    assert len(calls) == 1
+
+
+def test_both_arms_print_the_same_config():
+    w = W.WORKLOADS["prefill"]
+    c = bench.workload_config(w, 1)
+    assert c == bench.workload_config(w, 1)
+    assert c["parallelism"] == "replicas x1" and c["num_tokens"] == 4096
+    # the weights every step reads (at least k experts' 352.3 MB) exceed the L2
+    assert "0.70 GB" in c["l2"]
+
+
+def test_near_tie_tokens_counts_small_gaps_among_the_top_k_plus_one():
+    import torch
+    logits = torch.tensor([[3.0, 2.0, 1.0, 0.0],      # clear
+                           [3.0, 2.995, 1.0, 0.0],    # 1st-2nd tie
+                           [3.0, 2.0, 1.995, 0.0],    # 2nd-3rd tie (decides the top 2)
+                           [3.0, 2.0, 1.0, 0.995]])   # 3rd-4th: outside the k+1 largest
+    assert bench.near_tie_tokens(logits, 2) == 2
+    assert bench.near_tie_tokens(logits, 3) == 3
+    assert bench.near_tie_tokens(logits[:1], 2) == 0
+
+
+def test_layer_roofline_against_nominal_and_measured_peaks():
+    dec = W.WORKLOADS["decode"]
+    r = bench.layer_roofline(dec, 0.5, [4] * 8, PEAKS, "measured", False)
+    b = 8 * dec.expert_bytes() + 3 * 16 * 4096 * 2 + 8 * 4096 * 2 + 16 * 2 * 8
+    assert r["bound"] == "hbm" and r["algorithmic_bytes"] == b
+    assert abs(r["achieved"] - b / 0.5e-3 / 1e9) < 1e-9
+    assert abs(r["frac_of_nominal"] - r["achieved"] / 8000.0) < 1e-12
+    assert abs(r["frac_of_measured"] - r["achieved"] / 6556.2) < 1e-12
+    pre = W.WORKLOADS["prefill"]
+    r = bench.layer_roofline(pre, 2.14, [1024] * 8, PEAKS, "measured", False)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    flops = 6 * 8192 * 4096 * 14336 + 2 * 4096 * 4096 * 8
+    assert r["algorithmic_flops"] == flops
+    # the prefill target: 60% of 2.25 PFLOP/s is a 2.14 ms layer
+    assert abs(r["frac_of_nominal"] - 0.6) < 0.002
