@@ -144,8 +144,10 @@ moe_status_t moe_permute(const moe_shape_t* shape, const int32_t* topk_idx,
  * device array inside the library, which every GPU that loads the library holds
  * until the process exits. Shapes needing more than 65536 entries return
  * MOE_ERR_UNSUPPORTED. The first call on each device, made with that device
- * current, looks up the array's device address (cudaGetSymbolAddress); make that
- * first call before any stream capture. Every call shares the array: calls whose
+ * current, looks up the array's device address (cudaGetSymbolAddress) and keeps it
+ * for the life of the process; make that first call before any stream capture, and
+ * do not call this entry point again on a device after cudaDeviceReset (the kept
+ * address would be stale). Every call shares the array: calls whose
  * kernels overlap on the GPU race on it, so the caller must serialise them. A call
  * writes every table entry it reads, so nothing needs clearing between calls. */
 moe_status_t moe_permute_static(const moe_shape_t* shape, const int32_t* topk_idx,
@@ -235,8 +237,11 @@ moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_bf16_t* x_host
  * result, and x_host and residual_host may be reused, once the stream has reached this
  * point (for example after cudaStreamSynchronize). Calls on one stream with one ws are
  * ordered by the stream, so a serving loop can enqueue step after step and wait once;
- * calls that may overlap on different streams need separate workspaces. Host buffers
- * must be pinned for the copies to be asynchronous. */
+ * the steps may change shape (a workspace sized for the largest serves them all: a
+ * call whose shape differs from the previous call's copies in only after that call is
+ * done with the workspace, without the overlap). Calls that may overlap on different
+ * streams need separate workspaces. Host buffers must be pinned for the copies to be
+ * asynchronous. */
 moe_status_t moe_forward_host_async(const moe_shape_t* shape, const moe_bf16_t* x_host,
                                     const moe_bf16_t* w_router, const float* logit_bias,
                                     const moe_bf16_t* w1, const moe_bf16_t* w3,

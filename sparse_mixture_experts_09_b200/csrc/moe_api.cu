@@ -258,12 +258,17 @@ moe_status_t run_forward(const Shape& s, const uint16_t* x, const uint16_t* wr, 
 // Host-path overlap. The copies in of a host call run on a copy stream of the library's
 // own, into one of two staging slots of the workspace, so they overlap the previous
 // call's layer; the caller's stream waits for them (event `ready`) before the layer, and
-// a slot is refilled only after the layer two calls back has read it (event `freed`).
+// a slot is refilled only after the call two back has finished with the workspace: its
+// layer and its copy out (event `freed`). Every region's offset depends on the shape, so
+// when a call's shape differs from the previous call's on this workspace, its copies in
+// may land anywhere the previous call still reads or writes: they then also wait for the
+// previous call to finish.
 struct HostPath {
   cudaStream_t copy = nullptr;
   cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
   bool freed_recorded[2] = {false, false};
   unsigned calls = 0;
+  size_t prev_x_in = 0, prev_end_host = 0;  // staging layout of the previous call
 };
 
 std::mutex g_host_mutex;
@@ -311,9 +316,14 @@ moe_status_t forward_host_enqueue(const moe_shape_t* shape, const moe_bf16_t* x_
   uint16_t* xd = at<uint16_t>(ws, L.x_in[b]);
   uint16_t* rd = residual_host ? at<uint16_t>(ws, L.res_in[b]) : nullptr;
   uint16_t* od = at<uint16_t>(ws, L.out_st);
-  // copies in, on the copy stream, once the layer two calls back has read this slot
-  if (hp->freed_recorded[b]) {
-    e = cudaStreamWaitEvent(hp->copy, hp->freed[b], 0);
+  // copies in, on the copy stream, once the call two back is done with the workspace;
+  // after a change of shape, also once the previous call is
+  const bool moved = hp->calls > 1 && (hp->prev_x_in != L.x_in[0] || hp->prev_end_host != L.end_host);
+  hp->prev_x_in = L.x_in[0];
+  hp->prev_end_host = L.end_host;
+  for (int j = 0; j < 2; ++j) {
+    if (!hp->freed_recorded[j] || (j != b && !moved)) continue;
+    e = cudaStreamWaitEvent(hp->copy, hp->freed[j], 0);
     if (e != cudaSuccess) return cuda_fail(e, "copy-stream wait");
   }
   e = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, hp->copy);
@@ -327,11 +337,11 @@ moe_status_t forward_host_enqueue(const moe_shape_t* shape, const moe_bf16_t* x_
   if (e != cudaSuccess) return cuda_fail(e, "copy-in event");
   // the layer and the copy out, on the caller's stream
   MOE_TRY(run_forward(s, xd, w_router, logit_bias, bf16_experts(w1, w3, w2), rd, od, ws, st));
+  e = cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e, "copy of out to the host");
   e = cudaEventRecord(hp->freed[b], st);
   if (e != cudaSuccess) return cuda_fail(e, "slot event");
   hp->freed_recorded[b] = true;
-  e = cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, st);
-  if (e != cudaSuccess) return cuda_fail(e, "copy of out to the host");
   return MOE_OK;
 }
 

@@ -103,7 +103,27 @@ def test_forward_full_size(name):
     ok = np.ones(w.num_tokens, dtype=bool)
     ok[near.numpy()] = False
     assert np.array_equal(idx.cpu().numpy()[ok], ref_idx[ok])
-    count, offset, row_of, tok = O.stable_permute(ref_idx, w.num_experts)
+    # counts, padded offsets and the permutation, bit-exact against the oracle's
+    # counting sort. With no near-tie rows the GPU's indices are the oracle's, so this is
+    # the oracle's permutation of the oracle's routing; a near-tie row (at most one per
+    # thousand tokens) may go either way, and then the oracle permutes the GPU's choice.
+    gpu_idx = idx.cpu().numpy()
+    if near.numel() == 0:
+        assert np.array_equal(gpu_idx, ref_idx)
+    count, offset, row_of, tok = O.stable_permute(gpu_idx, w.num_experts)
+    ws = M.make_workspace(M.make_shape(*w.shape))
+    p = M.permute(idx, inp.x, w.num_experts, w.intermediate_size, ws)
+    M.device_status(ws)
+    assert np.array_equal(p["counts"].cpu().numpy(), count)
+    assert np.array_equal(p["offsets"].cpu().numpy(), offset)
+    assert np.array_equal(p["row_of"].cpu().numpy(), row_of)
+    n_rows = int(offset[-1])
+    assert np.array_equal(p["token_of_row"][:n_rows].cpu().numpy(), tok)
+    # the gathered rows: x_perm[row] = x[token], pad rows zero
+    tok_d = p["token_of_row"][:n_rows].long()
+    real = tok_d >= 0
+    assert torch.equal(p["x_perm"][:n_rows][real], inp.x[tok_d[real]])
+    assert not p["x_perm"][:n_rows][~real].any()
     if w.logit_bias is not None:
         assert count[0] > 0.4 * count.sum()          # about half the slots go to expert 0
     # outputs on sampled tokens (all tokens when T <= 256)
@@ -177,4 +197,28 @@ def test_forward_host_async_steps_queue_on_one_stream():
     for x, o in zip(xs, outs):
         want = M.forward(x.cuda(), inp.w_router, inp.w1, inp.w3, inp.w2, w.num_experts_per_tok,
                          residual=inp.residual)
+        assert torch.equal(o, want.cpu())
+
+
+def test_forward_host_async_steps_of_different_sizes_share_a_workspace():
+    # a serving loop whose batch size changes from step to step, enqueued back to back on
+    # one stream and one workspace sized for the largest batch: every region of the
+    # workspace moves with the batch size, so each step's copies in must not land on
+    # memory the step before is still using. Each output equals the device forward.
+    w = SMALL["ragged"]
+    inp, _ = screened(w)
+    t_max = w.num_tokens
+    sizes = [t_max, 7, t_max // 2 + 3, t_max, 1, t_max, t_max - 5, 33]
+    ws = M.make_workspace(M.make_shape(*w.shape), "cuda", host=True)
+    xs = [W.redraw_x_rows(w, torch.arange(t), a + 1).pin_memory() for a, t in enumerate(sizes)]
+    rs = [W.redraw_x_rows(w, torch.arange(t), a + 40).pin_memory() for a, t in enumerate(sizes)]
+    outs = [torch.empty_like(x).pin_memory() for x in xs]
+    for x, r, o in zip(xs, rs, outs):
+        M.forward_host(x, inp.w_router, inp.w1, inp.w3, inp.w2, w.num_experts_per_tok,
+                       residual_host=r, ws=ws, out_host=o, wait=False)
+    torch.cuda.synchronize()
+    M.device_status(ws)
+    for x, r, o in zip(xs, rs, outs):
+        want = M.forward(x.cuda(), inp.w_router, inp.w1, inp.w3, inp.w2, w.num_experts_per_tok,
+                         residual=r.cuda())
         assert torch.equal(o, want.cpu())
