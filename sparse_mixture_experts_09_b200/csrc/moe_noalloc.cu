@@ -76,7 +76,9 @@ moe_status_t moe_permute_static(const moe_shape_t* shape, const int32_t* topk_id
                 "shape needs %lld scratch entries (ceil(num_tokens/32) * num_experts) but the "
                 "static table holds %lld; use moe_permute with a workspace",
                 (long long)need, (long long)kStaticScratchInts);
-  // once per device, with that device current: the device address of the table
+  // once per device, with that device current: the device address of the table, kept
+  // for the life of the process (a cudaDeviceReset would make it stale; the header
+  // rules that out)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));

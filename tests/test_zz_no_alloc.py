@@ -2,14 +2,18 @@
 
 moe_permute_static serves callers that cannot call cudaMalloc (so cannot hand the
 library a workspace): its scratch table is a static device array inside libmoe.so.
-The GPU test calls it twice in a row, on two different shapes that both need the
-table (more than 1024 tokens), and compares every output with moe_permute's. It
+The GPU test calls it three times in a row, on different shapes that all need the
+table (more than 1024 tokens), the last one filling it exactly, and compares every
+output with moe_permute's and, for two of the shapes, with the oracle's. It
 sits in a file of its own, collected last, and needs nothing from other tests.
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
+
+from oracle import moe_oracle as O
 
 from sparse_mixture_experts_09_b200 import build_lib
 from sparse_mixture_experts_09_b200 import moe as M
@@ -25,8 +29,9 @@ def _routing(t, h, e, k, seed):
 
 @pytest.mark.gpu
 def test_static_permute_matches_workspace_permute_on_two_calls():
+    # the last shape fills the static table exactly: ceil(262144 / 32) * 8 = 65536 entries
     build_lib.build()
-    for t, h, e, k, seed in ((3000, 256, 8, 2, 1), (2500, 384, 5, 3, 2)):
+    for t, h, e, k, seed in ((3000, 256, 8, 2, 1), (2500, 384, 5, 3, 2), (262144, 128, 8, 2, 3)):
         idx, x = _routing(t, h, e, k, seed)
         ws = M.make_workspace(M.make_shape(t, h, 128, e, k))
         want = M.permute(idx, x, e, 128, ws)
@@ -34,6 +39,13 @@ def test_static_permute_matches_workspace_permute_on_two_calls():
         torch.cuda.synchronize()
         for key in ("counts", "offsets", "row_of", "token_of_row", "x_perm"):
             assert torch.equal(got[key], want[key]), (t, key)
+        if seed != 2:
+            # both share their kernels, so also against the oracle's counting sort
+            count, offset, row_of, tok = O.stable_permute(idx.cpu().numpy(), e)
+            assert np.array_equal(got["counts"].cpu().numpy(), count), t
+            assert np.array_equal(got["offsets"].cpu().numpy(), offset), t
+            assert np.array_equal(got["row_of"].cpu().numpy(), row_of), t
+            assert np.array_equal(got["token_of_row"][:int(offset[-1])].cpu().numpy(), tok), t
 
 
 def test_static_permute_rejects_oversized_shapes():
