@@ -170,7 +170,7 @@ def test_exchange_plan_sends_real_rows_and_pads_per_expert():
     # receives, for its experts 0 and 1, 3 and 0 rows from rank 0, 7 and 2 from rank 1
     offsets = [0, 128, 384, 384, 512]
     counts = [3, 130, 0, 5]
-    p = ep.exchange_plan(offsets, counts, 2, [[3, 0], [7, 2]])
+    p = _lists(ep.exchange_plan(offsets, counts, 2, [[3, 0], [7, 2]]))
     assert p["send_rows"] == [133, 5] and p["recv_rows"] == [3, 9]
     assert p["send_index"] == [0, 1, 2] + list(range(128, 258)) + [384, 385, 386, 387, 388]
     # every x_perm row maps to its place in the packed rows, pad rows to -1
@@ -186,8 +186,13 @@ def test_exchange_plan_sends_real_rows_and_pads_per_expert():
     assert all(tl[p["to_recv"][i]] == i for i in range(12))
 
 
+def _lists(plan):
+    """The plan with its index tensors as Python lists."""
+    return {k: v.tolist() if torch.is_tensor(v) else v for k, v in plan.items()}
+
+
 def test_exchange_plan_empty_rank():
-    p = ep.exchange_plan([0, 0, 0, 0, 0], [0, 0, 0, 0], 2, [[0, 0], [4, 0]])
+    p = _lists(ep.exchange_plan([0, 0, 0, 0, 0], [0, 0, 0, 0], 2, [[0, 0], [4, 0]]))
     assert p["send_rows"] == [0, 0] and p["send_index"] == [] and p["back_index"] == []
     assert p["local_offsets"] == [0, 128, 128] and p["to_recv"] == [0, 1, 2, 3]
 
@@ -210,7 +215,7 @@ def _simulate_world(counts):
             offs.append(len(rows))
         x_perm.append(rows)
         recv = [[counts[s][r * e_loc + e] for e in range(e_loc)] for s in range(world)]
-        plans.append(ep.exchange_plan(offs, counts[r], world, recv))
+        plans.append(_lists(ep.exchange_plan(offs, counts[r], world, recv)))
     sent = []
     for r in range(world):
         rows = [x_perm[r][i] for i in plans[r]["send_index"]]

@@ -1,6 +1,8 @@
-"""Expert parallelism on one GPU: the row-gather kernel, and the expert-parallel layer
-over a one-rank NCCL group, whose exchanges are then identities, equal to moe_forward
-bit for bit (same routing, same groups, same GEMM tiles)."""
+"""Expert parallelism on one GPU: the row-gather kernel; the expert-parallel layer over
+a one-rank NCCL group, whose exchanges are then identities, equal to moe_forward bit
+for bit (same routing, same groups, same GEMM tiles) and to the fp64 oracle; and the
+layer over two ranks (two processes on the GPU, rows exchanged through host memory)
+against the oracle, with bf16, int8 and 4-bit experts."""
 import datetime
 import socket
 
@@ -63,6 +65,26 @@ def test_expert_parallel_one_rank_equals_forward(one_rank_group, name):
                         residual=inp.residual, logit_bias=inp.logit_bias)
     torch.cuda.synchronize()
     assert torch.equal(got, want)
+    # and the routed output against the fp64 oracle
+    routed = ep.forward_ep(inp.x, inp.w_router, l1, l3, l2, k, w.num_experts,
+                           logit_bias=inp.logit_bias)
+    from oracle import moe_oracle as O
+    from ._cases import assert_layer_close
+    assert_layer_close(O.to_f64(routed.cpu()), _oracle_out(w, inp, "bf16"), name)
+
+
+@pytest.mark.parametrize("mode", ["int8", "int4"])
+def test_expert_parallel_quantized_one_rank_matches_oracle(one_rank_group, mode):
+    from oracle import moe_oracle as O
+    from ._cases import assert_layer_close
+    w = SMALL["ragged"]
+    inp, _ = screened(w)
+    quant = M.quantize_int8 if mode == "int8" else M.quantize_int4
+    local = ep.shard_quantized(quant(inp.w1, inp.w3, inp.w2), 0, 1)
+    got = ep.forward_ep_quantized(inp.x, inp.w_router, local, w.num_experts_per_tok,
+                                  w.num_experts, logit_bias=inp.logit_bias)
+    torch.cuda.synchronize()
+    assert_layer_close(O.to_f64(got.cpu()), _oracle_out(w, inp, mode), mode)
 
 
 def test_expert_parallel_one_rank_decode(one_rank_group):
@@ -73,3 +95,110 @@ def test_expert_parallel_one_rank_decode(one_rank_group):
                         residual=inp.residual)
     torch.cuda.synchronize()
     assert torch.equal(got, want)
+
+
+# ---- two ranks on one GPU, the exchange staged through gloo on the host ----
+#
+# Each rank is its own process with its own CUDA context on the same GPU. The rows cross
+# between ranks through torch.distributed's gloo all_to_all on host copies, so no kernel
+# ever waits on another rank: every wait is in the host collective. The layer's steps
+# are the library's kernels (CudaOps), the exchange plan is ep.exchange_plan, and the
+# two ranks' outputs together are checked against the fp64 oracle.
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _host_exchange(out, inp, out_splits=None, in_splits=None, group=None):
+    """all_to_all_single through host memory (gloo); rows of 2-D tensors move as bytes."""
+    cast = (lambda t: t.view(torch.uint8)) if inp.dim() == 2 else (lambda t: t)
+    got = torch.empty(out.shape, dtype=out.dtype)
+    dist.all_to_all_single(cast(got), cast(inp.contiguous().cpu()), out_splits, in_splits,
+                           group=group)
+    out.copy_(got)
+
+
+def _token_split(t, world):
+    cuts = [0, (3 * t) // 8, t] if world == 2 else [round(t * r / world) for r in range(world + 1)]
+    return [(cuts[r], cuts[r + 1]) for r in range(world)]
+
+
+def _ep_rank(rank, world, port, q, name, mode):
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import torch.distributed as D
+    from sparse_mixture_experts_09_b200 import ep as EP
+    from sparse_mixture_experts_09_b200 import moe as MM
+    from tests._cases import screened as scr
+    from tests.test_gpu_kernels import SMALL as S
+    D.init_process_group("gloo", rank=rank, world_size=world,
+                         timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(0)
+    w = S[name]
+    inp, _ = scr(w)
+    lo, hi = _token_split(w.num_tokens, world)[rank]
+    k, e = w.num_experts_per_tok, w.num_experts
+    if mode == "bf16":
+        l1, l3, l2 = EP.shard_experts(inp.w1, inp.w3, inp.w2, rank, world)
+        out = EP.forward_ep(inp.x[lo:hi], inp.w_router, l1, l3, l2, k, e,
+                            logit_bias=inp.logit_bias, exchange=_host_exchange)
+    else:
+        quant = MM.quantize_int8 if mode == "int8" else MM.quantize_int4
+        local = EP.shard_quantized(quant(inp.w1, inp.w3, inp.w2), rank, world)
+        out = EP.forward_ep_quantized(inp.x[lo:hi], inp.w_router, local, k, e,
+                                      logit_bias=inp.logit_bias, exchange=_host_exchange)
+    torch.cuda.synchronize()
+    q.put((rank, out.cpu().view(torch.int16).numpy().copy()))
+    D.barrier()
+    D.destroy_process_group()
+
+
+def _oracle_out(w, inp, mode):
+    import numpy as np
+    from oracle import moe_oracle as O
+    from ._cases import to_cpu
+    c = to_cpu(inp)
+    k = w.num_experts_per_tok
+    if mode == "bf16":
+        return O.moe_layer(c.x, c.w_router, c.w1, c.w3, c.w2, k, logit_bias=c.logit_bias,
+                           mode="bf16_storage")["out"]
+    if mode == "int8":
+        deq = []
+        for t in (c.w1, c.w3, c.w2):
+            qq, s = O.quantize_int8_rows(t)
+            deq.append(qq.astype(np.float64) * s.astype(np.float64)[..., None])
+    else:
+        deq = [O.dequantize_int4_groups(*O.quantize_int4_groups(t)) for t in (c.w1, c.w3, c.w2)]
+    return O.moe_layer(c.x, c.w_router, *deq, k, logit_bias=c.logit_bias, mode="f16_experts")["out"]
+
+
+@pytest.mark.parametrize("name,mode", [("ragged", "bf16"), ("e64k8", "bf16"), ("skewed", "bf16"),
+                                       ("ragged", "int8"), ("ragged", "int4")])
+def test_expert_parallel_two_ranks_matches_oracle(name, mode):
+    import numpy as np
+    import torch.multiprocessing as mp
+    from oracle import moe_oracle as O
+    from ._cases import assert_layer_close
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ep_rank, args=(r, world, port, q, name, mode))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=300) for _ in range(world))
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    bits = np.concatenate([got[r] for r in range(world)])
+    out = torch.from_numpy(bits).view(torch.bfloat16)
+    w = SMALL[name]
+    inp, near = screened(w)
+    assert near.numel() == 0
+    assert_layer_close(O.to_f64(out), _oracle_out(w, inp, mode), f"{name} {mode} over 2 ranks")
