@@ -502,10 +502,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 // tcgen05.mma.cta_group::2 (M = 256): each CTA stages its own 128 rows of A and its
 // 128 rows of B (gate/up: CTA 0 holds the w1 rows, CTA 1 the w3 rows; down: the two
 // 128-row halves of the w2 tile), so a CTA moves 32 KiB per 64-wide k-block instead
-// of 48 KiB and six stages fit in shared memory. The pair's two row tiles are
-// consecutive 128-row tiles of one expert; when an expert has an odd number, the
-// second CTA's rows of its last pair belong to the next group and are computed but
-// not stored.
+// of 48 KiB. A stage holds kPairKB = 2 k-blocks (K = 128: 64 KiB per CTA, three
+// stages), so every barrier handoff between the copies and the MMAs carries eight
+// MMAs instead of four. Measured on B200: with K = 64 stages a k-block took about 700
+// SM clocks against the tensor pipe's 512, whatever the stage count (4 to 7), the
+// number of busy SMs (37 to 148) or the clock; with K = 128 stages it takes about 570.
+// The pair's two row tiles are consecutive 128-row tiles of one expert; when an
+// expert has an odd number, the second CTA's rows of its last pair belong to the next
+// group and are computed but not stored.
 //
 // Synchronisation: CTA 0 (the leader) owns the full barriers (both CTAs' TMA loads
 // complete transactions on them; only the leader arrives, expecting both CTAs'
@@ -513,11 +517,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 // arrive). The leader's MMA thread commits to the empty and accumulator-full
 // barriers of both CTAs at once (multicast commit). No TMA load uses multicast.
 
-constexpr int kPairStages = 6;
+#ifndef MOE_PAIR_STAGES
+#define MOE_PAIR_STAGES 3
+#endif
+#ifndef MOE_PAIR_KB
+#define MOE_PAIR_KB 2
+#endif
+constexpr int kPairStages = MOE_PAIR_STAGES;
+constexpr int kPairKB = MOE_PAIR_KB;  // 64-wide k-blocks per stage
 
 struct PairTile {
-  static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = 128 * BK * 2;
+  static constexpr int A_BOX = BM * BK * 2;   // one 128-row x 64 box of A
+  static constexpr int B_BOX = 128 * BK * 2;  // one 128-row x 64 box of B
+  static constexpr int A_BYTES = A_BOX * kPairKB;
+  static constexpr int B_BYTES = B_BOX * kPairKB;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 512;
   static constexpr int SMEM_BYTES = 1024 + kPairStages * STAGE_BYTES + 256 + 4 * 144;
@@ -690,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           b_row = e * p.b_rows + n * 256 + (int)rank * 128;
           mb = &mapB0;
         }
-        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+        for (int kb = 0; kb < p.k_blocks; kb += kPairKB, ++it) {
           const int s = it % kPairStages;
           const uint32_t ph = (uint32_t)(it / kPairStages) & 1u;
           if (!wait_phase(empty_bar(s), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
@@ -700,10 +713,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
           if (rank == 0) mbar_expect_tx(full_bar(s), 2 * C::STAGE_BYTES);
           const uint32_t fb = mapa_shared(full_bar(s), 0);
-          tma_load_2d_pair(sa, &mapA, kb * BK, a_row, fb);
-          int wx, wy;
-          wcoord(kb, b_row, p.k_blocks, p.blocked, wx, wy);
-          tma_load_2d_pair(sa + C::A_BYTES, mb, wx, wy, fb);
+#pragma unroll
+          for (int j = 0; j < kPairKB; ++j) {
+            tma_load_2d_pair(sa + j * C::A_BOX, &mapA, (kb + j) * BK, a_row, fb);
+            int wx, wy;
+            wcoord(kb + j, b_row, p.k_blocks, p.blocked, wx, wy);
+            tma_load_2d_pair(sa + C::A_BYTES + j * C::B_BOX, mb, wx, wy, fb);
+          }
         }
       }
       if (!ok && rank == 0) {
@@ -724,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_phase(tempty_bar(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
         fence_after();
         const uint32_t d = tmem_base + (uint32_t)(a * 256);
-        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+        for (int kb = 0; kb < p.k_blocks; kb += kPairKB, ++it) {
           const int s = it % kPairStages;
           const uint32_t ph = (uint32_t)(it / kPairStages) & 1u;
           if (!wait_phase(full_bar(s), ph, abort_flag, p.status, p.timeout_ns)) {
@@ -735,10 +751,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
           const uint32_t sb = sa + C::A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            mma_bf16_pair(d, sdesc(sa + kk * 32), sdesc(sb + kk * 32), C::IDESC,
-                          (kb | kk) ? 1u : 0u);
-          }
+          for (int j = 0; j < kPairKB; ++j)
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              mma_bf16_pair(d, sdesc(sa + j * C::A_BOX + kk * 32),
+                            sdesc(sb + j * C::B_BOX + kk * 32), C::IDESC, (kb | j | kk) ? 1u : 0u);
           mma_commit_pair_both(empty_bar(s));
           issued = true;
         }
@@ -952,6 +969,7 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
+  if (p.k_blocks % kPairKB) return cudaErrorInvalidValue;  // K is a multiple of 128
   int64_t pairs = pair_capacity<MODE>();
   if (pairs > max_pair_tiles) pairs = max_pair_tiles;
   if (pairs < 1) pairs = 1;
@@ -972,10 +990,9 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
   return cudaLaunchKernelEx(&cfg, k_grouped_gemm_pair<MODE>, a, b0, b1, p);
 }
 
-// Measured on B200: the pair kernel speeds up the down GEMM by 4-7% once an average
-// expert has at least eight row tiles (1024 rows); with fewer, the half-empty pair of
-// every expert with an odd tile count and the coarser waves cost more than it saves.
-// The gate/up GEMM runs as fast with single CTAs, so it always uses them.
+// Measured on B200: the pair kernel speeds up both GEMMs once an average expert has at
+// least eight row tiles (1024 rows); with fewer, the half-empty pair of every expert
+// with an odd tile count and the coarser waves cost more than it saves.
 #ifndef MOE_PAIR_GEMM
 #define MOE_PAIR_GEMM 1
 #endif
@@ -1004,8 +1021,11 @@ cudaError_t launch_gate_up(const Shape& s, const GemmArgs& g, cudaStream_t st, c
   p.b_rows = s.I;
   p.blocked = s.blocked;
   p.timeout_ns = g.timeout_ns;
-  cudaError_t e =
-      launch_one<kSwiGLU, 256>(mx, mw1, mw3, mw1s, mw3s, p, (g.rmax / BM) * p.n_tiles, st);
+  cudaError_t e;
+  if (use_pair(s))
+    e = launch_pair<kSwiGLU>(mx, mw1, mw3, p, (g.rmax / BM / 2 + s.E) * p.n_tiles, st);
+  else
+    e = launch_one<kSwiGLU, 256>(mx, mw1, mw3, mw1s, mw3s, p, (g.rmax / BM) * p.n_tiles, st);
   if (e != cudaSuccess) *why = "gate/up GEMM launch failed";
   return e;
 }
