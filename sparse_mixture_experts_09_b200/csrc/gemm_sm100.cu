@@ -50,7 +50,7 @@ struct Tile {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + BAR_BYTES + 4 * 72;
+  static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + BAR_BYTES + 4 * 144;
   // instruction descriptor: D f32 (bit 4), A bf16 (bits 7-9 = 1), B bf16 (bits 10-12 = 1),
   // both K-major, N >> 3 at bit 17, M >> 4 at bit 24
   static constexpr uint32_t IDESC =
@@ -68,6 +68,13 @@ struct KParams {
   int b_rows;  // rows of the B tensor per expert
   int blocked;  // weights in the blocked layout (MOE_WEIGHTS_BLOCKED)
   unsigned long long timeout_ns;
+  // split-K (plain GEMM): counts [E] (null: no split), partial sums [kMaxSplitK, routed,
+  // out_ld] fp32, arrival counters [kSplitSems]; routed = total routed rows
+  const int32_t* counts;
+  float* partial;
+  int32_t* split_sem;
+  int64_t routed;
+  int32_t* zero_sem;  // gate/up: counters to zero for the down GEMM that follows (nullable)
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -190,12 +197,16 @@ __device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile 
   }
 }
 
-// Bounded wait used while unwinding: ignores the abort flag.
-__device__ __noinline__ void drain_phase(uint32_t bar, uint32_t parity,
+// Bounded wait used while unwinding: ignores the abort flag; if it runs out too, it
+// records kStatusUnwound.
+__device__ __noinline__ void drain_phase(uint32_t bar, uint32_t parity, int32_t* status,
                                          unsigned long long timeout_ns) {
   const unsigned long long t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > timeout_ns) return;
+    if (globaltimer() - t0 > timeout_ns) {
+      atomicOr(status, kStatusUnwound);
+      return;
+    }
   }
 }
 
@@ -230,10 +241,36 @@ __device__ __forceinline__ void tile_coords(int L, const int* row_tiles, int E, 
 // Work items. Whole waves of tiles run at full width (item = tile, round-robin over
 // the CTAs). When the tiles left over for the last wave would fill at most half of the
 // CTAs, each of them is cut into `split` (2 or 4) pieces along N, so the last wave is
-// shorter by that factor and more CTAs share it.
+// shorter by that factor and more CTAs share it. When split-K is allowed (max_ksplit >
+// 1) and the tiles do not fill one wave, each tile is instead cut into `ksplit` parts
+// along K (items tile * ksplit + part), ksplit chosen to minimise waves per part, at
+// least kMinSplitKBlocks k-blocks per part, the fewest parts on a tie, and taken only
+// when it shortens the GEMM to at most 3/4 of one wave of whole tiles (measured on
+// B200: 8 parts for 128 tiles on 148 SMs, 7/8 on paper, ran 4% slower; 3 parts for 48
+// tiles cut a one-token layer by 22%).
+constexpr int kMinSplitKBlocks = 8;
+
 struct Work {
-  int full_items, split, items;
-  __device__ void init(int total_tiles, int grid) {
+  int full_items, split, items, ksplit;
+  __device__ void init(int total_tiles, int grid, int max_ksplit = 1, int k_blocks = 0) {
+    ksplit = 1;
+    if (max_ksplit > 1 && total_tiles > 0 && total_tiles < grid) {
+      int best_waves = 1;  // ksplit = 1: one wave of whole tiles
+      for (int s = 2; s <= max_ksplit && k_blocks / s >= kMinSplitKBlocks; ++s) {
+        const int waves = (total_tiles * s + grid - 1) / grid;
+        if (waves * ksplit < best_waves * s) {  // waves / s < best_waves / ksplit
+          best_waves = waves;
+          ksplit = s;
+        }
+      }
+      if (4 * best_waves > 3 * ksplit) ksplit = 1;
+    }
+    if (ksplit > 1) {
+      full_items = 0;
+      split = 1;
+      items = total_tiles * ksplit;
+      return;
+    }
     full_items = (total_tiles / grid) * grid;
     const int rest = total_tiles - full_items;
     split = 1;
@@ -243,8 +280,16 @@ struct Work {
     }
     items = full_items + split * rest;
   }
-  // item -> (tile, piece, pieces)
-  __device__ void get(int item, int& tile, int& piece, int& pieces) const {
+  // item -> (tile, piece, pieces, K part)
+  __device__ void get(int item, int& tile, int& piece, int& pieces, int& part) const {
+    part = 0;
+    if (ksplit > 1) {
+      tile = item / ksplit;
+      part = item - tile * ksplit;
+      piece = 0;
+      pieces = 1;
+      return;
+    }
     if (item < full_items) {
       tile = item;
       piece = 0;
@@ -276,6 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* row_tiles = reinterpret_cast<int*>(tmem_holder + 2);
+  int* routed_start = row_tiles + 72;  // split-K: first compact routed row of each expert
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t bar0 = smem_u32(bars);
@@ -318,12 +364,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_trigger();
   pdl_wait();
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) row_tiles[i] = p.offsets[i] / BM;
+  if (p.zero_sem && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < kSplitSems; i += blockDim.x) p.zero_sem[i] = 0;
+  if (p.counts && threadIdx.x == 0) {
+    int acc = 0;
+    for (int e = 0; e < p.E; ++e) {
+      routed_start[e] = acc;
+      acc += p.counts[e];
+    }
+  }
   fence_before();
   __syncthreads();
   fence_after();
   const uint32_t tmem_base = *tmem_holder;
   Work work;
-  work.init(row_tiles[p.E] * p.n_tiles, gridDim.x);
+  work.init(row_tiles[p.E] * p.n_tiles, gridDim.x, (MODE == kPlain && p.counts) ? kMaxSplitK : 1,
+            p.k_blocks);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -331,14 +387,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < work.items && ok; w += gridDim.x) {
-        int tile, piece, pieces, e, m, n;
-        work.get(w, tile, piece, pieces);
+        int tile, piece, pieces, part, e, m, n;
+        work.get(w, tile, piece, pieces, part);
         tile_coords(tile, row_tiles, p.E, p.n_tiles, e, m, n);
         const int a_row = m * BM;
         const int rp = ROWS / pieces;  // B rows per weight matrix in this item
         const int b_row = e * p.b_rows + n * ROWS + piece * rp;
         const uint32_t bytes = C::A_BYTES + (MODE == kSwiGLU ? 2 : 1) * rp * BK * 2;
-        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+        const int kb_end = (part + 1) * p.k_blocks / work.ksplit;
+        for (int kb = part * p.k_blocks / work.ksplit; kb < kb_end; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
           if (!wait_phase(empty_bar(s), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
@@ -380,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // let the copies already issued land before the CTA can exit
         const int first = it > kStages ? it - kStages : 0;
         for (int i = first; i < it; ++i)
-          drain_phase(full_bar(i % kStages), (uint32_t)(i / kStages) & 1u, p.timeout_ns);
+          drain_phase(full_bar(i % kStages), (uint32_t)(i / kStages) & 1u, p.status, p.timeout_ns);
       }
     }
     __syncwarp();
@@ -390,8 +447,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0, tc = 0;
       bool ok = true, issued = false;
       for (int w = blockIdx.x; w < work.items && ok; w += gridDim.x, ++tc) {
-        int tile, piece, pieces;
-        work.get(w, tile, piece, pieces);
+        int tile, piece, pieces, part;
+        work.get(w, tile, piece, pieces, part);
         const uint32_t nmma = (uint32_t)((MODE == kSwiGLU ? 2 : 1) * (ROWS / pieces));
         const uint32_t idesc = (C::IDESC & ~(0x3Fu << 17)) | ((nmma >> 3) << 17);
         const int a = tc & 1;
@@ -399,7 +456,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_phase(tempty_bar(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
         fence_after();
         const uint32_t d = tmem_base + (uint32_t)(a * BN);
-        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+        const int kb0 = part * p.k_blocks / work.ksplit;
+        const int kb_end = (part + 1) * p.k_blocks / work.ksplit;
+        for (int kb = kb0; kb < kb_end; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
           if (!wait_phase(full_bar(s), ph, abort_flag, p.status, p.timeout_ns)) {
@@ -411,7 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sb = sa + C::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            mma_bf16(d, sdesc(sa + kk * 32), sdesc(sb + kk * 32), idesc, (kb | kk) ? 1u : 0u);
+            mma_bf16(d, sdesc(sa + kk * 32), sdesc(sb + kk * 32), idesc,
+                     (kb != kb0 || kk) ? 1u : 0u);
           }
           mma_commit(empty_bar(s));
           issued = true;
@@ -421,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every MMA issued so far completes before tensor memory is released
       if (issued) {
         mma_commit(final_bar);
-        drain_phase(final_bar, 0, p.timeout_ns);
+        drain_phase(final_bar, 0, p.status, p.timeout_ns);
       }
     }
     __syncwarp();
@@ -431,8 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row_in_tile = q * 32 + lane;
     int tc = 0;
     for (int w = blockIdx.x; w < work.items; w += gridDim.x, ++tc) {
-      int tile, piece, pieces, e, m, n;
-      work.get(w, tile, piece, pieces);
+      int tile, piece, pieces, part, e, m, n;
+      work.get(w, tile, piece, pieces, part);
       tile_coords(tile, row_tiles, p.E, p.n_tiles, e, m, n);
       const int rp = ROWS / pieces;  // output columns of this item
       const int a = tc & 1;
@@ -466,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
-      } else {
+      } else if (work.ksplit == 1) {
         float* y = reinterpret_cast<float*>(p.out) + row * p.out_ld + col0;
 #pragma unroll 1
         for (int c = 0; c < rp; c += 16) {
@@ -479,6 +539,71 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
                                  __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
         }
+      } else {
+        // split-K: this part's sums of the tile's real rows go to the partial buffer
+        // (compact routed rows; pad rows are neither stored nor summed)
+        const int local = (m - row_tiles[e]) * BM + row_in_tile;  // row within the expert
+        const bool real = local < p.counts[e];
+        const int64_t crow = (int64_t)routed_start[e] + local;
+        const int64_t part_ld = p.routed * p.out_ld;
+        float* mine = p.partial + (int64_t)part * part_ld + crow * p.out_ld + col0;
+#pragma unroll 1
+        for (int c = 0; c < rp; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(taddr + c, v);
+          tmem_wait_ld();
+          if (real) {
+            float4* dst = reinterpret_cast<float4*>(mine + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          }
+        }
+        // the accumulator is free once read
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(a));
+        // arrival of this warp's 32 rows; the warp of the last part to arrive sums the
+        // parts in part order (a fixed order, whichever part finishes last) into y
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        int32_t* sem = p.split_sem + tile * 4 + q;
+        if (lane == 0) last = atomicAdd(sem, 1) == work.ksplit - 1;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          __threadfence();
+          // the warp sums its real rows one at a time, lanes across the columns
+          // (coalesced), every part's load in flight before the adds
+          const int local0 = local - row_in_tile + q * 32;  // the warp's first row in the expert
+          const int nreal = min(32, max(0, p.counts[e] - local0));
+          const float* src0 = p.partial + ((int64_t)routed_start[e] + local0) * p.out_ld + col0;
+          float* y0 = reinterpret_cast<float*>(p.out) + ((int64_t)m * BM + q * 32) * p.out_ld + col0;
+#pragma unroll 1
+          for (int r = 0; r < nreal; ++r) {
+#pragma unroll 1
+            for (int c = lane * 4; c < rp; c += 128) {
+              float4 v[kMaxSplitK];
+#pragma unroll
+              for (int s = 0; s < kMaxSplitK; ++s)
+                if (s < work.ksplit)
+                  v[s] = __ldcg(reinterpret_cast<const float4*>(src0 + r * p.out_ld + s * part_ld + c));
+              float4 acc = v[0];
+#pragma unroll
+              for (int s = 1; s < kMaxSplitK; ++s)
+                if (s < work.ksplit) {
+                  acc.x += v[s].x;
+                  acc.y += v[s].y;
+                  acc.z += v[s].z;
+                  acc.w += v[s].w;
+                }
+              *reinterpret_cast<float4*>(y0 + r * p.out_ld + c) = acc;
+            }
+          }
+          if (lane == 0) *sem = 0;  // ready for the next launch
+        }
+        continue;
       }
       fence_before();
       __syncwarp();
@@ -631,6 +756,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  // a role that gives up a wait also raises the other CTA's abort flag, so the pair
+  // unwinds together (both CTAs stay resident until the final cluster barrier)
+  const uint32_t peer_abort = mapa_shared(smem_u32((const void*)abort_flag), rank ^ 1u);
+  auto abort_peer = [&]() {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer_abort), "r"(1) : "memory");
+  };
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kPairStages + s); };
@@ -707,6 +838,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = it % kPairStages;
           const uint32_t ph = (uint32_t)(it / kPairStages) & 1u;
           if (!wait_phase(empty_bar(s), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+            abort_peer();
             ok = false;
             break;
           }
@@ -725,7 +857,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok && rank == 0) {
         const int first = it > kPairStages ? it - kPairStages : 0;
         for (int i = first; i < it; ++i)
-          drain_phase(full_bar(i % kPairStages), (uint32_t)(i / kPairStages) & 1u, p.timeout_ns);
+          drain_phase(full_bar(i % kPairStages), (uint32_t)(i / kPairStages) & 1u, p.status,
+                      p.timeout_ns);
       }
     }
     __syncwarp();
@@ -737,13 +870,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int L = pair; L < total && ok; L += npairs, ++tc) {
         const int a = tc & 1;
         const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
-        if (!wait_phase(tempty_bar(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
+        if (!wait_phase(tempty_bar(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+          abort_peer();
+          break;
+        }
         fence_after();
         const uint32_t d = tmem_base + (uint32_t)(a * 256);
         for (int kb = 0; kb < p.k_blocks; kb += kPairKB, ++it) {
           const int s = it % kPairStages;
           const uint32_t ph = (uint32_t)(it / kPairStages) & 1u;
           if (!wait_phase(full_bar(s), ph, abort_flag, p.status, p.timeout_ns)) {
+            abort_peer();
             ok = false;
             break;
           }
@@ -763,7 +900,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (issued) {
         mma_commit_pair_local(final_bar);
-        drain_phase(final_bar, 0, p.timeout_ns);
+        drain_phase(final_bar, 0, p.status, p.timeout_ns);
       }
     }
     __syncwarp();
@@ -780,7 +917,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int a = tc & 1;
       const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
       int ok = 0;
-      if (lane == 0) ok = wait_phase(tfull_bar(a), aph, abort_flag, p.status, p.timeout_ns) ? 1 : 0;
+      if (lane == 0) {
+        ok = wait_phase(tfull_bar(a), aph, abort_flag, p.status, p.timeout_ns) ? 1 : 0;
+        if (!ok) abort_peer();
+      }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       fence_after();
@@ -1021,6 +1161,11 @@ cudaError_t launch_gate_up(const Shape& s, const GemmArgs& g, cudaStream_t st, c
   p.b_rows = s.I;
   p.blocked = s.blocked;
   p.timeout_ns = g.timeout_ns;
+  p.counts = nullptr;
+  p.partial = nullptr;
+  p.split_sem = nullptr;
+  p.routed = 0;
+  p.zero_sem = g.counts ? g.split_sem : nullptr;
   cudaError_t e;
   if (use_pair(s))
     e = launch_pair<kSwiGLU>(mx, mw1, mw3, p, (g.rmax / BM / 2 + s.E) * p.n_tiles, st);
@@ -1049,16 +1194,26 @@ cudaError_t launch_down(const Shape& s, const GemmArgs& g, cudaStream_t st, cons
   p.b_rows = s.H;
   p.blocked = s.blocked;
   p.timeout_ns = g.timeout_ns;
+  // split-K needs the counts (real rows), the partial buffer and the counters, which
+  // the gate/up GEMM before it has zeroed
+  const bool split = g.counts && g.partial && g.split_sem && s.T * s.k <= kSplitMaxRows;
+  p.counts = split ? g.counts : nullptr;
+  p.partial = g.partial;
+  p.split_sem = g.split_sem;
+  p.routed = s.T * s.k;
+  p.zero_sem = nullptr;
   cudaError_t e;
   if (s.H % 256 == 0 && use_pair(s)) {
     p.n_tiles = s.H / 256;
     e = launch_pair<kPlain>(mh, mw2, mw2, p, (g.rmax / BM / 2 + s.E) * p.n_tiles, st);
   } else if (s.H % 256 == 0) {
     p.n_tiles = s.H / 256;
-    e = launch_one<kPlain, 256>(mh, mw2, mw2, mw2s, mw2s, p, (g.rmax / BM) * p.n_tiles, st);
+    e = launch_one<kPlain, 256>(mh, mw2, mw2, mw2s, mw2s, p,
+                                (g.rmax / BM) * p.n_tiles * (split ? kMaxSplitK : 1), st);
   } else {
     p.n_tiles = s.H / 128;
-    e = launch_one<kPlain, 128>(mh, mw2, mw2, mw2s, mw2s, p, (g.rmax / BM) * p.n_tiles, st);
+    e = launch_one<kPlain, 128>(mh, mw2, mw2, mw2s, mw2s, p,
+                                (g.rmax / BM) * p.n_tiles * (split ? kMaxSplitK : 1), st);
   }
   if (e != cudaSuccess) *why = "down GEMM launch failed";
   return e;

@@ -237,10 +237,14 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatil
   return wait_w8(bar, parity, abort_flag, status, timeout_ns);
 }
 
-__device__ __noinline__ void drain_w8(uint32_t bar, uint32_t parity, unsigned long long timeout_ns) {
+__device__ __noinline__ void drain_w8(uint32_t bar, uint32_t parity, int32_t* status,
+                                      unsigned long long timeout_ns) {
   const unsigned long long t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > timeout_ns) return;
+    if (globaltimer() - t0 > timeout_ns) {
+      atomicOr(status, kStatusUnwound);
+      return;
+    }
   }
 }
 
@@ -443,7 +447,7 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
       if (!ok) {
         const int first = it > kCodeStages ? it - kCodeStages : 0;
         for (int i = first; i < it; ++i)
-          drain_w8(q_full(i % kCodeStages), (uint32_t)(i / kCodeStages) & 1u, p.timeout_ns);
+          drain_w8(q_full(i % kCodeStages), (uint32_t)(i / kCodeStages) & 1u, p.status, p.timeout_ns);
       }
     }
     __syncwarp();
@@ -481,7 +485,7 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
       }
       if (issued) {
         mma_commit(final_bar);
-        drain_w8(final_bar, 0, p.timeout_ns);
+        drain_w8(final_bar, 0, p.status, p.timeout_ns);
       }
     }
     __syncwarp();
@@ -507,7 +511,7 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
       if (!ok) {
         const int first = it > kAStages ? it - kAStages : 0;
         for (int i = first; i < it; ++i)
-          drain_w8(a_full(i % kAStages), (uint32_t)(i / kAStages) & 1u, p.timeout_ns);
+          drain_w8(a_full(i % kAStages), (uint32_t)(i / kAStages) & 1u, p.status, p.timeout_ns);
       }
     }
     __syncwarp();

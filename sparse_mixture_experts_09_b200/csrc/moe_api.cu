@@ -50,7 +50,7 @@ inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 // Workspace regions, in order; each starts on a 1024-byte boundary.
 struct Layout {
   size_t status, topk_idx, topk_w, block_base, counts, offsets, row_of, token_of_row, x_perm, h,
-      y, rnorm, end;
+      y, rnorm, split_sem, partial, end;
   size_t x_in[2], res_in[2], out_st, end_host;  // staging of the host entry points
 };
 
@@ -71,6 +71,10 @@ Layout layout(const Shape& s) {
   L.h = o; o += up(rmax * s.I * 2);
   L.y = o; o += up(rmax * s.H * 4);
   L.rnorm = o; o += up((size_t)s.T * 4);
+  // split-K of the down GEMM (small batches only): arrival counters and partial sums
+  const bool split = (int64_t)tk <= kSplitMaxRows;
+  L.split_sem = o; o += split ? up((size_t)kSplitSems * 4) : 0;
+  L.partial = o; o += split ? up((size_t)kMaxSplitK * tk * s.H * 4) : 0;
   L.end = o;
   for (int b = 0; b < 2; ++b) {
     L.x_in[b] = o; o += up((size_t)s.T * s.H * 2);
@@ -192,9 +196,16 @@ Experts int4_experts(const uint8_t* q1, const uint8_t* q3, const uint8_t* q2, co
   return x;
 }
 
+// split: the per-expert counts and the workspace's split-K regions, or null (no split)
+struct SplitK {
+  const int32_t* counts = nullptr;
+  float* partial = nullptr;
+  int32_t* sem = nullptr;
+};
+
 moe_status_t run_experts(const Shape& s, const uint16_t* x_perm, const int32_t* offsets,
                          const Experts& w, uint16_t* h, float* y, int32_t* status,
-                         cudaStream_t st) {
+                         cudaStream_t st, const SplitK& split = SplitK()) {
   const char* why = "";
   cudaError_t e;
   if (w.q1) {
@@ -229,6 +240,9 @@ moe_status_t run_experts(const Shape& s, const uint16_t* x_perm, const int32_t* 
     g.status = status;
     g.rmax = max_padded_rows(s);
     g.timeout_ns = kTimeoutNs;
+    g.counts = split.counts;
+    g.partial = split.partial;
+    g.split_sem = split.sem;
     e = launch_grouped_swiglu(s, g, st, &why);
   }
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, why);
@@ -247,8 +261,15 @@ moe_status_t run_forward(const Shape& s, const uint16_t* x, const uint16_t* wr, 
                      at<int32_t>(ws, L.token_of_row), at<uint16_t>(ws, L.x_perm),
                      at<int32_t>(ws, L.block_base), st, norm_w, rnorm, w.q1 != nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
+  SplitK split;
+  if (L.partial != L.end) {
+    split.counts = at<int32_t>(ws, L.counts);
+    split.partial = at<float>(ws, L.partial);
+    split.sem = at<int32_t>(ws, L.split_sem);
+  }
   MOE_TRY(run_experts(s, at<uint16_t>(ws, L.x_perm), at<int32_t>(ws, L.offsets), w,
-                      at<uint16_t>(ws, L.h), at<float>(ws, L.y), at<int32_t>(ws, L.status), st));
+                      at<uint16_t>(ws, L.h), at<float>(ws, L.y), at<int32_t>(ws, L.status), st,
+                      split));
   e = launch_combine(s, at<float>(ws, L.y), at<int32_t>(ws, L.row_of), at<float>(ws, L.topk_w), res,
                      out, st);
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
@@ -614,8 +635,10 @@ moe_status_t moe_device_status(void* ws, size_t ws_bytes, moe_stream_t stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "status clear");
   if (word & kStatusTimeout)
-    return fail(MOE_ERR_TIMEOUT, "a kernel gave up a bounded wait (device status 0x%x)",
-                (unsigned)word);
+    return fail(MOE_ERR_TIMEOUT, "a kernel gave up a bounded wait (device status 0x%x)%s",
+                (unsigned)word,
+                (word & kStatusUnwound) ? "; it exited with copies or MMAs possibly still in flight"
+                                        : "");
   return fail(MOE_ERR_CUDA, "unknown device status 0x%x", (unsigned)word);
 }
 

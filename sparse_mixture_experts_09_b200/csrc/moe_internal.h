@@ -14,8 +14,12 @@ constexpr int kTokensPerBlock = 32;
 constexpr int kRowPad = 128;
 
 
-// Device status word, first int32 of the workspace.
+// Device status word, first int32 of the workspace: a bounded wait ran out
+// (kStatusTimeout); while unwinding after it, a wait for the kernel's own copies or
+// MMAs ran out too, so they may still have been in flight when it released its tensor
+// memory and exited (kStatusUnwound).
 constexpr int32_t kStatusTimeout = 1;
+constexpr int32_t kStatusUnwound = 2;
 
 struct Shape {
   int64_t T;
@@ -52,6 +56,16 @@ cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16
 cudaError_t launch_rows_to_f16(const uint16_t* src, uint16_t* dst, int64_t rows, int H,
                                cudaStream_t st);
 
+// Split-K of the down GEMM for small batches. When its tiles would leave SMs idle, each
+// tile's K range is cut into S <= kMaxSplitK parts: every part writes fp32 partial sums
+// of its tile's real rows to a workspace region, and the part that finishes last sums
+// the S partials in part order and writes y (the result does not depend on which part
+// finishes last). Used for batches of at most kSplitMaxRows routed rows, when the
+// per-expert row counts are known (they bound the rows to store).
+constexpr int kMaxSplitK = 8;
+constexpr int64_t kSplitMaxRows = 512;
+constexpr int kSplitSems = 1024;  // arrival counters, one per (tile, epilogue warp)
+
 struct GemmArgs {
   const uint16_t* a;        // x_perm [Rmax, K1] (GEMM1) or h [Rmax, I] (GEMM2)
   const int32_t* offsets;   // [E+1], multiples of 128
@@ -63,6 +77,11 @@ struct GemmArgs {
   int32_t* status;          // device status word
   int64_t rmax;
   unsigned long long timeout_ns;
+  // split-K of GEMM2 (all null: no split): per-expert routed rows [E], partial sums
+  // [kMaxSplitK, T*k, H] fp32, arrival counters [kSplitSems] (GEMM1 zeroes them)
+  const int32_t* counts = nullptr;
+  float* partial = nullptr;
+  int32_t* split_sem = nullptr;
 };
 
 // GEMM1 (gate/up + SwiGLU -> h) then GEMM2 (h w2^T -> y), both persistent tcgen05.

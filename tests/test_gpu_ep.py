@@ -88,13 +88,23 @@ def test_expert_parallel_quantized_one_rank_matches_oracle(one_rank_group, mode)
 
 
 def test_expert_parallel_one_rank_decode(one_rank_group):
+    # moe_forward may split the down GEMM along K at small batches (its sums are then
+    # grouped differently) where the expert-parallel path does not: both against the
+    # oracle, and close to each other
+    from oracle import moe_oracle as O
+    from ._cases import assert_layer_close
     w = W.WORKLOADS["decode"]
-    inp = W.draw(w, "cuda")
-    want = M.forward(inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, 2, residual=inp.residual)
-    got = ep.forward_ep(inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, 2, w.num_experts,
-                        residual=inp.residual)
+    inp, near = screened(w)
+    assert near.numel() == 0
+    want = M.forward(inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, 2)
+    got = ep.forward_ep(inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, 2, w.num_experts)
     torch.cuda.synchronize()
-    assert torch.equal(got, want)
+    ref = _oracle_out(w, inp, "bf16")
+    assert_layer_close(O.to_f64(got.cpu()), ref, "decode, expert parallel")
+    assert_layer_close(O.to_f64(want.cpu()), ref, "decode, moe_forward")
+    from ._cases import layer_errors
+    max_rel, mae = layer_errors(O.to_f64(got.cpu()), O.to_f64(want.cpu()))
+    assert max_rel <= 2e-3 and mae <= 1e-4, (max_rel, mae)
 
 
 # ---- two ranks on one GPU, the exchange staged through gloo on the host ----

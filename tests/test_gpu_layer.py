@@ -222,3 +222,39 @@ def test_forward_host_async_steps_of_different_sizes_share_a_workspace():
         want = M.forward(x.cuda(), inp.w_router, inp.w1, inp.w3, inp.w2, w.num_experts_per_tok,
                          residual=r.cuda())
         assert torch.equal(o, want.cpu())
+
+
+# Few routed rows: the down GEMM's tiles do not fill the SMs, so moe_forward splits each
+# tile's K range into parts (at least 8 k-blocks each) and the last part of a tile sums
+# the parts in order. 8 parts; 3 uneven parts (26 k-blocks); 4 parts on 128-column tiles
+# (a hidden size that is not a multiple of 256).
+SPLIT_K = {
+    "sk_t5": W.Workload("sk_t5", 5, 256, 4096, 8, 2, seed=51),
+    "sk_uneven": W.Workload("sk_uneven", 3, 512, 1664, 8, 2, seed=52),
+    "sk_h384": W.Workload("sk_h384", 7, 384, 2048, 4, 2, seed=53),
+}
+
+
+@pytest.mark.parametrize("name", list(SPLIT_K))
+def test_split_k_down_gemm_matches_oracle_and_repeats_exactly(name):
+    w = SPLIT_K[name]
+    inp, near = screened(w)
+    assert near.numel() == 0
+    got, ref, out = _forward_and_check(w, inp, residual=False)
+    assert_layer_close(got, ref["out"], name)
+    # the parts are summed in a fixed order: a second call gives the same bits
+    again = M.forward(inp.x, inp.w_router, inp.w1, inp.w3, inp.w2, w.num_experts_per_tok,
+                      logit_bias=inp.logit_bias)
+    assert torch.equal(again, out)
+    # against the unsplit GEMM (the split entry points do not split): within a rounding
+    shape = M.make_shape(*w.shape)
+    ws = M.make_workspace(shape)
+    idx, wt = M.router_topk(inp.x, inp.w_router, w.num_experts_per_tok, inp.logit_bias)
+    p = M.permute(idx, inp.x, w.num_experts, w.intermediate_size, ws)
+    y = M.grouped_swiglu(p["x_perm"], p["offsets"], inp.w1, inp.w3, inp.w2, w.num_tokens,
+                         w.num_experts_per_tok, ws)
+    plain = M.combine(y, p["row_of"], wt, None, w.num_experts, w.intermediate_size)
+    g, f = out.float(), plain.float()
+    # one bf16 rounding step, or an fp32-sized difference where the output cancels to ~0
+    tol = 2.0 ** -7 * torch.maximum(g.abs(), f.abs()) + 1e-5 * f.pow(2).mean().sqrt()
+    assert ((g - f).abs() <= tol).all()
