@@ -69,7 +69,7 @@ constexpr int kConvWarps = MOE_W8_CONV_WARPS;
 // warp 0: code copies, 1: MMA, 2-5: epilogue, 6: activation TMA, 7..: converters
 constexpr int kConvWarp0 = 7;
 constexpr int kThreadsW8 = 32 * (kConvWarp0 + kConvWarps);
-constexpr int kSwiGLU = 0, kPlain = 1;
+constexpr int kSwiGLU = 0, kPlain = 1, kFused = 2;
 #ifndef MOE_W8_HALF_TILES
 #define MOE_W8_HALF_TILES 1
 #endif
@@ -124,6 +124,9 @@ struct W8Params {
   int64_t out_ld;
   int E, k_blocks, n_tiles, b_rows;
   unsigned long long timeout_ns;
+  // kFused: row_ready[m] counts the gate/up epilogue warps that have stored their rows
+  // of h for row tile m; a down tile waits for 4 * (gate/up column tiles) of them
+  int32_t* row_ready;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -219,6 +222,27 @@ __device__ __noinline__ bool wait_w8(uint32_t bar, uint32_t parity, volatile int
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > timeout_ns) {
+        *abort_flag = 1;
+        atomicOr(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// Wait until *ready >= target (an acquire load: the h rows the gate/up epilogues
+// stored before their release are then visible), bounded like the barrier waits.
+__device__ __noinline__ bool wait_ready(const int32_t* ready, int target, volatile int* abort_flag,
+                                        int32_t* status, unsigned long long timeout_ns) {
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t n = 0;; ++n) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ready) : "memory");
+    if (v >= target) return true;
+    __nanosleep(64);
+    if ((n & 63u) == 63u) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > timeout_ns) {
         *abort_flag = 1;
@@ -332,9 +356,17 @@ __device__ __forceinline__ uint32_t pack_f16x2_rn(float lo, float hi) {
 // MODE kSwiGLU: A = x_perm [rows, H] (half), weight tile = 128 rows of w1 then 128 rows
 //   of w3 (BN = 256), h = half(silu(s1 * gate) * (s3 * up)).
 // MODE kPlain:  A = h [rows, I], weight tile = BN rows of w2, y = s2 * acc (fp32).
+// MODE kFused:  both in one persistent grid: the gate/up tiles (parameters p, A map
+//   mapA) come first, then the down tiles (p2, mapA2, BN = 256). A down tile reads the
+//   h rows of its row tile only once every gate/up tile of that row tile has stored
+//   them (p.row_ready), so the down tiles fill the SMs the gate/up tail leaves idle.
+//   Every gate/up tile precedes every down tile in the order each CTA walks its tiles,
+//   so a down tile only ever waits for tiles that are running or done.
 template <int MODE, int BN, int MT, int BITS>
 __global__ void __launch_bounds__(kThreadsW8, 1)
-    k_grouped_gemm_w8(const __grid_constant__ CUtensorMap mapA, const W8Params p) {
+    k_grouped_gemm_w8(const __grid_constant__ CUtensorMap mapA,
+                      const __grid_constant__ CUtensorMap mapA2,
+                      const __grid_constant__ W8Params p, const __grid_constant__ W8Params p2) {
   using TL = TileW8<BN, MT, BITS>;
   constexpr int kAStages = TL::A_ST, kBStages = TL::B_ST, kCodeStages = TL::Q_ST;
   constexpr int A_BYTES = TL::A_BYTES;
@@ -401,7 +433,16 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
   __syncthreads();
   fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int total = row_tiles[p.E] * p.n_tiles;
+  // tiles L < total0 belong to the first GEMM (p), the rest (kFused) to the down GEMM (p2)
+  const int total0 = row_tiles[p.E] * p.n_tiles;
+  const int total = total0 + (MODE == kFused ? row_tiles[p.E] * p2.n_tiles : 0);
+  auto second = [&](int L) { return MODE == kFused && L >= total0; };
+  // tile L -> (expert, row tile, column tile) of its GEMM
+  auto coords = [&](int L, int& e, int& m, int& n) {
+    const bool d = second(L);
+    tile_coords_w8(d ? L - total0 : L, row_tiles, p.E, d ? p2.n_tiles : p.n_tiles, e, m, n);
+  };
+  auto kblocks = [&](int L) { return second(L) ? p2.k_blocks : p.k_blocks; };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -410,9 +451,13 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
       bool ok = true;
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
         int e, m, n;
-        tile_coords_w8(L, row_tiles, p.E, p.n_tiles, e, m, n);
-        const int row0 = MODE == kSwiGLU ? e * p.b_rows + n * 128 : e * p.b_rows + n * BN;
-        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+        coords(L, e, m, n);
+        const bool dn = second(L);
+        const bool sw = MODE == kSwiGLU || (MODE == kFused && !dn);
+        const W8Params& g = dn ? p2 : p;
+        const int k_blocks = g.k_blocks;
+        const int row0 = sw ? e * g.b_rows + n * 128 : e * g.b_rows + n * BN;
+        for (int kb = 0; kb < k_blocks; ++kb, ++it) {
           const int q = it % kCodeStages;
           const uint32_t ph = (uint32_t)(it / kCodeStages) & 1u;
           if (!wait_w8(q_empty(q), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
@@ -424,22 +469,22 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
           // code_y / 128 is the tile number: its codes start at byte tile * BOX_CODE
           // and (4-bit) its 128 scales at element tile * 128 = code_y
           constexpr int kBox = TL::BOX_CODE;
-          if (MODE == kSwiGLU) {
-            const int cy = code_y(row0, kb, p.k_blocks);
+          if (sw) {
+            const int cy = code_y(row0, kb, k_blocks);
             const size_t off = (size_t)cy * (kBox / 128);
-            bulk_load(dq, p.q0 + off, kBox, q_full(q));
-            bulk_load(dq + kBox, p.q1 + off, kBox, q_full(q));
+            bulk_load(dq, g.q0 + off, kBox, q_full(q));
+            bulk_load(dq + kBox, g.q1 + off, kBox, q_full(q));
             if constexpr (BITS == 4) {
-              bulk_load(dq + TL::Q_CODE, p.gscale_a + cy, 256, q_full(q));
-              bulk_load(dq + TL::Q_CODE + 256, p.gscale_b + cy, 256, q_full(q));
+              bulk_load(dq + TL::Q_CODE, g.gscale_a + cy, 256, q_full(q));
+              bulk_load(dq + TL::Q_CODE + 256, g.gscale_b + cy, 256, q_full(q));
             }
           } else {
 #pragma unroll
             for (int j = 0; j < BN / 128; ++j) {
-              const int cy = code_y(row0 + 128 * j, kb, p.k_blocks);
-              bulk_load(dq + j * kBox, p.q0 + (size_t)cy * (kBox / 128), kBox, q_full(q));
+              const int cy = code_y(row0 + 128 * j, kb, k_blocks);
+              bulk_load(dq + j * kBox, g.q0 + (size_t)cy * (kBox / 128), kBox, q_full(q));
               if constexpr (BITS == 4)
-                bulk_load(dq + TL::Q_CODE + j * 256, p.gscale_a + cy, 256, q_full(q));
+                bulk_load(dq + TL::Q_CODE + j * 256, g.gscale_a + cy, 256, q_full(q));
             }
           }
         }
@@ -462,7 +507,8 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
         if (!wait_w8(tempty(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
         fence_after();
         const uint32_t d = tmem_base + (uint32_t)(a * BN);
-        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+        const int k_blocks = kblocks(L);
+        for (int kb = 0; kb < k_blocks; ++kb, ++it) {
           const int sa = it % kAStages, sb = it % kBStages;
           if (!wait_w8(a_full(sa), (uint32_t)(it / kAStages) & 1u, abort_flag, p.status,
                        p.timeout_ns) ||
@@ -496,8 +542,20 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
       bool ok = true;
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
         int e, m, n;
-        tile_coords_w8(L, row_tiles, p.E, p.n_tiles, e, m, n);
-        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+        coords(L, e, m, n);
+        const bool dn = second(L);
+        if (dn) {
+          // the h rows of this row tile, once every gate/up tile of it has stored them;
+          // then a proxy fence, so the tensor copies (async proxy) see those stores
+          if (!wait_ready(p.row_ready + m, 4 * p.n_tiles, abort_flag, p.status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
+        const CUtensorMap* map = dn ? &mapA2 : &mapA;
+        const int k_blocks = kblocks(L);
+        for (int kb = 0; kb < k_blocks; ++kb, ++it) {
           const int sa = it % kAStages;
           const uint32_t ph = (uint32_t)(it / kAStages) & 1u;
           if (!wait_w8(a_empty(sa), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
@@ -505,7 +563,7 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
             break;
           }
           mbar_expect_tx(a_full(sa), A_BYTES);
-          tma_load_2d(smem_u32(smem + sa * A_BYTES), &mapA, kb * BK, m * BM, a_full(sa));
+          tma_load_2d(smem_u32(smem + sa * A_BYTES), map, kb * BK, m * BM, a_full(sa));
         }
       }
       if (!ok) {
@@ -526,7 +584,8 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
     int it = 0;
     bool ok = true;
     for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-      for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+      const int k_blocks = kblocks(L);
+      for (int kb = 0; kb < k_blocks; ++kb, ++it) {
         const int q = it % kCodeStages, sb = it % kBStages;
         if (!wait_warp(q_full(q), (uint32_t)(it / kCodeStages) & 1u, abort_flag, p.status,
                        p.timeout_ns)) {
@@ -597,17 +656,20 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
     int tc = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x, ++tc) {
       int e, m, n;
-      tile_coords_w8(L, row_tiles, p.E, p.n_tiles, e, m, n);
+      coords(L, e, m, n);
+      const bool dn = second(L);
+      const bool sw = MODE == kSwiGLU || (MODE == kFused && !dn);
+      const W8Params& g = dn ? p2 : p;
       const int a = tc & 1;
       const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
       if (!wait_warp(tfull(a), aph, abort_flag, p.status, p.timeout_ns)) break;
       fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(qd * 32) << 16) + (uint32_t)(a * BN);
       const int64_t row = (int64_t)m * BM + row_in_tile;
-      if (MODE == kSwiGLU) {
-        const float* sg = BITS == 8 ? p.scale_a + (size_t)e * p.b_rows + n * 128 : nullptr;
-        const float* su = BITS == 8 ? p.scale_b + (size_t)e * p.b_rows + n * 128 : nullptr;
-        uint16_t* h = reinterpret_cast<uint16_t*>(p.out) + row * p.out_ld + (int64_t)n * 128;
+      if (sw) {
+        const float* sg = BITS == 8 ? g.scale_a + (size_t)e * g.b_rows + n * 128 : nullptr;
+        const float* su = BITS == 8 ? g.scale_b + (size_t)e * g.b_rows + n * 128 : nullptr;
+        uint16_t* h = reinterpret_cast<uint16_t*>(g.out) + row * g.out_ld + (int64_t)n * 128;
 #pragma unroll 1
         for (int c = 0; c < 128; c += 16) {
           uint32_t g[16], u[16];
@@ -629,9 +691,18 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
             dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
           }
         }
+        if (MODE == kFused) {
+          // release this warp's rows of h to the down tiles of row tile m: the stores,
+          // a proxy fence (the readers copy with the async proxy) and a gpu-scope fence
+          // before the count
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) atomicAdd(p.row_ready + m, 1);
+        }
       } else {
-        const float* sc = BITS == 8 ? p.scale_a + (size_t)e * p.b_rows + n * BN : nullptr;
-        float* y = reinterpret_cast<float*>(p.out) + row * p.out_ld + (int64_t)n * BN;
+        const float* sc = BITS == 8 ? g.scale_a + (size_t)e * g.b_rows + n * BN : nullptr;
+        float* y = reinterpret_cast<float*>(g.out) + row * g.out_ld + (int64_t)n * BN;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 16) {
           uint32_t v[16];
@@ -813,8 +884,8 @@ bool map_act(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, ui
 }
 
 template <int MODE, int BN, int MT, int BITS>
-cudaError_t launch_w8(const CUtensorMap& a, const W8Params& p, int64_t max_tiles,
-                      cudaStream_t st) {
+cudaError_t launch_w8(const CUtensorMap& a, const W8Params& p, int64_t max_tiles, cudaStream_t st,
+                      const CUtensorMap* a2 = nullptr, const W8Params* p2 = nullptr) {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -829,7 +900,7 @@ cudaError_t launch_w8(const CUtensorMap& a, const W8Params& p, int64_t max_tiles
   if (grid > max_tiles) grid = max_tiles;
   if (grid < 1) grid = 1;
   return launch_pdl(k_grouped_gemm_w8<MODE, BN, MT, BITS>, dim3((unsigned)grid), dim3(kThreadsW8),
-                    (size_t)TileW8<BN, MT, BITS>::SMEM, st, a, p);
+                    (size_t)TileW8<BN, MT, BITS>::SMEM, st, a, a2 ? *a2 : a, p, p2 ? *p2 : p);
 }
 
 }  // namespace
@@ -889,11 +960,6 @@ cudaError_t launch_swiglu_w8_tiles(const Shape& s, const GemmArgsW8& g, cudaStre
   p1.n_tiles = s.I / 128;
   p1.b_rows = s.I;
   p1.timeout_ns = g.timeout_ns;
-  cudaError_t e = launch_w8<kSwiGLU, 256, MT, BITS>(mx, p1, mt_max * p1.n_tiles, st);
-  if (e != cudaSuccess) {
-    *why = BITS == 8 ? "int8 gate/up GEMM launch failed" : "4-bit gate/up GEMM launch failed";
-    return e;
-  }
   W8Params p2 = p1;
   p2.q0 = g.q2;
   p2.q1 = nullptr;
@@ -905,6 +971,23 @@ cudaError_t launch_swiglu_w8_tiles(const Shape& s, const GemmArgsW8& g, cudaStre
   p2.out_ld = s.H;
   p2.k_blocks = s.I / BK;
   p2.b_rows = s.H;
+  cudaError_t e;
+  if (s.H % 256 == 0 && g.row_ready) {
+    // one grid for both GEMMs; the row-tile counters start at zero
+    p2.n_tiles = s.H / 256;
+    p1.row_ready = g.row_ready;
+    e = cudaMemsetAsync(g.row_ready, 0, (size_t)mt_max * sizeof(int32_t), st);
+    if (e == cudaSuccess)
+      e = launch_w8<kFused, 256, MT, BITS>(mx, p1, mt_max * (p1.n_tiles + p2.n_tiles), st, &mh, &p2);
+    if (e != cudaSuccess)
+      *why = BITS == 8 ? "int8 expert GEMMs launch failed" : "4-bit expert GEMMs launch failed";
+    return e;
+  }
+  e = launch_w8<kSwiGLU, 256, MT, BITS>(mx, p1, mt_max * p1.n_tiles, st);
+  if (e != cudaSuccess) {
+    *why = BITS == 8 ? "int8 gate/up GEMM launch failed" : "4-bit gate/up GEMM launch failed";
+    return e;
+  }
   if (s.H % 256 == 0) {
     p2.n_tiles = s.H / 256;
     e = launch_w8<kPlain, 256, MT, BITS>(mh, p2, mt_max * p2.n_tiles, st);

@@ -50,7 +50,7 @@ inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 // Workspace regions, in order; each starts on a 1024-byte boundary.
 struct Layout {
   size_t status, topk_idx, topk_w, block_base, counts, offsets, row_of, token_of_row, x_perm, h,
-      y, rnorm, split_sem, partial, end;
+      y, rnorm, row_ready, split_sem, partial, end;
   size_t x_in[2], res_in[2], out_st, end_host;  // staging of the host entry points
 };
 
@@ -71,6 +71,7 @@ Layout layout(const Shape& s) {
   L.h = o; o += up(rmax * s.I * 2);
   L.y = o; o += up(rmax * s.H * 4);
   L.rnorm = o; o += up((size_t)s.T * 4);
+  L.row_ready = o; o += up((size_t)(rmax / kRowPad) * 4);  // quantised experts: row tiles of h done
   // split-K of the down GEMM (small batches only): arrival counters and partial sums
   const bool split = (int64_t)tk <= kSplitMaxRows;
   L.split_sem = o; o += split ? up((size_t)kSplitSems * 4) : 0;
@@ -196,11 +197,14 @@ Experts int4_experts(const uint8_t* q1, const uint8_t* q3, const uint8_t* q2, co
   return x;
 }
 
-// split: the per-expert counts and the workspace's split-K regions, or null (no split)
+// Workspace scratch of the expert GEMMs: the per-expert counts and the split-K regions
+// of the bf16 down GEMM (null: no split), and the row-tile counters that let the
+// quantised experts run both GEMMs as one grid (null: two grids).
 struct SplitK {
   const int32_t* counts = nullptr;
   float* partial = nullptr;
   int32_t* sem = nullptr;
+  int32_t* row_ready = nullptr;
 };
 
 moe_status_t run_experts(const Shape& s, const uint16_t* x_perm, const int32_t* offsets,
@@ -227,6 +231,7 @@ moe_status_t run_experts(const Shape& s, const uint16_t* x_perm, const int32_t* 
     g.status = status;
     g.rmax = max_padded_rows(s);
     g.timeout_ns = kTimeoutNs;
+    g.row_ready = split.row_ready;
     e = launch_grouped_swiglu_w8(s, g, st, &why);
   } else {
     GemmArgs g;
@@ -262,6 +267,7 @@ moe_status_t run_forward(const Shape& s, const uint16_t* x, const uint16_t* wr, 
                      at<int32_t>(ws, L.block_base), st, norm_w, rnorm, w.q1 != nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   SplitK split;
+  split.row_ready = at<int32_t>(ws, L.row_ready);
   if (L.partial != L.end) {
     split.counts = at<int32_t>(ws, L.counts);
     split.partial = at<float>(ws, L.partial);
@@ -689,9 +695,11 @@ moe_status_t moe_grouped_swiglu_w8(const moe_shape_t* shape, const moe_bf16_t* x
   uint16_t* xh = at<uint16_t>(ws, L.x_perm);
   cudaError_t e = launch_rows_to_f16(x_perm, xh, max_padded_rows(s), s.H, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "x_perm conversion launch");
+  SplitK scratch;
+  scratch.row_ready = at<int32_t>(ws, L.row_ready);
   return run_experts(s, xh, expert_offsets, int8_experts(q1, q3, q2, s1, s3, s2),
                      at<uint16_t>(ws, L.h), y_perm, at<int32_t>(ws, L.status),
-                     (cudaStream_t)stream);
+                     (cudaStream_t)stream, scratch);
 }
 
 moe_status_t moe_forward_w8(const moe_shape_t* shape, const moe_bf16_t* x,
@@ -766,9 +774,11 @@ moe_status_t moe_grouped_swiglu_w4(const moe_shape_t* shape, const moe_bf16_t* x
   uint16_t* xh = at<uint16_t>(ws, L.x_perm);
   cudaError_t e = launch_rows_to_f16(x_perm, xh, max_padded_rows(s), s.H, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "x_perm conversion launch");
+  SplitK scratch;
+  scratch.row_ready = at<int32_t>(ws, L.row_ready);
   return run_experts(s, xh, expert_offsets, int4_experts(q1, q3, q2, s1, s3, s2),
                      at<uint16_t>(ws, L.h), y_perm, at<int32_t>(ws, L.status),
-                     (cudaStream_t)stream);
+                     (cudaStream_t)stream, scratch);
 }
 
 moe_status_t moe_forward_w4(const moe_shape_t* shape, const moe_bf16_t* x,

@@ -122,6 +122,8 @@ struct GemmArgsW8 {
   int32_t* status = nullptr;
   int64_t rmax = 0;
   unsigned long long timeout_ns = 0;
+  // [rmax / 128] int32 scratch: given, both GEMMs run as one grid (hidden % 256 == 0)
+  int32_t* row_ready = nullptr;
 };
 
 // GEMM1 (int8 or 4-bit gate/up + SwiGLU -> h) then GEMM2 (h q2^T -> y), in float16.
