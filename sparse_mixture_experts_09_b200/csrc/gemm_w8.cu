@@ -31,6 +31,7 @@
 // half scales, and the converters widen each code to a half and multiply it by its
 // group's scale (the scale varies along K, so it cannot wait for the epilogue).
 // Every wait is bounded (timeout -> status word, abort flag, drained copies).
+#include <algorithm>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -74,6 +75,10 @@ constexpr int kSwiGLU = 0, kPlain = 1, kFused = 2;
 #define MOE_W8_HALF_TILES 1
 #endif
 constexpr bool kUseHalfTiles = MOE_W8_HALF_TILES != 0;
+#ifndef MOE_W8_DECODE_KERNEL
+#define MOE_W8_DECODE_KERNEL 1
+#endif
+constexpr bool kUseDecodeKernel = MOE_W8_DECODE_KERNEL != 0;
 
 // Shared-memory plan for an MT x BN tile: [A ring][B ring][code ring][barriers, TMEM
 // address, row tiles]. Three rings: activation tiles (TMA -> MMA), code tiles (bulk
@@ -733,6 +738,523 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
   }
 }
 
+// ---------------------------------------------------------------- small batches
+//
+// k_w8_decode: both expert GEMMs of a batch of at most 64 tokens, in one persistent
+// grid, with the operands swapped. A token reaches an expert at most once, so each
+// expert then has at most 64 routed rows, all in its one 128-row tile. The tile kernel
+// above spends a full M = 64 MMA and an 8 KiB activation tile on every 64-wide k-block
+// for those few rows. Here the weights are the tcgen05 M operand (128 weight rows per
+// tile) and the expert's routed rows the N operand (N = its row count rounded up to
+// 16), so the MMAs shrink with the batch. The widened weights never touch shared memory:
+//
+//   warp 0      streams code stages into a deep ring (bulk copies): a stage is four
+//               128-row x 64-code boxes, gate/up the w1 and w3 boxes of two k-blocks,
+//               down four consecutive k-blocks of one w2 box (4-bit: plus their scales);
+//   warps 7-22  widen them, one thread per weight row: converter warp c takes box c / 4
+//               and TMEM lanes 32 (warp % 4) .. + 31, reads its row's codes with 4
+//               (int8) or 2 (4-bit) conflict-free 16-byte loads and writes 32 columns of
+//               half pairs with one tcgen05.st: the tensor-memory layout of an M = 128
+//               A operand (lane = row, column c = K elements 2c and 2c + 1);
+//   warp 6      loads the routed rows' k-blocks (TMA, 16-row boxes, 128-byte swizzle);
+//               a down tile first waits until every gate/up tile of its row tile has
+//               released its rows of h (per-row-tile counters);
+//   warp 1      issues tcgen05.mma with A in tensor memory and B (the rows) in shared
+//               memory, M = 128, N = rows: gate/up into two accumulators (gate, up),
+//               down into one;
+//   warps 2-5   read the accumulators (lane = weight row, column = routed row): h =
+//               half(silu(s1 gate) * s3 up) at [row, i], y = s2 acc at [row, j].
+//
+// Tiles: gate/up tile (row tile, n) covers intermediate columns 128 n .. + 127 over
+// H / 128 stages; down tile (row tile, n) covers hidden columns 128 n .. + 127 over
+// I / 256 stages. Every gate/up tile precedes every down tile in the order each CTA
+// walks its tiles, and the grid is at most one CTA per SM, so a down tile only waits for
+// tiles that are running or done.
+//
+// Measured on B200, and what the plan does about it. (1) An MMA of this shape (M = 128,
+// N <= 64, K = 16) occupies the issuing thread for about 45 SM clocks whatever N is, so
+// sixteen are about 710 clocks: below the HBM time of the 32 KiB of int8 codes they
+// consume. (2) In the MMA thread, between MMAs, a commit costs about 55 clocks, a
+// non-blocking test_wait about 53, and a wait whose result steers the thread about 340
+// even on a phase that has long completed: barrier traffic, not the tensor pipe, set
+// the pace of small stages. So a stage is 128 columns of K (sixteen MMAs), each role
+// tests the barriers of its next stage with test_wait before it starts the current one
+// (the latency runs under its work) and blocks only if that test failed. (3) Separate
+// accumulators per MMA do not help (the pipe is not waiting on accumulation).
+template <int BITS, int NMAX>
+struct DecW8 {
+  static constexpr int BOX = 128 * BK * BITS / 8;                  // code bytes of a box
+  static constexpr int SUBS = 4;                                   // boxes per stage
+  static constexpr int Q_BYTES = SUBS * BOX + (BITS == 4 ? SUBS * 256 : 0);
+  static constexpr int ACT_UNIT = NMAX * 128;                      // NMAX rows of one k-block
+  static constexpr int ACC_COLS = 2 * NMAX;                        // one buffer: gate, up
+  static constexpr int W_COL0 = 2 * ACC_COLS;                      // two buffers
+  static constexpr int W_SLOT_COLS = SUBS * 32;                    // a widened stage
+  static constexpr int W_SLOTS = (512 - W_COL0) / W_SLOT_COLS;     // widened stages in TMEM
+  static constexpr int ACT_SLOT = SUBS * ACT_UNIT;                 // a slot's rows (down: 4 k-blocks)
+  static constexpr int Q_FIT = (200 * 1024 - W_SLOTS * ACT_SLOT) / Q_BYTES;
+  static constexpr int Q_ST = Q_FIT > 16 ? 16 : Q_FIT;
+  static constexpr int CONV_WARPS = 4 * SUBS;                      // one box per warp
+  static constexpr int THREADS = 32 * (7 + CONV_WARPS);
+  static constexpr int Q_OFF = W_SLOTS * ACT_SLOT;
+  static constexpr int BAR_OFF = Q_OFF + Q_ST * Q_BYTES;
+  static constexpr int NUM_BARS = 2 * Q_ST + 3 * W_SLOTS + 4 + 1;
+  static constexpr int SMEM = 1024 + BAR_OFF + NUM_BARS * 8 + 16 + 2 * 72 * 4;
+  // D f32, A and B f16, both K-major, M = 128; N is set per tile
+  static constexpr uint32_t IDESC_M128 = (1u << 4) | ((uint32_t)(128 >> 4) << 24);
+  static_assert(NMAX == 16 || NMAX == 32 || NMAX == 64, "rows per expert");
+  static_assert(W_SLOTS >= 2 && Q_ST >= 3, "pipeline plan");
+  static_assert(Q_BYTES % 16 == 0 && ACT_UNIT % 1024 == 0, "stage alignment");
+  static_assert(SMEM <= 232448, "shared memory plan exceeds 227 KiB");
+};
+
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+struct DecParams {
+  const uint8_t* q1;
+  const uint8_t* q3;
+  const uint8_t* q2;
+  const float* s1;   // int8: per-row scales
+  const float* s3;
+  const float* s2;
+  const uint16_t* g1;  // 4-bit: half group scales, tile order
+  const uint16_t* g3;
+  const uint16_t* g2;
+  const int32_t* offsets;  // [E+1], multiples of 128
+  const int32_t* counts;   // [E] routed rows per expert, or null (then NMAX rows)
+  uint16_t* h;             // [rows, I] half
+  float* y;                // [rows, H] fp32
+  int32_t* status;
+  int32_t* row_ready;      // [rows / 128], zero at launch
+  int E, H, I;
+  unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint16_t half_rn(float f) {
+  uint16_t v;
+  asm("cvt.rn.f16.f32 %0, %1;" : "=h"(v) : "f"(f));
+  return v;
+}
+
+// 4-bit word (8 columns) -> four half pairs times the scale pair s2, the same values
+// as widen_word4 with fewer instructions: the pairs in nibbles (1, 5) and (3, 7) are
+// masked in place, giving half 1024 + 16u, and one packed fma by 1/16 minus 72 leaves
+// q = u - 8 exactly (every intermediate is an integer below 2048); the pairs in
+// nibbles (0, 4) and (2, 6) give 1024 + u, minus 1032. One multiply by the scale then
+// rounds q * s once, as before.
+__device__ __forceinline__ void widen_word4_pairs(uint32_t w, uint32_t s2, uint32_t* out) {
+  const uint32_t ws = w >> 8;
+  const uint32_t x0 = (w & 0x000F000Fu) | 0x64006400u;
+  const uint32_t x1 = (w & 0x00F000F0u) | 0x64006400u;
+  const uint32_t x2 = (ws & 0x000F000Fu) | 0x64006400u;
+  const uint32_t x3 = (ws & 0x00F000F0u) | 0x64006400u;
+  uint32_t q0, q1, q2, q3;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(q0) : "r"(x0), "r"(0x64086408u));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(q1) : "r"(x1), "r"(0x2C002C00u), "r"(0xD480D480u));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(q2) : "r"(x2), "r"(0x64086408u));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(q3) : "r"(x3), "r"(0x2C002C00u), "r"(0xD480D480u));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[0]) : "r"(q0), "r"(s2));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[1]) : "r"(q1), "r"(s2));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[2]) : "r"(q2), "r"(s2));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[3]) : "r"(q3), "r"(s2));
+}
+
+template <int BITS, int NMAX>
+__global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
+    k_w8_decode(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapH,
+                const __grid_constant__ DecParams p) {
+  using D = DecW8<BITS, NMAX>;
+  constexpr int kQ = D::Q_ST, kW = D::W_SLOTS;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint8_t* qbase = smem + D::Q_OFF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + D::BAR_OFF);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + D::NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* row_tiles = reinterpret_cast<int*>(tmem_holder + 4);  // [E + 1]
+  int* ncols = row_tiles + 72;                                // [E]: N of the expert's tiles
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // barriers: q_full, q_empty [kQ]; w_full (widened slot), a_full (the slot's rows),
+  // w_empty (slot and rows free) [kW]; t_full, t_empty [2]; final
+  const uint32_t bar0 = smem_u32(bars);
+  constexpr int kW0 = 2 * kQ, kT0 = kW0 + 3 * kW;
+  auto q_full = [&](int s) { return bar0 + 8u * s; };
+  auto q_empty = [&](int s) { return bar0 + 8u * (kQ + s); };
+  auto w_full = [&](int s) { return bar0 + 8u * (kW0 + s); };
+  auto a_full = [&](int s) { return bar0 + 8u * (kW0 + kW + s); };
+  auto w_empty = [&](int s) { return bar0 + 8u * (kW0 + 2 * kW + s); };
+  auto t_full = [&](int b) { return bar0 + 8u * (kT0 + b); };
+  auto t_empty = [&](int b) { return bar0 + 8u * (kT0 + 2 + b); };
+  const uint32_t final_bar = bar0 + 8u * (kT0 + 4);
+  auto act = [&](int ws) { return smem_u32(smem + ws * D::ACT_SLOT); };
+  const int kb1 = p.H / BK, kb2 = p.I / BK;  // k-blocks of the gate/up and down weights
+  // phase parity of the barrier a stage uses (ring of n), and of its previous use
+  auto ph = [](int it, int n) { return (uint32_t)(it / n) & 1u; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQ; ++s) {
+      mbar_init(q_full(s), 1);
+      mbar_init(q_empty(s), D::CONV_WARPS);
+    }
+    for (int s = 0; s < kW; ++s) {
+      mbar_init(w_full(s), D::CONV_WARPS);
+      mbar_init(a_full(s), 1);
+      mbar_init(w_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(t_full(b), 1);
+      mbar_init(t_empty(b), 4);
+    }
+    mbar_init(final_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(512u)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  pdl_trigger();
+  pdl_wait();
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) row_tiles[i] = p.offsets[i] / BM;
+  for (int i = threadIdx.x; i < p.E; i += blockDim.x) {
+    int n = NMAX;
+    if (p.counts) {
+      n = (p.counts[i] + 15) & ~15;
+      n = n < 16 ? 16 : (n > NMAX ? NMAX : n);
+    }
+    ncols[i] = n;
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int n1 = p.I / 128, n2 = p.H / 128;  // column tiles per row tile
+  const int st1 = p.H / (2 * BK), st2 = p.I / (4 * BK);  // stages per tile
+  const int total0 = row_tiles[p.E] * n1;
+  const int total = total0 + row_tiles[p.E] * n2;
+  auto coords = [&](int L, bool& dn, int& e, int& m, int& n) {
+    dn = L >= total0;
+    tile_coords_w8(dn ? L - total0 : L, row_tiles, p.E, dn ? n2 : n1, e, m, n);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- code stages
+      int it = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        bool dn;
+        int e, m, n;
+        coords(L, dn, e, m, n);
+        const int nst = dn ? st2 : st1;
+        for (int s = 0; s < nst; ++s, ++it) {
+          const int q = it % kQ;
+          if (!wait_w8(q_empty(q), ph(it, kQ) ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dq = smem_u32(qbase + q * D::Q_BYTES);
+          mbar_expect_tx(q_full(q), D::Q_BYTES);
+          // boxes of one row tile and consecutive k-blocks are adjacent in memory (and
+          // so are their scales)
+          if (!dn) {
+            // boxes 0, 1: w1 rows 128 n .. of expert e, k-blocks 2s, 2s + 1; boxes 2, 3: w3
+            const int cy = code_y(e * p.I + n * 128, 2 * s, kb1);
+            const size_t off = (size_t)cy * (D::BOX / 128);
+            bulk_load(dq, p.q1 + off, 2 * D::BOX, q_full(q));
+            bulk_load(dq + 2 * D::BOX, p.q3 + off, 2 * D::BOX, q_full(q));
+            if constexpr (BITS == 4) {
+              bulk_load(dq + 4 * D::BOX, p.g1 + cy, 512, q_full(q));
+              bulk_load(dq + 4 * D::BOX + 512, p.g3 + cy, 512, q_full(q));
+            }
+          } else {
+            // boxes 0..3: k-blocks 4s .. 4s + 3 of the w2 box of rows 128 n ..
+            const int cy = code_y(e * p.H + n * 128, 4 * s, kb2);
+            bulk_load(dq, p.q2 + (size_t)cy * (D::BOX / 128), 4 * D::BOX, q_full(q));
+            if constexpr (BITS == 4) bulk_load(dq + 4 * D::BOX, p.g2 + cy, 1024, q_full(q));
+          }
+        }
+      }
+      if (!ok) {
+        const int first = it > kQ ? it - kQ : 0;
+        for (int i = first; i < it; ++i) drain_w8(q_full(i % kQ), ph(i, kQ), p.status, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    if (lane == 0) {
+      // ---------------- routed rows of each stage into its slot's buffer: two k-blocks
+      // (gate/up) or four (down), N rows in 16-row boxes
+      int it = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        bool dn;
+        int e, m, n;
+        coords(L, dn, e, m, n);
+        if (dn) {
+          // every gate/up tile of row tile m has stored its rows of h; the proxy fence
+          // orders those stores before the tensor copies (async proxy) that read them
+          if (!wait_ready(p.row_ready + m, 4 * n1, abort_flag, p.status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
+        const int nrow = ncols[e];
+        const CUtensorMap* map = dn ? &mapH : &mapX;
+        const int nst = dn ? st2 : st1;
+        const int nblk = dn ? 4 : 2;
+        for (int s = 0; s < nst; ++s, ++it) {
+          const int ws = it % kW;
+          if (!wait_w8(w_empty(ws), ph(it, kW) ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(a_full(ws), (uint32_t)(nblk * nrow * 128));
+          for (int b = 0; b < nblk; ++b) {
+            const int xk = (nblk * s + b) * BK;
+            for (int j = 0; j < nrow; j += 16)
+              tma_load_2d(act(ws) + b * D::ACT_UNIT + j * 128, map, xk, m * BM + j, a_full(ws));
+          }
+        }
+      }
+      if (!ok) {
+        const int first = it > kW ? it - kW : 0;
+        for (int i = first; i < it; ++i) drain_w8(a_full(i % kW), ph(i, kW), p.status, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer. The next stage's barriers are tested before this
+      // stage's MMAs issue, so their latency runs under the MMAs.
+      int it = 0, tc = 0;
+      bool ok = true, issued = false, pre_w = false, pre_a = false;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tc) {
+        bool dn;
+        int e, m, n;
+        coords(L, dn, e, m, n);
+        const uint32_t idesc = D::IDESC_M128 | ((uint32_t)(ncols[e] >> 3) << 17);
+        const int b = tc & 1;
+        if (!wait_w8(t_empty(b), ph(tc, 2) ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
+        fence_after();
+        const uint32_t dacc = tmem_base + (uint32_t)(b * D::ACC_COLS);
+        const int nst = dn ? st2 : st1;
+        for (int s = 0; s < nst; ++s, ++it) {
+          const int ws = it % kW;
+          if ((!pre_w && !wait_w8(w_full(ws), ph(it, kW), abort_flag, p.status, p.timeout_ns)) ||
+              (!pre_a && !wait_w8(a_full(ws), ph(it, kW), abort_flag, p.status, p.timeout_ns))) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          pre_w = mbar_test_wait(w_full((it + 1) % kW), ph(it + 1, kW));
+          pre_a = mbar_test_wait(a_full((it + 1) % kW), ph(it + 1, kW));
+          const uint32_t wcol = tmem_base + (uint32_t)(D::W_COL0 + ws * D::W_SLOT_COLS);
+          const uint32_t da = act(ws);
+          if (!dn) {
+            // gate from boxes 0, 1 (w1), up from boxes 2, 3 (w3), rows of k-blocks 0, 1
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t bd = sdesc(da + kb * D::ACT_UNIT + kk * 32);
+                const uint32_t acc = (s | kb | kk) ? 1u : 0u;
+                mma_f16_ts(dacc, wcol + kb * 32 + kk * 8, bd, idesc, acc);
+                mma_f16_ts(dacc + NMAX, wcol + (2 + kb) * 32 + kk * 8, bd, idesc, acc);
+              }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk)
+              mma_f16_ts(dacc, wcol + kk * 8, sdesc(da + (kk >> 2) * D::ACT_UNIT + (kk & 3) * 32),
+                         idesc, (s | kk) ? 1u : 0u);
+          }
+          mma_commit(w_empty(ws));
+          issued = true;
+        }
+        if (ok) mma_commit(t_full(b));
+      }
+      if (issued) {
+        mma_commit(final_bar);
+        drain_w8(final_bar, 0, p.status, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 7) {
+    // ---------------- converters: thread = one weight row of box (warp - 7) / 4. The
+    // next stage's barriers are tested before this stage's widening.
+    const int sub = (warp - 7) >> 2, quarter = warp & 3;
+    const int r = 32 * quarter + lane;
+    const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
+    int it = 0;
+    bool ok = true, pre_q = false, pre_w = false;
+    for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+      const int nst = L >= total0 ? st2 : st1;
+      for (int s = 0; s < nst; ++s, ++it) {
+        const int q = it % kQ, ws = it % kW;
+        if (!pre_q && !wait_warp(q_full(q), ph(it, kQ), abort_flag, p.status, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        const int nx = it + 1;
+        pre_q = mbar_test_wait(q_full(nx % kQ), ph(nx, kQ));
+        const uint8_t* box = qbase + q * D::Q_BYTES + sub * D::BOX;
+        uint32_t out[32];
+        if constexpr (BITS == 8) {
+          // chunk v: columns 16 v .. 16 v + 15 of the 128 rows, 16 bytes per row
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint4 c = *reinterpret_cast<const uint4*>(box + v * 2048 + r * 16);
+            uint4 lo8, hi8;
+            widen16(c, lo8, hi8);
+            out[8 * v + 0] = lo8.x;
+            out[8 * v + 1] = lo8.y;
+            out[8 * v + 2] = lo8.z;
+            out[8 * v + 3] = lo8.w;
+            out[8 * v + 4] = hi8.x;
+            out[8 * v + 5] = hi8.y;
+            out[8 * v + 6] = hi8.z;
+            out[8 * v + 7] = hi8.w;
+          }
+        } else {
+          // half hf: columns 32 hf .. 32 hf + 31, one 32-bit word per 8 columns
+          const uint16_t* sc =
+              reinterpret_cast<const uint16_t*>(qbase + q * D::Q_BYTES + D::SUBS * D::BOX + sub * 256);
+          const uint32_t s2 = (uint32_t)sc[r] * 0x10001u;
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const uint4 c = *reinterpret_cast<const uint4*>(box + hf * 2048 + r * 16);
+            widen_word4_pairs(c.x, s2, out + 16 * hf + 0);
+            widen_word4_pairs(c.y, s2, out + 16 * hf + 4);
+            widen_word4_pairs(c.z, s2, out + 16 * hf + 8);
+            widen_word4_pairs(c.w, s2, out + 16 * hf + 12);
+          }
+        }
+        // the codes are in registers: the stage may be refilled
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_empty(q));
+        if (!pre_w && !wait_warp(w_empty(ws), ph(it, kW) ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        pre_w = mbar_test_wait(w_empty(nx % kW), ph(nx, kW) ^ 1u);
+        __syncwarp();
+        fence_after();
+        tmem_st32(tmem_base + lane_addr + (uint32_t)(D::W_COL0 + ws * D::W_SLOT_COLS + sub * 32), out);
+        tmem_wait_st();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(w_full(ws));
+      }
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5, TMEM lanes 32 (warp % 4) .. = weight rows
+    const int quarter = warp & 3;
+    const int r = 32 * quarter + lane;
+    int tc = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x, ++tc) {
+      bool dn;
+      int e, m, n;
+      coords(L, dn, e, m, n);
+      const int nrow = ncols[e];
+      const int b = tc & 1;
+      if (!wait_warp(t_full(b), ph(tc, 2), abort_flag, p.status, p.timeout_ns)) break;
+      fence_after();
+      const uint32_t tacc =
+          tmem_base + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(b * D::ACC_COLS);
+      const int64_t row0 = (int64_t)m * BM;
+      if (!dn) {
+        const int i = n * 128 + r;  // intermediate column
+        const float sg = BITS == 8 ? __ldg(p.s1 + (size_t)e * p.I + i) : 1.f;
+        const float su = BITS == 8 ? __ldg(p.s3 + (size_t)e * p.I + i) : 1.f;
+        uint16_t* hcol = p.h + row0 * p.I + i;
+        for (int c0 = 0; c0 < nrow; c0 += 16) {
+          uint32_t g[16], u[16];
+          tmem_ld16(tacc + c0, g);
+          tmem_ld16(tacc + NMAX + c0, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const float gv = __uint_as_float(g[t]) * sg, uv = __uint_as_float(u[t]) * su;
+            hcol[(int64_t)(c0 + t) * p.I] = half_rn(gv / (1.f + __expf(-gv)) * uv);
+          }
+        }
+        // release this warp's rows of h to the down tiles of row tile m
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(p.row_ready + m, 1);
+      } else {
+        const int j = n * 128 + r;  // hidden column
+        const float sc = BITS == 8 ? __ldg(p.s2 + (size_t)e * p.H + j) : 1.f;
+        float* ycol = p.y + row0 * p.H + j;
+        for (int c0 = 0; c0 < nrow; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(tacc + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 16; ++t) ycol[(int64_t)(c0 + t) * p.H] = __uint_as_float(v[t]) * sc;
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(t_empty(b));
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512u)
+                 : "memory");
+  }
+}
+
 // bf16 rows -> IEEE half rows (round to nearest even), 8 values per thread-step
 __global__ void __launch_bounds__(256) k_rows_to_f16(const uint4* __restrict__ src,
                                                      uint4* __restrict__ dst, int64_t n8) {
@@ -1000,6 +1522,64 @@ cudaError_t launch_swiglu_w8_tiles(const Shape& s, const GemmArgsW8& g, cudaStre
   return e;
 }
 
+// Both GEMMs of a batch of at most NMAX tokens on the swap-operand kernel
+template <int BITS, int NMAX>
+cudaError_t launch_w8_decode(const Shape& s, const GemmArgsW8& g, cudaStream_t st,
+                             const char** why) {
+  using D = DecW8<BITS, NMAX>;
+  CUtensorMap mx, mh;
+  if (!map_act(&mx, g.a, s.H, g.rmax, 16) || !map_act(&mh, g.h, s.I, g.rmax, 16)) {
+    *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad tensor)";
+    return cudaErrorInvalidValue;
+  }
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_w8_decode<BITS, NMAX>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM);
+    if (e != cudaSuccess) {
+      *why = "expert GEMM shared-memory attribute";
+      return e;
+    }
+    attr_set[dev] = true;
+  }
+  DecParams p = {};
+  p.q1 = g.q1;
+  p.q3 = g.q3;
+  p.q2 = g.q2;
+  p.s1 = g.s1;
+  p.s3 = g.s3;
+  p.s2 = g.s2;
+  p.g1 = g.g1;
+  p.g3 = g.g3;
+  p.g2 = g.g2;
+  p.offsets = g.offsets;
+  p.counts = g.counts;
+  p.h = g.h;
+  p.y = g.y;
+  p.status = g.status;
+  p.row_ready = g.row_ready;
+  p.E = s.E;
+  p.H = s.H;
+  p.I = s.I;
+  p.timeout_ns = g.timeout_ns;
+  // the row-tile counters start at zero
+  cudaError_t e = cudaMemsetAsync(g.row_ready, 0, (size_t)(g.rmax / BM) * sizeof(int32_t), st);
+  if (e == cudaSuccess) {
+    // at most one row tile per expert with rows, at most T * k experts with rows
+    const int64_t active = std::min<int64_t>(s.E, (int64_t)s.T * s.k);
+    const int64_t tiles = active * (s.I / 128 + s.H / 128);
+    int64_t grid = std::min<int64_t>(num_sms(), tiles);
+    if (grid < 1) grid = 1;
+    e = launch_pdl(k_w8_decode<BITS, NMAX>, dim3((unsigned)grid), dim3(D::THREADS),
+                   (size_t)D::SMEM, st, mx, mh, p);
+  }
+  if (e != cudaSuccess)
+    *why = BITS == 8 ? "int8 expert GEMMs launch failed" : "4-bit expert GEMMs launch failed";
+  return e;
+}
+
 }  // namespace
 
 cudaError_t launch_grouped_swiglu_w8(const Shape& s, const GemmArgsW8& g, cudaStream_t st,
@@ -1007,6 +1587,17 @@ cudaError_t launch_grouped_swiglu_w8(const Shape& s, const GemmArgsW8& g, cudaSt
   // a token is routed to an expert at most once, so with at most 64 tokens every expert
   // has at most 64 rows, all in the first half of its 128-row tile
   const bool half_tiles = s.T <= 64 && kUseHalfTiles;
+  // with at most 64 tokens, hidden % 128 == 0 and intermediate % 256 == 0, the
+  // swap-operand kernel
+  if (s.T <= 64 && s.H % 128 == 0 && s.I % 256 == 0 && g.row_ready && kUseDecodeKernel) {
+    if (g.bits == 4)
+      return s.T <= 16   ? launch_w8_decode<4, 16>(s, g, st, why)
+             : s.T <= 32 ? launch_w8_decode<4, 32>(s, g, st, why)
+                         : launch_w8_decode<4, 64>(s, g, st, why);
+    return s.T <= 16   ? launch_w8_decode<8, 16>(s, g, st, why)
+           : s.T <= 32 ? launch_w8_decode<8, 32>(s, g, st, why)
+                       : launch_w8_decode<8, 64>(s, g, st, why);
+  }
   if (g.bits == 4)
     return half_tiles ? launch_swiglu_w8_tiles<64, 4>(s, g, st, why)
                       : launch_swiglu_w8_tiles<128, 4>(s, g, st, why);

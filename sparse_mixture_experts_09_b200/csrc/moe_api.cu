@@ -205,6 +205,7 @@ struct SplitK {
   float* partial = nullptr;
   int32_t* sem = nullptr;
   int32_t* row_ready = nullptr;
+  const int32_t* q_counts = nullptr;  // quantised experts: routed rows per expert
 };
 
 moe_status_t run_experts(const Shape& s, const uint16_t* x_perm, const int32_t* offsets,
@@ -232,6 +233,7 @@ moe_status_t run_experts(const Shape& s, const uint16_t* x_perm, const int32_t* 
     g.rmax = max_padded_rows(s);
     g.timeout_ns = kTimeoutNs;
     g.row_ready = split.row_ready;
+    g.counts = split.q_counts;
     e = launch_grouped_swiglu_w8(s, g, st, &why);
   } else {
     GemmArgs g;
@@ -268,6 +270,7 @@ moe_status_t run_forward(const Shape& s, const uint16_t* x, const uint16_t* wr, 
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   SplitK split;
   split.row_ready = at<int32_t>(ws, L.row_ready);
+  split.q_counts = at<int32_t>(ws, L.counts);
   if (L.partial != L.end) {
     split.counts = at<int32_t>(ws, L.counts);
     split.partial = at<float>(ws, L.partial);

@@ -124,6 +124,9 @@ struct GemmArgsW8 {
   unsigned long long timeout_ns = 0;
   // [rmax / 128] int32 scratch: given, both GEMMs run as one grid (hidden % 256 == 0)
   int32_t* row_ready = nullptr;
+  // [E] routed rows per expert (nullable): at most 64 tokens, they size each expert's
+  // tiles (16-row steps); null: every expert is sized for the whole batch
+  const int32_t* counts = nullptr;
 };
 
 // GEMM1 (int8 or 4-bit gate/up + SwiGLU -> h) then GEMM2 (h q2^T -> y), in float16.
