@@ -156,6 +156,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -503,9 +514,10 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer
+      // ---------------- MMA issuer (the next stage's barriers are tested before this
+      // stage's MMAs issue, so their latency runs under the MMAs)
       int it = 0, tc = 0;
-      bool ok = true, issued = false;
+      bool ok = true, issued = false, pre_a = false, pre_b = false;
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tc) {
         const int a = tc & 1;
         const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
@@ -515,14 +527,16 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
         const int k_blocks = kblocks(L);
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
           const int sa = it % kAStages, sb = it % kBStages;
-          if (!wait_w8(a_full(sa), (uint32_t)(it / kAStages) & 1u, abort_flag, p.status,
-                       p.timeout_ns) ||
-              !wait_w8(b_full(sb), (uint32_t)(it / kBStages) & 1u, abort_flag, p.status,
-                       p.timeout_ns)) {
+          if ((!pre_a && !wait_w8(a_full(sa), (uint32_t)(it / kAStages) & 1u, abort_flag,
+                                  p.status, p.timeout_ns)) ||
+              (!pre_b && !wait_w8(b_full(sb), (uint32_t)(it / kBStages) & 1u, abort_flag,
+                                  p.status, p.timeout_ns))) {
             ok = false;
             break;
           }
           fence_after();
+          pre_a = mbar_test_wait(a_full((it + 1) % kAStages), (uint32_t)((it + 1) / kAStages) & 1u);
+          pre_b = mbar_test_wait(b_full((it + 1) % kBStages), (uint32_t)((it + 1) / kBStages) & 1u);
           const uint32_t da = smem_u32(smem + sa * A_BYTES);
           const uint32_t db = smem_u32(bbase + sb * TL::B_BYTES);
 #pragma unroll
@@ -808,17 +822,6 @@ struct DecW8 {
   static_assert(SMEM <= 232448, "shared memory plan exceeds 227 KiB");
 };
 
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
 
 struct DecParams {
   const uint8_t* q1;
