@@ -843,13 +843,110 @@ struct DecParams {
   unsigned long long timeout_ns;
 };
 
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
-                                           uint32_t idesc, uint32_t accumulate) {
+// The sixteen MMAs of a gate/up stage in one asm block (few instructions per MMA: the
+// issuing thread shares its scheduler with the converter warps). Gate: boxes 0, 1 at
+// TMEM columns a + 0 .. 63, up: boxes 2, 3 at a + 64 .. 127; rows of k-block kb at the
+// B descriptor + kb * unit16 (the unit in 16-byte steps); a K step moves A by 8
+// columns and the B descriptor by 2 (32 bytes). Only the stage's first MMA of each
+// accumulator honours `acc` (0 starts the tile); the others accumulate.
+template <int UNIT16>
+__device__ __forceinline__ void mma_stage_gate_up(uint32_t d_gate, uint32_t d_up, uint32_t a,
+                                                  uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+      "{\n\t.reg .pred p0, p1;\n\t.reg .b32 ag, au;\n\t.reg .b64 bk;\n\t"
+      "setp.ne.b32 p0, %5, 0;\n\tsetp.eq.b32 p1, %5, %5;\n\t"
+      "mov.b64 bk, %3;\n\t"
+      "add.u32 ag, %2, 0;\n\tadd.u32 au, %2, 64;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p0;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ag, %2, 8;\n\tadd.u32 au, %2, 72;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ag, %2, 16;\n\tadd.u32 au, %2, 80;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ag, %2, 24;\n\tadd.u32 au, %2, 88;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p1;\n\t"
+      "add.s64 bk, %3, %6;\n\t"
+      "add.u32 ag, %2, 32;\n\tadd.u32 au, %2, 96;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ag, %2, 40;\n\tadd.u32 au, %2, 104;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ag, %2, 48;\n\tadd.u32 au, %2, 112;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ag, %2, 56;\n\tadd.u32 au, %2, 120;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p1;\n\t"
+      "}" ::"r"(d_gate), "r"(d_up), "r"(a), "l"(b), "r"(idesc), "r"(acc), "n"(UNIT16)
+      : "memory");
+}
+
+// The sixteen MMAs of a down stage in one asm block: boxes 0..3 are k-blocks 0..3 at
+// TMEM columns a + 32 j, their rows at the B descriptor + j * unit16.
+template <int UNIT16>
+__device__ __forceinline__ void mma_stage_down(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
+                                               uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t.reg .b32 ak;\n\t.reg .b64 bk;\n\t"
+      "setp.ne.b32 p0, %4, 0;\n\tsetp.eq.b32 p1, %4, %4;\n\t"
+      "mov.b64 bk, %2;\n\tmov.b32 ak, %1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p0;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "add.s64 bk, bk, %6;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "add.s64 bk, bk, %6;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "add.s64 bk, bk, %6;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "add.s64 bk, bk, 2;\n\t"
+      "add.u32 ak, ak, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
+      "}" ::"r"(d), "r"(a), "l"(b), "r"(idesc), "r"(acc), "n"(UNIT16), "n"(UNIT16 - 6)
       : "memory");
 }
 
@@ -1098,24 +1195,11 @@ __global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
           pre_w = mbar_test_wait(w_full((it + 1) % kW), ph(it + 1, kW));
           pre_a = mbar_test_wait(a_full((it + 1) % kW), ph(it + 1, kW));
           const uint32_t wcol = tmem_base + (uint32_t)(D::W_COL0 + ws * D::W_SLOT_COLS);
-          const uint32_t da = act(ws);
-          if (!dn) {
-            // gate from boxes 0, 1 (w1), up from boxes 2, 3 (w3), rows of k-blocks 0, 1
-#pragma unroll
-            for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t bd = sdesc(da + kb * D::ACT_UNIT + kk * 32);
-                const uint32_t acc = (s | kb | kk) ? 1u : 0u;
-                mma_f16_ts(dacc, wcol + kb * 32 + kk * 8, bd, idesc, acc);
-                mma_f16_ts(dacc + NMAX, wcol + (2 + kb) * 32 + kk * 8, bd, idesc, acc);
-              }
-          } else {
-#pragma unroll
-            for (int kk = 0; kk < 16; ++kk)
-              mma_f16_ts(dacc, wcol + kk * 8, sdesc(da + (kk >> 2) * D::ACT_UNIT + (kk & 3) * 32),
-                         idesc, (s | kk) ? 1u : 0u);
-          }
+          const uint64_t bd = sdesc(act(ws));
+          if (!dn)  // gate from boxes 0, 1 (w1), up from boxes 2, 3 (w3)
+            mma_stage_gate_up<D::ACT_UNIT / 16>(dacc, dacc + NMAX, wcol, bd, idesc, s ? 1u : 0u);
+          else
+            mma_stage_down<D::ACT_UNIT / 16>(dacc, wcol, bd, idesc, s ? 1u : 0u);
           mma_commit(w_empty(ws));
           issued = true;
         }
