@@ -100,7 +100,8 @@ def test_grouped_swiglu_w4_matches_oracle(name):
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged", "e5k3", "one_token", "skewed", "bn128_split",
-                                  "ts_t33", "ts_e64k8", "ts_h640", "ts_k1", "t64_edge", "t65_edge"])
+                                  "ts_t33", "ts_e64k8", "ts_h640", "ts_k1", "t64_edge", "t65_edge",
+                                  "t17_e4", "t24_e2", "t48_e2"])
 def test_forward_w4_matches_oracle(name):
     w = CASES[name]
     inp, near = screened(w)
@@ -120,9 +121,9 @@ def test_forward_w4_matches_oracle(name):
         assert_layer_close(O.to_f64(out.cpu()), ref["out"], name)
 
 
-@pytest.mark.parametrize("name", ["decode", "prefill"])
+@pytest.mark.parametrize("name", ["decode", "prefill", "larger_decode_T1", "larger_decode_T64"])
 def test_forward_w4_full_size_against_oracle(name):
-    w = W.WORKLOADS[name]
+    w = W.workload(name)
     inp, near = screened(w)
     assert near.numel() == 0
     ex = M.quantize_int4(inp.w1, inp.w3, inp.w2)

@@ -73,6 +73,11 @@ SMALL_BATCH = {
     # 64 tokens is the last batch on 64-row tiles; 65 takes the 128-row tiles
     "t64_edge": W.Workload("t64_edge", 64, 256, 256, 2, 2, seed=35),
     "t65_edge": W.Workload("t65_edge", 65, 256, 256, 2, 2, seed=36),
+    # the swap-operand kernel's row widths: 17 and 24 tokens take its 32-row variant (24
+    # rows per expert: N = 32), 48 tokens its 64-row variant with N = 48
+    "t17_e4": W.Workload("t17_e4", 17, 512, 512, 4, 2, seed=37),
+    "t24_e2": W.Workload("t24_e2", 24, 256, 512, 2, 2, seed=38),
+    "t48_e2": W.Workload("t48_e2", 48, 384, 768, 2, 2, seed=39),
 }
 CASES = {**SMALL, **SMALL_BATCH}
 
@@ -100,7 +105,8 @@ def test_grouped_swiglu_w8_matches_oracle(name):
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged", "e5k3", "one_token", "skewed", "bn128_split",
-                                  "ts_t33", "ts_e64k8", "ts_h640", "t64_edge", "t65_edge"])
+                                  "ts_t33", "ts_e64k8", "ts_h640", "t64_edge", "t65_edge",
+                                  "t17_e4", "t24_e2", "t48_e2"])
 def test_forward_w8_matches_oracle(name):
     w = CASES[name]
     inp, near = screened(w)
@@ -120,9 +126,9 @@ def test_forward_w8_matches_oracle(name):
         assert_layer_close(O.to_f64(out.cpu()), ref["out"], name)
 
 
-@pytest.mark.parametrize("name", ["decode", "prefill"])
+@pytest.mark.parametrize("name", ["decode", "prefill", "larger_decode_T1", "larger_decode_T64"])
 def test_forward_w8_full_size_against_oracle(name):
-    w = W.WORKLOADS[name]
+    w = W.workload(name)
     inp, near = screened(w)
     assert near.numel() == 0
     ex = M.quantize_int8(inp.w1, inp.w3, inp.w2)
