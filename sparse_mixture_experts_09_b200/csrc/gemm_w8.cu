@@ -773,9 +773,10 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
 //   warp 6      loads the routed rows' k-blocks (TMA, 16-row boxes, 128-byte swizzle);
 //               a down tile first waits until every gate/up tile of its row tile has
 //               released its rows of h (per-row-tile counters);
-//   warp 1      issues tcgen05.mma with A in tensor memory and B (the rows) in shared
-//               memory, M = 128, N = rows: gate/up into two accumulators (gate, up),
-//               down into one;
+//   warps 1, 23 issue tcgen05.mma with A in tensor memory and B (the rows) in shared
+//               memory, M = 128, N = rows, each half of every stage: gate/up the first
+//               issues gate and the second up, down each issues two of the four k-blocks
+//               into its own partial sum (the epilogue adds the two);
 //   warps 2-5   read the accumulators (lane = weight row, column = routed row): h =
 //               half(silu(s1 gate) * s3 up) at [row, i], y = s2 acc at [row, j].
 //
@@ -794,7 +795,9 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
 // the pace of small stages. So a stage is 128 columns of K (sixteen MMAs), each role
 // tests the barriers of its next stage with test_wait before it starts the current one
 // (the latency runs under its work) and blocks only if that test failed. (3) Separate
-// accumulators per MMA do not help (the pipe is not waiting on accumulation).
+// accumulators per MMA do not help (the pipe is not waiting on accumulation), but a
+// second issuing thread does: two threads issue N = 16 MMAs at about 38 clocks each
+// against 51 for one, so two threads split every stage.
 template <int BITS, int NMAX>
 struct DecW8 {
   static constexpr int BOX = 128 * BK * BITS / 8;                  // code bytes of a box
@@ -809,10 +812,11 @@ struct DecW8 {
   static constexpr int Q_FIT = (200 * 1024 - W_SLOTS * ACT_SLOT) / Q_BYTES;
   static constexpr int Q_ST = Q_FIT > 16 ? 16 : Q_FIT;
   static constexpr int CONV_WARPS = 4 * SUBS;                      // one box per warp
-  static constexpr int THREADS = 32 * (7 + CONV_WARPS);
+  static constexpr int MMA_WARP2 = 7 + CONV_WARPS;                 // the second MMA issuer
+  static constexpr int THREADS = 32 * (8 + CONV_WARPS);
   static constexpr int Q_OFF = W_SLOTS * ACT_SLOT;
   static constexpr int BAR_OFF = Q_OFF + Q_ST * Q_BYTES;
-  static constexpr int NUM_BARS = 2 * Q_ST + 3 * W_SLOTS + 4 + 1;
+  static constexpr int NUM_BARS = 2 * Q_ST + 3 * W_SLOTS + 4 + 2;
   static constexpr int SMEM = 1024 + BAR_OFF + NUM_BARS * 8 + 16 + 2 * 72 * 4;
   // D f32, A and B f16, both K-major, M = 128; N is set per tile
   static constexpr uint32_t IDESC_M128 = (1u << 4) | ((uint32_t)(128 >> 4) << 24);
@@ -843,58 +847,12 @@ struct DecParams {
   unsigned long long timeout_ns;
 };
 
-// The sixteen MMAs of a gate/up stage in one asm block (few instructions per MMA: the
-// issuing thread shares its scheduler with the converter warps). Gate: boxes 0, 1 at
-// TMEM columns a + 0 .. 63, up: boxes 2, 3 at a + 64 .. 127; rows of k-block kb at the
-// B descriptor + kb * unit16 (the unit in 16-byte steps); a K step moves A by 8
-// columns and the B descriptor by 2 (32 bytes). Only the stage's first MMA of each
-// accumulator honours `acc` (0 starts the tile); the others accumulate.
+// Eight MMAs of one issuer's half of a stage in one asm block: boxes j = 0, 1 at TMEM
+// columns a + 32 j, the rows of k-block j at the B descriptor + j * unit16; a K step
+// moves A by 8 columns and the B descriptor by 2 (32 bytes). Only the first MMA honours
+// `acc` (0 starts the tile's accumulator); the others accumulate.
 template <int UNIT16>
-__device__ __forceinline__ void mma_stage_gate_up(uint32_t d_gate, uint32_t d_up, uint32_t a,
-                                                  uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p0, p1;\n\t.reg .b32 ag, au;\n\t.reg .b64 bk;\n\t"
-      "setp.ne.b32 p0, %5, 0;\n\tsetp.eq.b32 p1, %5, %5;\n\t"
-      "mov.b64 bk, %3;\n\t"
-      "add.u32 ag, %2, 0;\n\tadd.u32 au, %2, 64;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p0;\n\t"
-      "add.s64 bk, bk, 2;\n\t"
-      "add.u32 ag, %2, 8;\n\tadd.u32 au, %2, 72;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p1;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p1;\n\t"
-      "add.s64 bk, bk, 2;\n\t"
-      "add.u32 ag, %2, 16;\n\tadd.u32 au, %2, 80;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p1;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p1;\n\t"
-      "add.s64 bk, bk, 2;\n\t"
-      "add.u32 ag, %2, 24;\n\tadd.u32 au, %2, 88;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p1;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p1;\n\t"
-      "add.s64 bk, %3, %6;\n\t"
-      "add.u32 ag, %2, 32;\n\tadd.u32 au, %2, 96;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p1;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p1;\n\t"
-      "add.s64 bk, bk, 2;\n\t"
-      "add.u32 ag, %2, 40;\n\tadd.u32 au, %2, 104;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p1;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p1;\n\t"
-      "add.s64 bk, bk, 2;\n\t"
-      "add.u32 ag, %2, 48;\n\tadd.u32 au, %2, 112;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p1;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p1;\n\t"
-      "add.s64 bk, bk, 2;\n\t"
-      "add.u32 ag, %2, 56;\n\tadd.u32 au, %2, 120;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ag], bk, %4, p1;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%1], [au], bk, %4, p1;\n\t"
-      "}" ::"r"(d_gate), "r"(d_up), "r"(a), "l"(b), "r"(idesc), "r"(acc), "n"(UNIT16)
-      : "memory");
-}
-
-// The sixteen MMAs of a down stage in one asm block: boxes 0..3 are k-blocks 0..3 at
-// TMEM columns a + 32 j, their rows at the B descriptor + j * unit16.
-template <int UNIT16>
-__device__ __forceinline__ void mma_stage_down(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
+__device__ __forceinline__ void mma_stage_half(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
                                                uint32_t acc) {
   asm volatile(
       "{\n\t.reg .pred p0, p1;\n\t.reg .b32 ak;\n\t.reg .b64 bk;\n\t"
@@ -910,7 +868,7 @@ __device__ __forceinline__ void mma_stage_down(uint32_t d, uint32_t a, uint64_t 
       "add.s64 bk, bk, 2;\n\t"
       "add.u32 ak, ak, 8;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
-      "add.s64 bk, bk, %6;\n\t"
+      "add.s64 bk, bk, %5;\n\t"
       "add.u32 ak, ak, 8;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
       "add.s64 bk, bk, 2;\n\t"
@@ -922,31 +880,7 @@ __device__ __forceinline__ void mma_stage_down(uint32_t d, uint32_t a, uint64_t 
       "add.s64 bk, bk, 2;\n\t"
       "add.u32 ak, ak, 8;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
-      "add.s64 bk, bk, %6;\n\t"
-      "add.u32 ak, ak, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
-      "add.s64 bk, bk, 2;\n\t"
-      "add.u32 ak, ak, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
-      "add.s64 bk, bk, 2;\n\t"
-      "add.u32 ak, ak, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
-      "add.s64 bk, bk, 2;\n\t"
-      "add.u32 ak, ak, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
-      "add.s64 bk, bk, %6;\n\t"
-      "add.u32 ak, ak, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
-      "add.s64 bk, bk, 2;\n\t"
-      "add.u32 ak, ak, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
-      "add.s64 bk, bk, 2;\n\t"
-      "add.u32 ak, ak, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
-      "add.s64 bk, bk, 2;\n\t"
-      "add.u32 ak, ak, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], bk, %3, p1;\n\t"
-      "}" ::"r"(d), "r"(a), "l"(b), "r"(idesc), "r"(acc), "n"(UNIT16), "n"(UNIT16 - 6)
+      "}" ::"r"(d), "r"(a), "l"(b), "r"(idesc), "r"(acc), "n"(UNIT16 - 6)
       : "memory");
 }
 
@@ -1024,7 +958,7 @@ __global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
   auto w_empty = [&](int s) { return bar0 + 8u * (kW0 + 2 * kW + s); };
   auto t_full = [&](int b) { return bar0 + 8u * (kT0 + b); };
   auto t_empty = [&](int b) { return bar0 + 8u * (kT0 + 2 + b); };
-  const uint32_t final_bar = bar0 + 8u * (kT0 + 4);
+  const uint32_t final_bar = bar0 + 8u * (kT0 + 4);  // and final_bar + 8: one per issuer
   auto act = [&](int ws) { return smem_u32(smem + ws * D::ACT_SLOT); };
   const int kb1 = p.H / BK, kb2 = p.I / BK;  // k-blocks of the gate/up and down weights
   // phase parity of the barrier a stage uses (ring of n), and of its previous use
@@ -1038,13 +972,14 @@ __global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
     for (int s = 0; s < kW; ++s) {
       mbar_init(w_full(s), D::CONV_WARPS);
       mbar_init(a_full(s), 1);
-      mbar_init(w_empty(s), 1);
+      mbar_init(w_empty(s), 2);  // both issuers' commits
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(t_full(b), 1);
+      mbar_init(t_full(b), 2);
       mbar_init(t_empty(b), 4);
     }
     mbar_init(final_bar, 1);
+    mbar_init(final_bar + 8u, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -1168,10 +1103,12 @@ __global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == D::MMA_WARP2) {
     if (lane == 0) {
-      // ---------------- MMA issuer. The next stage's barriers are tested before this
-      // stage's MMAs issue, so their latency runs under the MMAs.
+      // ---------------- MMA issuers (mi = 0, 1), each half of every stage. The next
+      // stage's barriers are tested before this stage's MMAs issue, so their latency
+      // runs under the MMAs.
+      const int mi = warp == 1 ? 0 : 1;
       int it = 0, tc = 0;
       bool ok = true, issued = false, pre_w = false, pre_a = false;
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tc) {
@@ -1194,24 +1131,25 @@ __global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
           fence_after();
           pre_w = mbar_test_wait(w_full((it + 1) % kW), ph(it + 1, kW));
           pre_a = mbar_test_wait(a_full((it + 1) % kW), ph(it + 1, kW));
-          const uint32_t wcol = tmem_base + (uint32_t)(D::W_COL0 + ws * D::W_SLOT_COLS);
-          const uint64_t bd = sdesc(act(ws));
-          if (!dn)  // gate from boxes 0, 1 (w1), up from boxes 2, 3 (w3)
-            mma_stage_gate_up<D::ACT_UNIT / 16>(dacc, dacc + NMAX, wcol, bd, idesc, s ? 1u : 0u);
-          else
-            mma_stage_down<D::ACT_UNIT / 16>(dacc, wcol, bd, idesc, s ? 1u : 0u);
+          // gate/up: issuer 0 gate (boxes 0, 1: w1), issuer 1 up (boxes 2, 3: w3), both
+          // over the rows of k-blocks 0, 1; down: issuer mi boxes (k-blocks) 2 mi, 2 mi + 1
+          // into partial sum mi
+          const uint32_t wcol =
+              tmem_base + (uint32_t)(D::W_COL0 + ws * D::W_SLOT_COLS + mi * 64);
+          const uint64_t bd = sdesc(act(ws) + (dn ? mi * 2 * D::ACT_UNIT : 0));
+          mma_stage_half<D::ACT_UNIT / 16>(dacc + mi * NMAX, wcol, bd, idesc, s ? 1u : 0u);
           mma_commit(w_empty(ws));
           issued = true;
         }
         if (ok) mma_commit(t_full(b));
       }
       if (issued) {
-        mma_commit(final_bar);
-        drain_w8(final_bar, 0, p.status, p.timeout_ns);
+        mma_commit(final_bar + 8u * mi);
+        drain_w8(final_bar + 8u * mi, 0, p.status, p.timeout_ns);
       }
     }
     __syncwarp();
-  } else if (warp >= 7) {
+  } else if (warp >= 7 && warp < D::MMA_WARP2) {
     // ---------------- converters: thread = one weight row of box (warp - 7) / 4. The
     // next stage's barriers are tested before this stage's widening.
     const int sub = (warp - 7) >> 2, quarter = warp & 3;
@@ -1320,11 +1258,13 @@ __global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
         const float sc = BITS == 8 ? __ldg(p.s2 + (size_t)e * p.H + j) : 1.f;
         float* ycol = p.y + row0 * p.H + j;
         for (int c0 = 0; c0 < nrow; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld16(tacc + c0, v);
+          uint32_t v0[16], v1[16];
+          tmem_ld16(tacc + c0, v0);
+          tmem_ld16(tacc + NMAX + c0, v1);
           tmem_wait_ld();
 #pragma unroll
-          for (int t = 0; t < 16; ++t) ycol[(int64_t)(c0 + t) * p.H] = __uint_as_float(v[t]) * sc;
+          for (int t = 0; t < 16; ++t)
+            ycol[(int64_t)(c0 + t) * p.H] = (__uint_as_float(v0[t]) + __uint_as_float(v1[t])) * sc;
         }
       }
       fence_before();
