@@ -318,6 +318,24 @@ def layer_roofline(w, ms, counts, peaks, peak_kind, long_run):
             "measured_peak_source": peak_kind, "algorithmic_bytes": bytes_}
 
 
+def quant_layer_roofline(w, ms, counts, peaks, peak_kind, bits):
+    """Whole-layer fraction of the HBM roofline for weight-only int8 (bits = 8) or 4-bit
+    (bits = 4, plus one 2-byte scale per 64 weights) experts: the active experts' code
+    and scale bytes plus the activations' bytes, over the step time. The int8 per-row
+    fp32 scales (4 bytes per weight row) are counted too."""
+    H, I, k, T, E = (w.hidden_size, w.intermediate_size, w.num_experts_per_tok, w.num_tokens,
+                     w.num_experts)
+    n_active = int(sum(1 for c in counts if c > 0))
+    elems = 3 * H * I  # weights per expert
+    per_expert = elems * bits // 8 + (elems // 64 * 2 if bits == 4 else (2 * I + H) * 4)
+    bytes_ = n_active * per_expert + 3 * T * H * 2 + E * H * 2 + T * k * 8
+    achieved = bytes_ / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "unit": "GB/s",
+            "nominal_peak": NOMINAL["hbm_gbs"], "frac_of_nominal": achieved / NOMINAL["hbm_gbs"],
+            "measured_peak": peaks["hbm_gbs"], "frac_of_measured": achieved / peaks["hbm_gbs"],
+            "measured_peak_source": peak_kind, "algorithmic_bytes": bytes_}
+
+
 def near_tie_tokens(logits, k, margin=1e-2):
     """Tokens whose float32 router logits have a gap below ``margin`` between any two
     neighbours among their k + 1 largest (the ranks that decide the top-k and its slot
@@ -612,6 +630,8 @@ def run_ours(args):
                              "value": job_throughput(w.num_tokens, world, w8_ms),
                              "api": "moe_forward_w8",
                              "weight_gb_per_step": n_active * w.expert_bytes() / 2e9,
+                             "layer_roofline": quant_layer_roofline(w, w8_ms, counts, peaks,
+                                                                    peak_kind, 8),
                              "note": "weight-only int8 experts, half-precision expert math, "
                                      "quantised once at load (untimed); not the headline"},
             "int4_experts": {"ms_per_step": w4_ms,
@@ -619,6 +639,8 @@ def run_ours(args):
                              "api": "moe_forward_w4",
                              "weight_gb_per_step": (n_active * w.expert_bytes()
                                                     * (1 / 4 + 1 / 64) / 1e9),
+                             "layer_roofline": quant_layer_roofline(w, w4_ms, counts, peaks,
+                                                                    peak_kind, 4),
                              "note": "weight-only 4-bit experts (a half scale per 64-column "
                                      "group), half-precision expert math, quantised once at "
                                      "load (untimed); not the headline"},

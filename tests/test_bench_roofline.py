@@ -140,3 +140,22 @@ def test_layer_roofline_against_nominal_and_measured_peaks():
     assert r["algorithmic_flops"] == flops
     # the prefill target: 60% of 2.25 PFLOP/s is a 2.14 ms layer
     assert abs(r["frac_of_nominal"] - 0.6) < 0.002
+
+
+def test_quantised_layer_roofline_counts_codes_and_scales():
+    # decode workload, all 8 experts active: int8 codes are 1 byte per weight plus 4-byte
+    # row scales, 4-bit codes half a byte plus one 2-byte scale per 64 weights
+    w = W.WORKLOADS["decode"]
+    H, I, T = w.hidden_size, w.intermediate_size, w.num_tokens
+    peaks = {"hbm_gbs": 6556.0}
+    acts = 3 * T * H * 2 + w.num_experts * H * 2 + T * 2 * 8
+    r8 = bench.quant_layer_roofline(w, 1.0, [1] * 8, peaks, "measured", 8)
+    assert r8["algorithmic_bytes"] == 8 * (3 * H * I + (2 * I + H) * 4) + acts
+    r4 = bench.quant_layer_roofline(w, 1.0, [1] * 8, peaks, "measured", 4)
+    assert r4["algorithmic_bytes"] == 8 * (3 * H * I // 2 + 3 * H * I // 32) + acts
+    # 1 ms per step: GB/s = bytes / 1e6
+    assert abs(r8["achieved"] - r8["algorithmic_bytes"] / 1e6) < 1e-6
+    assert r4["bound"] == "hbm" and abs(r4["frac_of_measured"] - r4["achieved"] / 6556.0) < 1e-12
+    # inactive experts carry no weight bytes
+    r8_two = bench.quant_layer_roofline(w, 1.0, [3, 0, 0, 0, 0, 0, 0, 2], peaks, "measured", 8)
+    assert r8_two["algorithmic_bytes"] == 2 * (3 * H * I + (2 * I + H) * 4) + acts
