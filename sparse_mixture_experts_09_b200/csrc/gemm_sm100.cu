@@ -1003,6 +1003,381 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------- small batches
+//
+// k_decode_swap: both expert GEMMs of a batch of at most 64 tokens in one persistent
+// grid, with the operands swapped: the weights are the tcgen05 M operand (128 weight
+// rows per tile, loaded by TMA straight into the 128-byte swizzled K-major layout the
+// MMA reads) and the expert's routed rows the N operand (N = its row count rounded up to
+// 16; a token reaches an expert at most once, so each expert has at most T rows, in one
+// 128-row tile). A stage holds four 128 x 64 weight boxes (gate/up: the w1 and w3 boxes
+// of two k-blocks; down: four k-blocks of one w2 box; 64 KiB) and its k-blocks of rows.
+// Against the tile kernels this moves 2 KiB of routed rows per 64 KiB of weights
+// instead of a 16 KiB activation tile per 32 KiB, and runs both GEMMs as one grid.
+//
+//   warp 0      weight boxes (TMA);
+//   warp 6      routed rows (TMA, 16-row boxes); a down tile first waits until every
+//               gate/up tile of its row tile has released its rows of h;
+//   warps 1, 7  issue the MMAs (M = 128, N = rows): gate/up the first issues gate, the
+//               second up; down each issues two of the four k-blocks into its own
+//               partial sum;
+//   warps 2-5   read the accumulators (lane = weight row, column = routed row): h =
+//               bf16(silu(gate) * up) at [row, i], y = the two partial sums' sum at
+//               [row, j].
+// Each role tests its next stage's barriers with test_wait before starting the current
+// one (measured on B200: a wait whose result steers the MMA thread costs about 340 SM
+// clocks between MMAs). Every gate/up tile precedes every down tile in the order each
+// CTA walks its tiles and the grid is at most one CTA per SM, so a down tile only waits
+// for tiles that are running or done.
+template <int NMAX>
+struct DecBf16 {
+  static constexpr int WBOX = 128 * BK * 2;                    // one 128 x 64 weight box
+  static constexpr int ACT_UNIT = NMAX * 128;                  // NMAX rows of one k-block
+  static constexpr int STAGE = 4 * WBOX + 4 * ACT_UNIT;
+  static constexpr int STAGES = (220 * 1024) / STAGE;          // 3 (NMAX 16) or 2 (32, 64)
+  static constexpr int ACC_COLS = 2 * NMAX;                    // gate, up (or two partials)
+  static constexpr int TMEM_COLS =
+      2 * ACC_COLS <= 32 ? 32 : (2 * ACC_COLS <= 64 ? 64 : (2 * ACC_COLS <= 128 ? 128 : 256));
+  static constexpr int NUM_BARS = 3 * STAGES + 6;
+  static constexpr int SMEM = 1024 + STAGES * STAGE + NUM_BARS * 8 + 16 + 2 * 72 * 4;
+  // D f32, A and B bf16, both K-major, M = 128; N is set per tile
+  static constexpr uint32_t IDESC_M128 =
+      (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 4) << 24);
+  static_assert(NMAX == 16 || NMAX == 32 || NMAX == 64, "rows per expert");
+  static_assert(STAGES >= 2 && STAGE % 1024 == 0, "stage plan");
+  static_assert(SMEM <= 232448, "shared memory plan exceeds 227 KiB");
+};
+
+struct DecBf16Params {
+  const int32_t* offsets;  // [E+1], multiples of 128
+  const int32_t* counts;   // [E] routed rows per expert, or null (then NMAX rows)
+  uint16_t* h;             // [rows, I] bf16
+  float* y;                // [rows, H] fp32
+  int32_t* status;
+  int32_t* row_ready;      // [rows / 128], zero at launch
+  int E, H, I, blocked;
+  unsigned long long timeout_ns;
+};
+
+// Tile L -> (expert e, row tile m, column tile n) of a grid whose tiles are n_tiles per
+// row tile (one row tile per expert with rows at these batch sizes)
+__device__ __forceinline__ void swap_coords(int L, const int* row_tiles, int E, int n_tiles,
+                                            int& e, int& m, int& n) {
+  const int mrow = L / n_tiles;
+  e = 0;
+  while (e + 1 < E && row_tiles[e + 1] <= mrow) ++e;
+  const int cnt = row_tiles[e + 1] - row_tiles[e];
+  const int local = L - row_tiles[e] * n_tiles;
+  n = local / cnt;
+  m = row_tiles[e] + local % cnt;
+}
+
+// Wait until *ready >= target (acquire: the h rows stored before the release are then
+// visible), bounded like the barrier waits.
+__device__ __noinline__ bool wait_count(const int32_t* ready, int target, volatile int* abort_flag,
+                                        int32_t* status, unsigned long long timeout_ns) {
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t n = 0;; ++n) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ready) : "memory");
+    if (v >= target) return true;
+    __nanosleep(64);
+    if ((n & 63u) == 63u) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > timeout_ns) {
+        *abort_flag = 1;
+        atomicOr(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+template <int NMAX>
+__global__ void __launch_bounds__(256, 1)
+    k_decode_swap(const __grid_constant__ CUtensorMap mw1, const __grid_constant__ CUtensorMap mw3,
+                  const __grid_constant__ CUtensorMap mw2, const __grid_constant__ CUtensorMap mx,
+                  const __grid_constant__ CUtensorMap mh, const __grid_constant__ DecBf16Params p) {
+  using D = DecBf16<NMAX>;
+  constexpr int kS = D::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kS * D::STAGE);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + D::NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* row_tiles = reinterpret_cast<int*>(tmem_holder + 4);  // [E + 1]
+  int* ncols = row_tiles + 72;                                // [E]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // barriers: w_full (weights), a_full (rows), empty (both; the two issuers' commits) [kS];
+  // t_full, t_empty [2]; final [2] (one per issuer)
+  const uint32_t bar0 = smem_u32(bars);
+  auto w_full = [&](int s) { return bar0 + 8u * s; };
+  auto a_full = [&](int s) { return bar0 + 8u * (kS + s); };
+  auto empty = [&](int s) { return bar0 + 8u * (2 * kS + s); };
+  auto t_full = [&](int b) { return bar0 + 8u * (3 * kS + b); };
+  auto t_empty = [&](int b) { return bar0 + 8u * (3 * kS + 2 + b); };
+  const uint32_t final_bar = bar0 + 8u * (3 * kS + 4);
+  auto stage = [&](int s) { return smem_u32(smem + s * D::STAGE); };
+  auto ph = [](int it, int n) { return (uint32_t)(it / n) & 1u; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kS; ++s) {
+      mbar_init(w_full(s), 1);
+      mbar_init(a_full(s), 1);
+      mbar_init(empty(s), 2);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(t_full(b), 2);
+      mbar_init(t_empty(b), 4);
+    }
+    mbar_init(final_bar, 1);
+    mbar_init(final_bar + 8u, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (threadIdx.x == 32) {
+    prefetch_map(&mw1);
+    prefetch_map(&mw3);
+    prefetch_map(&mw2);
+    prefetch_map(&mx);
+    prefetch_map(&mh);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"((uint32_t)D::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  pdl_trigger();
+  pdl_wait();
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) row_tiles[i] = p.offsets[i] / BM;
+  for (int i = threadIdx.x; i < p.E; i += blockDim.x) {
+    int n = NMAX;
+    if (p.counts) {
+      n = (p.counts[i] + 15) & ~15;
+      n = n < 16 ? 16 : (n > NMAX ? NMAX : n);
+    }
+    ncols[i] = n;
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int n1 = p.I / 128, n2 = p.H / 128;          // column tiles per row tile
+  const int kb1 = p.H / BK, kb2 = p.I / BK;          // k-blocks of w1/w3 and of w2
+  const int st1 = kb1 / 2, st2 = kb2 / 4;            // stages per tile
+  const int total0 = row_tiles[p.E] * n1;
+  const int total = total0 + row_tiles[p.E] * n2;
+  auto coords = [&](int L, bool& dn, int& e, int& m, int& n) {
+    dn = L >= total0;
+    swap_coords(dn ? L - total0 : L, row_tiles, p.E, dn ? n2 : n1, e, m, n);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- weight boxes
+      int it = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        bool dn;
+        int e, m, n;
+        coords(L, dn, e, m, n);
+        const int nst = dn ? st2 : st1;
+        for (int s = 0; s < nst; ++s, ++it) {
+          const int q = it % kS;
+          if (!wait_phase(empty(q), ph(it, kS) ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(w_full(q), 4 * D::WBOX);
+          const uint32_t dst = stage(q);
+          int wx, wy;
+          if (!dn) {
+            // boxes 0, 1: w1 rows 128 n .. of expert e, k-blocks 2s, 2s + 1; boxes 2, 3: w3
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              wcoord(2 * s + j, e * p.I + n * 128, kb1, p.blocked, wx, wy);
+              tma_load_2d(dst + j * D::WBOX, &mw1, wx, wy, w_full(q));
+              tma_load_2d(dst + (2 + j) * D::WBOX, &mw3, wx, wy, w_full(q));
+            }
+          } else {
+            // boxes 0..3: k-blocks 4s .. 4s + 3 of w2 rows 128 n .. of expert e
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              wcoord(4 * s + j, e * p.H + n * 128, kb2, p.blocked, wx, wy);
+              tma_load_2d(dst + j * D::WBOX, &mw2, wx, wy, w_full(q));
+            }
+          }
+        }
+      }
+      if (!ok) {
+        const int first = it > kS ? it - kS : 0;
+        for (int i = first; i < it; ++i) drain_phase(w_full(i % kS), ph(i, kS), p.status, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    if (lane == 0) {
+      // ---------------- routed rows of each stage's k-blocks: two (gate/up) or four
+      // (down), N rows in 16-row boxes
+      int it = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        bool dn;
+        int e, m, n;
+        coords(L, dn, e, m, n);
+        if (dn) {
+          // every gate/up tile of row tile m has stored its rows of h; the proxy fence
+          // orders those stores before the tensor copies (async proxy) that read them
+          if (!wait_count(p.row_ready + m, 4 * n1, abort_flag, p.status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
+        const int nrow = ncols[e];
+        const CUtensorMap* map = dn ? &mh : &mx;
+        const int nst = dn ? st2 : st1;
+        const int nblk = dn ? 4 : 2;
+        for (int s = 0; s < nst; ++s, ++it) {
+          const int q = it % kS;
+          if (!wait_phase(empty(q), ph(it, kS) ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(a_full(q), (uint32_t)(nblk * nrow * 128));
+          const uint32_t dst = stage(q) + 4 * D::WBOX;
+          for (int b = 0; b < nblk; ++b)
+            for (int j = 0; j < nrow; j += 16)
+              tma_load_2d(dst + b * D::ACT_UNIT + j * 128, map, (nblk * s + b) * BK, m * BM + j,
+                          a_full(q));
+        }
+      }
+      if (!ok) {
+        const int first = it > kS ? it - kS : 0;
+        for (int i = first; i < it; ++i) drain_phase(a_full(i % kS), ph(i, kS), p.status, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1 || warp == 7) {
+    if (lane == 0) {
+      // ---------------- MMA issuers (mi = 0, 1): gate/up: mi 0 gate (boxes 0, 1), mi 1
+      // up (boxes 2, 3), both over the rows of k-blocks 0, 1; down: mi's boxes (k-blocks)
+      // 2 mi, 2 mi + 1 into partial sum mi. The next stage's barriers are tested before
+      // this stage's MMAs issue.
+      const int mi = warp == 1 ? 0 : 1;
+      int it = 0, tc = 0;
+      bool ok = true, issued = false, pre_w = false, pre_a = false;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tc) {
+        bool dn;
+        int e, m, n;
+        coords(L, dn, e, m, n);
+        const uint32_t idesc = D::IDESC_M128 | ((uint32_t)(ncols[e] >> 3) << 17);
+        const int b = tc & 1;
+        if (!wait_phase(t_empty(b), ph(tc, 2) ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
+        fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(b * D::ACC_COLS + mi * NMAX);
+        const int nst = dn ? st2 : st1;
+        for (int s = 0; s < nst; ++s, ++it) {
+          const int q = it % kS;
+          if ((!pre_w && !wait_phase(w_full(q), ph(it, kS), abort_flag, p.status, p.timeout_ns)) ||
+              (!pre_a && !wait_phase(a_full(q), ph(it, kS), abort_flag, p.status, p.timeout_ns))) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          pre_w = mbar_test_wait(w_full((it + 1) % kS), ph(it + 1, kS));
+          pre_a = mbar_test_wait(a_full((it + 1) % kS), ph(it + 1, kS));
+          const uint32_t sw = stage(q), sa = sw + 4 * D::WBOX;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int box = 2 * mi + j, unit = dn ? 2 * mi + j : j;
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              mma_bf16(d, sdesc(sw + box * D::WBOX + kk * 32), sdesc(sa + unit * D::ACT_UNIT + kk * 32),
+                       idesc, (s | j | kk) ? 1u : 0u);
+          }
+          mma_commit(empty(q));
+          issued = true;
+        }
+        if (ok) mma_commit(t_full(b));
+      }
+      if (issued) {
+        mma_commit(final_bar + 8u * mi);
+        drain_phase(final_bar + 8u * mi, 0, p.status, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 2 && warp <= 5) {
+    // ---------------- epilogue: TMEM lanes 32 (warp % 4) .. = weight rows
+    const int quarter = warp & 3;
+    const int r = 32 * quarter + lane;
+    int tc = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x, ++tc) {
+      bool dn;
+      int e, m, n;
+      coords(L, dn, e, m, n);
+      const int nrow = ncols[e];
+      const int b = tc & 1;
+      int ok = 0;
+      if (lane == 0) ok = wait_phase(t_full(b), ph(tc, 2), abort_flag, p.status, p.timeout_ns) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      fence_after();
+      const uint32_t tacc =
+          tmem_base + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(b * D::ACC_COLS);
+      const int64_t row0 = (int64_t)m * BM;
+      if (!dn) {
+        uint16_t* hcol = p.h + row0 * p.I + n * 128 + r;  // intermediate column n 128 + r
+        for (int c0 = 0; c0 < nrow; c0 += 16) {
+          uint32_t g[16], u[16];
+          tmem_ld16(tacc + c0, g);
+          tmem_ld16(tacc + NMAX + c0, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const float gv = __uint_as_float(g[t]), uv = __uint_as_float(u[t]);
+            hcol[(int64_t)(c0 + t) * p.I] =
+                (uint16_t)(pack_bf16x2_rn(gv / (1.f + __expf(-gv)) * uv, 0.f) & 0xFFFFu);
+          }
+        }
+        // release this warp's rows of h to the down tiles of row tile m
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(p.row_ready + m, 1);
+      } else {
+        float* ycol = p.y + row0 * p.H + n * 128 + r;  // hidden column n 128 + r
+        for (int c0 = 0; c0 < nrow; c0 += 16) {
+          uint32_t v0[16], v1[16];
+          tmem_ld16(tacc + c0, v0);
+          tmem_ld16(tacc + NMAX + c0, v1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            ycol[(int64_t)(c0 + t) * p.H] = __uint_as_float(v0[t]) + __uint_as_float(v1[t]);
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(t_empty(b));
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"((uint32_t)D::TMEM_COLS)
+                 : "memory");
+  }
+}
+
 // ---------------------------------------------------------------- bounded-wait check
 // One thread waits, with the same bounded wait the GEMMs use, on a barrier phase that
 // nothing completes; after timeout_ns it records kStatusTimeout and returns.
@@ -1157,6 +1532,64 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
 #endif
 bool use_pair(const Shape& s) { return MOE_PAIR_GEMM && s.T * s.k >= (int64_t)1024 * s.E; }
 
+// Both expert GEMMs of a batch of at most NMAX tokens on the swap-operand kernel
+template <int NMAX>
+cudaError_t launch_decode_swap(const Shape& s, const GemmArgs& g, cudaStream_t st,
+                               const char** why) {
+  using D = DecBf16<NMAX>;
+  CUtensorMap mx, mh, mw1, mw3, mw2;
+  const uint64_t EI = (uint64_t)s.E * s.I, EH = (uint64_t)s.E * s.H;
+  const uint64_t wi1 = s.blocked ? BK : s.H, wr1 = s.blocked ? EI * s.H / BK : EI;
+  const uint64_t wi2 = s.blocked ? BK : s.I, wr2 = s.blocked ? EH * s.I / BK : EH;
+  if (!make_map(&mx, g.a, s.H, g.rmax, 16) || !make_map(&mh, g.h, s.I, g.rmax, 16) ||
+      !make_map(&mw1, g.w1, wi1, wr1, 128) || !make_map(&mw3, g.w3, wi1, wr1, 128) ||
+      !make_map(&mw2, g.w2, wi2, wr2, 128)) {
+    *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad tensor)";
+    return cudaErrorInvalidValue;
+  }
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_decode_swap<NMAX>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM);
+    if (e != cudaSuccess) {
+      *why = "expert GEMM shared-memory attribute";
+      return e;
+    }
+    attr_set[dev] = true;
+  }
+  DecBf16Params p;
+  p.offsets = g.offsets;
+  p.counts = g.counts;
+  p.h = g.h;
+  p.y = g.y;
+  p.status = g.status;
+  p.row_ready = g.row_ready;
+  p.E = s.E;
+  p.H = s.H;
+  p.I = s.I;
+  p.blocked = s.blocked;
+  p.timeout_ns = g.timeout_ns;
+  // the row-tile counters start at zero
+  cudaError_t e = cudaMemsetAsync(g.row_ready, 0, (size_t)(g.rmax / BM) * sizeof(int32_t), st);
+  if (e == cudaSuccess) {
+    // at most one row tile per expert with rows, at most T * k experts with rows
+    const int64_t active = s.E < s.T * s.k ? s.E : s.T * s.k;
+    const int64_t tiles = active * (s.I / 128 + s.H / 128);
+    int64_t grid = num_sms() < tiles ? num_sms() : tiles;
+    if (grid < 1) grid = 1;
+    e = launch_pdl(k_decode_swap<NMAX>, dim3((unsigned)grid), dim3(256), (size_t)D::SMEM, st, mw1,
+                   mw3, mw2, mx, mh, p);
+  }
+  if (e != cudaSuccess) *why = "expert GEMMs launch failed";
+  return e;
+}
+
+#ifndef MOE_SWAP_DECODE
+#define MOE_SWAP_DECODE 1
+#endif
+
 }  // namespace
 
 cudaError_t launch_gate_up(const Shape& s, const GemmArgs& g, cudaStream_t st, const char** why) {
@@ -1255,6 +1688,11 @@ cudaError_t launch_wait_selftest(int32_t* status, unsigned long long timeout_ns,
 
 cudaError_t launch_grouped_swiglu(const Shape& s, const GemmArgs& g, cudaStream_t st,
                                   const char** why) {
+  // at most 64 tokens, hidden % 128 == 0, intermediate % 256 == 0: the swap-operand kernel
+  if (MOE_SWAP_DECODE && s.T <= 64 && s.H % 128 == 0 && s.I % 256 == 0 && g.row_ready)
+    return s.T <= 16   ? launch_decode_swap<16>(s, g, st, why)
+           : s.T <= 32 ? launch_decode_swap<32>(s, g, st, why)
+                       : launch_decode_swap<64>(s, g, st, why);
   cudaError_t e = launch_gate_up(s, g, st, why);
   if (e != cudaSuccess) return e;
   return launch_down(s, g, st, why);

@@ -250,6 +250,7 @@ moe_status_t run_experts(const Shape& s, const uint16_t* x_perm, const int32_t* 
     g.counts = split.counts;
     g.partial = split.partial;
     g.split_sem = split.sem;
+    g.row_ready = split.row_ready;
     e = launch_grouped_swiglu(s, g, st, &why);
   }
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, why);
@@ -462,8 +463,10 @@ moe_status_t moe_grouped_swiglu(const moe_shape_t* shape, const moe_bf16_t* x_pe
   MOE_TRY(check_ptr(y_perm, "y_perm"));
   const Layout L = layout(s);
   MOE_TRY(check_ws(ws, ws_bytes, L.end));
+  SplitK scratch;
+  scratch.row_ready = at<int32_t>(ws, L.row_ready);
   return run_experts(s, x_perm, expert_offsets, bf16_experts(w1, w3, w2), at<uint16_t>(ws, L.h),
-                     y_perm, at<int32_t>(ws, L.status), (cudaStream_t)stream);
+                     y_perm, at<int32_t>(ws, L.status), (cudaStream_t)stream, scratch);
 }
 
 moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* x_perm,

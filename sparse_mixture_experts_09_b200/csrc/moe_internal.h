@@ -82,6 +82,8 @@ struct GemmArgs {
   const int32_t* counts = nullptr;
   float* partial = nullptr;
   int32_t* split_sem = nullptr;
+  // [Rmax / 128] int32 scratch: given, at most 64 tokens run both GEMMs as one grid
+  int32_t* row_ready = nullptr;
 };
 
 // GEMM1 (gate/up + SwiGLU -> h) then GEMM2 (h w2^T -> y), both persistent tcgen05.

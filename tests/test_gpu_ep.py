@@ -88,9 +88,11 @@ def test_expert_parallel_quantized_one_rank_matches_oracle(one_rank_group, mode)
 
 
 def test_expert_parallel_one_rank_decode(one_rank_group):
-    # moe_forward may split the down GEMM along K at small batches (its sums are then
-    # grouped differently) where the expert-parallel path does not: both against the
-    # oracle, and close to each other
+    # moe_forward sums the experts' products in another fp32 order than the expert-
+    # parallel path at small batches (a split down GEMM, or the swap-operand kernel's
+    # partial sums), so a few outputs may round to the neighbouring bf16 value: both
+    # against the oracle, and within one bf16 unit in the last place of each other (at
+    # most 2^-7 of the largest output), with a tight mean
     from oracle import moe_oracle as O
     from ._cases import assert_layer_close
     w = W.WORKLOADS["decode"]
@@ -104,7 +106,7 @@ def test_expert_parallel_one_rank_decode(one_rank_group):
     assert_layer_close(O.to_f64(want.cpu()), ref, "decode, moe_forward")
     from ._cases import layer_errors
     max_rel, mae = layer_errors(O.to_f64(got.cpu()), O.to_f64(want.cpu()))
-    assert max_rel <= 2e-3 and mae <= 1e-4, (max_rel, mae)
+    assert max_rel <= 2.0 ** -7 and mae <= 1e-4, (max_rel, mae)
 
 
 # ---- two ranks on one GPU, the exchange staged through gloo on the host ----
