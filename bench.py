@@ -37,12 +37,19 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 GEMM_SOURCE = os.path.join(ROOT, "sparse_mixture_experts_09_b200", "csrc", "gemm_sm100.cu")
 
 
-def kernels_per_forward(num_tokens: int) -> int:
+def fused_experts(num_tokens: int, hidden: int, inter: int) -> bool:
+    """Whether the bf16 layer runs both expert GEMMs as one swap-operand kernel (at most
+    64 tokens, hidden % 128 == 0, intermediate % 256 == 0)."""
+    return num_tokens <= 64 and hidden % 128 == 0 and inter % 256 == 0
+
+
+def kernels_per_forward(num_tokens: int, hidden: int = 4096, inter: int = 14336) -> int:
     """Kernels one moe_forward launches: router, the permutation (one planning kernel
-    up to 1024 tokens, else histogram + scan + rank; then the gather), the two expert
-    GEMMs and the combine."""
+    up to 1024 tokens, else histogram + scan + rank; then the gather), the expert GEMMs
+    (one swap-operand kernel at small batches, else gate/up and down) and the combine."""
     plan = 1 if (num_tokens + 31) // 32 <= 32 else 3
-    return 1 + plan + 1 + 2 + 1
+    gemms = 1 if fused_experts(num_tokens, hidden, inter) else 2
+    return 1 + plan + 1 + gemms + 1
 
 
 def parse_args():
@@ -234,6 +241,10 @@ def kernel_roofline(w, stage_ms, counts, peaks, peak_kind, long_run):
         "permute": (2 * R * H * wbytes + T * k * 12, 0),
         "gate_up": (n_active * 2 * I * H * wbytes + R * H * wbytes + R * I * wbytes, 4 * R * H * I),
         "down": (n_active * H * I * wbytes + R * I * wbytes + R * H * 4, 2 * R * H * I),
+        # both GEMMs as one kernel: the weights once, the routed rows, h written and read
+        # back, y written
+        "experts": (n_active * 3 * I * H * wbytes + R * H * wbytes + 2 * R * I * wbytes + R * H * 4,
+                    6 * R * H * I),
         "combine": (R * H * 4 + 2 * T * H * wbytes + T * k * 8, 2 * R * H),
     }
     name = max(stage_ms, key=stage_ms.get)
@@ -243,7 +254,7 @@ def kernel_roofline(w, stage_ms, counts, peaks, peak_kind, long_run):
     tensor_peak = peaks["bf16_tflops_sustained" if long_run else "bf16_tflops"]
     hbm_time = bytes_ / (hbm_peak * 1e9)
     tensor_time = flops / (tensor_peak * 1e12) if flops else 0.0
-    if name in ("gate_up", "down") and tensor_time > hbm_time:
+    if name in ("gate_up", "down", "experts") and tensor_time > hbm_time:
         r = {"bound": "tensor", "achieved": flops / sec / 1e12, "peak": tensor_peak,
              "unit": "TFLOP/s"}
     else:
@@ -394,6 +405,11 @@ class Bf16Layer:
                      "x_perm": torch.empty((rmax, w.hidden_size), dtype=torch.bfloat16, device=dev)}
         self.hbuf = torch.empty((rmax, w.intermediate_size), dtype=torch.bfloat16, device=dev)
         self.ybuf = torch.empty((rmax, w.hidden_size), dtype=torch.float32, device=dev)
+        # at small batches the forward runs both expert GEMMs as one kernel: the split
+        # timing then takes them together (the grouped entry point) as stage "experts"
+        self.fused = fused_experts(T, w.hidden_size, w.intermediate_size)
+        self.stage_names = (["router", "permute", "experts", "combine"] if self.fused
+                            else ["router", "permute", "gate_up", "down", "combine"])
 
     def step(self):
         i, (b1, b3, b2) = self.inp, self.bw
@@ -416,15 +432,21 @@ class Bf16Layer:
                                  p(perm["row_of"]), p(perm["token_of_row"]), p(perm["x_perm"]),
                                  p(ws), ws.numel(), st))
         ev[2].record(self.stream)
-        moe._check(L.moe_expert_gate_up(sp, p(perm["x_perm"]), p(perm["offsets"]), p(self.bw[0]),
-                                        p(self.bw[1]), p(self.hbuf), p(ws), ws.numel(), st))
-        ev[3].record(self.stream)
-        moe._check(L.moe_expert_down(sp, p(self.hbuf), p(perm["offsets"]), p(self.bw[2]),
-                                     p(self.ybuf), p(ws), ws.numel(), st))
-        ev[4].record(self.stream)
+        if self.fused:
+            moe._check(L.moe_grouped_swiglu(sp, p(perm["x_perm"]), p(perm["offsets"]),
+                                            p(self.bw[0]), p(self.bw[1]), p(self.bw[2]),
+                                            p(self.ybuf), p(ws), ws.numel(), st))
+        else:
+            moe._check(L.moe_expert_gate_up(sp, p(perm["x_perm"]), p(perm["offsets"]),
+                                            p(self.bw[0]), p(self.bw[1]), p(self.hbuf), p(ws),
+                                            ws.numel(), st))
+            ev[3].record(self.stream)
+            moe._check(L.moe_expert_down(sp, p(self.hbuf), p(perm["offsets"]), p(self.bw[2]),
+                                         p(self.ybuf), p(ws), ws.numel(), st))
+        ev[4 if not self.fused else 3].record(self.stream)
         moe._check(L.moe_combine(sp, p(self.ybuf), p(perm["row_of"]), p(self.wt), p(i.residual),
                                  p(self.out), st))
-        ev[5].record(self.stream)
+        ev[5 if not self.fused else 4].record(self.stream)
 
     def warm(self, n):
         import torch
@@ -446,9 +468,8 @@ class Bf16Layer:
             self.split_step(evs[i])
         torch.cuda.synchronize(self.dev)
         self.moe.device_status(self.ws)
-        names = ["router", "permute", "gate_up", "down", "combine"]
         return {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
-                for j, n in enumerate(names)}
+                for j, n in enumerate(self.stage_names)}
 
     def routing_report(self):
         """Expert counts and near-tie tokens of the last split step (untimed)."""
@@ -594,7 +615,8 @@ def run_ours(args):
                    "roofline": kernel_roofline(pre.w, pstage, pcounts, peaks, peak_kind, plong),
                    "kernels_ms": pstage, "expert_counts": pcounts, "near_ties": pnear,
                    "clocks": pclocks,
-                   "gpu_launches": kernels_per_forward(pre.w.num_tokens) * K}
+                   "gpu_launches": kernels_per_forward(pre.w.num_tokens, pre.w.hidden_size,
+                                                       pre.w.intermediate_size) * K}
 
     ms, e2e_ms = slowest_rank(ms, e2e_ms, world, dev)
     e2e_sync_ms, _ = slowest_rank(e2e_sync_ms, e2e_sync_ms, world, dev)
@@ -649,7 +671,8 @@ def run_ours(args):
                     "api": "moe_forward_host_async, steps enqueued back to back, one wait",
                     "per_call_wait": {"value": job_throughput(w.num_tokens, world, e2e_sync_ms),
                                       "api": "moe_forward_host (waits every step)"}},
-            "gpu_launches": kernels_per_forward(w.num_tokens) * K,
+            "gpu_launches": kernels_per_forward(w.num_tokens, w.hidden_size,
+                                                w.intermediate_size) * K,
             "clocks": clk,
             "expert_counts": counts,
             "near_ties": {"tokens": near_ties, "margin": 1e-2,

@@ -79,12 +79,28 @@ def test_clock_sampler_reports_slowdowns_and_tolerates_no_samples():
 
 
 def test_kernels_per_forward_matches_the_launch_lists():
-    # the ncu launch lists: 6 kernels per forward at decode (router, plan, gather, two
-    # GEMMs, combine); 8 above 1024 tokens (histogram, scan and rank replace the plan)
-    assert bench.kernels_per_forward(16) == 6
+    # the ncu launch lists: 5 kernels per forward at decode (router, plan, gather, the
+    # swap-operand kernel for both GEMMs, combine); 6 from 65 tokens (two GEMMs) or when
+    # the intermediate size is not a multiple of 256; 8 above 1024 tokens (histogram,
+    # scan and rank replace the plan)
+    assert bench.kernels_per_forward(16) == 5
+    assert bench.kernels_per_forward(64) == 5
+    assert bench.kernels_per_forward(65) == 6
+    assert bench.kernels_per_forward(16, 4096, 384) == 6
     assert bench.kernels_per_forward(1024) == 6
     assert bench.kernels_per_forward(1025) == 8
     assert bench.kernels_per_forward(4096) == 8
+    assert bench.fused_experts(64, 6144, 16384) and not bench.fused_experts(16, 4160, 14336)
+
+
+def test_experts_stage_roofline_counts_both_gemms():
+    w = W.WORKLOADS["decode"]
+    H, I, T = w.hidden_size, w.intermediate_size, w.num_tokens
+    R = T * 2
+    r = bench.kernel_roofline(w, {"router": 0.01, "experts": 0.4}, [4] * 8, PEAKS, "measured", False)
+    assert r["kernel"] == "experts" and r["bound"] == "hbm"
+    assert r["algorithmic_bytes"] == 8 * 3 * I * H * 2 + R * H * 2 + 2 * R * I * 2 + R * H * 4
+    assert r["algorithmic_flops"] == 6 * R * H * I
 
 
 class _Inputs:
