@@ -1005,13 +1005,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------- small batches
 //
-// k_decode_swap: both expert GEMMs of a batch of at most 64 tokens in one persistent
+// k_decode_swap: both expert GEMMs of a batch of at most 256 tokens in one persistent
 // grid, with the operands swapped: the weights are the tcgen05 M operand (128 weight
 // rows per tile, loaded by TMA straight into the 128-byte swizzled K-major layout the
-// MMA reads) and the expert's routed rows the N operand (N = its row count rounded up to
-// 16; a token reaches an expert at most once, so each expert has at most T rows, in one
-// 128-row tile). A stage holds four 128 x 64 weight boxes (gate/up: the w1 and w3 boxes
-// of two k-blocks; down: four k-blocks of one w2 box; 64 KiB) and its k-blocks of rows.
+// MMA reads) and a row tile's routed rows the N operand (N = the tile's row count
+// rounded up to 16, at most NMAX; a token reaches an expert at most once, so up to 64
+// tokens every expert has one row tile). A stage holds 4 KB 128 x 64 weight boxes
+// (gate/up: the w1 and w3 boxes of KB k-blocks; down: 2 KB k-blocks of one w2 box; KB =
+// 2, or 1 for NMAX = 128 so that three stages of rows still fit) and its k-blocks of
+// rows.
 // Against the tile kernels this moves 2 KiB of routed rows per 64 KiB of weights
 // instead of a 16 KiB activation tile per 32 KiB, and runs both GEMMs as one grid.
 //
@@ -1019,8 +1021,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   warp 6      routed rows (TMA, 16-row boxes); a down tile first waits until every
 //               gate/up tile of its row tile has released its rows of h;
 //   warps 1, 7  issue the MMAs (M = 128, N = rows): gate/up the first issues gate, the
-//               second up; down each issues two of the four k-blocks into its own
-//               partial sum;
+//               second up; down each issues KB of the stage's 2 KB k-blocks into its
+//               own partial sum;
 //   warps 2-5   read the accumulators (lane = weight row, column = routed row): h =
 //               bf16(silu(gate) * up) at [row, i], y = the two partial sums' sum at
 //               [row, j].
@@ -1031,26 +1033,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 // for tiles that are running or done.
 template <int NMAX>
 struct DecBf16 {
+  static constexpr int KB = NMAX <= 64 ? 2 : 1;                // k-blocks per matrix per stage
+  static constexpr int BOXES = 2 * KB;                         // weight boxes per stage
   static constexpr int WBOX = 128 * BK * 2;                    // one 128 x 64 weight box
   static constexpr int ACT_UNIT = NMAX * 128;                  // NMAX rows of one k-block
-  static constexpr int STAGE = 4 * WBOX + 4 * ACT_UNIT;
-  static constexpr int STAGES = (220 * 1024) / STAGE;          // 3 (NMAX 16) or 2 (32, 64)
+  static constexpr int STAGE = BOXES * WBOX + BOXES * ACT_UNIT;
+  static constexpr int STAGES = (220 * 1024) / STAGE;          // 3 (NMAX 16, 128), 2 (32, 64)
   static constexpr int ACC_COLS = 2 * NMAX;                    // gate, up (or two partials)
-  static constexpr int TMEM_COLS =
-      2 * ACC_COLS <= 32 ? 32 : (2 * ACC_COLS <= 64 ? 64 : (2 * ACC_COLS <= 128 ? 128 : 256));
+  static constexpr int TMEM_COLS = 2 * ACC_COLS <= 32    ? 32
+                                   : 2 * ACC_COLS <= 64  ? 64
+                                   : 2 * ACC_COLS <= 128 ? 128
+                                   : 2 * ACC_COLS <= 256 ? 256
+                                                         : 512;
   static constexpr int NUM_BARS = 3 * STAGES + 6;
   static constexpr int SMEM = 1024 + STAGES * STAGE + NUM_BARS * 8 + 16 + 2 * 72 * 4;
   // D f32, A and B bf16, both K-major, M = 128; N is set per tile
   static constexpr uint32_t IDESC_M128 =
       (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 4) << 24);
-  static_assert(NMAX == 16 || NMAX == 32 || NMAX == 64, "rows per expert");
+  static_assert(NMAX == 16 || NMAX == 32 || NMAX == 64 || NMAX == 128, "rows per tile");
   static_assert(STAGES >= 2 && STAGE % 1024 == 0, "stage plan");
+  static_assert(TMEM_COLS >= 2 * ACC_COLS && TMEM_COLS <= 512, "two accumulator buffers");
   static_assert(SMEM <= 232448, "shared memory plan exceeds 227 KiB");
 };
 
 struct DecBf16Params {
   const int32_t* offsets;  // [E+1], multiples of 128
-  const int32_t* counts;   // [E] routed rows per expert, or null (then NMAX rows)
+  const int32_t* counts;   // [E] routed rows per expert, or null (then NMAX rows a tile)
   uint16_t* h;             // [rows, I] bf16
   float* y;                // [rows, H] fp32
   int32_t* status;
@@ -1060,7 +1068,8 @@ struct DecBf16Params {
 };
 
 // Tile L -> (expert e, row tile m, column tile n) of a grid whose tiles are n_tiles per
-// row tile (one row tile per expert with rows at these batch sizes)
+// row tile; an expert's row tiles of one column tile are consecutive, so its weight tile
+// is read from HBM once and from L2 for the other row tiles
 __device__ __forceinline__ void swap_coords(int L, const int* row_tiles, int E, int n_tiles,
                                             int& e, int& m, int& n) {
   const int mrow = L / n_tiles;
@@ -1107,9 +1116,10 @@ __global__ void __launch_bounds__(256, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + D::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* row_tiles = reinterpret_cast<int*>(tmem_holder + 4);  // [E + 1]
-  int* ncols = row_tiles + 72;                                // [E]
+  int* nrows = row_tiles + 72;                                // [E]: routed rows (or -1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int KB = D::KB;
   // barriers: w_full (weights), a_full (rows), empty (both; the two issuers' commits) [kS];
   // t_full, t_empty [2]; final [2] (one per issuer)
   const uint32_t bar0 = smem_u32(bars);
@@ -1155,22 +1165,22 @@ __global__ void __launch_bounds__(256, 1)
   pdl_trigger();
   pdl_wait();
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) row_tiles[i] = p.offsets[i] / BM;
-  for (int i = threadIdx.x; i < p.E; i += blockDim.x) {
-    int n = NMAX;
-    if (p.counts) {
-      n = (p.counts[i] + 15) & ~15;
-      n = n < 16 ? 16 : (n > NMAX ? NMAX : n);
-    }
-    ncols[i] = n;
-  }
+  for (int i = threadIdx.x; i < p.E; i += blockDim.x) nrows[i] = p.counts ? p.counts[i] : -1;
   fence_before();
   __syncthreads();
   fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // N of row tile m of expert e: its routed rows rounded up to 16, at most NMAX (NMAX
+  // when the counts are not given)
+  auto tile_n = [&](int e, int m) {
+    if (nrows[e] < 0) return NMAX;
+    int n = (nrows[e] - (m - row_tiles[e]) * BM + 15) & ~15;
+    return n < 16 ? 16 : (n > NMAX ? NMAX : n);
+  };
 
   const int n1 = p.I / 128, n2 = p.H / 128;          // column tiles per row tile
   const int kb1 = p.H / BK, kb2 = p.I / BK;          // k-blocks of w1/w3 and of w2
-  const int st1 = kb1 / 2, st2 = kb2 / 4;            // stages per tile
+  const int st1 = kb1 / KB, st2 = kb2 / (2 * KB);    // stages per tile
   const int total0 = row_tiles[p.E] * n1;
   const int total = total0 + row_tiles[p.E] * n2;
   auto coords = [&](int L, bool& dn, int& e, int& m, int& n) {
@@ -1194,22 +1204,23 @@ __global__ void __launch_bounds__(256, 1)
             ok = false;
             break;
           }
-          mbar_expect_tx(w_full(q), 4 * D::WBOX);
+          mbar_expect_tx(w_full(q), D::BOXES * D::WBOX);
           const uint32_t dst = stage(q);
           int wx, wy;
           if (!dn) {
-            // boxes 0, 1: w1 rows 128 n .. of expert e, k-blocks 2s, 2s + 1; boxes 2, 3: w3
+            // boxes 0 .. KB-1: w1 rows 128 n .. of expert e, k-blocks KB s ..; boxes KB ..:
+            // the same of w3
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              wcoord(2 * s + j, e * p.I + n * 128, kb1, p.blocked, wx, wy);
+            for (int j = 0; j < KB; ++j) {
+              wcoord(KB * s + j, e * p.I + n * 128, kb1, p.blocked, wx, wy);
               tma_load_2d(dst + j * D::WBOX, &mw1, wx, wy, w_full(q));
-              tma_load_2d(dst + (2 + j) * D::WBOX, &mw3, wx, wy, w_full(q));
+              tma_load_2d(dst + (KB + j) * D::WBOX, &mw3, wx, wy, w_full(q));
             }
           } else {
-            // boxes 0..3: k-blocks 4s .. 4s + 3 of w2 rows 128 n .. of expert e
+            // boxes 0 .. 2KB-1: k-blocks 2KB s .. of w2 rows 128 n .. of expert e
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              wcoord(4 * s + j, e * p.H + n * 128, kb2, p.blocked, wx, wy);
+            for (int j = 0; j < 2 * KB; ++j) {
+              wcoord(2 * KB * s + j, e * p.H + n * 128, kb2, p.blocked, wx, wy);
               tma_load_2d(dst + j * D::WBOX, &mw2, wx, wy, w_full(q));
             }
           }
@@ -1223,7 +1234,7 @@ __global__ void __launch_bounds__(256, 1)
     __syncwarp();
   } else if (warp == 6) {
     if (lane == 0) {
-      // ---------------- routed rows of each stage's k-blocks: two (gate/up) or four
+      // ---------------- routed rows of each stage's k-blocks: KB (gate/up) or 2 KB
       // (down), N rows in 16-row boxes
       int it = 0;
       bool ok = true;
@@ -1240,10 +1251,10 @@ __global__ void __launch_bounds__(256, 1)
           }
           asm volatile("fence.proxy.async.global;" ::: "memory");
         }
-        const int nrow = ncols[e];
+        const int nrow = tile_n(e, m);
         const CUtensorMap* map = dn ? &mh : &mx;
         const int nst = dn ? st2 : st1;
-        const int nblk = dn ? 4 : 2;
+        const int nblk = dn ? 2 * KB : KB;
         for (int s = 0; s < nst; ++s, ++it) {
           const int q = it % kS;
           if (!wait_phase(empty(q), ph(it, kS) ^ 1u, abort_flag, p.status, p.timeout_ns)) {
@@ -1251,7 +1262,7 @@ __global__ void __launch_bounds__(256, 1)
             break;
           }
           mbar_expect_tx(a_full(q), (uint32_t)(nblk * nrow * 128));
-          const uint32_t dst = stage(q) + 4 * D::WBOX;
+          const uint32_t dst = stage(q) + D::BOXES * D::WBOX;
           for (int b = 0; b < nblk; ++b)
             for (int j = 0; j < nrow; j += 16)
               tma_load_2d(dst + b * D::ACT_UNIT + j * 128, map, (nblk * s + b) * BK, m * BM + j,
@@ -1266,10 +1277,10 @@ __global__ void __launch_bounds__(256, 1)
     __syncwarp();
   } else if (warp == 1 || warp == 7) {
     if (lane == 0) {
-      // ---------------- MMA issuers (mi = 0, 1): gate/up: mi 0 gate (boxes 0, 1), mi 1
-      // up (boxes 2, 3), both over the rows of k-blocks 0, 1; down: mi's boxes (k-blocks)
-      // 2 mi, 2 mi + 1 into partial sum mi. The next stage's barriers are tested before
-      // this stage's MMAs issue.
+      // ---------------- MMA issuers (mi = 0, 1): gate/up: mi 0 gate (w1 boxes), mi 1 up
+      // (w3 boxes), both over the rows of the stage's KB k-blocks; down: mi's KB boxes
+      // (k-blocks) into partial sum mi. The next stage's barriers are tested before this
+      // stage's MMAs issue.
       const int mi = warp == 1 ? 0 : 1;
       int it = 0, tc = 0;
       bool ok = true, issued = false, pre_w = false, pre_a = false;
@@ -1277,7 +1288,7 @@ __global__ void __launch_bounds__(256, 1)
         bool dn;
         int e, m, n;
         coords(L, dn, e, m, n);
-        const uint32_t idesc = D::IDESC_M128 | ((uint32_t)(ncols[e] >> 3) << 17);
+        const uint32_t idesc = D::IDESC_M128 | ((uint32_t)(tile_n(e, m) >> 3) << 17);
         const int b = tc & 1;
         if (!wait_phase(t_empty(b), ph(tc, 2) ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
         fence_after();
@@ -1293,10 +1304,10 @@ __global__ void __launch_bounds__(256, 1)
           fence_after();
           pre_w = mbar_test_wait(w_full((it + 1) % kS), ph(it + 1, kS));
           pre_a = mbar_test_wait(a_full((it + 1) % kS), ph(it + 1, kS));
-          const uint32_t sw = stage(q), sa = sw + 4 * D::WBOX;
+          const uint32_t sw = stage(q), sa = sw + D::BOXES * D::WBOX;
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int box = 2 * mi + j, unit = dn ? 2 * mi + j : j;
+          for (int j = 0; j < KB; ++j) {
+            const int box = KB * mi + j, unit = dn ? KB * mi + j : j;
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
               mma_bf16(d, sdesc(sw + box * D::WBOX + kk * 32), sdesc(sa + unit * D::ACT_UNIT + kk * 32),
@@ -1322,7 +1333,7 @@ __global__ void __launch_bounds__(256, 1)
       bool dn;
       int e, m, n;
       coords(L, dn, e, m, n);
-      const int nrow = ncols[e];
+      const int nrow = tile_n(e, m);
       const int b = tc & 1;
       int ok = 0;
       if (lane == 0) ok = wait_phase(t_full(b), ph(tc, 2), abort_flag, p.status, p.timeout_ns) ? 1 : 0;
@@ -1532,7 +1543,7 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
 #endif
 bool use_pair(const Shape& s) { return MOE_PAIR_GEMM && s.T * s.k >= (int64_t)1024 * s.E; }
 
-// Both expert GEMMs of a batch of at most NMAX tokens on the swap-operand kernel
+// Both expert GEMMs on the swap-operand kernel (row tiles of at most NMAX routed rows)
 template <int NMAX>
 cudaError_t launch_decode_swap(const Shape& s, const GemmArgs& g, cudaStream_t st,
                                const char** why) {
@@ -1561,7 +1572,7 @@ cudaError_t launch_decode_swap(const Shape& s, const GemmArgs& g, cudaStream_t s
   }
   DecBf16Params p;
   p.offsets = g.offsets;
-  p.counts = g.counts;
+  p.counts = g.expert_rows ? g.expert_rows : g.counts;
   p.h = g.h;
   p.y = g.y;
   p.status = g.status;
@@ -1574,9 +1585,7 @@ cudaError_t launch_decode_swap(const Shape& s, const GemmArgs& g, cudaStream_t s
   // the row-tile counters start at zero
   cudaError_t e = cudaMemsetAsync(g.row_ready, 0, (size_t)(g.rmax / BM) * sizeof(int32_t), st);
   if (e == cudaSuccess) {
-    // at most one row tile per expert with rows, at most T * k experts with rows
-    const int64_t active = s.E < s.T * s.k ? s.E : s.T * s.k;
-    const int64_t tiles = active * (s.I / 128 + s.H / 128);
+    const int64_t tiles = (g.rmax / BM) * (s.I / 128 + s.H / 128);
     int64_t grid = num_sms() < tiles ? num_sms() : tiles;
     if (grid < 1) grid = 1;
     e = launch_pdl(k_decode_swap<NMAX>, dim3((unsigned)grid), dim3(256), (size_t)D::SMEM, st, mw1,
@@ -1688,11 +1697,15 @@ cudaError_t launch_wait_selftest(int32_t* status, unsigned long long timeout_ns,
 
 cudaError_t launch_grouped_swiglu(const Shape& s, const GemmArgs& g, cudaStream_t st,
                                   const char** why) {
-  // at most 64 tokens, hidden % 128 == 0, intermediate % 256 == 0: the swap-operand kernel
-  if (MOE_SWAP_DECODE && s.T <= 64 && s.H % 128 == 0 && s.I % 256 == 0 && g.row_ready)
+  // the swap-operand kernel: at most 64 tokens with hidden % 128 == 0 and intermediate
+  // % 256 == 0 (two k-blocks per stage), or up to 256 tokens with 128-row tiles (one
+  // k-block per stage)
+  if (MOE_SWAP_DECODE && g.row_ready && s.T <= 64 && s.H % 128 == 0 && s.I % 256 == 0)
     return s.T <= 16   ? launch_decode_swap<16>(s, g, st, why)
            : s.T <= 32 ? launch_decode_swap<32>(s, g, st, why)
                        : launch_decode_swap<64>(s, g, st, why);
+  if (MOE_SWAP_DECODE && g.row_ready && s.T <= 256 && s.H % 128 == 0 && s.I % 128 == 0)
+    return launch_decode_swap<128>(s, g, st, why);
   cudaError_t e = launch_gate_up(s, g, st, why);
   if (e != cudaSuccess) return e;
   return launch_down(s, g, st, why);

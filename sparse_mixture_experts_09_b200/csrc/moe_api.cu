@@ -205,7 +205,7 @@ struct SplitK {
   float* partial = nullptr;
   int32_t* sem = nullptr;
   int32_t* row_ready = nullptr;
-  const int32_t* q_counts = nullptr;  // quantised experts: routed rows per expert
+  const int32_t* q_counts = nullptr;  // routed rows per expert (sizes one-grid row tiles)
 };
 
 moe_status_t run_experts(const Shape& s, const uint16_t* x_perm, const int32_t* offsets,
@@ -251,6 +251,7 @@ moe_status_t run_experts(const Shape& s, const uint16_t* x_perm, const int32_t* 
     g.partial = split.partial;
     g.split_sem = split.sem;
     g.row_ready = split.row_ready;
+    g.expert_rows = split.q_counts;
     e = launch_grouped_swiglu(s, g, st, &why);
   }
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, why);

@@ -82,8 +82,11 @@ struct GemmArgs {
   const int32_t* counts = nullptr;
   float* partial = nullptr;
   int32_t* split_sem = nullptr;
-  // [Rmax / 128] int32 scratch: given, at most 64 tokens run both GEMMs as one grid
+  // [Rmax / 128] int32 scratch: given, at most 256 tokens run both GEMMs as one grid
   int32_t* row_ready = nullptr;
+  // [E] routed rows per expert (nullable): they size the one-grid kernel's row tiles
+  // (16-row steps); null: every row tile is sized for its full 128 rows or the batch
+  const int32_t* expert_rows = nullptr;
 };
 
 // GEMM1 (gate/up + SwiGLU -> h) then GEMM2 (h w2^T -> y), both persistent tcgen05.
