@@ -754,13 +754,16 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
 
 // ---------------------------------------------------------------- small batches
 //
-// k_w8_decode: both expert GEMMs of a batch of at most 64 tokens, in one persistent
-// grid, with the operands swapped. A token reaches an expert at most once, so each
-// expert then has at most 64 routed rows, all in its one 128-row tile. The tile kernel
-// above spends a full M = 64 MMA and an 8 KiB activation tile on every 64-wide k-block
-// for those few rows. Here the weights are the tcgen05 M operand (128 weight rows per
-// tile) and the expert's routed rows the N operand (N = its row count rounded up to
-// 16), so the MMAs shrink with the batch. The widened weights never touch shared memory:
+// k_w8_decode: both expert GEMMs of a batch of at most 256 tokens, in one persistent
+// grid, with the operands swapped. A token reaches an expert at most once, so up to 64
+// tokens each expert has at most 64 routed rows, all in its one 128-row tile. The tile
+// kernel above spends a full M = 64 MMA and an 8 KiB activation tile on every 64-wide
+// k-block for those few rows. Here the weights are the tcgen05 M operand (128 weight
+// rows per tile) and a sub-tile of at most NMAX of the expert's routed rows the N
+// operand (N = the sub-tile's row count rounded up to 16), so the MMAs shrink with the
+// batch. An expert with more than NMAX rows has several sub-tiles over the same weight
+// tiles: consecutive tiles, so the codes of all but the first come from L2 (the widening
+// is repeated). The widened weights never touch shared memory:
 //
 //   warp 0      streams code stages into a deep ring (bulk copies): a stage is four
 //               128-row x 64-code boxes, gate/up the w1 and w3 boxes of two k-blocks,
@@ -771,8 +774,8 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
 //               half pairs with one tcgen05.st: the tensor-memory layout of an M = 128
 //               A operand (lane = row, column c = K elements 2c and 2c + 1);
 //   warp 6      loads the routed rows' k-blocks (TMA, 16-row boxes, 128-byte swizzle);
-//               a down tile first waits until every gate/up tile of its row tile has
-//               released its rows of h (per-row-tile counters);
+//               a down tile first waits until every gate/up tile of its sub-tile has
+//               released its rows of h (per-sub-tile counters);
 //   warps 1, 23 issue tcgen05.mma with A in tensor memory and B (the rows) in shared
 //               memory, M = 128, N = rows, each half of every stage: gate/up the first
 //               issues gate and the second up, down each issues two of the four k-blocks
@@ -780,8 +783,8 @@ __global__ void __launch_bounds__(kThreadsW8, 1)
 //   warps 2-5   read the accumulators (lane = weight row, column = routed row): h =
 //               half(silu(s1 gate) * s3 up) at [row, i], y = s2 acc at [row, j].
 //
-// Tiles: gate/up tile (row tile, n) covers intermediate columns 128 n .. + 127 over
-// H / 128 stages; down tile (row tile, n) covers hidden columns 128 n .. + 127 over
+// Tiles: gate/up tile (sub-tile, n) covers intermediate columns 128 n .. + 127 over
+// H / 128 stages; down tile (sub-tile, n) covers hidden columns 128 n .. + 127 over
 // I / 256 stages. Every gate/up tile precedes every down tile in the order each CTA
 // walks its tiles, and the grid is at most one CTA per SM, so a down tile only waits for
 // tiles that are running or done.
@@ -817,10 +820,10 @@ struct DecW8 {
   static constexpr int Q_OFF = W_SLOTS * ACT_SLOT;
   static constexpr int BAR_OFF = Q_OFF + Q_ST * Q_BYTES;
   static constexpr int NUM_BARS = 2 * Q_ST + 3 * W_SLOTS + 4 + 2;
-  static constexpr int SMEM = 1024 + BAR_OFF + NUM_BARS * 8 + 16 + 2 * 72 * 4;
+  static constexpr int SMEM = 1024 + BAR_OFF + NUM_BARS * 8 + 16 + 3 * 72 * 4;
   // D f32, A and B f16, both K-major, M = 128; N is set per tile
   static constexpr uint32_t IDESC_M128 = (1u << 4) | ((uint32_t)(128 >> 4) << 24);
-  static_assert(NMAX == 16 || NMAX == 32 || NMAX == 64, "rows per expert");
+  static_assert(NMAX == 16 || NMAX == 32 || NMAX == 64, "rows per sub-tile");
   static_assert(W_SLOTS >= 2 && Q_ST >= 3, "pipeline plan");
   static_assert(Q_BYTES % 16 == 0 && ACT_UNIT % 1024 == 0, "stage alignment");
   static_assert(SMEM <= 232448, "shared memory plan exceeds 227 KiB");
@@ -838,12 +841,13 @@ struct DecParams {
   const uint16_t* g3;
   const uint16_t* g2;
   const int32_t* offsets;  // [E+1], multiples of 128
-  const int32_t* counts;   // [E] routed rows per expert, or null (then NMAX rows)
+  const int32_t* counts;   // [E] routed rows per expert, or null (then min(max_rows, padded))
   uint16_t* h;             // [rows, I] half
   float* y;                // [rows, H] fp32
   int32_t* status;
-  int32_t* row_ready;      // [rows / 128], zero at launch
+  int32_t* row_ready;      // [rows / 64] per-sub-tile counters, zero at launch
   int E, H, I;
+  int max_rows;            // most rows an expert can have: the tokens
   unsigned long long timeout_ns;
 };
 
@@ -943,8 +947,9 @@ __global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + D::BAR_OFF);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + D::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  int* row_tiles = reinterpret_cast<int*>(tmem_holder + 4);  // [E + 1]
-  int* ncols = row_tiles + 72;                                // [E]: N of the expert's tiles
+  int* sub0 = reinterpret_cast<int*>(tmem_holder + 4);  // [E + 1]: first sub-tile of each expert
+  int* nrows = sub0 + 72;                                // [E]: routed rows of each expert
+  int* row_off = nrows + 72;                             // [E]: first row of each expert
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // barriers: q_full, q_empty [kQ]; w_full (widened slot), a_full (the slot's rows),
@@ -993,27 +998,39 @@ __global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
   }
   pdl_trigger();
   pdl_wait();
-  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) row_tiles[i] = p.offsets[i] / BM;
   for (int i = threadIdx.x; i < p.E; i += blockDim.x) {
-    int n = NMAX;
-    if (p.counts) {
-      n = (p.counts[i] + 15) & ~15;
-      n = n < 16 ? 16 : (n > NMAX ? NMAX : n);
+    const int padded = p.offsets[i + 1] - p.offsets[i];
+    nrows[i] = p.counts ? p.counts[i] : (padded < p.max_rows ? padded : p.max_rows);
+    row_off[i] = p.offsets[i];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int i = 0; i < p.E; ++i) {
+      sub0[i] = acc;
+      acc += (nrows[i] + NMAX - 1) / NMAX;
     }
-    ncols[i] = n;
+    sub0[p.E] = acc;
   }
   fence_before();
   __syncthreads();
   fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // sub-tile m of expert e: its first row, and N = its rows rounded up to 16 (at most NMAX)
+  auto sub_row0 = [&](int e, int m) { return row_off[e] + (m - sub0[e]) * NMAX; };
+  auto sub_rows = [&](int e, int m) {
+    const int n = (nrows[e] - (m - sub0[e]) * NMAX + 15) & ~15;
+    return n < 16 ? 16 : (n > NMAX ? NMAX : n);
+  };
 
-  const int n1 = p.I / 128, n2 = p.H / 128;  // column tiles per row tile
+  const int n1 = p.I / 128, n2 = p.H / 128;  // column tiles per sub-tile
   const int st1 = p.H / (2 * BK), st2 = p.I / (4 * BK);  // stages per tile
-  const int total0 = row_tiles[p.E] * n1;
-  const int total = total0 + row_tiles[p.E] * n2;
+  const int total0 = sub0[p.E] * n1;
+  const int total = total0 + sub0[p.E] * n2;
+  // the sub-tiles of one expert and column tile are consecutive tiles
   auto coords = [&](int L, bool& dn, int& e, int& m, int& n) {
     dn = L >= total0;
-    tile_coords_w8(dn ? L - total0 : L, row_tiles, p.E, dn ? n2 : n1, e, m, n);
+    tile_coords_w8(dn ? L - total0 : L, sub0, p.E, dn ? n2 : n1, e, m, n);
   };
 
   if (warp == 0) {
@@ -1071,7 +1088,7 @@ __global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
         int e, m, n;
         coords(L, dn, e, m, n);
         if (dn) {
-          // every gate/up tile of row tile m has stored its rows of h; the proxy fence
+          // every gate/up tile of sub-tile m has stored its rows of h; the proxy fence
           // orders those stores before the tensor copies (async proxy) that read them
           if (!wait_ready(p.row_ready + m, 4 * n1, abort_flag, p.status, p.timeout_ns)) {
             ok = false;
@@ -1079,7 +1096,7 @@ __global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
           }
           asm volatile("fence.proxy.async.global;" ::: "memory");
         }
-        const int nrow = ncols[e];
+        const int nrow = sub_rows(e, m), row0 = sub_row0(e, m);
         const CUtensorMap* map = dn ? &mapH : &mapX;
         const int nst = dn ? st2 : st1;
         const int nblk = dn ? 4 : 2;
@@ -1093,7 +1110,7 @@ __global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
           for (int b = 0; b < nblk; ++b) {
             const int xk = (nblk * s + b) * BK;
             for (int j = 0; j < nrow; j += 16)
-              tma_load_2d(act(ws) + b * D::ACT_UNIT + j * 128, map, xk, m * BM + j, a_full(ws));
+              tma_load_2d(act(ws) + b * D::ACT_UNIT + j * 128, map, xk, row0 + j, a_full(ws));
           }
         }
       }
@@ -1115,7 +1132,7 @@ __global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
         bool dn;
         int e, m, n;
         coords(L, dn, e, m, n);
-        const uint32_t idesc = D::IDESC_M128 | ((uint32_t)(ncols[e] >> 3) << 17);
+        const uint32_t idesc = D::IDESC_M128 | ((uint32_t)(sub_rows(e, m) >> 3) << 17);
         const int b = tc & 1;
         if (!wait_w8(t_empty(b), ph(tc, 2) ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
         fence_after();
@@ -1225,13 +1242,13 @@ __global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
       bool dn;
       int e, m, n;
       coords(L, dn, e, m, n);
-      const int nrow = ncols[e];
+      const int nrow = sub_rows(e, m);
       const int b = tc & 1;
       if (!wait_warp(t_full(b), ph(tc, 2), abort_flag, p.status, p.timeout_ns)) break;
       fence_after();
       const uint32_t tacc =
           tmem_base + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(b * D::ACC_COLS);
-      const int64_t row0 = (int64_t)m * BM;
+      const int64_t row0 = sub_row0(e, m);
       if (!dn) {
         const int i = n * 128 + r;  // intermediate column
         const float sg = BITS == 8 ? __ldg(p.s1 + (size_t)e * p.I + i) : 1.f;
@@ -1248,7 +1265,7 @@ __global__ void __launch_bounds__(DecW8<BITS, NMAX>::THREADS, 1)
             hcol[(int64_t)(c0 + t) * p.I] = half_rn(gv / (1.f + __expf(-gv)) * uv);
           }
         }
-        // release this warp's rows of h to the down tiles of row tile m
+        // release this warp's rows of h to the down tiles of sub-tile m
         asm volatile("fence.proxy.async.global;" ::: "memory");
         __threadfence();
         __syncwarp();
@@ -1549,7 +1566,7 @@ cudaError_t launch_swiglu_w8_tiles(const Shape& s, const GemmArgsW8& g, cudaStre
   return e;
 }
 
-// Both GEMMs of a batch of at most NMAX tokens on the swap-operand kernel
+// Both GEMMs on the swap-operand kernel (sub-tiles of at most NMAX routed rows)
 template <int BITS, int NMAX>
 cudaError_t launch_w8_decode(const Shape& s, const GemmArgsW8& g, cudaStream_t st,
                              const char** why) {
@@ -1590,13 +1607,14 @@ cudaError_t launch_w8_decode(const Shape& s, const GemmArgsW8& g, cudaStream_t s
   p.E = s.E;
   p.H = s.H;
   p.I = s.I;
+  p.max_rows = (int)s.T;
   p.timeout_ns = g.timeout_ns;
-  // the row-tile counters start at zero
-  cudaError_t e = cudaMemsetAsync(g.row_ready, 0, (size_t)(g.rmax / BM) * sizeof(int32_t), st);
+  // the sub-tile counters start at zero; an expert of c rows has ceil(c / NMAX) sub-tiles,
+  // so there are at most T k / NMAX + E of them, within rmax / 64 (rmax >= T k + 128 E)
+  const int64_t subs = (int64_t)s.T * s.k / NMAX + s.E;
+  cudaError_t e = cudaMemsetAsync(g.row_ready, 0, (size_t)(g.rmax / 64) * sizeof(int32_t), st);
   if (e == cudaSuccess) {
-    // at most one row tile per expert with rows, at most T * k experts with rows
-    const int64_t active = std::min<int64_t>(s.E, (int64_t)s.T * s.k);
-    const int64_t tiles = active * (s.I / 128 + s.H / 128);
+    const int64_t tiles = subs * (s.I / 128 + s.H / 128);
     int64_t grid = std::min<int64_t>(num_sms(), tiles);
     if (grid < 1) grid = 1;
     e = launch_pdl(k_w8_decode<BITS, NMAX>, dim3((unsigned)grid), dim3(D::THREADS),
@@ -1614,9 +1632,12 @@ cudaError_t launch_grouped_swiglu_w8(const Shape& s, const GemmArgsW8& g, cudaSt
   // a token is routed to an expert at most once, so with at most 64 tokens every expert
   // has at most 64 rows, all in the first half of its 128-row tile
   const bool half_tiles = s.T <= 64 && kUseHalfTiles;
-  // with at most 64 tokens, hidden % 128 == 0 and intermediate % 256 == 0, the
-  // swap-operand kernel
-  if (s.T <= 64 && s.H % 128 == 0 && s.I % 256 == 0 && g.row_ready && kUseDecodeKernel) {
+  // the swap-operand kernel: at most 64 tokens, or at most 256 tokens averaging at most
+  // 48 routed rows per expert (above that most experts take two 64-row sub-tiles, each
+  // widening the same weights, and the tile kernels are as fast); hidden % 128 == 0 and
+  // intermediate % 256 == 0
+  const bool swap_rows = s.T <= 64 || (s.T <= 256 && (int64_t)s.T * s.k <= 48 * (int64_t)s.E);
+  if (swap_rows && s.H % 128 == 0 && s.I % 256 == 0 && g.row_ready && kUseDecodeKernel) {
     if (g.bits == 4)
       return s.T <= 16   ? launch_w8_decode<4, 16>(s, g, st, why)
              : s.T <= 32 ? launch_w8_decode<4, 32>(s, g, st, why)

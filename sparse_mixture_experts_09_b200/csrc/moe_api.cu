@@ -71,7 +71,7 @@ Layout layout(const Shape& s) {
   L.h = o; o += up(rmax * s.I * 2);
   L.y = o; o += up(rmax * s.H * 4);
   L.rnorm = o; o += up((size_t)s.T * 4);
-  L.row_ready = o; o += up((size_t)(rmax / kRowPad) * 4);  // quantised experts: row tiles of h done
+  L.row_ready = o; o += up((size_t)(rmax / 64) * 4);  // one-grid experts: sub-tiles of h done
   // split-K of the down GEMM (small batches only): arrival counters and partial sums
   const bool split = (int64_t)tk <= kSplitMaxRows;
   L.split_sem = o; o += split ? up((size_t)kSplitSems * 4) : 0;

@@ -82,7 +82,7 @@ struct GemmArgs {
   const int32_t* counts = nullptr;
   float* partial = nullptr;
   int32_t* split_sem = nullptr;
-  // [Rmax / 128] int32 scratch: given, at most 256 tokens run both GEMMs as one grid
+  // [Rmax / 64] int32 scratch: given, at most 256 tokens run both GEMMs as one grid
   int32_t* row_ready = nullptr;
   // [E] routed rows per expert (nullable): they size the one-grid kernel's row tiles
   // (16-row steps); null: every row tile is sized for its full 128 rows or the batch
@@ -127,10 +127,11 @@ struct GemmArgsW8 {
   int32_t* status = nullptr;
   int64_t rmax = 0;
   unsigned long long timeout_ns = 0;
-  // [rmax / 128] int32 scratch: given, both GEMMs run as one grid (hidden % 256 == 0)
+  // [rmax / 64] int32 scratch: given, at most 256 tokens run both GEMMs as one grid
+  // (intermediate % 256 == 0)
   int32_t* row_ready = nullptr;
-  // [E] routed rows per expert (nullable): at most 64 tokens, they size each expert's
-  // tiles (16-row steps); null: every expert is sized for the whole batch
+  // [E] routed rows per expert (nullable): they size the one-grid kernel's sub-tiles
+  // (16-row steps); null: an expert is taken to have min(T, its padded rows) rows
   const int32_t* counts = nullptr;
 };
 

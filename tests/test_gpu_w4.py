@@ -101,7 +101,7 @@ def test_grouped_swiglu_w4_matches_oracle(name):
 
 @pytest.mark.parametrize("name", ["tiny", "ragged", "e5k3", "one_token", "skewed", "bn128_split",
                                   "ts_t33", "ts_e64k8", "ts_h640", "ts_k1", "t64_edge", "t65_edge",
-                                  "t17_e4", "t24_e2", "t48_e2"])
+                                  "t17_e4", "t24_e2", "t48_e2", "t160_skew", "t96_e4"])
 def test_forward_w4_matches_oracle(name):
     w = CASES[name]
     inp, near = screened(w)
@@ -121,7 +121,8 @@ def test_forward_w4_matches_oracle(name):
         assert_layer_close(O.to_f64(out.cpu()), ref["out"], name)
 
 
-@pytest.mark.parametrize("name", ["decode", "prefill", "larger_decode_T1", "larger_decode_T64"])
+@pytest.mark.parametrize("name", ["decode", "prefill", "larger_decode_T1", "larger_decode_T64",
+                                  "larger_decode_T256"])
 def test_forward_w4_full_size_against_oracle(name):
     w = W.workload(name)
     inp, near = screened(w)

@@ -78,6 +78,13 @@ SMALL_BATCH = {
     "t17_e4": W.Workload("t17_e4", 17, 512, 512, 4, 2, seed=37),
     "t24_e2": W.Workload("t24_e2", 24, 256, 512, 2, 2, seed=38),
     "t48_e2": W.Workload("t48_e2", 48, 384, 768, 2, 2, seed=39),
+    # above 64 tokens (at most 48 routed rows per expert on average) an expert's rows are
+    # cut into 64-row sub-tiles over the same weight tiles: 160 tokens with expert 0
+    # favoured give it 155 rows (sub-tiles of 64, 64 and 27); 96 tokens on 4 experts
+    # with expert 0 slightly favoured give it 66 rows (64 and 2)
+    "t160_skew": W.Workload("t160_skew", 160, 256, 512, 8, 2, seed=45,
+                            logit_bias=(3.0, 0, 0, 0, 0, 0, 0, 0)),
+    "t96_e4": W.Workload("t96_e4", 96, 384, 512, 4, 2, seed=46, logit_bias=(0.5, 0, 0, 0)),
 }
 CASES = {**SMALL, **SMALL_BATCH}
 
@@ -106,7 +113,7 @@ def test_grouped_swiglu_w8_matches_oracle(name):
 
 @pytest.mark.parametrize("name", ["tiny", "ragged", "e5k3", "one_token", "skewed", "bn128_split",
                                   "ts_t33", "ts_e64k8", "ts_h640", "t64_edge", "t65_edge",
-                                  "t17_e4", "t24_e2", "t48_e2"])
+                                  "t17_e4", "t24_e2", "t48_e2", "t160_skew", "t96_e4"])
 def test_forward_w8_matches_oracle(name):
     w = CASES[name]
     inp, near = screened(w)
@@ -126,7 +133,8 @@ def test_forward_w8_matches_oracle(name):
         assert_layer_close(O.to_f64(out.cpu()), ref["out"], name)
 
 
-@pytest.mark.parametrize("name", ["decode", "prefill", "larger_decode_T1", "larger_decode_T64"])
+@pytest.mark.parametrize("name", ["decode", "prefill", "larger_decode_T1", "larger_decode_T64",
+                                  "larger_decode_T256"])
 def test_forward_w8_full_size_against_oracle(name):
     w = W.workload(name)
     inp, near = screened(w)
