@@ -1582,8 +1582,11 @@ cudaError_t launch_decode_swap(const Shape& s, const GemmArgs& g, cudaStream_t s
   p.I = s.I;
   p.blocked = s.blocked;
   p.timeout_ns = g.timeout_ns;
-  // the row-tile counters start at zero
-  cudaError_t e = cudaMemsetAsync(g.row_ready, 0, (size_t)(g.rmax / BM) * sizeof(int32_t), st);
+  // the row-tile counters start at zero (unless a kernel before this one zeroed them: a
+  // memset between the two would keep this launch from overlapping that kernel's tail)
+  cudaError_t e = g.row_ready_zeroed
+                      ? cudaSuccess
+                      : cudaMemsetAsync(g.row_ready, 0, (size_t)(g.rmax / BM) * sizeof(int32_t), st);
   if (e == cudaSuccess) {
     const int64_t tiles = (g.rmax / BM) * (s.I / 128 + s.H / 128);
     int64_t grid = num_sms() < tiles ? num_sms() : tiles;

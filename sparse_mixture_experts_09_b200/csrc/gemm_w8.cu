@@ -1611,8 +1611,11 @@ cudaError_t launch_w8_decode(const Shape& s, const GemmArgsW8& g, cudaStream_t s
   p.timeout_ns = g.timeout_ns;
   // the sub-tile counters start at zero; an expert of c rows has ceil(c / NMAX) sub-tiles,
   // so there are at most T k / NMAX + E of them, within rmax / 64 (rmax >= T k + 128 E)
+  // (unless a kernel before this one zeroed them, so that this launch overlaps its tail)
   const int64_t subs = (int64_t)s.T * s.k / NMAX + s.E;
-  cudaError_t e = cudaMemsetAsync(g.row_ready, 0, (size_t)(g.rmax / 64) * sizeof(int32_t), st);
+  cudaError_t e = g.row_ready_zeroed
+                      ? cudaSuccess
+                      : cudaMemsetAsync(g.row_ready, 0, (size_t)(g.rmax / 64) * sizeof(int32_t), st);
   if (e == cudaSuccess) {
     const int64_t tiles = subs * (s.I / 128 + s.H / 128);
     int64_t grid = std::min<int64_t>(num_sms(), tiles);

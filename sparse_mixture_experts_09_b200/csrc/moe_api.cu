@@ -206,6 +206,7 @@ struct SplitK {
   int32_t* sem = nullptr;
   int32_t* row_ready = nullptr;
   const int32_t* q_counts = nullptr;  // routed rows per expert (sizes one-grid row tiles)
+  bool row_ready_zeroed = false;      // the gather kernel zeroed row_ready
 };
 
 moe_status_t run_experts(const Shape& s, const uint16_t* x_perm, const int32_t* offsets,
@@ -233,6 +234,7 @@ moe_status_t run_experts(const Shape& s, const uint16_t* x_perm, const int32_t* 
     g.rmax = max_padded_rows(s);
     g.timeout_ns = kTimeoutNs;
     g.row_ready = split.row_ready;
+    g.row_ready_zeroed = split.row_ready_zeroed;
     g.counts = split.q_counts;
     e = launch_grouped_swiglu_w8(s, g, st, &why);
   } else {
@@ -251,6 +253,7 @@ moe_status_t run_experts(const Shape& s, const uint16_t* x_perm, const int32_t* 
     g.partial = split.partial;
     g.split_sem = split.sem;
     g.row_ready = split.row_ready;
+    g.row_ready_zeroed = split.row_ready_zeroed;
     g.expert_rows = split.q_counts;
     e = launch_grouped_swiglu(s, g, st, &why);
   }
@@ -268,10 +271,12 @@ moe_status_t run_forward(const Shape& s, const uint16_t* x, const uint16_t* wr, 
   e = launch_permute(s, at<int32_t>(ws, L.topk_idx), x, at<int32_t>(ws, L.counts),
                      at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.row_of),
                      at<int32_t>(ws, L.token_of_row), at<uint16_t>(ws, L.x_perm),
-                     at<int32_t>(ws, L.block_base), st, norm_w, rnorm, w.q1 != nullptr);
+                     at<int32_t>(ws, L.block_base), st, norm_w, rnorm, w.q1 != nullptr,
+                     at<int32_t>(ws, L.row_ready), (int)(max_padded_rows(s) / 64));
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   SplitK split;
   split.row_ready = at<int32_t>(ws, L.row_ready);
+  split.row_ready_zeroed = true;
   split.q_counts = at<int32_t>(ws, L.counts);
   if (L.partial != L.end) {
     split.counts = at<int32_t>(ws, L.counts);

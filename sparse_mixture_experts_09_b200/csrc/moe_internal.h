@@ -50,7 +50,8 @@ cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16
                            int32_t* counts, int32_t* offsets, int32_t* row_of,
                            int32_t* token_of_row, uint16_t* x_perm, int32_t* block_base,
                            cudaStream_t st, const uint16_t* norm_w = nullptr,
-                           const float* rnorm = nullptr, bool f16_out = false);
+                           const float* rnorm = nullptr, bool f16_out = false,
+                           int32_t* zero_buf = nullptr, int zero_n = 0);
 
 // x_perm rows [0, rows) of width H: bf16 -> IEEE half (the int8 experts' input).
 cudaError_t launch_rows_to_f16(const uint16_t* src, uint16_t* dst, int64_t rows, int H,
@@ -87,6 +88,9 @@ struct GemmArgs {
   // [E] routed rows per expert (nullable): they size the one-grid kernel's row tiles
   // (16-row steps); null: every row tile is sized for its full 128 rows or the batch
   const int32_t* expert_rows = nullptr;
+  // row_ready was zeroed by an earlier kernel in the stream (the gather): no memset,
+  // so the one-grid kernel's launch overlaps the kernels before it
+  bool row_ready_zeroed = false;
 };
 
 // GEMM1 (gate/up + SwiGLU -> h) then GEMM2 (h w2^T -> y), both persistent tcgen05.
@@ -133,6 +137,8 @@ struct GemmArgsW8 {
   // [E] routed rows per expert (nullable): they size the one-grid kernel's sub-tiles
   // (16-row steps); null: an expert is taken to have min(T, its padded rows) rows
   const int32_t* counts = nullptr;
+  // row_ready was zeroed by an earlier kernel in the stream (the gather): no memset
+  bool row_ready_zeroed = false;
 };
 
 // GEMM1 (int8 or 4-bit gate/up + SwiGLU -> h) then GEMM2 (h q2^T -> y), in float16.

@@ -409,9 +409,14 @@ __global__ void __launch_bounds__(256) k_gather(const uint16_t* __restrict__ x, 
                                                 int32_t* __restrict__ token_of_row,
                                                 uint16_t* __restrict__ x_perm,
                                                 const uint16_t* __restrict__ norm_w,
-                                                const float* __restrict__ rnorm) {
+                                                const float* __restrict__ rnorm,
+                                                int32_t* __restrict__ zero_buf, int zero_n) {
   pdl_trigger();
   pdl_wait();
+  // the expert GEMMs' sub-tile counters start at zero (their previous users have
+  // finished: every kernel before this one in the stream has)
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < zero_n; i += blockDim.x) zero_buf[i] = 0;
   __shared__ int32_t s_off[65], s_cnt[64];
   for (int e = threadIdx.x; e <= E; e += blockDim.x) {
     s_off[e] = offsets[e];
@@ -503,7 +508,7 @@ cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16
                            int32_t* counts, int32_t* offsets, int32_t* row_of,
                            int32_t* token_of_row, uint16_t* x_perm, int32_t* block_base,
                            cudaStream_t st, const uint16_t* norm_w, const float* rnorm,
-                           bool f16_out) {
+                           bool f16_out, int32_t* zero_buf, int zero_n) {
   const int64_t nb = num_token_blocks(s);
   cudaError_t e;
   if (nb <= 32) {
@@ -527,7 +532,7 @@ cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16
   if (gblocks > cap) gblocks = cap;
 #define MOE_GATHER(NM, FH)                                                                   \
   launch_pdl(k_gather<NM, FH>, dim3((unsigned)gblocks), dim3(256), 0, st, x, s.H, s.E, counts, \
-             offsets, token_of_row, x_perm, norm_w, rnorm)
+             offsets, token_of_row, x_perm, norm_w, rnorm, zero_buf, zero_n)
   if (norm_w) return f16_out ? MOE_GATHER(true, true) : MOE_GATHER(true, false);
   return f16_out ? MOE_GATHER(false, true) : MOE_GATHER(false, false);
 #undef MOE_GATHER
