@@ -1008,18 +1008,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 // k_decode_swap: both expert GEMMs of a batch of at most 256 tokens in one persistent
 // grid, with the operands swapped: the weights are the tcgen05 M operand (128 weight
 // rows per tile, loaded by TMA straight into the 128-byte swizzled K-major layout the
-// MMA reads) and a row tile's routed rows the N operand (N = the tile's row count
-// rounded up to 16, at most NMAX; a token reaches an expert at most once, so up to 64
-// tokens every expert has one row tile). A stage holds 4 KB 128 x 64 weight boxes
-// (gate/up: the w1 and w3 boxes of KB k-blocks; down: 2 KB k-blocks of one w2 box; KB =
-// 2, or 1 for NMAX = 128 so that three stages of rows still fit) and its k-blocks of
-// rows.
+// MMA reads) and a sub-tile of at most NMAX of an expert's routed rows the N operand (N
+// = the sub-tile's row count rounded up to 16; a token reaches an expert at most once,
+// so up to NMAX tokens every expert has one sub-tile). An expert with more rows has
+// several sub-tiles over the same weight tiles, consecutive tiles, so the weights cross
+// HBM once. A stage holds twice KB weight boxes of 128 x 64 (gate/up: the w1 and w3
+// boxes of KB k-blocks; down: twice KB k-blocks of one w2 box; KB = 2, or 1 for NMAX =
+// 128 so that three stages of rows still fit) and its k-blocks of rows.
 // Against the tile kernels this moves 2 KiB of routed rows per 64 KiB of weights
 // instead of a 16 KiB activation tile per 32 KiB, and runs both GEMMs as one grid.
 //
 //   warp 0      weight boxes (TMA);
 //   warp 6      routed rows (TMA, 16-row boxes); a down tile first waits until every
-//               gate/up tile of its row tile has released its rows of h;
+//               gate/up tile of its sub-tile has released its rows of h;
 //   warps 1, 7  issue the MMAs (M = 128, N = rows): gate/up the first issues gate, the
 //               second up; down each issues KB of the stage's 2 KB k-blocks into its
 //               own partial sum;
@@ -1046,7 +1047,7 @@ struct DecBf16 {
                                    : 2 * ACC_COLS <= 256 ? 256
                                                          : 512;
   static constexpr int NUM_BARS = 3 * STAGES + 6;
-  static constexpr int SMEM = 1024 + STAGES * STAGE + NUM_BARS * 8 + 16 + 2 * 72 * 4;
+  static constexpr int SMEM = 1024 + STAGES * STAGE + NUM_BARS * 8 + 16 + 3 * 72 * 4;
   // D f32, A and B bf16, both K-major, M = 128; N is set per tile
   static constexpr uint32_t IDESC_M128 =
       (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 4) << 24);
@@ -1062,23 +1063,25 @@ struct DecBf16Params {
   uint16_t* h;             // [rows, I] bf16
   float* y;                // [rows, H] fp32
   int32_t* status;
-  int32_t* row_ready;      // [rows / 128], zero at launch
+  int32_t* row_ready;      // [rows / 64] per-sub-tile counters, zero at launch
   int E, H, I, blocked;
+  int max_rows;            // most rows an expert can have: the tokens
   unsigned long long timeout_ns;
 };
 
-// Tile L -> (expert e, row tile m, column tile n) of a grid whose tiles are n_tiles per
-// row tile; an expert's row tiles of one column tile are consecutive, so its weight tile
-// is read from HBM once and from L2 for the other row tiles
-__device__ __forceinline__ void swap_coords(int L, const int* row_tiles, int E, int n_tiles,
+// Tile L -> (expert e, sub-tile m, column tile n) of a grid whose tiles are n_tiles per
+// sub-tile (first_sub[e]: the expert's first sub-tile); an expert's sub-tiles of one
+// column tile are consecutive, so its weight tile is read from HBM once and from L2 for
+// the other sub-tiles
+__device__ __forceinline__ void swap_coords(int L, const int* first_sub, int E, int n_tiles,
                                             int& e, int& m, int& n) {
   const int mrow = L / n_tiles;
   e = 0;
-  while (e + 1 < E && row_tiles[e + 1] <= mrow) ++e;
-  const int cnt = row_tiles[e + 1] - row_tiles[e];
-  const int local = L - row_tiles[e] * n_tiles;
+  while (e + 1 < E && first_sub[e + 1] <= mrow) ++e;
+  const int cnt = first_sub[e + 1] - first_sub[e];
+  const int local = L - first_sub[e] * n_tiles;
   n = local / cnt;
-  m = row_tiles[e] + local % cnt;
+  m = first_sub[e] + local % cnt;
 }
 
 // Wait until *ready >= target (acquire: the h rows stored before the release are then
@@ -1115,8 +1118,9 @@ __global__ void __launch_bounds__(256, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kS * D::STAGE);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + D::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  int* row_tiles = reinterpret_cast<int*>(tmem_holder + 4);  // [E + 1]
-  int* nrows = row_tiles + 72;                                // [E]: routed rows (or -1)
+  int* sub0 = reinterpret_cast<int*>(tmem_holder + 4);  // [E + 1]: first sub-tile of each expert
+  int* nrows = sub0 + 72;                                // [E]: routed rows of each expert
+  int* row_off = nrows + 72;                             // [E]: first row of each expert
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int KB = D::KB;
@@ -1164,28 +1168,39 @@ __global__ void __launch_bounds__(256, 1)
   }
   pdl_trigger();
   pdl_wait();
-  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) row_tiles[i] = p.offsets[i] / BM;
-  for (int i = threadIdx.x; i < p.E; i += blockDim.x) nrows[i] = p.counts ? p.counts[i] : -1;
+  for (int i = threadIdx.x; i < p.E; i += blockDim.x) {
+    const int padded = p.offsets[i + 1] - p.offsets[i];
+    nrows[i] = p.counts ? p.counts[i] : (padded < p.max_rows ? padded : p.max_rows);
+    row_off[i] = p.offsets[i];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int i = 0; i < p.E; ++i) {
+      sub0[i] = acc;
+      acc += (nrows[i] + NMAX - 1) / NMAX;
+    }
+    sub0[p.E] = acc;
+  }
   fence_before();
   __syncthreads();
   fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  // N of row tile m of expert e: its routed rows rounded up to 16, at most NMAX (NMAX
-  // when the counts are not given)
+  // sub-tile m of expert e: its first row, and N = its rows rounded up to 16 (at most NMAX)
+  auto sub_row0 = [&](int e, int m) { return row_off[e] + (m - sub0[e]) * NMAX; };
   auto tile_n = [&](int e, int m) {
-    if (nrows[e] < 0) return NMAX;
-    int n = (nrows[e] - (m - row_tiles[e]) * BM + 15) & ~15;
+    const int n = (nrows[e] - (m - sub0[e]) * NMAX + 15) & ~15;
     return n < 16 ? 16 : (n > NMAX ? NMAX : n);
   };
 
-  const int n1 = p.I / 128, n2 = p.H / 128;          // column tiles per row tile
+  const int n1 = p.I / 128, n2 = p.H / 128;          // column tiles per sub-tile
   const int kb1 = p.H / BK, kb2 = p.I / BK;          // k-blocks of w1/w3 and of w2
   const int st1 = kb1 / KB, st2 = kb2 / (2 * KB);    // stages per tile
-  const int total0 = row_tiles[p.E] * n1;
-  const int total = total0 + row_tiles[p.E] * n2;
+  const int total0 = sub0[p.E] * n1;
+  const int total = total0 + sub0[p.E] * n2;
   auto coords = [&](int L, bool& dn, int& e, int& m, int& n) {
     dn = L >= total0;
-    swap_coords(dn ? L - total0 : L, row_tiles, p.E, dn ? n2 : n1, e, m, n);
+    swap_coords(dn ? L - total0 : L, sub0, p.E, dn ? n2 : n1, e, m, n);
   };
 
   if (warp == 0) {
@@ -1243,7 +1258,7 @@ __global__ void __launch_bounds__(256, 1)
         int e, m, n;
         coords(L, dn, e, m, n);
         if (dn) {
-          // every gate/up tile of row tile m has stored its rows of h; the proxy fence
+          // every gate/up tile of sub-tile m has stored its rows of h; the proxy fence
           // orders those stores before the tensor copies (async proxy) that read them
           if (!wait_count(p.row_ready + m, 4 * n1, abort_flag, p.status, p.timeout_ns)) {
             ok = false;
@@ -1251,7 +1266,7 @@ __global__ void __launch_bounds__(256, 1)
           }
           asm volatile("fence.proxy.async.global;" ::: "memory");
         }
-        const int nrow = tile_n(e, m);
+        const int nrow = tile_n(e, m), row0 = sub_row0(e, m);
         const CUtensorMap* map = dn ? &mh : &mx;
         const int nst = dn ? st2 : st1;
         const int nblk = dn ? 2 * KB : KB;
@@ -1265,7 +1280,7 @@ __global__ void __launch_bounds__(256, 1)
           const uint32_t dst = stage(q) + D::BOXES * D::WBOX;
           for (int b = 0; b < nblk; ++b)
             for (int j = 0; j < nrow; j += 16)
-              tma_load_2d(dst + b * D::ACT_UNIT + j * 128, map, (nblk * s + b) * BK, m * BM + j,
+              tma_load_2d(dst + b * D::ACT_UNIT + j * 128, map, (nblk * s + b) * BK, row0 + j,
                           a_full(q));
         }
       }
@@ -1341,7 +1356,7 @@ __global__ void __launch_bounds__(256, 1)
       fence_after();
       const uint32_t tacc =
           tmem_base + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(b * D::ACC_COLS);
-      const int64_t row0 = (int64_t)m * BM;
+      const int64_t row0 = sub_row0(e, m);
       if (!dn) {
         uint16_t* hcol = p.h + row0 * p.I + n * 128 + r;  // intermediate column n 128 + r
         for (int c0 = 0; c0 < nrow; c0 += 16) {
@@ -1356,7 +1371,7 @@ __global__ void __launch_bounds__(256, 1)
                 (uint16_t)(pack_bf16x2_rn(gv / (1.f + __expf(-gv)) * uv, 0.f) & 0xFFFFu);
           }
         }
-        // release this warp's rows of h to the down tiles of row tile m
+        // release this warp's rows of h to the down tiles of sub-tile m
         asm volatile("fence.proxy.async.global;" ::: "memory");
         __threadfence();
         __syncwarp();
@@ -1581,14 +1596,17 @@ cudaError_t launch_decode_swap(const Shape& s, const GemmArgs& g, cudaStream_t s
   p.H = s.H;
   p.I = s.I;
   p.blocked = s.blocked;
+  p.max_rows = (int)s.T;
   p.timeout_ns = g.timeout_ns;
-  // the row-tile counters start at zero (unless a kernel before this one zeroed them: a
-  // memset between the two would keep this launch from overlapping that kernel's tail)
+  // the sub-tile counters start at zero (unless a kernel before this one zeroed them: a
+  // memset between the two would keep this launch from overlapping that kernel's tail);
+  // an expert of c rows has ceil(c / NMAX) sub-tiles, at most T k / NMAX + E in all,
+  // within rmax / 64 (rmax >= T k + 128 E)
   cudaError_t e = g.row_ready_zeroed
                       ? cudaSuccess
-                      : cudaMemsetAsync(g.row_ready, 0, (size_t)(g.rmax / BM) * sizeof(int32_t), st);
+                      : cudaMemsetAsync(g.row_ready, 0, (size_t)(g.rmax / 64) * sizeof(int32_t), st);
   if (e == cudaSuccess) {
-    const int64_t tiles = (g.rmax / BM) * (s.I / 128 + s.H / 128);
+    const int64_t tiles = ((int64_t)s.T * s.k / NMAX + s.E) * (s.I / 128 + s.H / 128);
     int64_t grid = num_sms() < tiles ? num_sms() : tiles;
     if (grid < 1) grid = 1;
     e = launch_pdl(k_decode_swap<NMAX>, dim3((unsigned)grid), dim3(256), (size_t)D::SMEM, st, mw1,
@@ -1700,10 +1718,13 @@ cudaError_t launch_wait_selftest(int32_t* status, unsigned long long timeout_ns,
 
 cudaError_t launch_grouped_swiglu(const Shape& s, const GemmArgs& g, cudaStream_t st,
                                   const char** why) {
-  // the swap-operand kernel: at most 64 tokens with hidden % 128 == 0 and intermediate
-  // % 256 == 0 (two k-blocks per stage), or up to 256 tokens with 128-row tiles (one
-  // k-block per stage)
-  if (MOE_SWAP_DECODE && g.row_ready && s.T <= 64 && s.H % 128 == 0 && s.I % 256 == 0)
+  // the swap-operand kernel, hidden % 128 == 0: sub-tiles of 16, 32 or 64 rows (two
+  // k-blocks per stage, intermediate % 256 == 0) up to 64 tokens, and up to 256 tokens
+  // while the batch averages at most 56 routed rows per expert (measured: above that most
+  // experts take two 64-row sub-tiles and the 128-row ones are faster); otherwise up to
+  // 256 tokens 128-row sub-tiles (one k-block per stage, intermediate % 128 == 0)
+  const bool rows64 = s.T <= 64 || (int64_t)s.T * s.k <= 56 * (int64_t)s.E;
+  if (MOE_SWAP_DECODE && g.row_ready && s.T <= 256 && s.H % 128 == 0 && s.I % 256 == 0 && rows64)
     return s.T <= 16   ? launch_decode_swap<16>(s, g, st, why)
            : s.T <= 32 ? launch_decode_swap<32>(s, g, st, why)
                        : launch_decode_swap<64>(s, g, st, why);

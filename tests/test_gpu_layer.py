@@ -47,11 +47,13 @@ def test_forward_small(name):
 
 
 # At most 256 tokens the bf16 layer runs both expert GEMMs as one swap-operand kernel:
-# up to 64 tokens its 16-, 32- and 64-row variants (7, 17, 24, 48, 50 and 64 tokens), N =
-# 16 .. 64 per expert (2 experts at 24 and 48 tokens: N = 32 and 48), E = 64 with k = 8
-# and a hidden size that is not a multiple of 256; above 64 tokens its 128-row tiles (65
-# tokens on 2 experts: N = 80; 200 tokens on 2 experts: row tiles of 128 and 72 rows, an
-# intermediate size that is not a multiple of 256; 256 tokens on 8 experts).
+# 16-, 32- and 64-row sub-tiles up to 64 tokens (7, 17, 24, 48, 50 and 64 tokens; N = 32
+# and 48 on 2 experts at 24 and 48 tokens; E = 64 with k = 8; a hidden size that is not
+# a multiple of 256), 64-row sub-tiles above that while experts average at most 56 rows
+# (160 tokens with one expert holding 155 rows: sub-tiles of 64, 64 and 27; 96 tokens
+# with one at 66), else 128-row sub-tiles (65 tokens on 2 experts: N = 80; 200 tokens on
+# 2 experts: 128 and 72 rows, an intermediate size that is not a multiple of 256; 256
+# tokens on 8 experts).
 SWAP_128 = {
     "t200_e2": W.Workload("t200_e2", 200, 256, 384, 2, 2, seed=43),
     "t256_e8": W.Workload("t256_e8", 256, 512, 768, 8, 2, seed=44),
@@ -59,7 +61,8 @@ SWAP_128 = {
 
 
 @pytest.mark.parametrize("name", ["ts_k1", "t17_e4", "t24_e2", "t48_e2", "ts_e64k8", "ts_h640",
-                                  "t64_edge", "t65_edge", "t200_e2", "t256_e8"])
+                                  "t64_edge", "t160_skew", "t96_e4", "t65_edge", "t200_e2",
+                                  "t256_e8"])
 def test_forward_swap_operand_widths(name):
     from .test_gpu_w8 import SMALL_BATCH
     w = SWAP_128[name] if name in SWAP_128 else SMALL_BATCH[name]
