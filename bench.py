@@ -38,9 +38,10 @@ GEMM_SOURCE = os.path.join(ROOT, "sparse_mixture_experts_09_b200", "csrc", "gemm
 
 
 def fused_experts(num_tokens: int, hidden: int, inter: int) -> bool:
-    """Whether the bf16 layer runs both expert GEMMs as one swap-operand kernel (at most
-    64 tokens, hidden % 128 == 0, intermediate % 256 == 0)."""
-    return num_tokens <= 64 and hidden % 128 == 0 and inter % 256 == 0
+    """Whether the bf16 layer runs both expert GEMMs as one swap-operand kernel: at most
+    256 tokens, hidden and intermediate multiples of 128 (64-row sub-tiles when the
+    intermediate size is a multiple of 256 and the batch is small, else 128-row ones)."""
+    return num_tokens <= 256 and hidden % 128 == 0 and inter % 128 == 0
 
 
 def kernels_per_forward(num_tokens: int, hidden: int = 4096, inter: int = 14336) -> int:

@@ -80,13 +80,14 @@ def test_clock_sampler_reports_slowdowns_and_tolerates_no_samples():
 
 def test_kernels_per_forward_matches_the_launch_lists():
     # the ncu launch lists: 5 kernels per forward at decode (router, plan, gather, the
-    # swap-operand kernel for both GEMMs, combine); 6 from 65 tokens (two GEMMs) or when
-    # the intermediate size is not a multiple of 256; 8 above 1024 tokens (histogram,
-    # scan and rank replace the plan)
+    # swap-operand kernel for both GEMMs, combine), up to 256 tokens; 6 from 257 tokens
+    # (two GEMMs); 8 above 1024 tokens (histogram, scan and rank replace the plan)
     assert bench.kernels_per_forward(16) == 5
     assert bench.kernels_per_forward(64) == 5
-    assert bench.kernels_per_forward(65) == 6
-    assert bench.kernels_per_forward(16, 4096, 384) == 6
+    assert bench.kernels_per_forward(65) == 5
+    assert bench.kernels_per_forward(256) == 5
+    assert bench.kernels_per_forward(257) == 6
+    assert bench.kernels_per_forward(16, 4096, 384) == 5
     assert bench.kernels_per_forward(1024) == 6
     assert bench.kernels_per_forward(1025) == 8
     assert bench.kernels_per_forward(4096) == 8
