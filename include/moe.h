@@ -376,6 +376,69 @@ moe_status_t moe_gather_rows(const void* src, int64_t src_rows, const int64_t* i
                              int64_t n_rows, int64_t row_bytes, void* dst,
                              moe_stream_t stream);
 
+/* ---- expert parallelism over peer memory (this library's own steps; the pages say
+ * only that experts may be spread over devices, Hugging Face "Mixtral", MixtralConfig
+ * num_local_experts). Rank r's receive buffers are allocated here and shared with the
+ * other ranks' processes through CUDA IPC handles; a rank then stores the rows bound
+ * for rank r straight into r's expert groups, and reads the experts' outputs back from
+ * r's buffer in its combine. Between the steps the caller orders the ranks (a barrier
+ * after each rank's stream has finished the previous step): no kernel here waits on
+ * another rank. */
+
+/* Bytes of an IPC handle (a cudaIpcMemHandle_t). */
+#define MOE_IPC_HANDLE_BYTES 64
+
+/* Allocates `bytes` (> 0) of device memory on the current device that other processes
+ * may map (cudaMalloc; 256-byte aligned) and writes its handle, MOE_IPC_HANDLE_BYTES
+ * bytes, to `handle` (host memory). *dev_ptr receives the buffer (NULL on failure). The
+ * caller owns it: moe_ipc_free. */
+moe_status_t moe_ipc_alloc(size_t bytes, void** dev_ptr, void* handle);
+
+/* Maps a buffer that moe_ipc_alloc made in another process (on this GPU or a peer that
+ * this device can access) and writes its address in this process to *dev_ptr. Opening
+ * a handle in the process that made it fails (MOE_ERR_CUDA). Unmap with moe_ipc_close
+ * before the owner frees it. */
+moe_status_t moe_ipc_open(const void* handle, void** dev_ptr);
+
+/* Unmaps a buffer that moe_ipc_open mapped (NULL: no-op). */
+moe_status_t moe_ipc_close(void* dev_ptr);
+
+/* Frees a buffer that moe_ipc_alloc made (NULL: no-op); every other process must have
+ * unmapped it first. */
+moe_status_t moe_ipc_free(void* dev_ptr);
+
+/* Row scatter into several ranks' buffers: for 0 <= i < n_rows, row dst_row[i] of the
+ * buffer dst_bases[dst_rank[i]] = row src_index[i] of src. Rows are row_bytes bytes (a
+ * positive multiple of 16). src [src_rows] rows, 16-byte aligned, on this device;
+ * src_index [n_rows] int64, dst_rank [n_rows] int32, dst_row [n_rows] int64 device
+ * arrays; dst_bases a device array of `world` device pointers (16-byte aligned; this
+ * device's buffers or peers' mappings from moe_ipc_open), each buffer dst_rows rows. A
+ * row whose source index, rank or destination row is out of range is skipped and
+ * counted into *bad_rows (a device int32, may be NULL). The stores are plain stores:
+ * they are visible to the owner once this launch has finished on `stream`. */
+moe_status_t moe_scatter_rows_peer(const void* src, int64_t src_rows, const int64_t* src_index,
+                                   const int32_t* dst_rank, const int64_t* dst_row,
+                                   int64_t n_rows, void* const* dst_bases, int world,
+                                   int64_t dst_rows, int64_t row_bytes, int32_t* bad_rows,
+                                   moe_stream_t stream);
+
+/* Combine reading the experts' outputs from several ranks' buffers, with moe_combine's
+ * arithmetic (nnterp "Mixtral": slot outputs scaled by their float32 weights, summed,
+ * added to the residual; fp32 in slot order, one rounding to bf16):
+ *   out[t, :] = bf16(residual[t, :] + sum_j topk_w[t, j] * y_j)
+ * with y_j = row slot_row[t k + j] of the fp32 buffer y_bases[slot_rank[t k + j]].
+ *   y_bases: device array of `world` device pointers, each buffer [y_rows, hidden] fp32
+ *   (16-byte aligned); slot_rank [T k] int32 and slot_row [T k] int64 device arrays;
+ *   topk_w [T, k] fp32; residual [T, hidden] bf16 or NULL; out [T, hidden] bf16.
+ *   1 <= k <= 8, hidden a positive multiple of 8. A slot whose rank or row is out of
+ *   range adds nothing and is counted into *bad_slots (device int32, may be NULL).
+ *   num_tokens = 0 is a no-op. */
+moe_status_t moe_combine_peer(const float* const* y_bases, int world, int64_t y_rows,
+                              const int32_t* slot_rank, const int64_t* slot_row,
+                              const float* topk_w, const moe_bf16_t* residual, moe_bf16_t* out,
+                              int64_t num_tokens, int k, int hidden, int32_t* bad_slots,
+                              moe_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the device status word in `ws`:
  * MOE_OK, or MOE_ERR_TIMEOUT if a kernel gave up a bounded wait since the last
  * call. */

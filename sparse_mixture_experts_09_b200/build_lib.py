@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoe.so")
 SOURCES = ["moe_api.cu", "routing.cu", "gemm_sm100.cu", "gemm_w8.cu", "combine.cu", "moe_noalloc.cu",
-           "gather_rows.cu"]
+           "gather_rows.cu", "ep_peer.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -834,4 +834,92 @@ moe_status_t moe_gather_rows(const void* src, int64_t src_rows, const int64_t* i
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "row gather launch");
 }
 
+moe_status_t moe_ipc_alloc(size_t bytes, void** dev_ptr, void* handle) {
+  g_err[0] = 0;
+  if (!dev_ptr || !handle) return fail(MOE_ERR_INVALID_ARG, "dev_ptr and handle must not be NULL");
+  *dev_ptr = nullptr;
+  if (bytes == 0) return fail(MOE_ERR_INVALID_ARG, "bytes must be > 0");
+  void* p = nullptr;
+  cudaError_t e = cudaMalloc(&p, bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc of a shareable buffer");
+  cudaIpcMemHandle_t h;
+  e = cudaIpcGetMemHandle(&h, p);
+  if (e != cudaSuccess) {
+    cudaFree(p);
+    return cuda_fail(e, "cudaIpcGetMemHandle");
+  }
+  memcpy(handle, &h, sizeof h);
+  *dev_ptr = p;
+  return MOE_OK;
+}
+
+moe_status_t moe_ipc_open(const void* handle, void** dev_ptr) {
+  g_err[0] = 0;
+  if (!dev_ptr || !handle) return fail(MOE_ERR_INVALID_ARG, "dev_ptr and handle must not be NULL");
+  *dev_ptr = nullptr;
+  cudaIpcMemHandle_t h;
+  memcpy(&h, handle, sizeof h);
+  cudaError_t e = cudaIpcOpenMemHandle(dev_ptr, h, cudaIpcMemLazyEnablePeerAccess);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "cudaIpcOpenMemHandle");
+}
+
+moe_status_t moe_ipc_close(void* dev_ptr) {
+  g_err[0] = 0;
+  if (!dev_ptr) return MOE_OK;
+  cudaError_t e = cudaIpcCloseMemHandle(dev_ptr);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "cudaIpcCloseMemHandle");
+}
+
+moe_status_t moe_ipc_free(void* dev_ptr) {
+  g_err[0] = 0;
+  if (!dev_ptr) return MOE_OK;
+  cudaError_t e = cudaFree(dev_ptr);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "cudaFree of a shareable buffer");
+}
+
+moe_status_t moe_scatter_rows_peer(const void* src, int64_t src_rows, const int64_t* src_index,
+                                   const int32_t* dst_rank, const int64_t* dst_row,
+                                   int64_t n_rows, void* const* dst_bases, int world,
+                                   int64_t dst_rows, int64_t row_bytes, int32_t* bad_rows,
+                                   moe_stream_t stream) {
+  g_err[0] = 0;
+  if (n_rows < 0 || src_rows < 0 || dst_rows < 0)
+    return fail(MOE_ERR_INVALID_ARG, "row counts must be >= 0");
+  if (world < 1) return fail(MOE_ERR_INVALID_ARG, "world must be >= 1 (got %d)", world);
+  if (row_bytes <= 0 || row_bytes % 16)
+    return fail(MOE_ERR_INVALID_ARG, "row_bytes must be a positive multiple of 16 (got %lld)",
+                (long long)row_bytes);
+  if (n_rows == 0) return MOE_OK;
+  MOE_TRY(check_ptr(src, "src", src_rows == 0));
+  MOE_TRY(check_ptr(src_index, "src_index"));
+  if (!dst_rank || !dst_row || !dst_bases)
+    return fail(MOE_ERR_INVALID_ARG, "dst_rank, dst_row and dst_bases must not be NULL");
+  cudaError_t e = launch_scatter_rows_peer(src, src_rows, src_index, dst_rank, dst_row, n_rows,
+                                           dst_bases, world, dst_rows, row_bytes, bad_rows,
+                                           (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "peer row scatter launch");
+}
+
+moe_status_t moe_combine_peer(const float* const* y_bases, int world, int64_t y_rows,
+                              const int32_t* slot_rank, const int64_t* slot_row,
+                              const float* topk_w, const moe_bf16_t* residual, moe_bf16_t* out,
+                              int64_t num_tokens, int k, int hidden, int32_t* bad_slots,
+                              moe_stream_t stream) {
+  g_err[0] = 0;
+  if (num_tokens < 0 || y_rows < 0) return fail(MOE_ERR_INVALID_ARG, "sizes must be >= 0");
+  if (world < 1) return fail(MOE_ERR_INVALID_ARG, "world must be >= 1 (got %d)", world);
+  if (k < 1 || k > 8) return fail(MOE_ERR_UNSUPPORTED, "k must be in [1, 8] (got %d)", k);
+  if (hidden <= 0 || hidden % 8)
+    return fail(MOE_ERR_UNSUPPORTED, "hidden must be a positive multiple of 8 (got %d)", hidden);
+  if (num_tokens == 0) return MOE_OK;
+  if (!y_bases || !slot_rank || !slot_row || !topk_w)
+    return fail(MOE_ERR_INVALID_ARG, "y_bases, slot_rank, slot_row and topk_w must not be NULL");
+  MOE_TRY(check_ptr(residual, "residual", true));
+  MOE_TRY(check_ptr(out, "out"));
+  cudaError_t e = launch_combine_peer(y_bases, world, y_rows, slot_rank, slot_row, topk_w,
+                                      residual, out, num_tokens, hidden, k, bad_slots,
+                                      (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "peer combine launch");
+}
+
 }  // extern "C"

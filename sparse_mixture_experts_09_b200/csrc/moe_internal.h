@@ -162,6 +162,18 @@ cudaError_t launch_combine(const Shape& s, const float* y, const int32_t* row_of
 cudaError_t launch_gather_rows(const void* src, void* dst, const int64_t* index, int64_t n_rows,
                                int64_t src_rows, int64_t row_bytes, cudaStream_t st);
 
+// Peer-memory exchange of the expert-parallel layer (ep_peer.cu). dst_bases and y_bases
+// are device arrays of `world` device pointers (this GPU's buffers or peers' mappings).
+cudaError_t launch_scatter_rows_peer(const void* src, int64_t src_rows, const int64_t* src_index,
+                                     const int32_t* dst_rank, const int64_t* dst_row,
+                                     int64_t n_rows, void* const* dst_bases, int world,
+                                     int64_t dst_rows, int64_t row_bytes, int32_t* bad,
+                                     cudaStream_t st);
+cudaError_t launch_combine_peer(const float* const* y_bases, int world, int64_t y_rows,
+                                const int32_t* slot_rank, const int64_t* slot_row,
+                                const float* topk_w, const uint16_t* residual, uint16_t* out,
+                                int64_t T, int H, int k, int32_t* bad, cudaStream_t st);
+
 int num_sms();
 
 // Host helpers of the C ABI (moe_api.cu): shape validation returning a moe_status_t

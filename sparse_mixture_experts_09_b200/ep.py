@@ -65,16 +65,16 @@ class CudaOps:
     def gather_rows(self, src, index):
         return self.moe.gather_rows(src, index)
 
-    def grouped_swiglu(self, x_groups, offsets, w1, w3, w2, rows):
+    def grouped_swiglu(self, x_groups, offsets, w1, w3, w2, rows, y=None):
         """The experts on `rows` routed rows in expert groups (x_groups holds
-        padded_rows(rows, E) rows)."""
+        padded_rows(rows, E) rows); into `y` when given."""
         e, i, h = w1.shape
         rows = max(rows, 1)
         shape = self.moe.make_shape(rows, h, i, e, 1)
         ws = self._workspace("experts", shape, x_groups.device)
-        return self.moe.grouped_swiglu(x_groups, offsets, w1, w3, w2, rows, 1, ws)
+        return self.moe.grouped_swiglu(x_groups, offsets, w1, w3, w2, rows, 1, ws, y=y)
 
-    def grouped_swiglu_quantized(self, x_groups, offsets, experts, rows):
+    def grouped_swiglu_quantized(self, x_groups, offsets, experts, rows, y=None):
         """The same with int8 (Int8Experts) or 4-bit (Int4Experts) expert weights."""
         e, i, _ = experts.q1.shape
         h = x_groups.shape[1]
@@ -83,7 +83,14 @@ class CudaOps:
         ws = self._workspace("experts", shape, x_groups.device)
         fn = (self.moe.grouped_swiglu_w4 if isinstance(experts, self.moe.Int4Experts)
               else self.moe.grouped_swiglu_w8)
-        return fn(x_groups, offsets, experts, rows, 1, ws)
+        return fn(x_groups, offsets, experts, rows, 1, ws, y=y)
+
+    def scatter_rows_peer(self, src, src_index, dst_rank, dst_row, dst_bases, dst_rows):
+        self.moe.scatter_rows_peer(src, src_index, dst_rank, dst_row, dst_bases, dst_rows)
+
+    def combine_peer(self, y_bases, y_rows, slot_rank, slot_row, topk_w, hidden, residual):
+        return self.moe.combine_peer(y_bases, y_rows, slot_rank, slot_row, topk_w, hidden,
+                                     residual)
 
     def combine(self, y_perm, row_of, topk_w, residual, num_experts, intermediate_size):
         return self.moe.combine(y_perm, row_of, topk_w, residual, num_experts, intermediate_size)
@@ -292,3 +299,232 @@ def shard_experts(w1, w3, w2, rank: int, world: int):
     lo, hi = rank * e // world, (rank + 1) * e // world
     return w1[lo:hi].contiguous(), w3[lo:hi].contiguous(), w2[lo:hi].contiguous()
 
+
+
+# ---- the same layer with the exchanges as peer-memory loads and stores ----
+#
+# Every rank allocates its receive buffers once (PeerBuffers: x_local [rows, H] bf16,
+# the expert groups the grouped GEMM reads, and y_local [rows, H] fp32, what it writes)
+# and maps every other rank's through CUDA IPC. One layer, after routing and permuting
+# as above:
+#
+# 1. all-gather every rank's routed rows per expert (world x E integers), so each rank
+#    knows every owner's group layout;
+# 2. store each real routed row straight into its owner's x_local, at its final place:
+#    the owner's group for that expert, after the rows of lower source ranks (one
+#    kernel of plain stores; it replaces the all-to-all and both regrouping gathers);
+# 3. barrier; every owner runs its experts from x_local into y_local;
+# 4. barrier; each rank's combine reads its slots' outputs from the owners' y_local
+#    (plain loads) and adds them into the residual; barrier, so the buffers are free
+#    for the next layer.
+#
+# The barriers order the ranks between kernels: no kernel waits on another rank.
+
+
+def peer_plan(offsets, counts_all, rank: int, world: int, device=None):
+    """Plan of the peer-memory exchange for rank `rank`, in whole-tensor index
+    arithmetic. offsets: this rank's padded group offsets [E+1]; counts_all [world, E]:
+    every rank's routed rows per expert (E = world * E_loc). Returns a dict:
+      send_index [n_send] int64: this rank's x_perm rows to send (real rows, expert order);
+      dst_rank [n_send] int32: the owner of each; dst_row [n_send] int64: its row in the
+        owner's x_local (the owner's group for the expert, each group padded to 128 rows
+        and holding the source ranks' rows in rank order);
+      local_offsets [E_loc+1] (ints): this rank's own groups as an owner;
+      n_recv (int): the real rows this rank receives in them;
+      row_rank [offsets[-1]] int32, row_dst [offsets[-1]] int64: for each x_perm row,
+        the owner and row of its expert output (-1 on pad rows).
+    The sizes come to the host in one read."""
+    i64 = dict(dtype=torch.int64, device=device)
+    offsets = torch.as_tensor(offsets, **i64).reshape(-1)
+    c = torch.as_tensor(counts_all, **i64).reshape(world, -1)
+    e_total = c.shape[1]
+    if e_total % world:
+        raise ValueError(f"{e_total} experts do not split over {world} ranks")
+    e_loc = e_total // world
+    padded = _pad(c.sum(0)).reshape(world, e_loc)            # rows of each owner's groups
+    group_start = (torch.cumsum(padded, 1) - padded).reshape(-1)
+    before = (torch.cumsum(c, 0) - c)[rank]                  # rows of expert e from ranks < rank
+    counts = c[rank]
+    mine = c[:, rank * e_loc:(rank + 1) * e_loc].sum().reshape(1)
+    host = torch.cat([offsets[-1:], counts.sum().reshape(1), mine, padded[rank]]).cpu()
+    n_rows, n_send, n_recv = int(host[0]), int(host[1]), int(host[2])
+    local_offsets = [0] + torch.cumsum(host[3:], 0).tolist()
+    grp, j = _segment_ranks(counts, n_send)
+    send_index = offsets[:-1][grp] + j
+    dst_rank = (grp // e_loc).to(torch.int32)
+    dst_row = group_start[grp] + before[grp] + j
+    row_rank = torch.full((n_rows,), -1, dtype=torch.int32, device=device)
+    row_rank[send_index] = dst_rank
+    row_dst = torch.full((n_rows,), -1, **i64)
+    row_dst[send_index] = dst_row
+    return {"send_index": send_index, "dst_rank": dst_rank, "dst_row": dst_row,
+            "local_offsets": local_offsets, "n_recv": n_recv, "row_rank": row_rank,
+            "row_dst": row_dst}
+
+
+def peer_rows_needed(max_tokens: int, k: int, world: int, e_loc: int) -> int:
+    """Rows an owner's buffers need: every rank's tokens all routed to this owner
+    (world * max_tokens * k rows) in E_loc groups, as the grouped GEMM sizes them."""
+    r = world * max_tokens * k
+    return (r + 127) // 128 * 128 + 128 * e_loc
+
+
+class PeerBuffers:
+    """This rank's receive buffers of the peer-memory layer and every rank's addresses.
+
+    x_local [rows, hidden] bf16 and y_local [rows, hidden] fp32 are allocated by the
+    library (moe_ipc_alloc) and zeroed; ``share`` (default: all_gather_object over
+    ``group``) gives every rank's IPC handles, and the other ranks' buffers are mapped
+    (moe_ipc_open). x_bases / y_bases: int64 device tensors of the world's addresses,
+    indexed by rank. ``close()`` unmaps, waits for every rank, and frees."""
+
+    def __init__(self, rows: int, hidden: int, group=None, device=None, share=None):
+        from . import moe
+        self.moe = moe
+        self.rows, self.hidden, self.group = rows, hidden, group
+        self.device = device or torch.device("cuda", torch.cuda.current_device())
+        self.rank = dist.get_rank(group)
+        world = dist.get_world_size(group)
+        x_ptr, x_h = moe.ipc_alloc(rows * hidden * 2)
+        y_ptr, y_h = moe.ipc_alloc(rows * hidden * 4)
+        self._own = [x_ptr, y_ptr]
+        self._mapped = []
+        self.x_local = moe.tensor_at(x_ptr, (rows, hidden), torch.bfloat16, self.device)
+        self.y_local = moe.tensor_at(y_ptr, (rows, hidden), torch.float32, self.device)
+        self.x_local.zero_()
+        self.y_local.zero_()
+        torch.cuda.synchronize(self.device)
+        if share is None:
+            def share(obj):
+                out = [None] * world
+                dist.all_gather_object(out, obj, group=group)
+                return out
+        handles = share((x_h, y_h, rows, hidden))
+        # the stores and loads index every rank's buffers with this rank's row count
+        if any((rr, hh) != (rows, hidden) for _, _, rr, hh in handles):
+            for p in self._own:
+                moe.ipc_free(p)
+            raise ValueError("every rank's PeerBuffers must have the same rows and hidden size: "
+                             f"{[(rr, hh) for _, _, rr, hh in handles]}")
+        xs, ys = [], []
+        for r, (xh, yh, _, _) in enumerate(handles):
+            if r == self.rank:
+                xs.append(x_ptr)
+                ys.append(y_ptr)
+            else:
+                xs.append(moe.ipc_open(xh))
+                ys.append(moe.ipc_open(yh))
+                self._mapped += [xs[-1], ys[-1]]
+        self.x_bases = torch.tensor(xs, dtype=torch.int64, device=self.device)
+        self.y_bases = torch.tensor(ys, dtype=torch.int64, device=self.device)
+
+    def close(self, barrier=None):
+        """Unmap the other ranks' buffers, wait at ``barrier`` (default: a group
+        barrier) until every rank has done the same, then free this rank's."""
+        for p in self._mapped:
+            self.moe.ipc_close(p)
+        self._mapped = []
+        (barrier or (lambda: dist.barrier(group=self.group)))()
+        self.x_local = self.y_local = None
+        for p in self._own:
+            self.moe.ipc_free(p)
+        self._own = []
+
+
+def _default_barrier(group, device):
+    def barrier():
+        torch.cuda.current_stream(device).synchronize()
+        dist.barrier(group=group)
+    return barrier
+
+
+def _default_gather_counts(group, world):
+    def gather(counts):
+        parts = [torch.empty_like(counts) for _ in range(world)]
+        dist.all_gather(parts, counts, group=group)
+        return torch.stack(parts)
+    return gather
+
+
+def forward_ep_peer(x, w_router, w1_local, w3_local, w2_local, k: int, num_experts: int,
+                    bufs: PeerBuffers, group=None, residual=None, logit_bias=None, ops=None,
+                    gather_counts=None, barrier=None):
+    """forward_ep with the exchanges as peer-memory stores and loads (PeerBuffers).
+    ``gather_counts(counts [E] int64) -> [world, E]`` (default: all_gather over
+    ``group``) and ``barrier()`` (default: wait for this rank's stream, then a group
+    barrier) can be replaced, e.g. by host-side collectives in tests."""
+    ops = ops or _default_ops()
+    return _forward_ep_peer(
+        x, w_router, k, num_experts, w1_local.shape[0], w1_local.shape[1],
+        lambda xl, off, n, y: ops.grouped_swiglu(xl, off, w1_local, w3_local, w2_local, n, y=y),
+        bufs, group, residual, logit_bias, ops, gather_counts, barrier)
+
+
+def forward_ep_peer_quantized(x, w_router, experts_local, k: int, num_experts: int,
+                              bufs: PeerBuffers, group=None, residual=None, logit_bias=None,
+                              ops=None, gather_counts=None, barrier=None):
+    """forward_ep_peer with this rank's experts as int8 or 4-bit codes."""
+    ops = ops or _default_ops()
+    e_loc, inter = experts_local.q1.shape[0], experts_local.q1.shape[1]
+    return _forward_ep_peer(
+        x, w_router, k, num_experts, e_loc, inter,
+        lambda xl, off, n, y: ops.grouped_swiglu_quantized(xl, off, experts_local, n, y=y),
+        bufs, group, residual, logit_bias, ops, gather_counts, barrier)
+
+
+def _forward_ep_peer(x, w_router, k, num_experts, held, inter, run_experts, bufs, group,
+                     residual, logit_bias, ops, gather_counts, barrier):
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    if num_experts % world:
+        raise ValueError(f"num_experts {num_experts} is not a multiple of the group size {world}")
+    e_loc = num_experts // world
+    if held != e_loc:
+        raise ValueError(f"this rank must hold {e_loc} experts, got {held}")
+    hidden = x.shape[1]
+    if hidden != bufs.hidden:
+        raise ValueError(f"the buffers hold rows of {bufs.hidden}, x has {hidden}")
+    dev = x.device
+    gather_counts = gather_counts or _default_gather_counts(group, world)
+    barrier = barrier or _default_barrier(group, dev)
+
+    # routing and permutation of this rank's tokens (none: it only takes part)
+    if x.shape[0] == 0:
+        wt = None
+        perm = {"offsets": torch.zeros(num_experts + 1, dtype=torch.int64, device=dev),
+                "counts": torch.zeros(num_experts, dtype=torch.int64, device=dev),
+                "x_perm": torch.empty((0, hidden), dtype=x.dtype, device=dev)}
+    else:
+        idx, wt = ops.router_topk(x, w_router, k, logit_bias)
+        perm = ops.permute(idx, x, num_experts, inter)
+    offsets = perm["offsets"].to(dev, torch.int64)
+    counts = perm["counts"].to(dev, torch.int64)
+
+    # 1. every rank's counts; 2. the rows into their owners' groups
+    counts_all = gather_counts(counts).to(dev, torch.int64).reshape(world, num_experts)
+    plan = peer_plan(offsets, counts_all, rank, world, device=dev)
+    n_recv = plan["n_recv"]
+    # the grouped GEMM's buffer rows for n_recv rows in E_loc groups (they cover the
+    # padded groups: local_offsets[-1] <= n_recv + 127 E_loc)
+    rows_buf = ops.padded_rows(n_recv, e_loc)
+    if rows_buf > bufs.rows:
+        raise ValueError(f"this rank receives {n_recv} rows; the grouped GEMM needs "
+                         f"{rows_buf} buffer rows, the buffers hold {bufs.rows}")
+    ops.scatter_rows_peer(perm["x_perm"], plan["send_index"], plan["dst_rank"], plan["dst_row"],
+                          bufs.x_bases, bufs.rows)
+    barrier()
+    # 3. this rank's experts on the rows every rank stored here
+    loc_off = torch.tensor(plan["local_offsets"], dtype=torch.int32, device=dev)
+    run_experts(bufs.x_local[:rows_buf], loc_off, n_recv, bufs.y_local[:rows_buf])
+    barrier()
+    # 4. the combine reads each slot's output where its owner wrote it
+    if x.shape[0] == 0:
+        out = torch.empty((0, hidden), dtype=x.dtype, device=dev)
+    else:
+        row_of = perm["row_of"].to(dev, torch.int64).reshape(-1)
+        slot_rank = plan["row_rank"][row_of].contiguous()
+        slot_row = plan["row_dst"][row_of].contiguous()
+        out = ops.combine_peer(bufs.y_bases, bufs.rows, slot_rank, slot_row, wt, hidden,
+                               residual)
+    barrier()
+    return out

@@ -28,7 +28,9 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_size_host", "moe_max_padded_rows
            "moe_forward_host", "moe_device_status", "moe_last_error", "moe_permute_static",
            "moe_selftest_wait_timeout", "moe_forward_rmsnorm", "moe_pack_weights",
            "moe_quantize_int8", "moe_grouped_swiglu_w8", "moe_forward_w8", "moe_gather_rows",
-           "moe_forward_host_async", "moe_quantize_int4", "moe_grouped_swiglu_w4", "moe_forward_w4")
+           "moe_forward_host_async", "moe_quantize_int4", "moe_grouped_swiglu_w4", "moe_forward_w4",
+           "moe_ipc_alloc", "moe_ipc_open", "moe_ipc_close", "moe_ipc_free",
+           "moe_scatter_rows_peer", "moe_combine_peer")
 
 
 @dataclass
@@ -149,6 +151,20 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_w4.restype = st
         L.moe_gather_rows.argtypes = [_P, ctypes.c_int64, _P, ctypes.c_int64, ctypes.c_int64, _P, _P]
         L.moe_gather_rows.restype = st
+        L.moe_ipc_alloc.argtypes = [_SZ, ctypes.POINTER(_P), _P]
+        L.moe_ipc_alloc.restype = st
+        L.moe_ipc_open.argtypes = [_P, ctypes.POINTER(_P)]
+        L.moe_ipc_open.restype = st
+        L.moe_ipc_close.argtypes = [_P]
+        L.moe_ipc_close.restype = st
+        L.moe_ipc_free.argtypes = [_P]
+        L.moe_ipc_free.restype = st
+        L.moe_scatter_rows_peer.argtypes = [_P, ctypes.c_int64, _P, _P, _P, ctypes.c_int64, _P,
+                                            ctypes.c_int, ctypes.c_int64, ctypes.c_int64, _P, _P]
+        L.moe_scatter_rows_peer.restype = st
+        L.moe_combine_peer.argtypes = [_P, ctypes.c_int, ctypes.c_int64, _P, _P, _P, _P, _P,
+                                       ctypes.c_int64, ctypes.c_int, ctypes.c_int, _P, _P]
+        L.moe_combine_peer.restype = st
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         _lib = L
@@ -309,14 +325,24 @@ def permute_static(topk_idx, x, num_experts: int, intermediate_size: int, stream
     return out
 
 
+def _out_rows(y, rows: int, h: int, device):
+    """The experts' fp32 output: y itself (its first rows x h elements are written; it
+    must hold at least that many), or a new zeroed [rows, h] tensor."""
+    if y is None:
+        return torch.zeros((rows, h), dtype=torch.float32, device=device)
+    _sized("y_perm", y, rows * h, at_least=True)
+    return y
+
+
 def grouped_swiglu(x_perm, offsets, w1, w3, w2, num_tokens: int, k: int, ws, stream=None,
-                   weight_layout: int = ROW_MAJOR):
-    """y_perm [R_max, H] fp32 = w2[e] (silu(w1[e] x) * w3[e] x) per routed row."""
+                   weight_layout: int = ROW_MAJOR, y=None):
+    """y_perm [R_max, H] fp32 = w2[e] (silu(w1[e] x) * w3[e] x) per routed row (into
+    `y` when given: an fp32 CUDA tensor of at least R_max x H elements)."""
     e, i, h = w1.shape
     shape = make_shape(num_tokens, h, i, e, k, weight_layout)
     _layer_sizes(0, h, e, i, x_perm=(x_perm, max_padded_rows(shape) * h),
                  offsets=(offsets, e + 1), **_bf16_weights(e, i, h, w1, w3, w2))
-    y = torch.zeros((max_padded_rows(shape), h), dtype=torch.float32, device=x_perm.device)
+    y = _out_rows(y, max_padded_rows(shape), h, x_perm.device)
     _check(lib().moe_grouped_swiglu(ctypes.byref(shape), _dev(x_perm, "x_perm", torch.bfloat16),
                                     _dev(offsets, "offsets", torch.int32),
                                     _dev(w1, "w1", torch.bfloat16), _dev(w3, "w3", torch.bfloat16),
@@ -484,13 +510,14 @@ def quantize_int8(w1, w3, w2, stream=None) -> Int8Experts:
 
 
 def grouped_swiglu_w8(x_perm, offsets, experts: Int8Experts, num_tokens: int, k: int, ws,
-                      stream=None):
-    """grouped_swiglu with int8 expert weights: y_perm [R_max, H] fp32."""
+                      stream=None, y=None):
+    """grouped_swiglu with int8 expert weights: y_perm [R_max, H] fp32 (into `y` when
+    given)."""
     e, i, h = experts.q1.shape
     shape = make_shape(num_tokens, h, i, e, k)
     _layer_sizes(0, h, e, i, x_perm=(x_perm, max_padded_rows(shape) * h),
                  offsets=(offsets, e + 1), **_quant_weights(e, i, h, experts, 8))
-    y = torch.zeros((max_padded_rows(shape), h), dtype=torch.float32, device=x_perm.device)
+    y = _out_rows(y, max_padded_rows(shape), h, x_perm.device)
     _check(lib().moe_grouped_swiglu_w8(ctypes.byref(shape), _dev(x_perm, "x_perm", torch.bfloat16),
                                        _dev(offsets, "offsets", torch.int32), *experts.pointers(),
                                        _dev(y, "y_perm"), _dev(ws, "ws"), ws.numel(),
@@ -539,13 +566,14 @@ def quantize_int4(w1, w3, w2, stream=None) -> Int4Experts:
 
 
 def grouped_swiglu_w4(x_perm, offsets, experts: Int4Experts, num_tokens: int, k: int, ws,
-                      stream=None):
-    """grouped_swiglu with 4-bit expert weights: y_perm [R_max, H] fp32."""
+                      stream=None, y=None):
+    """grouped_swiglu with 4-bit expert weights: y_perm [R_max, H] fp32 (into `y` when
+    given)."""
     e, i, h2 = experts.q1.shape
     shape = make_shape(num_tokens, 2 * h2, i, e, k)
     _layer_sizes(0, 2 * h2, e, i, x_perm=(x_perm, max_padded_rows(shape) * 2 * h2),
                  offsets=(offsets, e + 1), **_quant_weights(e, i, 2 * h2, experts, 4))
-    y = torch.zeros((max_padded_rows(shape), 2 * h2), dtype=torch.float32, device=x_perm.device)
+    y = _out_rows(y, max_padded_rows(shape), 2 * h2, x_perm.device)
     _check(lib().moe_grouped_swiglu_w4(ctypes.byref(shape), _dev(x_perm, "x_perm", torch.bfloat16),
                                        _dev(offsets, "offsets", torch.int32), *experts.pointers(),
                                        _dev(y, "y_perm"), _dev(ws, "ws"), ws.numel(),
@@ -586,3 +614,101 @@ def gather_rows(src, index, stream=None):
                                  _dev(index, "index", torch.int64) if n else None, n, row_bytes,
                                  _dev(out, "dst") if n else None, _stream(stream)))
     return out
+
+
+# ---- expert parallelism over peer memory ----
+
+IPC_HANDLE_BYTES = 64
+
+
+def ipc_alloc(nbytes: int):
+    """A device buffer other processes can map: (device address, IPC handle bytes). The
+    caller frees it with ipc_free once every other process has unmapped it."""
+    ptr = _P()
+    handle = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    _check(lib().moe_ipc_alloc(int(nbytes), ctypes.byref(ptr), ctypes.cast(handle, _P)))
+    return int(ptr.value), handle.raw
+
+
+def ipc_open(handle: bytes) -> int:
+    """Address in this process of another process's ipc_alloc buffer."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError(f"an IPC handle has {IPC_HANDLE_BYTES} bytes, got {len(handle)}")
+    buf = ctypes.create_string_buffer(bytes(handle), IPC_HANDLE_BYTES)
+    ptr = _P()
+    _check(lib().moe_ipc_open(ctypes.cast(buf, _P), ctypes.byref(ptr)))
+    return int(ptr.value)
+
+
+def ipc_close(ptr: int) -> None:
+    _check(lib().moe_ipc_close(ptr))
+
+
+def ipc_free(ptr: int) -> None:
+    _check(lib().moe_ipc_free(ptr))
+
+
+class _DeviceArray:
+    """A contiguous device array described to torch by its address
+    (__cuda_array_interface__); torch.as_tensor then wraps it without copying."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (int(ptr), False), "version": 2, "strides": None}
+
+
+_TYPESTR = {torch.bfloat16: ("<i2", torch.int16), torch.float32: ("<f4", torch.float32),
+            torch.int32: ("<i4", torch.int32), torch.int64: ("<i8", torch.int64)}
+
+
+def tensor_at(ptr: int, shape, dtype, device) -> torch.Tensor:
+    """A tensor over device memory this library allocated (it does not own the memory:
+    keep the buffer alive while the tensor is used)."""
+    typestr, base = _TYPESTR[dtype]
+    t = torch.as_tensor(_DeviceArray(ptr, shape, typestr), device=device)
+    return t.view(dtype) if base != dtype else t
+
+
+def scatter_rows_peer(src, src_index, dst_rank, dst_row, dst_bases, dst_rows: int, bad=None,
+                      stream=None) -> None:
+    """Row dst_row[i] of buffer dst_bases[dst_rank[i]] = src[src_index[i]] for every i.
+    src: 2-D CUDA tensor (rows a multiple of 16 bytes); src_index, dst_row int64 and
+    dst_rank int32 CUDA tensors of one length; dst_bases: int64 CUDA tensor of device
+    addresses (this GPU's buffers or ipc_open mappings), each buffer dst_rows rows of
+    src's row size. Out-of-range rows are skipped and counted into `bad` (int32 CUDA
+    tensor of one element) when given."""
+    if src.dim() != 2:
+        raise ValueError("src must be 2-D")
+    n = src_index.numel()
+    if dst_rank.numel() != n or dst_row.numel() != n:
+        raise ValueError("src_index, dst_rank and dst_row must have the same length")
+    if n == 0:
+        return
+    _check(lib().moe_scatter_rows_peer(
+        _dev(src, "src") if src.shape[0] else None, src.shape[0],
+        _dev(src_index, "src_index", torch.int64), _dev(dst_rank, "dst_rank", torch.int32),
+        _dev(dst_row, "dst_row", torch.int64), n, _dev(dst_bases, "dst_bases", torch.int64),
+        dst_bases.numel(), int(dst_rows), src.shape[1] * src.element_size(),
+        _dev(bad, "bad", torch.int32, True), _stream(stream)))
+
+
+def combine_peer(y_bases, y_rows: int, slot_rank, slot_row, topk_w, hidden: int, residual=None,
+                 bad=None, stream=None):
+    """out [T, hidden] bf16 = residual + sum_j topk_w[:, j] * (row slot_row[t k + j] of
+    the fp32 buffer y_bases[slot_rank[t k + j]]), moe_combine's arithmetic. y_bases:
+    int64 CUDA tensor of device addresses, each buffer y_rows x hidden fp32; slot_rank
+    int32 and slot_row int64 CUDA tensors [T, k]; topk_w fp32 [T, k]."""
+    t, k = topk_w.shape
+    _sized("slot_rank", slot_rank, t * k)
+    _sized("slot_row", slot_row, t * k)
+    _sized("residual", residual, t * hidden)
+    out = torch.empty((t, hidden), dtype=torch.bfloat16, device=topk_w.device)
+    if t == 0:
+        return out
+    _check(lib().moe_combine_peer(
+        _dev(y_bases, "y_bases", torch.int64), y_bases.numel(), int(y_rows),
+        _dev(slot_rank, "slot_rank", torch.int32), _dev(slot_row, "slot_row", torch.int64),
+        _dev(topk_w, "topk_w", torch.float32), _dev(residual, "residual", torch.bfloat16, True),
+        _dev(out, "out"), t, k, hidden, _dev(bad, "bad", torch.int32, True), _stream(stream)))
+    return out
+

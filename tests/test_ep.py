@@ -47,15 +47,35 @@ class OracleOps:
         out[ok] = src[index[ok]]
         return out
 
-    def grouped_swiglu(self, x_groups, offsets, w1, w3, w2, rows):
-        y = torch.zeros((x_groups.shape[0], w2.shape[1]), dtype=torch.float64)
+    def grouped_swiglu(self, x_groups, offsets, w1, w3, w2, rows, y=None):
+        out = torch.zeros((x_groups.shape[0], w2.shape[1]), dtype=torch.float64)
         off = offsets.tolist()
         for e in range(w1.shape[0]):
             a, b = off[e], off[e + 1]
             if b > a:
                 rows_e = self.O.to_f64(x_groups[a:b])
-                y[a:b] = torch.from_numpy(self.O.swiglu_expert(rows_e, w1[e], w3[e], w2[e]))
+                out[a:b] = torch.from_numpy(self.O.swiglu_expert(rows_e, w1[e], w3[e], w2[e]))
+        if y is None:
+            return out
+        y[:out.shape[0]] = out
         return y
+
+    def scatter_rows_peer(self, src, src_index, dst_rank, dst_row, dst_bases, dst_rows):
+        """dst_bases: every rank's x_local (CPU tensors in shared memory)."""
+        for i, r, d in zip(src_index.tolist(), dst_rank.tolist(), dst_row.tolist()):
+            assert 0 <= d < dst_rows
+            dst_bases[r][d] = src[i]
+
+    def combine_peer(self, y_bases, y_rows, slot_rank, slot_row, topk_w, hidden, residual):
+        t, k = topk_w.shape
+        out = torch.zeros((t, hidden), dtype=torch.float64)
+        ranks, rows = slot_rank.reshape(t, k), slot_row.reshape(t, k)
+        for i in range(t):
+            for j in range(k):
+                out[i] += topk_w[i, j] * y_bases[int(ranks[i, j])][int(rows[i, j])]
+        if residual is not None:
+            out += residual.double()
+        return out
 
     def grouped_swiglu_quantized(self, x_groups, offsets, experts, rows):
         """Half-precision experts on dequantised weights (experts.deq = fp64 w1, w3, w2
@@ -311,3 +331,106 @@ def test_shard_quantized_slices_are_valid_layouts():
             assert np.array_equal(got_s.reshape(-1, kk // 64), s16[lo * r:hi * r])
     with pytest.raises(ValueError):
         ep.shard_quantized(ex, 0, 3)
+
+
+# ---- the peer-memory exchange (ep.peer_plan, ep.forward_ep_peer) ----
+
+def test_peer_plan_random_worlds_place_rows_as_the_exchange_does():
+    # every rank stores its rows straight into the owners' groups; the owners' groups
+    # must hold what the all-to-all path regroups there, pad rows untouched, and every
+    # x_perm row must know where its output is
+    rng = np.random.default_rng(43)
+    for trial in range(60):
+        world = int(rng.choice([1, 2, 4]))
+        e_loc = int(rng.integers(1, 4))
+        e_total = world * e_loc
+        counts = rng.choice([0, 1, 3, 17, 127, 128, 129, 260], size=(world, e_total)).tolist()
+        x_perm, plans, local, _ = _simulate_world(counts)
+        offs = [[0] + np.cumsum([(n + 127) // 128 * 128 for n in counts[r]]).tolist()
+                for r in range(world)]
+        peer = [_lists(ep.peer_plan(offs[r], counts, r, world)) for r in range(world)]
+        owners = [[None] * peer[s]["local_offsets"][-1] for s in range(world)]
+        for r in range(world):
+            p = peer[r]
+            assert p["send_index"] == plans[r]["send_index"]
+            for i, d, row in zip(p["send_index"], p["dst_rank"], p["dst_row"]):
+                assert owners[d][row] is None          # no row is written twice
+                owners[d][row] = x_perm[r][i]
+            n_rows = len(x_perm[r])
+            assert len(p["row_rank"]) == n_rows and len(p["row_dst"]) == n_rows
+            for i in range(n_rows):
+                if x_perm[r][i] is None:
+                    assert p["row_rank"][i] == -1 and p["row_dst"][i] == -1
+        for s in range(world):
+            assert peer[s]["local_offsets"] == plans[s]["local_offsets"]
+            assert peer[s]["n_recv"] == sum(plans[s]["recv_rows"])
+            assert owners[s] == local[s]
+        for r in range(world):
+            for i, row in enumerate(x_perm[r]):
+                if row is not None:
+                    assert owners[peer[r]["row_rank"][i]][peer[r]["row_dst"][i]] == row
+
+
+def test_peer_rows_needed_covers_every_routing():
+    # all of every rank's rows routed to one owner, in E_loc groups
+    for world, t, k, e_loc in ((1, 5, 2, 4), (2, 300, 2, 4), (4, 129, 8, 2)):
+        worst = world * t * k
+        groups = [(worst + 127) // 128 * 128] + [0] * (e_loc - 1)
+        assert sum(groups) <= ep.peer_rows_needed(t, k, world, e_loc)
+
+
+def _rank_peer(rank, world, port, q, tokens, e, k, bias, shared):
+    import datetime
+    import sys
+    from types import SimpleNamespace
+    import torch.distributed as dist
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from sparse_mixture_experts_09_b200 import ep as EP
+    from tests.test_ep import OracleOps, _layer_inputs
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    x, wr, w1, w3, w2, res = _layer_inputs(sum(tokens), 32, 48, e, seed=7)
+    lo = sum(tokens[:rank])
+    mine = slice(lo, lo + tokens[rank])
+    b = None if bias is None else torch.tensor(bias, dtype=torch.float64)
+    # the world's receive buffers: CPU tensors in shared memory, indexed by rank
+    bufs = SimpleNamespace(rows=shared[0][0].shape[0], hidden=32, x_local=shared[rank][0],
+                           y_local=shared[rank][1], x_bases=[t[0] for t in shared],
+                           y_bases=[t[1] for t in shared])
+    l1, l3, l2 = EP.shard_experts(w1, w3, w2, rank, world)
+    out = EP.forward_ep_peer(x[mine], wr, l1, l3, l2, k, e, bufs, residual=res[mine],
+                             logit_bias=b, ops=OracleOps(), barrier=dist.barrier)
+    q.put((rank, out.double().numpy()))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,tokens,e,k,bias", [
+    (2, [5, 9], 4, 2, None),
+    (4, [3, 0, 11, 6], 8, 2, None),
+    (2, [7, 4], 4, 2, [30.0, 30.0, -30.0, -30.0]),
+])
+def test_peer_layer_equals_single_process_layer(world, tokens, e, k, bias):
+    from oracle import moe_oracle as O
+    rows = ep.peer_rows_needed(max(tokens), k, world, e // world)
+    shared = [(torch.zeros((rows, 32), dtype=torch.bfloat16).share_memory_(),
+               torch.zeros((rows, 32), dtype=torch.float64).share_memory_()) for _ in range(world)]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_peer, args=(r, world, port, q, tokens, e, k, bias, shared))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    got = np.concatenate([got[r] for r in range(world)])
+    x, wr, w1, w3, w2, res = _layer_inputs(sum(tokens), 32, 48, e, seed=7)
+    b = None if bias is None else np.asarray(bias)
+    ref = O.moe_layer(x, wr, w1, w3, w2, k, residual=res, logit_bias=b, mode="exact")
+    np.testing.assert_allclose(got, ref["out"], rtol=1e-12, atol=1e-12)
+
