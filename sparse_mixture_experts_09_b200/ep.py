@@ -330,7 +330,8 @@ def peer_plan(offsets, counts_all, rank: int, world: int, device=None):
         owner's x_local (the owner's group for the expert, each group padded to 128 rows
         and holding the source ranks' rows in rank order);
       local_offsets [E_loc+1] (ints): this rank's own groups as an owner;
-      n_recv (int): the real rows this rank receives in them;
+      n_recv (int): the real rows this rank receives in them; owner_recv [world] (ints):
+        the real rows every owner receives (the same list on every rank);
       row_rank [offsets[-1]] int32, row_dst [offsets[-1]] int64: for each x_perm row,
         the owner and row of its expert output (-1 on pad rows).
     The sizes come to the host in one read."""
@@ -345,10 +346,12 @@ def peer_plan(offsets, counts_all, rank: int, world: int, device=None):
     group_start = (torch.cumsum(padded, 1) - padded).reshape(-1)
     before = (torch.cumsum(c, 0) - c)[rank]                  # rows of expert e from ranks < rank
     counts = c[rank]
-    mine = c[:, rank * e_loc:(rank + 1) * e_loc].sum().reshape(1)
-    host = torch.cat([offsets[-1:], counts.sum().reshape(1), mine, padded[rank]]).cpu()
-    n_rows, n_send, n_recv = int(host[0]), int(host[1]), int(host[2])
-    local_offsets = [0] + torch.cumsum(host[3:], 0).tolist()
+    owners = c.sum(0).reshape(world, e_loc).sum(1)             # real rows each owner receives
+    host = torch.cat([offsets[-1:], counts.sum().reshape(1), owners, padded[rank]]).cpu()
+    n_rows, n_send = int(host[0]), int(host[1])
+    owner_recv = host[2:2 + world].tolist()
+    n_recv = owner_recv[rank]
+    local_offsets = [0] + torch.cumsum(host[2 + world:], 0).tolist()
     grp, j = _segment_ranks(counts, n_send)
     send_index = offsets[:-1][grp] + j
     dst_rank = (grp // e_loc).to(torch.int32)
@@ -358,8 +361,8 @@ def peer_plan(offsets, counts_all, rank: int, world: int, device=None):
     row_dst = torch.full((n_rows,), -1, **i64)
     row_dst[send_index] = dst_row
     return {"send_index": send_index, "dst_rank": dst_rank, "dst_row": dst_row,
-            "local_offsets": local_offsets, "n_recv": n_recv, "row_rank": row_rank,
-            "row_dst": row_dst}
+            "local_offsets": local_offsets, "n_recv": n_recv, "owner_recv": owner_recv,
+            "row_rank": row_rank, "row_dst": row_dst}
 
 
 def peer_rows_needed(max_tokens: int, k: int, world: int, e_loc: int) -> int:
@@ -385,10 +388,11 @@ class PeerBuffers:
         self.device = device or torch.device("cuda", torch.cuda.current_device())
         self.rank = dist.get_rank(group)
         world = dist.get_world_size(group)
+        self._own, self._mapped = [], []
         x_ptr, x_h = moe.ipc_alloc(rows * hidden * 2)
+        self._own.append(x_ptr)
         y_ptr, y_h = moe.ipc_alloc(rows * hidden * 4)
-        self._own = [x_ptr, y_ptr]
-        self._mapped = []
+        self._own.append(y_ptr)
         self.x_local = moe.tensor_at(x_ptr, (rows, hidden), torch.bfloat16, self.device)
         self.y_local = moe.tensor_at(y_ptr, (rows, hidden), torch.float32, self.device)
         self.x_local.zero_()
@@ -505,11 +509,13 @@ def _forward_ep_peer(x, w_router, k, num_experts, held, inter, run_experts, bufs
     plan = peer_plan(offsets, counts_all, rank, world, device=dev)
     n_recv = plan["n_recv"]
     # the grouped GEMM's buffer rows for n_recv rows in E_loc groups (they cover the
-    # padded groups: local_offsets[-1] <= n_recv + 127 E_loc)
+    # padded groups: local_offsets[-1] <= n_recv + 127 E_loc). Every rank checks every
+    # owner from the same counts, so all ranks raise together and none is left waiting.
+    need = max(ops.padded_rows(n, e_loc) for n in plan["owner_recv"])
+    if need > bufs.rows:
+        raise ValueError(f"an owner receives {max(plan['owner_recv'])} rows; the grouped GEMM "
+                         f"needs {need} buffer rows, the buffers hold {bufs.rows}")
     rows_buf = ops.padded_rows(n_recv, e_loc)
-    if rows_buf > bufs.rows:
-        raise ValueError(f"this rank receives {n_recv} rows; the grouped GEMM needs "
-                         f"{rows_buf} buffer rows, the buffers hold {bufs.rows}")
     ops.scatter_rows_peer(perm["x_perm"], plan["send_index"], plan["dst_rank"], plan["dst_row"],
                           bufs.x_bases, bufs.rows)
     barrier()

@@ -364,6 +364,7 @@ def test_peer_plan_random_worlds_place_rows_as_the_exchange_does():
         for s in range(world):
             assert peer[s]["local_offsets"] == plans[s]["local_offsets"]
             assert peer[s]["n_recv"] == sum(plans[s]["recv_rows"])
+            assert peer[s]["owner_recv"] == [sum(plans[o]["recv_rows"]) for o in range(world)]
             assert owners[s] == local[s]
         for r in range(world):
             for i, row in enumerate(x_perm[r]):
@@ -400,9 +401,12 @@ def _rank_peer(rank, world, port, q, tokens, e, k, bias, shared):
                            y_local=shared[rank][1], x_bases=[t[0] for t in shared],
                            y_bases=[t[1] for t in shared])
     l1, l3, l2 = EP.shard_experts(w1, w3, w2, rank, world)
-    out = EP.forward_ep_peer(x[mine], wr, l1, l3, l2, k, e, bufs, residual=res[mine],
-                             logit_bias=b, ops=OracleOps(), barrier=dist.barrier)
-    q.put((rank, out.double().numpy()))
+    try:
+        out = EP.forward_ep_peer(x[mine], wr, l1, l3, l2, k, e, bufs, residual=res[mine],
+                                 logit_bias=b, ops=OracleOps(), barrier=dist.barrier)
+        q.put((rank, out.double().numpy()))
+    except ValueError as err:
+        q.put((rank, f"raised: {err}"))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -415,6 +419,22 @@ def _rank_peer(rank, world, port, q, tokens, e, k, bias, shared):
 def test_peer_layer_equals_single_process_layer(world, tokens, e, k, bias):
     from oracle import moe_oracle as O
     rows = ep.peer_rows_needed(max(tokens), k, world, e // world)
+    got = _run_peer(world, tokens, e, k, bias, rows)
+    got = np.concatenate([got[r] for r in range(world)])
+    x, wr, w1, w3, w2, res = _layer_inputs(sum(tokens), 32, 48, e, seed=7)
+    b = None if bias is None else np.asarray(bias)
+    ref = O.moe_layer(x, wr, w1, w3, w2, k, residual=res, logit_bias=b, mode="exact")
+    np.testing.assert_allclose(got, ref["out"], rtol=1e-12, atol=1e-12)
+
+
+def test_peer_layer_too_small_buffers_raise_on_every_rank():
+    # all tokens routed to rank 0's experts: rank 0 would need more rows than the
+    # buffers hold; every rank sees it from the gathered counts and raises (none waits)
+    got = _run_peer(2, [7, 4], 4, 2, [30.0, 30.0, -30.0, -30.0], rows=256)
+    assert all(isinstance(v, str) and v.startswith("raised") for v in got.values()), got
+
+
+def _run_peer(world, tokens, e, k, bias, rows):
     shared = [(torch.zeros((rows, 32), dtype=torch.bfloat16).share_memory_(),
                torch.zeros((rows, 32), dtype=torch.float64).share_memory_()) for _ in range(world)]
     ctx = mp.get_context("spawn")
@@ -428,9 +448,5 @@ def test_peer_layer_equals_single_process_layer(world, tokens, e, k, bias):
     for p in procs:
         p.join(120)
         assert p.exitcode == 0
-    got = np.concatenate([got[r] for r in range(world)])
-    x, wr, w1, w3, w2, res = _layer_inputs(sum(tokens), 32, 48, e, seed=7)
-    b = None if bias is None else np.asarray(bias)
-    ref = O.moe_layer(x, wr, w1, w3, w2, k, residual=res, logit_bias=b, mode="exact")
-    np.testing.assert_allclose(got, ref["out"], rtol=1e-12, atol=1e-12)
+    return got
 
