@@ -389,6 +389,18 @@ class PeerBuffers:
         self.rank = dist.get_rank(group)
         world = dist.get_world_size(group)
         self._own, self._mapped = [], []
+        try:
+            self._setup(moe, rows, hidden, group, world, share)
+        except BaseException:
+            # nothing half-made stays behind: unmap what was mapped, free what was made
+            for p in self._mapped:
+                moe.ipc_close(p)
+            for p in self._own:
+                moe.ipc_free(p)
+            self._own, self._mapped = [], []
+            raise
+
+    def _setup(self, moe, rows, hidden, group, world, share):
         x_ptr, x_h = moe.ipc_alloc(rows * hidden * 2)
         self._own.append(x_ptr)
         y_ptr, y_h = moe.ipc_alloc(rows * hidden * 4)
@@ -406,8 +418,6 @@ class PeerBuffers:
         handles = share((x_h, y_h, rows, hidden))
         # the stores and loads index every rank's buffers with this rank's row count
         if any((rr, hh) != (rows, hidden) for _, _, rr, hh in handles):
-            for p in self._own:
-                moe.ipc_free(p)
             raise ValueError("every rank's PeerBuffers must have the same rows and hidden size: "
                              f"{[(rr, hh) for _, _, rr, hh in handles]}")
         xs, ys = [], []
@@ -417,8 +427,9 @@ class PeerBuffers:
                 ys.append(y_ptr)
             else:
                 xs.append(moe.ipc_open(xh))
+                self._mapped.append(xs[-1])
                 ys.append(moe.ipc_open(yh))
-                self._mapped += [xs[-1], ys[-1]]
+                self._mapped.append(ys[-1])
         self.x_bases = torch.tensor(xs, dtype=torch.int64, device=self.device)
         self.y_bases = torch.tensor(ys, dtype=torch.int64, device=self.device)
 
