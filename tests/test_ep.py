@@ -77,19 +77,22 @@ class OracleOps:
             out += residual.double()
         return out
 
-    def grouped_swiglu_quantized(self, x_groups, offsets, experts, rows):
+    def grouped_swiglu_quantized(self, x_groups, offsets, experts, rows, y=None):
         """Half-precision experts on dequantised weights (experts.deq = fp64 w1, w3, w2
         of this rank's experts), as the oracle's f16_experts mode computes them."""
         O = self.O
         d1, d3, d2 = experts.deq
-        y = torch.zeros((x_groups.shape[0], d2.shape[1]), dtype=torch.float64)
+        out = torch.zeros((x_groups.shape[0], d2.shape[1]), dtype=torch.float64)
         off = offsets.tolist()
         for e in range(d1.shape[0]):
             a, b = off[e], off[e + 1]
             if b > a:
                 x16 = O.round_f16(O.to_f64(x_groups[a:b]))
                 h = O.silu(x16 @ d1[e].T) * (x16 @ d3[e].T)
-                y[a:b] = torch.from_numpy(O.round_f16(h) @ d2[e].T)
+                out[a:b] = torch.from_numpy(O.round_f16(h) @ d2[e].T)
+        if y is None:
+            return out
+        y[:out.shape[0]] = out
         return y
 
     def combine(self, y_perm, row_of, topk_w, residual, num_experts, intermediate_size):
@@ -380,7 +383,7 @@ def test_peer_rows_needed_covers_every_routing():
         assert sum(groups) <= ep.peer_rows_needed(t, k, world, e_loc)
 
 
-def _rank_peer(rank, world, port, q, tokens, e, k, bias, shared):
+def _rank_peer(rank, world, port, q, tokens, e, k, bias, shared, quant=False):
     import datetime
     import sys
     from types import SimpleNamespace
@@ -392,18 +395,29 @@ def _rank_peer(rank, world, port, q, tokens, e, k, bias, shared):
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
-    x, wr, w1, w3, w2, res = _layer_inputs(sum(tokens), 32, 48, e, seed=7)
+    hd, inter = (128, 128) if quant else (32, 48)
+    x, wr, w1, w3, w2, res = _layer_inputs(sum(tokens), hd, inter, e, seed=7)
     lo = sum(tokens[:rank])
     mine = slice(lo, lo + tokens[rank])
     b = None if bias is None else torch.tensor(bias, dtype=torch.float64)
     # the world's receive buffers: CPU tensors in shared memory, indexed by rank
-    bufs = SimpleNamespace(rows=shared[0][0].shape[0], hidden=32, x_local=shared[rank][0],
+    bufs = SimpleNamespace(rows=shared[0][0].shape[0], hidden=hd, x_local=shared[rank][0],
                            y_local=shared[rank][1], x_bases=[t[0] for t in shared],
                            y_bases=[t[1] for t in shared])
-    l1, l3, l2 = EP.shard_experts(w1, w3, w2, rank, world)
     try:
-        out = EP.forward_ep_peer(x[mine], wr, l1, l3, l2, k, e, bufs, residual=res[mine],
-                                 logit_bias=b, ops=OracleOps(), barrier=dist.barrier)
+        if quant:
+            from tests.test_ep import _dequantised_4bit
+            d = _dequantised_4bit(w1, w3, w2)
+            el = e // world
+            part = [t[rank * el:(rank + 1) * el] for t in d]
+            local = SimpleNamespace(q1=torch.from_numpy(part[0]), deq=part)
+            out = EP.forward_ep_peer_quantized(x[mine], wr, local, k, e, bufs,
+                                               residual=res[mine], logit_bias=b,
+                                               ops=OracleOps(), barrier=dist.barrier)
+        else:
+            l1, l3, l2 = EP.shard_experts(w1, w3, w2, rank, world)
+            out = EP.forward_ep_peer(x[mine], wr, l1, l3, l2, k, e, bufs, residual=res[mine],
+                                     logit_bias=b, ops=OracleOps(), barrier=dist.barrier)
         q.put((rank, out.double().numpy()))
     except ValueError as err:
         q.put((rank, f"raised: {err}"))
@@ -434,13 +448,15 @@ def test_peer_layer_too_small_buffers_raise_on_every_rank():
     assert all(isinstance(v, str) and v.startswith("raised") for v in got.values()), got
 
 
-def _run_peer(world, tokens, e, k, bias, rows):
-    shared = [(torch.zeros((rows, 32), dtype=torch.bfloat16).share_memory_(),
-               torch.zeros((rows, 32), dtype=torch.float64).share_memory_()) for _ in range(world)]
+def _run_peer(world, tokens, e, k, bias, rows, quant=False):
+    hd = 128 if quant else 32
+    shared = [(torch.zeros((rows, hd), dtype=torch.bfloat16).share_memory_(),
+               torch.zeros((rows, hd), dtype=torch.float64).share_memory_()) for _ in range(world)]
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_peer, args=(r, world, port, q, tokens, e, k, bias, shared))
+    procs = [ctx.Process(target=_rank_peer, args=(r, world, port, q, tokens, e, k, bias, shared,
+                                                  quant))
              for r in range(world)]
     for p in procs:
         p.start()
@@ -449,4 +465,18 @@ def _run_peer(world, tokens, e, k, bias, rows):
         p.join(120)
         assert p.exitcode == 0
     return got
+
+
+def test_peer_layer_4bit_equals_single_process_layer():
+    # forward_ep_peer_quantized: each owner computes its experts in half precision on
+    # the dequantised weights, from the rows the ranks stored into its buffer
+    from oracle import moe_oracle as O
+    tokens, e, k = [6, 11], 4, 2
+    rows = ep.peer_rows_needed(max(tokens), k, 2, e // 2)
+    got = _run_peer(2, tokens, e, k, None, rows, quant=True)
+    got = np.concatenate([got[r] for r in range(2)])
+    x, wr, w1, w3, w2, res = _layer_inputs(sum(tokens), 128, 128, e, seed=7)
+    d1, d3, d2 = _dequantised_4bit(w1, w3, w2)
+    ref = O.moe_layer(x, wr, d1, d3, d2, k, mode="f16_experts")
+    np.testing.assert_allclose(got, O.to_f64(res) + ref["routed"], rtol=1e-12, atol=1e-12)
 
