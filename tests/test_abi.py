@@ -105,3 +105,29 @@ def test_workspace_holds_every_region(L, t, h, i, e, k):
     # host entry points: two staging slots for x and the residual, one for the output
     assert M.workspace_size_host(s) - ws >= 5 * t * h * 2
     assert ws % 256 == 0 and M.workspace_size_host(s) % 256 == 0
+
+
+def test_peer_memory_entry_points_validate_on_the_host(L):
+    # every rejection below happens before any CUDA call
+    ok, invalid, unsupported = 0, 1, 2
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: each call fails validation first
+    ptr = ctypes.c_void_p()
+    handle = ctypes.create_string_buffer(64)
+    assert L.moe_ipc_alloc(0, ctypes.byref(ptr), ctypes.cast(handle, ctypes.c_void_p)) == invalid
+    assert L.moe_ipc_alloc(16, None, ctypes.cast(handle, ctypes.c_void_p)) == invalid
+    assert L.moe_ipc_open(None, ctypes.byref(ptr)) == invalid
+    assert L.moe_ipc_close(None) == ok and L.moe_ipc_free(None) == ok
+    # scatter: bad row size, bad world, negative counts; zero rows is a no-op
+    assert L.moe_scatter_rows_peer(fake, 4, fake, fake, fake, 2, fake, 2, 4, 10, None, None) == invalid
+    assert L.moe_scatter_rows_peer(fake, 4, fake, fake, fake, 2, fake, 0, 4, 16, None, None) == invalid
+    assert L.moe_scatter_rows_peer(fake, 4, fake, fake, fake, -1, fake, 2, 4, 16, None, None) == invalid
+    assert L.moe_scatter_rows_peer(None, 0, None, None, None, 0, None, 2, 4, 16, None, None) == ok
+    assert L.moe_scatter_rows_peer(fake, 4, None, fake, fake, 2, fake, 2, 4, 16, None, None) == invalid
+    # combine: k outside [1, 8], hidden not a multiple of 8, bad world; no tokens is a no-op
+    args = lambda k, h, world, t=3: (fake, world, 4, fake, fake, fake, None, fake, t, k, h, None, None)
+    assert L.moe_combine_peer(*args(9, 64, 2)) == unsupported
+    assert b"k must be in [1, 8]" in L.moe_last_error()
+    assert L.moe_combine_peer(*args(2, 60, 2)) == unsupported
+    assert b"hidden" in L.moe_last_error()
+    assert L.moe_combine_peer(*args(2, 64, 0)) == invalid
+    assert L.moe_combine_peer(*args(2, 64, 2, t=0)) == ok
